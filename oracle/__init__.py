@@ -1,0 +1,152 @@
+"""float64 CPU oracle for the selective scan (S6) forward and the recurrent step.
+
+TEST INFRASTRUCTURE. Only tests/, the package smoke check and the benchmark's
+CPU-baseline leg may import this package. It shares no code with the CUDA path.
+
+The arithmetic lives in ``ssm_oracle.c`` (one sequential loop over time per
+channel, in double); this module only marshals numpy arrays into it.
+Storage dtypes: ``"f32"`` (numpy float32) or ``"bf16"`` (numpy uint16 holding
+bfloat16 bit patterns). Results come back as float64.
+"""
+import ctypes
+import os
+
+import numpy as np
+
+from . import build as _build
+
+DELTA_SOFTPLUS = 1
+EXACT_ZOH = 2
+
+
+def _open(path):
+    lib = ctypes.CDLL(path)
+    vp, i64, c_int, c_uint = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.c_uint
+    lib.oracle_scan_f64.argtypes = [i64, i64, i64, i64, c_int, c_uint] + [vp] * 11 + [c_int]
+    lib.oracle_scan_f64.restype = c_int
+    lib.oracle_step_f64.argtypes = [i64, i64, i64, c_int, c_uint] + [vp] * 10 + [c_int]
+    lib.oracle_step_f64.restype = c_int
+    return lib
+
+
+def _ptr(a):
+    return None if a is None else a.ctypes.data_as(ctypes.c_void_p)
+
+
+def _tok(a, dtype, shape, name):
+    """Check a token-type array (x, dt, z, B, C) and return it contiguous."""
+    want = np.float32 if dtype == "f32" else np.uint16
+    a = np.ascontiguousarray(a)
+    if a.dtype != want or a.shape != tuple(shape):
+        raise ValueError(f"{name}: expected {want.__name__}{tuple(shape)}, got {a.dtype}{a.shape}")
+    return a
+
+
+def _f32(a, shape, name):
+    if a is None:
+        return None
+    a = np.ascontiguousarray(a, dtype=np.float32)
+    if a.shape != tuple(shape):
+        raise ValueError(f"{name}: expected shape {tuple(shape)}, got {a.shape}")
+    return a
+
+
+def default_threads():
+    return len(os.sched_getaffinity(0)) if hasattr(os, "sched_getaffinity") else (os.cpu_count() or 1)
+
+
+class Oracle:
+    """The oracle bound to one compiled library (the default build, or a test's variant)."""
+
+    def __init__(self, path=None):
+        self.path = path or _build.build()
+        self.lib = _open(self.path)
+
+    def scan(self, x, dt, A, B, C, D=None, z=None, dt_bias=None, h0=None, dtype="f32",
+             delta_softplus=True, exact_zoh=False, nthreads=None):
+        return _scan(self.lib, x, dt, A, B, C, D, z, dt_bias, h0, dtype, delta_softplus,
+                     exact_zoh, nthreads)
+
+    def step(self, x, dt, A, B, C, h, D=None, z=None, dt_bias=None, dtype="f32",
+             delta_softplus=True, exact_zoh=False, nthreads=None):
+        return _step(self.lib, x, dt, A, B, C, h, D, z, dt_bias, dtype, delta_softplus,
+                     exact_zoh, nthreads)
+
+
+_default = None
+
+
+def default():
+    global _default
+    if _default is None:
+        _default = Oracle()
+    return _default
+
+
+def scan(*args, **kw):
+    """Selective scan with the default oracle build; see ``_scan``."""
+    return default().scan(*args, **kw)
+
+
+def step(*args, **kw):
+    """One decode step with the default oracle build; see ``_step``."""
+    return default().step(*args, **kw)
+
+
+def _scan(lib, x, dt, A, B, C, D=None, z=None, dt_bias=None, h0=None, dtype="f32",
+          delta_softplus=True, exact_zoh=False, nthreads=None):
+    """Selective scan over a whole sequence.
+
+    x, dt, z: [Bsz, L, Dm]; B, C: [Bsz, L, N]; A: [Dm, N]; D, dt_bias: [Dm];
+    h0: [Bsz, Dm, N] (float32) or None for a zero initial state.
+    Returns (y [Bsz, L, Dm] float64, h_last [Bsz, Dm, N] float64).
+    """
+    Bsz, L, Dm = np.shape(x)
+    N = np.shape(A)[1]
+    x = _tok(x, dtype, (Bsz, L, Dm), "x")
+    dt = _tok(dt, dtype, (Bsz, L, Dm), "dt")
+    z = None if z is None else _tok(z, dtype, (Bsz, L, Dm), "z")
+    B = _tok(B, dtype, (Bsz, L, N), "B")
+    C = _tok(C, dtype, (Bsz, L, N), "C")
+    A = _f32(A, (Dm, N), "A")
+    D = _f32(D, (Dm,), "D")
+    dt_bias = _f32(dt_bias, (Dm,), "dt_bias")
+    h0 = _f32(h0, (Bsz, Dm, N), "h0")
+    y = np.empty((Bsz, L, Dm), dtype=np.float64)
+    h_last = np.empty((Bsz, Dm, N), dtype=np.float64)
+    flags = (DELTA_SOFTPLUS if delta_softplus else 0) | (EXACT_ZOH if exact_zoh else 0)
+    rc = lib.oracle_scan_f64(Bsz, L, Dm, N, 0 if dtype == "f32" else 1, flags,
+                             _ptr(x), _ptr(dt), _ptr(z), _ptr(B), _ptr(C), _ptr(A), _ptr(D),
+                             _ptr(dt_bias), _ptr(h0), _ptr(y), _ptr(h_last),
+                             default_threads() if nthreads is None else nthreads)
+    if rc != 0:
+        raise ValueError("oracle_scan_f64 rejected its arguments")
+    return y, h_last
+
+
+def _step(lib, x, dt, A, B, C, h, D=None, z=None, dt_bias=None, dtype="f32",
+          delta_softplus=True, exact_zoh=False, nthreads=None):
+    """One recurrent decode step. x, dt, z: [Bsz, Dm]; B, C: [Bsz, N];
+    h: float64 [Bsz, Dm, N], updated in place. Returns y [Bsz, Dm] float64."""
+    Bsz, Dm = np.shape(x)
+    N = np.shape(A)[1]
+    x = _tok(x, dtype, (Bsz, Dm), "x")
+    dt = _tok(dt, dtype, (Bsz, Dm), "dt")
+    z = None if z is None else _tok(z, dtype, (Bsz, Dm), "z")
+    B = _tok(B, dtype, (Bsz, N), "B")
+    C = _tok(C, dtype, (Bsz, N), "C")
+    A = _f32(A, (Dm, N), "A")
+    D = _f32(D, (Dm,), "D")
+    dt_bias = _f32(dt_bias, (Dm,), "dt_bias")
+    if not (isinstance(h, np.ndarray) and h.dtype == np.float64 and h.shape == (Bsz, Dm, N)
+            and h.flags.c_contiguous):
+        raise ValueError("h must be a C-contiguous float64 array of shape [Bsz, Dm, N]")
+    y = np.empty((Bsz, Dm), dtype=np.float64)
+    flags = (DELTA_SOFTPLUS if delta_softplus else 0) | (EXACT_ZOH if exact_zoh else 0)
+    rc = lib.oracle_step_f64(Bsz, Dm, N, 0 if dtype == "f32" else 1, flags,
+                             _ptr(x), _ptr(dt), _ptr(z), _ptr(B), _ptr(C), _ptr(A), _ptr(D),
+                             _ptr(dt_bias), _ptr(h), _ptr(y),
+                             default_threads() if nthreads is None else nthreads)
+    if rc != 0:
+        raise ValueError("oracle_step_f64 rejected its arguments")
+    return y

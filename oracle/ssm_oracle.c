@@ -1,0 +1,188 @@
+/*
+ * ssm_oracle.c -- float64 CPU oracle for the selective state space (S6) scan.
+ *
+ * TEST INFRASTRUCTURE. Only the test suite, the package's smoke check and the
+ * benchmark's CPU-baseline leg may load this code. It shares no source, header,
+ * table or helper with the CUDA path, and the CUDA path never calls it.
+ *
+ * What it computes is the plain definition, written out as a sequential loop
+ * over time for every channel, in double precision:
+ *
+ *   continuous model  h'(t) = A h(t) + B x(t),  y(t) = C h(t) + D x(t)
+ *       [SSM glossary (yapayzekasozluk.tr), "Temel Matematiksel Cerceve"]
+ *   selection         Delta_t = softplus(dt_raw_t + dt_bias), B_t, C_t per token,
+ *                     A fixed and acting through Delta
+ *       [Mamba summary (azimuth.plus), the selectivity paragraph]
+ *   discretisation    zero-order hold: Abar = exp(Delta * A); Bbar = Delta * B
+ *       (the pages name ZOH but print no Bbar formula; Delta * B is the reading
+ *        used for the scan. The exact-ZOH Bbar = (exp(Delta A) - 1) / A * B is
+ *        selectable because it is the form under which Theorem 1 holds exactly.)
+ *   recurrence        h_t = Abar_t (.) h_{t-1} + Bbar_t x_t
+ *       [Mamba summary, hardware-aware algorithm paragraph (parallel scan)]
+ *   readout           y_t = C_t . h_t + D x_t  (after the update of h_t)
+ *   gate              y_t <- y_t * silu(z_t),  silu(z) = z * sigma(z)
+ *       [Mamba summary, block-architecture paragraph (gate branch: SiLU, multiply)]
+ *   recurrent decode  one token: the same update with the state carried in place
+ *       [SSM blog (shakilmahmud.com), section 3 "dual form": recurrence at O(1)]
+ *
+ * Inputs are read in their storage type (float32, or bfloat16 given as raw
+ * 16-bit patterns) and widened exactly to double, so a comparison measures the
+ * error of the computation under test, not the quantisation of its inputs.
+ *
+ * Layouts (all row-major, contiguous):
+ *   x, dt, z : [Bsz, L, Dm]     B, C : [Bsz, L, N]
+ *   A : [Dm, N]   Dskip, dt_bias : [Dm]   h0, h_last : [Bsz, Dm, N]
+ *   y (double) : [Bsz, L, Dm]
+ */
+#include <math.h>
+#include <pthread.h>
+#include <stdint.h>
+#include <string.h>
+
+#define ORACLE_DELTA_SOFTPLUS 1u /* Delta = softplus(dt + dt_bias); else Delta = dt + dt_bias */
+#define ORACLE_EXACT_ZOH 2u      /* Bbar = (exp(Delta A) - 1) / A * B instead of Delta * B */
+
+/* Widen element i of a float32 (dtype 0) or bfloat16 (dtype 1) array to double. */
+static double widen(const void *p, int dtype, int64_t i) {
+    if (dtype == 0) return (double)((const float *)p)[i];
+    uint32_t bits = (uint32_t)((const uint16_t *)p)[i] << 16;
+    float f;
+    memcpy(&f, &bits, sizeof f);
+    return (double)f;
+}
+
+/* softplus(v) = log(1 + exp(v)), evaluated without overflow. */
+static double softplus(double v) {
+    return v > 0.0 ? v + log1p(exp(-v)) : log1p(exp(v));
+}
+
+static double sigmoid(double v) { return 1.0 / (1.0 + exp(-v)); }
+
+typedef struct {
+    int64_t Bsz, L, Dm, N;
+    int dtype;
+    unsigned flags;
+    const void *x, *dt, *z, *Bm, *Cm;
+    const float *A, *Dskip, *dt_bias, *h0;
+    double *y, *h_last;
+    const double *h0_f64; /* optional double initial state (used by the decode oracle) */
+    int64_t ch_begin, ch_end; /* channel range [begin, end) over b * Dm + d */
+} scan_job;
+
+/* One channel (b, d): the whole sequence, in time order. */
+static void scan_channel(const scan_job *J, int64_t b, int64_t d, double *h) {
+    const int64_t L = J->L, Dm = J->Dm, N = J->N;
+    for (int64_t n = 0; n < N; n++) {
+        int64_t hi = (b * Dm + d) * N + n;
+        h[n] = J->h0_f64 ? J->h0_f64[hi] : (J->h0 ? (double)J->h0[hi] : 0.0);
+    }
+    const double bias = J->dt_bias ? (double)J->dt_bias[d] : 0.0;
+    const double dskip = J->Dskip ? (double)J->Dskip[d] : 0.0;
+    for (int64_t t = 0; t < L; t++) {
+        const int64_t i = (b * L + t) * Dm + d;        /* token element (b, t, d) */
+        const int64_t bc = (b * L + t) * N;            /* row of B_t and C_t      */
+        const double v = widen(J->dt, J->dtype, i) + bias;
+        const double delta = (J->flags & ORACLE_DELTA_SOFTPLUS) ? softplus(v) : v;
+        const double xv = widen(J->x, J->dtype, i);
+        double y = 0.0;
+        for (int64_t n = 0; n < N; n++) {
+            const double a = (double)J->A[d * N + n];
+            const double abar = exp(delta * a);
+            double bbar;
+            if (J->flags & ORACLE_EXACT_ZOH)
+                bbar = (a != 0.0 ? expm1(delta * a) / a : delta) * widen(J->Bm, J->dtype, bc + n);
+            else
+                bbar = delta * widen(J->Bm, J->dtype, bc + n);
+            h[n] = abar * h[n] + bbar * xv;
+            y += widen(J->Cm, J->dtype, bc + n) * h[n];
+        }
+        y += dskip * xv;
+        if (J->z) {
+            const double zv = widen(J->z, J->dtype, i);
+            y *= zv * sigmoid(zv);
+        }
+        J->y[i] = y;
+    }
+    if (J->h_last)
+        for (int64_t n = 0; n < N; n++) J->h_last[(b * Dm + d) * N + n] = h[n];
+}
+
+static void *scan_worker(void *arg) {
+    const scan_job *J = (const scan_job *)arg;
+    double h[256];
+    for (int64_t c = J->ch_begin; c < J->ch_end; c++) scan_channel(J, c / J->Dm, c % J->Dm, h);
+    return NULL;
+}
+
+/*
+ * Full-sequence scan. Returns 0 on success, -1 on invalid arguments.
+ * Channels (b, d) are independent and are split over `nthreads` POSIX threads
+ * (nthreads <= 1 runs on the calling thread). Each channel is one plain loop.
+ */
+int oracle_scan_f64(int64_t Bsz, int64_t L, int64_t Dm, int64_t N, int dtype, unsigned flags,
+                    const void *x, const void *dt, const void *z, const void *Bm, const void *Cm,
+                    const float *A, const float *Dskip, const float *dt_bias, const float *h0,
+                    double *y, double *h_last, int nthreads) {
+    if (Bsz < 0 || L < 0 || Dm < 0 || N < 1 || N > 256 || (dtype != 0 && dtype != 1)) return -1;
+    if (!x || !dt || !Bm || !Cm || !A || !y) return -1;
+    scan_job base = {Bsz, L, Dm, N, dtype, flags, x, dt, z, Bm, Cm, A, Dskip, dt_bias, h0,
+                     y, h_last, NULL, 0, Bsz * Dm};
+    const int64_t nch = Bsz * Dm;
+    if (nthreads <= 1 || nch < 2) {
+        scan_worker(&base);
+        return 0;
+    }
+    if (nthreads > 512) nthreads = 512;
+    if (nthreads > nch) nthreads = (int)nch;
+    pthread_t tid[512];
+    scan_job jobs[512];
+    for (int k = 0; k < nthreads; k++) {
+        jobs[k] = base;
+        jobs[k].ch_begin = nch * k / nthreads;
+        jobs[k].ch_end = nch * (k + 1) / nthreads;
+        if (pthread_create(&tid[k], NULL, scan_worker, &jobs[k]) != 0) {
+            scan_worker(&jobs[k]); /* run inline if a thread cannot be started */
+            tid[k] = 0;
+        }
+    }
+    for (int k = 0; k < nthreads; k++)
+        if (tid[k]) pthread_join(tid[k], NULL);
+    return 0;
+}
+
+/*
+ * One recurrent decode step for every (b, d): a scan of length 1 whose state is
+ * read from and written back to `h` (double, [Bsz, Dm, N]). x, dt, z : [Bsz, Dm];
+ * B, C : [Bsz, N]; y (double) : [Bsz, Dm]. Returns 0, or -1 on invalid arguments.
+ */
+int oracle_step_f64(int64_t Bsz, int64_t Dm, int64_t N, int dtype, unsigned flags,
+                    const void *x, const void *dt, const void *z, const void *Bm, const void *Cm,
+                    const float *A, const float *Dskip, const float *dt_bias,
+                    double *h, double *y, int nthreads) {
+    if (Bsz < 0 || Dm < 0 || N < 1 || N > 256 || (dtype != 0 && dtype != 1)) return -1;
+    if (!x || !dt || !Bm || !Cm || !A || !h || !y) return -1;
+    /* A step is the scan with L = 1, started from h and writing its end state to h. */
+    scan_job base = {Bsz, 1, Dm, N, dtype, flags, x, dt, z, Bm, Cm, A, Dskip, dt_bias, NULL,
+                     y, h, h, 0, Bsz * Dm};
+    const int64_t nch = Bsz * Dm;
+    if (nthreads <= 1 || nch < 2) {
+        scan_worker(&base);
+        return 0;
+    }
+    if (nthreads > 512) nthreads = 512;
+    if (nthreads > nch) nthreads = (int)nch;
+    pthread_t tid[512];
+    scan_job jobs[512];
+    for (int k = 0; k < nthreads; k++) {
+        jobs[k] = base;
+        jobs[k].ch_begin = nch * k / nthreads;
+        jobs[k].ch_end = nch * (k + 1) / nthreads;
+        if (pthread_create(&tid[k], NULL, scan_worker, &jobs[k]) != 0) {
+            scan_worker(&jobs[k]);
+            tid[k] = 0;
+        }
+    }
+    for (int k = 0; k < nthreads; k++)
+        if (tid[k]) pthread_join(tid[k], NULL);
+    return 0;
+}

@@ -1,0 +1,77 @@
+"""Each plausible mistake planted in a copy of the oracle's C source must fail a pin.
+
+The copy is compiled into a temporary directory; the oracle as built is untouched.
+This shows that the pins constrain every term of the oracle: a dropped term, a
+wrong sign, a swapped or shifted index, a transposed operand.
+"""
+import os
+import subprocess
+
+import pytest
+
+import oracle
+from oracle import build as oracle_build
+from tests import oracle_pins
+
+MUTANTS = {
+    "drop_D_skip": ("y += dskip * xv;", "y += 0.0 * dskip * xv;"),
+    "wrong_sign_of_A": ("const double abar = exp(delta * a);", "const double abar = exp(-delta * a);"),
+    "drop_x_in_input": ("h[n] = abar * h[n] + bbar * xv;", "h[n] = abar * h[n] + bbar;"),
+    "readout_uses_B": ("y += widen(J->Cm, J->dtype, bc + n) * h[n];",
+                       "y += widen(J->Bm, J->dtype, bc + n) * h[n];"),
+    "gate_is_sigmoid": ("y *= zv * sigmoid(zv);", "y *= sigmoid(zv);"),
+    "softplus_negative_branch": ("return v > 0.0 ? v + log1p(exp(-v)) : log1p(exp(v));",
+                                 "return v > 0.0 ? v + log1p(exp(-v)) : log(exp(v));"),
+    "A_transposed": ("const double a = (double)J->A[d * N + n];",
+                     "const double a = (double)J->A[n * Dm + d];"),
+    "B_C_lagged_one_token": ("const int64_t bc = (b * L + t) * N;",
+                             "const int64_t bc = (b * L + (t > 0 ? t - 1 : 0)) * N;"),
+    "dt_bias_ignored": ("const double bias = J->dt_bias ? (double)J->dt_bias[d] : 0.0;",
+                        "const double bias = 0.0;"),
+    "h0_ignored": ("h[n] = J->h0_f64 ? J->h0_f64[hi] : (J->h0 ? (double)J->h0[hi] : 0.0);",
+                   "h[n] = J->h0_f64 ? J->h0_f64[hi] : 0.0;"),
+    "readout_before_update": ("h[n] = abar * h[n] + bbar * xv;\n            y += widen(J->Cm, J->dtype, bc + n) * h[n];",
+                              "y += widen(J->Cm, J->dtype, bc + n) * h[n];\n            h[n] = abar * h[n] + bbar * xv;"),
+    "bf16_widening_shift": ("uint32_t bits = (uint32_t)((const uint16_t *)p)[i] << 16;",
+                            "uint32_t bits = (uint32_t)((const uint16_t *)p)[i] << 15;"),
+    "exact_zoh_sign": ("expm1(delta * a) / a", "expm1(delta * a) / (-a)"),
+    "final_state_not_written": ("    if (J->h_last)\n", "    if (0)\n"),
+    "batch_time_transposed": ("const int64_t i = (b * L + t) * Dm + d;",
+                              "const int64_t i = (t * J->Bsz + b) * Dm + d;"),
+    "sigmoid_sign": ("static double sigmoid(double v) { return 1.0 / (1.0 + exp(-v)); }",
+                     "static double sigmoid(double v) { return 1.0 / (1.0 + exp(v)); }"),
+    "delta_times_A_squared": ("const double abar = exp(delta * a);", "const double abar = exp(delta * a * a);"),
+}
+
+
+def _build_variant(tmp_path, name, src):
+    c = tmp_path / f"{name}.c"
+    so = tmp_path / f"{name}.so"
+    c.write_text(src)
+    subprocess.check_call(["gcc", "-O2", "-std=c11", "-fPIC", "-shared", "-fno-fast-math",
+                           "-o", str(so), str(c), "-lm", "-lpthread"])
+    return oracle.Oracle(str(so))
+
+
+def _failed_pins(orc):
+    failed = []
+    for pin in oracle_pins.ALL_PINS:
+        try:
+            pin(orc)
+        except AssertionError:
+            failed.append(pin.__name__)
+    return failed
+
+
+def test_unmodified_copy_passes(tmp_path):
+    src = open(oracle_build.SRC).read()
+    assert _failed_pins(_build_variant(tmp_path, "same", src)) == []
+
+
+@pytest.mark.parametrize("name", sorted(MUTANTS))
+def test_mutant_is_caught(tmp_path, name):
+    src = open(oracle_build.SRC).read()
+    old, new = MUTANTS[name]
+    assert src.count(old) >= 1, f"mutation pattern for {name} not found in the oracle source"
+    failed = _failed_pins(_build_variant(tmp_path, name, src.replace(old, new)))
+    assert failed, f"mutant {name} passed every pin"
