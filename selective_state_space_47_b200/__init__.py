@@ -1,0 +1,173 @@
+"""B200-native selective state space (S6) scan: Python binding of libssmscan.so.
+
+Every step of the computation runs in the library's CUDA kernels; this module
+only checks tensors and passes their device pointers and the current CUDA stream
+through the C ABI (include/ssm_scan.h). PyTorch provides device memory and
+streams. There is no CPU fallback: without the built library, or without a CUDA
+device, the calls raise.
+
+    y = scan_fwd(x, dt, A, B, C, D, z, dt_bias)              # [B, L, D]
+    y, h_last = scan_fwd(..., return_last_state=True)         # h_last [B, D, N] fp32
+    y = step(x_t, dt_t, A, B_t, C_t, h, D, z_t, dt_bias)     # h [B, D, N] updated in place
+"""
+import ctypes
+
+import torch
+
+from . import _native
+from ._native import SSM_A_GENERAL, SSM_DELTA_SOFTPLUS
+
+__all__ = ["scan_fwd", "step", "workspace_size", "workspace_status", "ScanWorkspace"]
+
+_TOKEN_DTYPES = {torch.float32: _native.SSM_F32, torch.bfloat16: _native.SSM_BF16}
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream_handle(stream):
+    s = torch.cuda.current_stream() if stream is None else stream
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _need(t, name, shape, dtype, device):
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name}: expected shape {tuple(shape)}, got {tuple(t.shape)}")
+    if t.dtype != dtype:
+        raise TypeError(f"{name}: expected {dtype}, got {t.dtype}")
+    if t.device != device or t.device.type != "cuda":
+        raise ValueError(f"{name}: must be on {device} (a CUDA device)")
+    if not t.is_contiguous():
+        raise ValueError(f"{name}: must be contiguous")
+
+
+def _flags(delta_softplus, general_A):
+    return (SSM_DELTA_SOFTPLUS if delta_softplus else 0) | (SSM_A_GENERAL if general_A else 0)
+
+
+def _scan_args(x, dt, A, B, C, D, z, dt_bias, h0, y, h_last, flags):
+    a = _native.ScanArgs()
+    a.batch, a.seqlen, a.dim = x.shape
+    a.dstate = A.shape[1]
+    a.dtype = _TOKEN_DTYPES[x.dtype]
+    a.flags = flags
+    a.x, a.dt, a.z, a.Bm, a.Cm = (_ptr(t) for t in (x, dt, z, B, C))
+    a.A, a.Dskip, a.dt_bias, a.h0 = (_ptr(t) for t in (A, D, dt_bias, h0))
+    a.y, a.h_last = _ptr(y), _ptr(h_last)
+    return a
+
+
+def workspace_size(batch, seqlen, dim, dstate, dtype=torch.bfloat16):
+    """Bytes of device workspace a scan of these shapes needs."""
+    a = _native.ScanArgs()
+    a.batch, a.seqlen, a.dim, a.dstate = batch, seqlen, dim, dstate
+    a.dtype = _TOKEN_DTYPES[dtype]
+    return int(_native.lib().ssm_scan_workspace_size(ctypes.byref(a)))
+
+
+class ScanWorkspace:
+    """A reusable device workspace (grown on demand) for one stream's scans."""
+
+    def __init__(self, device=None):
+        self.device = torch.device(device) if device is not None else None
+        self.buf = None
+
+    def get(self, nbytes, device):
+        if self.buf is None or self.buf.numel() < nbytes or self.buf.device != device:
+            self.buf = torch.empty(max(nbytes, 256), dtype=torch.uint8, device=device)
+        return self.buf
+
+
+_default_ws = {}
+
+
+def scan_fwd(x, dt, A, B, C, D=None, z=None, dt_bias=None, h0=None, *, delta_softplus=True,
+             general_A=False, return_last_state=False, out=None, h_last=None, workspace=None,
+             stream=None):
+    """Selective scan forward over whole sequences (see include/ssm_scan.h, ssm_scan_fwd).
+
+    x, dt, z: [B, L, D] float32 or bfloat16; B, C: [B, L, N] same dtype; A: [D, N]
+    float32; D, dt_bias: [D] float32; h0: [B, D, N] float32. Returns y (same dtype
+    as x) and, with return_last_state, the final state [B, D, N] float32.
+    """
+    dev = x.device
+    if x.dtype not in _TOKEN_DTYPES:
+        raise TypeError(f"x: dtype must be float32 or bfloat16, got {x.dtype}")
+    if x.dim() != 3 or A.dim() != 2:
+        raise ValueError("x must be [B, L, D] and A [D, N]")
+    Bsz, L, Dm = x.shape
+    N = A.shape[1]
+    tok = x.dtype
+    _need(x, "x", (Bsz, L, Dm), tok, dev)
+    _need(dt, "dt", (Bsz, L, Dm), tok, dev)
+    if z is not None:
+        _need(z, "z", (Bsz, L, Dm), tok, dev)
+    _need(B, "B", (Bsz, L, N), tok, dev)
+    _need(C, "C", (Bsz, L, N), tok, dev)
+    _need(A, "A", (Dm, N), torch.float32, dev)
+    if D is not None:
+        _need(D, "D", (Dm,), torch.float32, dev)
+    if dt_bias is not None:
+        _need(dt_bias, "dt_bias", (Dm,), torch.float32, dev)
+    if h0 is not None:
+        _need(h0, "h0", (Bsz, Dm, N), torch.float32, dev)
+    y = torch.empty_like(x) if out is None else out
+    _need(y, "out", (Bsz, L, Dm), tok, dev)
+    if return_last_state and h_last is None:
+        h_last = torch.empty((Bsz, Dm, N), dtype=torch.float32, device=dev)
+    if h_last is not None:
+        _need(h_last, "h_last", (Bsz, Dm, N), torch.float32, dev)
+    args = _scan_args(x, dt, A, B, C, D, z, dt_bias, h0, y, h_last, _flags(delta_softplus, general_A))
+    nbytes = int(_native.lib().ssm_scan_workspace_size(ctypes.byref(args)))
+    if workspace is None:
+        key = (dev, torch.cuda.current_stream(dev).cuda_stream if stream is None else stream.cuda_stream)
+        workspace = _default_ws.setdefault(key, ScanWorkspace())
+    ws = workspace.get(nbytes, dev) if isinstance(workspace, ScanWorkspace) else workspace
+    if ws.numel() * ws.element_size() < nbytes:
+        raise ValueError(f"workspace too small: {ws.numel() * ws.element_size()} < {nbytes} bytes")
+    args.workspace = ctypes.c_void_p(ws.data_ptr())
+    args.workspace_bytes = ws.numel() * ws.element_size()
+    _native.check(_native.lib().ssm_scan_fwd(ctypes.byref(args), _stream_handle(stream)), "ssm_scan_fwd")
+    return (y, h_last) if return_last_state else y
+
+
+def workspace_status(workspace, stream=None):
+    """Synchronise and return the device status code of the last scan on this workspace."""
+    ws = workspace.buf if isinstance(workspace, ScanWorkspace) else workspace
+    return int(_native.lib().ssm_workspace_status(ctypes.c_void_p(ws.data_ptr()), _stream_handle(stream)))
+
+
+def step(x, dt, A, B, C, h, D=None, z=None, dt_bias=None, *, delta_softplus=True, general_A=False,
+         out=None, stream=None):
+    """One recurrent decode step (see include/ssm_scan.h, ssm_step); h is updated in place.
+
+    x, dt, z: [B, D]; B, C: [B, N]; A: [D, N]; h: [B, D, N] float32. Returns y [B, D].
+    """
+    dev = x.device
+    if x.dtype not in _TOKEN_DTYPES:
+        raise TypeError(f"x: dtype must be float32 or bfloat16, got {x.dtype}")
+    Bsz, Dm = x.shape
+    N = A.shape[1]
+    tok = x.dtype
+    _need(x, "x", (Bsz, Dm), tok, dev)
+    _need(dt, "dt", (Bsz, Dm), tok, dev)
+    if z is not None:
+        _need(z, "z", (Bsz, Dm), tok, dev)
+    _need(B, "B", (Bsz, N), tok, dev)
+    _need(C, "C", (Bsz, N), tok, dev)
+    _need(A, "A", (Dm, N), torch.float32, dev)
+    _need(h, "h", (Bsz, Dm, N), torch.float32, dev)
+    if D is not None:
+        _need(D, "D", (Dm,), torch.float32, dev)
+    if dt_bias is not None:
+        _need(dt_bias, "dt_bias", (Dm,), torch.float32, dev)
+    y = torch.empty_like(x) if out is None else out
+    _need(y, "out", (Bsz, Dm), tok, dev)
+    rc = _native.lib().ssm_step(Bsz, Dm, N, _TOKEN_DTYPES[tok], _flags(delta_softplus, general_A),
+                                _ptr(x), _ptr(dt), _ptr(z), _ptr(B), _ptr(C), _ptr(A), _ptr(D),
+                                _ptr(dt_bias), _ptr(h), _ptr(y), _stream_handle(stream))
+    _native.check(rc, "ssm_step")
+    return y

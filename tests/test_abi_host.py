@@ -1,0 +1,141 @@
+"""CPU checks of the C ABI: the library loads, exports what the header declares, and
+rejects bad arguments on the host before any CUDA call. No compute runs here."""
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+
+from selective_state_space_47_b200 import _native
+from selective_state_space_47_b200 import build as lib_build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "ssm_scan.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    lib_build.build()
+    return _native.lib()
+
+
+def _declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return set(re.findall(r"^\s*(?:const\s+)?\w+\s*\*?\s*(ssm_\w+)\s*\(", text, flags=re.M))
+
+
+def test_header_and_exports_agree(lib):
+    declared = _declared_functions()
+    assert declared == set(_native.EXPORTS)
+    out = subprocess.check_output(["nm", "-D", "--defined-only", _native.LIB_PATH]).decode()
+    exported = set(re.findall(r"\bT (ssm_\w+)$", out, flags=re.M))
+    assert declared <= exported, f"missing exports: {declared - exported}"
+    for name in declared:
+        assert hasattr(lib, name)
+
+
+def test_header_compiles_as_c(tmp_path):
+    src = tmp_path / "use.c"
+    src.write_text('#include "ssm_scan.h"\nint main(void){ ssm_scan_args a = {0}; (void)a;'
+                   ' return (int)ssm_scan_workspace_size(&a) * 0; }\n')
+    subprocess.check_call(["gcc", "-std=c99", "-Wall", "-Werror", "-fsyntax-only",
+                           "-I", os.path.join(ROOT, "include"), str(src)])
+
+
+def test_status_strings(lib):
+    for code in range(5):
+        assert _native.status_string(code).startswith("SSM_")
+    assert "unknown" in _native.status_string(99)
+
+
+def _args(**kw):
+    a = _native.ScanArgs()
+    a.batch, a.seqlen, a.dim, a.dstate = 2, 64, 32, 16
+    a.dtype = _native.SSM_BF16
+    a.flags = _native.SSM_DELTA_SOFTPLUS
+    fake = 1 << 20  # host-side stand-ins: never dereferenced, the calls must fail first
+    for name in ("x", "dt", "z", "Bm", "Cm", "A", "Dskip", "dt_bias", "h0", "y", "h_last"):
+        setattr(a, name, fake)
+        fake += 1 << 16
+    a.workspace = fake
+    a.workspace_bytes = lib_ws(a)
+    for k, v in kw.items():
+        setattr(a, k, v)
+    return a
+
+
+def lib_ws(a):
+    return _native.lib().ssm_scan_workspace_size(ctypes.byref(a))
+
+
+def test_workspace_size(lib):
+    a = _args()
+    a.batch, a.seqlen, a.dim = 1, 262144, 5120
+    n = lib_ws(a)
+    # per-group flags (rounded) plus one float32 state of 16 per channel
+    assert n == 256 * ((256 + 4 * (5120 // 16) + 255) // 256) + 5120 * 16 * 4
+    assert n < 400_000
+    a.batch = -1
+    assert lib_ws(a) == 0
+    assert lib.ssm_scan_workspace_size(None) == 0
+
+
+@pytest.mark.parametrize("bad,code", [
+    (dict(dstate=17), _native.SSM_ERR_UNSUPPORTED),
+    (dict(dstate=0), _native.SSM_ERR_INVALID),
+    (dict(dim=12), _native.SSM_ERR_UNSUPPORTED),          # bf16 needs dim % 8 == 0
+    (dict(dtype=7), _native.SSM_ERR_INVALID),
+    (dict(flags=0x40), _native.SSM_ERR_INVALID),
+    (dict(seqlen=-1), _native.SSM_ERR_INVALID),
+    (dict(x=None), _native.SSM_ERR_INVALID),
+    (dict(Bm=None), _native.SSM_ERR_INVALID),
+    (dict(y=None), _native.SSM_ERR_INVALID),
+    (dict(A=None), _native.SSM_ERR_INVALID),
+    (dict(x=(1 << 20) + 4), _native.SSM_ERR_UNSUPPORTED),  # misaligned
+    (dict(y=(1 << 20) + 8), _native.SSM_ERR_UNSUPPORTED),
+    (dict(h_last=(1 << 20) + 2), _native.SSM_ERR_UNSUPPORTED),
+    (dict(Bm=(1 << 20) + 1), _native.SSM_ERR_UNSUPPORTED),
+    (dict(workspace=(1 << 20) + 8), _native.SSM_ERR_UNSUPPORTED),
+    (dict(workspace=None), _native.SSM_ERR_INVALID),
+    (dict(workspace_bytes=100), _native.SSM_ERR_INVALID),
+])
+def test_scan_rejects_on_host(lib, bad, code):
+    a = _args(**bad)
+    assert lib.ssm_scan_fwd(ctypes.byref(a), None) == code
+    assert lib.ssm_scan_fwd(None, None) == _native.SSM_ERR_INVALID
+
+
+def test_scan_empty_batch_is_a_no_op(lib):
+    a = _args(batch=0)
+    assert lib.ssm_scan_fwd(ctypes.byref(a), None) == _native.SSM_OK
+
+
+def test_step_rejects_on_host(lib):
+    f = 1 << 20
+    ptrs = [f + (i << 16) for i in range(10)]
+    call = lambda *a: lib.ssm_step(*a)
+    assert call(2, 32, 17, 1, 1, *ptrs, None) == _native.SSM_ERR_UNSUPPORTED
+    assert call(2, 32, 16, 3, 1, *ptrs, None) == _native.SSM_ERR_INVALID
+    assert call(-1, 32, 16, 1, 1, *ptrs, None) == _native.SSM_ERR_INVALID
+    bad = list(ptrs)
+    bad[0] = None
+    assert call(2, 32, 16, 1, 1, *bad, None) == _native.SSM_ERR_INVALID
+    bad = list(ptrs)
+    bad[8] = f + 4                      # h must start on 16 bytes when dstate == 16
+    assert call(2, 32, 16, 1, 1, *bad, None) == _native.SSM_ERR_UNSUPPORTED
+    bad[8] = f + 2                      # and on 4 bytes otherwise
+    assert call(2, 32, 5, 1, 1, *bad, None) == _native.SSM_ERR_UNSUPPORTED
+    bad = list(ptrs)
+    bad[0] = f + 1                      # bf16 token pointer not on its element size
+    assert call(2, 32, 16, 1, 1, *bad, None) == _native.SSM_ERR_UNSUPPORTED
+    assert call(0, 32, 16, 1, 1, *ptrs, None) == _native.SSM_OK
+
+
+def test_python_binding_refuses_cpu_tensors():
+    import torch
+    import selective_state_space_47_b200 as ssm
+    x = torch.zeros(1, 4, 8)
+    with pytest.raises(ValueError):
+        ssm.scan_fwd(x, x, torch.zeros(8, 16), torch.zeros(1, 4, 16), torch.zeros(1, 4, 16))
