@@ -136,6 +136,29 @@ ssm_status ssm_step(int64_t batch, int64_t dim, int64_t dstate, ssm_dtype dtype,
  */
 ssm_status ssm_workspace_status(const void *workspace, void *stream);
 
+/*
+ * The scan for callers that must not allocate device memory: a host runtime
+ * whose memory pool owns all of the GPU's memory (a cudaMalloc there fails or
+ * fragments the pool), or a real-time loop that cannot accept the device-wide
+ * synchronisation cudaMalloc/cudaFree may imply. It computes exactly what
+ * ssm_scan_fwd computes and takes the same arguments, but ignores
+ * args->workspace: its scratch is a fixed 2 MiB array in the library's device
+ * memory, which every GPU that loads the library keeps until the process
+ * exits. Shapes for which ssm_scan_workspace_size() exceeds 2 MiB (a little over
+ * 32,000 channels B x D) return SSM_ERR_UNSUPPORTED, with nothing launched. The
+ * caller still provides all inputs
+ * and outputs. Nothing is allocated: no cudaMalloc, cudaFree or allocating
+ * library routine is called.
+ *  - The first call on each device looks up the array's device address (with
+ *    that device current); make that first call before any stream capture.
+ *  - All calls share the one array and the library clears what must start at
+ *    zero at each call, so calls that can overlap on the GPU (other streams,
+ *    other host threads) race and must be serialised by the caller.
+ *  - Its device-side status word also lives in that array; no call reports it.
+ * The pages have no counterpart: this entry point exists only for such callers.
+ */
+ssm_status ssm_scan_fwd_noalloc(const ssm_scan_args *args, void *stream);
+
 /* Human-readable name of a status code (static storage). */
 const char *ssm_status_string(ssm_status status);
 

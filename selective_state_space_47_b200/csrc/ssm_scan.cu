@@ -26,6 +26,7 @@
 #include <string.h>
 
 #include <algorithm>
+#include <mutex>
 
 #include "../../include/ssm_scan.h"
 #include "ssm_device.cuh"
@@ -531,6 +532,32 @@ ssm_status validate_scan(const ssm_scan_args *a) {
     return SSM_OK;
 }
 
+// ------------------------------------------------ allocation-free variant
+// Scratch for ssm_scan_fwd_noalloc: a fixed device array that every GPU which
+// loads this library holds until the process exits. 2 MiB covers the hand-over
+// state of a little over 32,000 channels (B x D).
+constexpr size_t kStaticScratchBytes = size_t(2) << 20;
+__device__ __align__(256) unsigned char g_scan_scratch[kStaticScratchBytes];
+
+constexpr int kMaxDevices = 64;
+std::mutex g_scratch_mu;
+unsigned char *g_scratch_ptr[kMaxDevices] = {};
+
+// Device address of g_scan_scratch on the current device. The host-side symbol
+// is only a stand-in, so the address is looked up once per device (with that
+// device current) and cached.
+unsigned char *static_scratch() {
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+    std::lock_guard<std::mutex> lock(g_scratch_mu);
+    if (!g_scratch_ptr[dev]) {
+        void *p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_scan_scratch) != cudaSuccess || !p) return nullptr;
+        g_scratch_ptr[dev] = static_cast<unsigned char *>(p);
+    }
+    return g_scratch_ptr[dev];
+}
+
 }  // namespace
 
 // ======================================================================= C ABI
@@ -642,6 +669,17 @@ ssm_status ssm_workspace_status(const void *workspace, void *stream_) {
         cudaStreamSynchronize(stream) != cudaSuccess)
         return SSM_ERR_CUDA;
     return v == 0 ? SSM_OK : static_cast<ssm_status>(v);
+}
+
+ssm_status ssm_scan_fwd_noalloc(const ssm_scan_args *a, void *stream) {
+    if (!a || a->batch < 0 || a->dim < 0) return SSM_ERR_INVALID;
+    if (ws_total(a->batch, a->dim) > kStaticScratchBytes) return SSM_ERR_UNSUPPORTED;
+    unsigned char *scratch = static_scratch();
+    if (!scratch) return SSM_ERR_CUDA;
+    ssm_scan_args b = *a;
+    b.workspace = scratch;
+    b.workspace_bytes = kStaticScratchBytes;
+    return ssm_scan_fwd(&b, stream);
 }
 
 const char *ssm_status_string(ssm_status s) {
