@@ -31,6 +31,7 @@ METRIC = "selective-scan state-updates/s (B·L·D·N) and % of B200 HBM roofline
 UNIT = "state-updates/s"
 FALLBACK_HBM_GBS = 6650.0
 SCAN_SOURCES = ["selective_state_space_47_b200/csrc/ssm_scan.cu",
+                "selective_state_space_47_b200/csrc/ssm_scan_kernel.cuh",
                 "selective_state_space_47_b200/csrc/ssm_device.cuh"]
 TRAFFIC_FILE = os.path.join(ROOT, "profiles", "scan_fwd_traffic.json")
 
