@@ -329,7 +329,7 @@ def run_ours(args):
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
                          "frac": achieved / hbm_peak, "traffic": recorded_traffic(w.name, path),
                          "peak_source": peak_src, "algorithmic_bytes_per_launch": nbytes,
-                         "kernel": "scan_fwd_kernel", "launch_ms": per_launch_ms},
+                         "kernel": "scan_ws_kernel", "launch_ms": per_launch_ms},
             "gpu_launches": args.steps,
             "clocks": clk}
 

@@ -57,17 +57,8 @@ struct Tok<float> {
     static __device__ __forceinline__ float ldg(const float *p) { return __ldg(p); }
     static __device__ __forceinline__ float to_f(float v) { return v; }
     static __device__ __forceinline__ float from_f(float v) { return v; }
-    // 16 consecutive elements (64 bytes, 16-byte aligned) widened to float.
-    static __device__ __forceinline__ void row16(const float *p, float *out) {
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            const float4 v = reinterpret_cast<const float4 *>(p)[i];
-            out[4 * i] = v.x;
-            out[4 * i + 1] = v.y;
-            out[4 * i + 2] = v.z;
-            out[4 * i + 3] = v.w;
-        }
-    }
+    // 4 consecutive elements (16-byte aligned).
+    static __device__ __forceinline__ float4 quad(const float *p) { return *reinterpret_cast<const float4 *>(p); }
 };
 template <>
 struct Tok<__nv_bfloat16> {
@@ -75,19 +66,12 @@ struct Tok<__nv_bfloat16> {
     static __device__ __forceinline__ float ldg(const __nv_bfloat16 *p) { return __bfloat162float(__ldg(p)); }
     static __device__ __forceinline__ float to_f(__nv_bfloat16 v) { return __bfloat162float(v); }
     static __device__ __forceinline__ __nv_bfloat16 from_f(float v) { return __float2bfloat16_rn(v); }
-    // 16 consecutive elements (32 bytes, 16-byte aligned) widened to float: a bfloat16
-    // is the upper half of the float with the same bits.
-    static __device__ __forceinline__ void row16(const __nv_bfloat16 *p, float *out) {
-#pragma unroll
-        for (int i = 0; i < 2; ++i) {
-            const uint4 w = reinterpret_cast<const uint4 *>(p)[i];
-            const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
-#pragma unroll
-            for (int k = 0; k < 4; ++k) {
-                out[8 * i + 2 * k] = __uint_as_float(ws[k] << 16);
-                out[8 * i + 2 * k + 1] = __uint_as_float(ws[k] & 0xffff0000u);
-            }
-        }
+    // 4 consecutive elements (8-byte aligned) widened to float: a bfloat16 is the upper
+    // half of the float with the same bits.
+    static __device__ __forceinline__ float4 quad(const __nv_bfloat16 *p) {
+        const uint2 w = *reinterpret_cast<const uint2 *>(p);
+        return make_float4(__uint_as_float(w.x << 16), __uint_as_float(w.x & 0xffff0000u),
+                           __uint_as_float(w.y << 16), __uint_as_float(w.y & 0xffff0000u));
     }
 };
 

@@ -3,7 +3,7 @@
 // plan of the warp-specialised scan kernel (ssm_scan_kernel.cuh), the one-token
 // decode kernel, and the allocation-free scan variant.
 //
-// Sequence parallelism: the sequence of every group of 16 channels is cut into
+// Sequence parallelism: the sequence of every group of 32 channels is cut into
 // time segments; (group, segment) items are handed out in order by an atomic
 // counter, and an item starts from the state its predecessor publishes in the
 // workspace (bounded wait on a release/acquire flag). The recurrence is
@@ -23,13 +23,12 @@
 
 using namespace ssm;
 
-#ifndef SSM_SEG_TILES
-#define SSM_SEG_TILES 64  // tiles per time segment (upper bound)
-#endif
 
 namespace {
 
 constexpr int kMaxN = 16;   // states per channel handled by the kernels
+constexpr int kMinSegTiles = 32;  // shortest time segment, in tiles (unless the sequence is shorter)
+constexpr int kMaxSegTiles = 64;  // longest time segment, in tiles
 
 // ------------------------------------------------------------- workspace
 // [0, 4) item counter; [4, 8) device status; [256, ...) per-group flags;
@@ -160,12 +159,15 @@ bool plan_scan(const ssm_scan_args *a, ScanPlan *pl) {
         occ <= 0)
         return false;
     pl->grid = int(std::min<int64_t>(pl->G, int64_t(occ) * sms));
-    // Short segments keep all blocks inside a narrow window of the sequence (items are
-    // handed out segment-major), so neighbouring channel groups read the same rows at
-    // about the same time; enough items also balance the blocks.
-    const int64_t want_k = std::max<int64_t>(1, (64 * int64_t(pl->grid) + pl->G - 1) / pl->G);
+    // Segments: about four items per block, between kMinSegTiles and kMaxSegTiles tiles
+    // long. Each item start waits for its predecessor's state (a few microseconds), which
+    // bounds them from below; dynamic claiming balances the blocks only if items are short
+    // against the whole run, which bounds them from above.
+    const int64_t want_k = std::max<int64_t>(1, (4 * int64_t(pl->grid) + pl->G - 1) / pl->G);
     const int64_t per = (a->seqlen + want_k - 1) / want_k;
-    pl->seg_len = std::max<int64_t>(TT, std::min<int64_t>(int64_t(SSM_SEG_TILES) * TT, (per + TT - 1) / TT * TT));
+    const int64_t lmin = std::min<int64_t>((a->seqlen + TT - 1) / TT * TT, int64_t(kMinSegTiles) * TT);
+    pl->seg_len = std::min<int64_t>(int64_t(kMaxSegTiles) * TT,
+                                    std::max<int64_t>(std::max<int64_t>(TT, lmin), (per + TT - 1) / TT * TT));
     pl->K = (a->seqlen + pl->seg_len - 1) / pl->seg_len;
     pl->items = pl->G * pl->K;
     return true;

@@ -1,34 +1,42 @@
 // ssm_scan_kernel.cuh -- warp-specialised selective-scan forward kernel for sm_100a.
 //
 // One thread block owns one group of CH = 32 channels of one sequence at a time
-// and walks the item's time segment tile by tile (TT steps per tile). Six warps
-// with fixed roles, connected by mbarrier rings (every wait bounded in time and
-// suspended in hardware while it waits):
+// and walks the item's time segment tile by tile (TT = 32 steps per tile). Nine
+// warps with fixed roles, connected by mbarrier rings (every wait bounded in time
+// and suspended in hardware while it waits):
 //
-//   W0..W3  consumers    the recurrence. Lane c is channel c of the group; warp w
+//   C0..C3  consumers    the recurrence. Lane c is channel c of the group; warp w
 //                        keeps states 4w .. 4w+3 of its lane's channel in registers.
 //                        Per step a lane reads its channel's 8-byte record (u, Delta
 //                        log2 e) and, with one warp-uniform broadcast load each, the
 //                        B_t and C_t values of the warp's four states; it forms Abar,
 //                        updates h = Abar h + u B and its partial readout sum_n C_n h_n
 //                        (one 16-byte store per four steps).
-//   P       prologue     per (t, channel), once: Delta = softplus(dt + bias), u = Delta
-//                        x, Delta log2 e; widens the B and C rows to float32.
-//   E       epilogue     per (t, channel): sums the four warps' partials, adds D x,
-//                        applies the SiLU gate, rounds, stores the y tile with TMA; it
-//                        also claims the (group, segment) items and issues the TMA
-//                        loads of x, dt, z, B, C into a STAGES-deep ring (it is the last
-//                        reader of a stage, so it refills it).
+//   P0, P1  prologue     per (t, channel), once: Delta = softplus(dt + bias), u =
+//                        Delta x, Delta log2 e; widens the B and C rows to float32.
+//                        P0 takes the first half of every tile's steps, P1 the second.
+//   E0, E1  epilogue     per (t, channel): sums the four consumer partials, adds D x,
+//                        applies the SiLU gate, rounds, and (E0) stores the y tile
+//                        with TMA. Halves of the tile as for P.
+//   L       loads        claims the (group, segment) items and streams x, dt, z, B, C
+//                        of every tile with TMA into a STAGES-deep ring; a stage is
+//                        refilled once both prologue and both epilogue warps have
+//                        released it.
 //
 // Why this shape: shared memory delivers 128 bytes per clock per SM to registers,
 // and a 16-byte load whose 32 lanes read different addresses costs four of those
 // clocks, while one whose lanes all read the same address costs one. With lanes
 // over channels and warps over states, B_t and C_t (shared by all channels) are
 // warp-uniform, and the only lane-distinct data per step is the 8-byte record.
+// Every loop is written operation by operation over a block of steps (all loads,
+// then each arithmetic stage for all steps of the block, then the stores): a warp
+// issues in order, and this order gives it independent instructions back to back
+// instead of one step's dependency chain at a time.
 //
 // Rings: stage (TMA, STAGES deep) -> P -> record ring (R_REC deep) -> consumers ->
-// partial ring (R_PART deep) -> E. Between blocks, an item (group g, segment k)
-// starts from the state its predecessor (g, k-1) published in the workspace.
+// partial ring (R_PART deep) -> E, which also reads x and z from the stage. Between
+// blocks, an item (group g, segment k) starts from the state its predecessor (g,
+// k-1) published in the workspace.
 //
 // Exponentials: Abar_n = 2^(Delta log2 e * A[d,n]) on the SFU (ex2.approx). Where
 // every row of A in the block is an arithmetic progression in n (A[d,n] = A[d,0] +
@@ -45,16 +53,18 @@ namespace ssm {
 namespace scan {
 
 constexpr int CW = 4;                             // consumer warps (4 states each)
+constexpr int NP = 2;                             // prologue warps
+constexpr int NE = 2;                             // epilogue warps
 constexpr int CH = 32;                            // channels per block (one per lane)
-constexpr int NTHREADS = (CW + 2) * 32;           // consumers + P + E
-constexpr int WARP_P = CW, WARP_E = CW + 1;
+constexpr int WARP_P0 = CW, WARP_E0 = CW + NP, WARP_L = CW + NP + NE;
+constexpr int NTHREADS = (CW + NP + NE + 1) * 32;
 constexpr int TT = 32;                            // time steps per tile
-#ifndef SSM_STAGES
-#define SSM_STAGES 4
-#endif
-constexpr int STAGES = SSM_STAGES;                // TMA ring depth (tiles)
-constexpr int R_REC = 3;                          // record ring depth
+constexpr int TP = TT / NP;                       // steps per prologue warp and tile
+constexpr int TE = TT / NE;                       // steps per epilogue warp and tile
+constexpr int STAGES = 6;                         // TMA ring depth (tiles)
+constexpr int R_REC = 2;                          // record ring depth
 constexpr int R_PART = 2;                         // partial-sum ring depth
+constexpr int YBUF = 3;                           // y staging buffers for the TMA store
 constexpr int kMaxN = 16;                         // state slots per channel
 constexpr uint64_t kWaitLimitNs = 2000000000ull;  // every device-side wait gives up after 2 s
 constexpr uint32_t kSuspendNs = 20000;            // hardware suspend hint per try_wait
@@ -91,6 +101,9 @@ struct Layout {
     static constexpr int BCBOX = TT * kMaxN;      // elements of one B or C box [TT][16]
     static constexpr size_t tok_bytes = size_t(BOX) * sizeof(T);
     static constexpr size_t bc_bytes = size_t(BCBOX) * sizeof(T);
+    // stage: x | dt | z | B | C
+    static constexpr size_t st_x = 0, st_dt = tok_bytes, st_z = 2 * tok_bytes, st_b = 3 * tok_bytes,
+                            st_c = 3 * tok_bytes + bc_bytes;
     static constexpr size_t stage_bytes = 3 * tok_bytes + 2 * bc_bytes;
     static constexpr size_t stage_off = 0;
     static constexpr size_t rec_off = stage_off + STAGES * stage_bytes;
@@ -101,13 +114,13 @@ struct Layout {
     static constexpr size_t part_bytes = size_t(CW) * (TT / 4) * CH * 16;  // [w][t/4][c] float4
     static constexpr size_t yout_off = part_off + R_PART * part_bytes;
     static constexpr size_t yout_bytes = tok_bytes;
-    static constexpr size_t dsk_off = yout_off + 2 * yout_bytes;
-    static constexpr size_t smeta_off = dsk_off + STAGES * CH * 4;
+    static constexpr size_t smeta_off = yout_off + YBUF * yout_bytes;
     static constexpr size_t tmeta_off = smeta_off + STAGES * sizeof(TileMeta);
     static constexpr size_t bar_off = (tmeta_off + R_REC * sizeof(TileMeta) + 15) / 16 * 16;
-    static constexpr int NBARS = STAGES + 2 * R_REC + 2 * R_PART;
+    static constexpr int NBARS = 2 * STAGES + 2 * R_REC + 2 * R_PART;
     static constexpr size_t total = bar_off + NBARS * 8;
-    static_assert(stage_bytes % 128 == 0 && tok_bytes % 128 == 0, "TMA boxes must stay 128-byte aligned");
+    static_assert(stage_bytes % 128 == 0 && tok_bytes % 128 == 0 && bc_bytes % 128 == 0,
+                  "TMA boxes must stay 128-byte aligned");
     static_assert(rec_off % 128 == 0 && yout_off % 128 == 0, "TMA/vector buffers must stay aligned");
 };
 
@@ -139,113 +152,264 @@ __device__ __forceinline__ void mbar_arrive(uint64_t *bar) {
     asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
 }
 
+// One arrival per warp: the warp's shared-memory accesses are ordered before lane 0's
+// release-arrive by __syncwarp (a 32-lane arrive costs the shared-memory pipe far more).
+__device__ __forceinline__ void warp_arrive(uint64_t *bar) {
+    __syncwarp();
+    if ((threadIdx.x & 31) == 0) mbar_arrive(bar);
+}
+
 __device__ __forceinline__ void consumer_sync() {  // named barrier 1: the consumer warps only
     asm volatile("bar.sync 1, %0;" ::"n"(CW * 32) : "memory");
+}
+__device__ __forceinline__ void epilogue_sync() {  // named barrier 2: the epilogue warps only
+    asm volatile("bar.sync 2, %0;" ::"n"(NE * 32) : "memory");
 }
 
 __device__ __forceinline__ float2 f2(float a, float b) { return make_float2(a, b); }
 
-// softplus of two values: log(1 + e^v), series for e^v < 2^-6, v itself above 15.
-__device__ __forceinline__ float2 softplus2(float2 v) {
-    const float2 x = __fmul2_rn(v, f2(kLog2e, kLog2e));
-    const float2 e = f2(ex2_approx(x.x), ex2_approx(x.y));
-    float2 s = __ffma2_rn(e, f2(-0.25f, -0.25f), f2(0.33333334f, 0.33333334f));
-    s = __ffma2_rn(e, s, f2(-0.5f, -0.5f));
-    s = __ffma2_rn(e, s, f2(1.f, 1.f));
-    s = __fmul2_rn(e, s);
-    const float2 one_e = __fadd2_rn(e, f2(1.f, 1.f));
-    const float2 lg = __fmul2_rn(f2(lg2_approx(one_e.x), lg2_approx(one_e.y)), f2(kLn2, kLn2));
-    float2 r;
-    r.x = v.x > 15.f ? v.x : (e.x < 0.015625f ? s.x : lg.x);
-    r.y = v.y > 15.f ? v.y : (e.y < 0.015625f ? s.y : lg.y);
-    return r;
-}
-
-// silu of two values: z / (1 + e^-z).
-__device__ __forceinline__ float2 silu2(float2 z) {
-    const float2 nz = __fmul2_rn(z, f2(-kLog2e, -kLog2e));
-    const float2 den = __fadd2_rn(f2(ex2_approx(nz.x), ex2_approx(nz.y)), f2(1.f, 1.f));
-    return __fmul2_rn(z, f2(rcp_approx(den.x), rcp_approx(den.y)));
+__device__ __forceinline__ void set_timeout(uint32_t *status, int lane) {
+    if (lane == 0) atomicExch(status, uint32_t(SSM_ERR_TIMEOUT));
 }
 
 // ---------------------------------------------------------------- consumers
-// TT steps of one tile for one lane (its channel, the warp's four states).
-// rec: this lane's records (stride CH float2 per step); bc: B of the warp's states
-// (stride 32 floats per step; C at +16); part: this lane's partials (stride CH
-// float4 per block of four steps). Aq: A[c][4w .. 4w+3]; del: A[c][1] - A[c][0].
+// TT steps of one tile for one lane (its channel, the warp's four states), in
+// blocks of four steps. rec: this lane's records (stride CH float2 per step); bc: B
+// of the warp's states (stride 32 floats per step; C at +16); part: this lane's
+// partials (stride CH float4 per block of four steps). Aq: A[c][4w .. 4w+3]; del:
+// A[c][1] - A[c][0].
 template <bool STRUCT>
 __device__ __forceinline__ void consume_tile(const float2 *__restrict__ rec, const float *__restrict__ bc,
                                              float4 *__restrict__ part, const float4 Aq, const float del,
                                              float2 &h01, float2 &h23) {
+    constexpr int S = 4;
+#pragma unroll 2
+    for (int t0 = 0; t0 < TT; t0 += S) {
+        float2 p[S];
+        float4 b4[S], c4[S];
 #pragma unroll
-    for (int t4 = 0; t4 < TT; t4 += 4) {
-        float yv[4];
+        for (int s = 0; s < S; ++s) p[s] = rec[(t0 + s) * CH];
 #pragma unroll
-        for (int s = 0; s < 4; ++s) {
-            const int t = t4 + s;
-            const float2 p = rec[t * CH];  // (u, Delta log2 e)
-            const float4 b4 = *reinterpret_cast<const float4 *>(bc + t * 32);       // warp-uniform
-            const float4 c4 = *reinterpret_cast<const float4 *>(bc + t * 32 + 16);  // warp-uniform
-            float2 a01, a23;
-            if (STRUCT) {
-                const float2 x = __fmul2_rn(f2(p.y, p.y), f2(Aq.x, del));
-                const float a0 = ex2_approx(x.x), r = ex2_approx(x.y);
-                a01 = f2(a0, a0 * r);
-                a23 = __fmul2_rn(a01, f2(r * r, r * r));
-            } else {
-                const float2 x01 = __fmul2_rn(f2(p.y, p.y), f2(Aq.x, Aq.y));
-                const float2 x23 = __fmul2_rn(f2(p.y, p.y), f2(Aq.z, Aq.w));
-                a01 = f2(ex2_approx(x01.x), ex2_approx(x01.y));
-                a23 = f2(ex2_approx(x23.x), ex2_approx(x23.y));
+        for (int s = 0; s < S; ++s) b4[s] = *reinterpret_cast<const float4 *>(bc + (t0 + s) * 32);  // uniform
+#pragma unroll
+        for (int s = 0; s < S; ++s) c4[s] = *reinterpret_cast<const float4 *>(bc + (t0 + s) * 32 + 16);
+        float2 a01[S], a23[S];
+        if (STRUCT) {
+            float2 x[S];
+#pragma unroll
+            for (int s = 0; s < S; ++s) x[s] = __fmul2_rn(f2(p[s].y, p[s].y), f2(Aq.x, del));
+            float a0[S], r[S];
+#pragma unroll
+            for (int s = 0; s < S; ++s) {
+                a0[s] = ex2_approx(x[s].x);
+                r[s] = ex2_approx(x[s].y);
             }
-            const float2 u2 = f2(p.x, p.x);
-            h01 = __ffma2_rn(a01, h01, __fmul2_rn(u2, f2(b4.x, b4.y)));
-            h23 = __ffma2_rn(a23, h23, __fmul2_rn(u2, f2(b4.z, b4.w)));
-            const float2 yy = __ffma2_rn(f2(c4.z, c4.w), h23, __fmul2_rn(f2(c4.x, c4.y), h01));
+#pragma unroll
+            for (int s = 0; s < S; ++s) a01[s] = f2(a0[s], a0[s] * r[s]);
+#pragma unroll
+            for (int s = 0; s < S; ++s) a23[s] = __fmul2_rn(a01[s], f2(r[s] * r[s], r[s] * r[s]));
+        } else {
+            float2 x01[S], x23[S];
+#pragma unroll
+            for (int s = 0; s < S; ++s) {
+                x01[s] = __fmul2_rn(f2(p[s].y, p[s].y), f2(Aq.x, Aq.y));
+                x23[s] = __fmul2_rn(f2(p[s].y, p[s].y), f2(Aq.z, Aq.w));
+            }
+#pragma unroll
+            for (int s = 0; s < S; ++s) {
+                a01[s] = f2(ex2_approx(x01[s].x), ex2_approx(x01[s].y));
+                a23[s] = f2(ex2_approx(x23[s].x), ex2_approx(x23[s].y));
+            }
+        }
+        float2 ub01[S], ub23[S];
+#pragma unroll
+        for (int s = 0; s < S; ++s) {
+            ub01[s] = __fmul2_rn(f2(p[s].x, p[s].x), f2(b4[s].x, b4[s].y));
+            ub23[s] = __fmul2_rn(f2(p[s].x, p[s].x), f2(b4[s].z, b4[s].w));
+        }
+        float2 g01[S], g23[S];
+#pragma unroll
+        for (int s = 0; s < S; ++s) {
+            h01 = __ffma2_rn(a01[s], h01, ub01[s]);
+            h23 = __ffma2_rn(a23[s], h23, ub23[s]);
+            g01[s] = h01;
+            g23[s] = h23;
+        }
+        float yv[S];
+#pragma unroll
+        for (int s = 0; s < S; ++s) {
+            const float2 yy = __ffma2_rn(f2(c4[s].z, c4[s].w), g23[s], __fmul2_rn(f2(c4[s].x, c4[s].y), g01[s]));
             yv[s] = yy.x + yy.y;
         }
-        part[(t4 / 4) * CH] = make_float4(yv[0], yv[1], yv[2], yv[3]);
+        part[(t0 / 4) * CH] = make_float4(yv[0], yv[1], yv[2], yv[3]);
+    }
+}
+
+// ---------------------------------------------------------------- prologue
+// Records of TP steps (rows t0 .. t0+TP-1 of a tile) for channel c: (u = Delta x,
+// Delta log2 e), with Delta = softplus(dt + bias) (or dt + bias), all steps of the
+// half tile stage by stage. Rows at or past tlen get (0, 0): Abar = 1, no input.
+template <typename T>
+__device__ __forceinline__ void prologue_rows(const T *__restrict__ sx, const T *__restrict__ sdt,
+                                              float2 *__restrict__ rec, const int t0, const int tlen,
+                                              const float bias, const bool softplus) {
+    constexpr int NPR = TP / 2;  // pairs of steps
+    float2 v[NPR], xv[NPR];
+#pragma unroll
+    for (int q = 0; q < NPR; ++q) {
+        const int t = t0 + 2 * q;
+        v[q] = f2(Tok<T>::to_f(sdt[t * CH]), Tok<T>::to_f(sdt[(t + 1) * CH]));
+        xv[q] = f2(Tok<T>::to_f(sx[t * CH]), Tok<T>::to_f(sx[(t + 1) * CH]));
+    }
+#pragma unroll
+    for (int q = 0; q < NPR; ++q) v[q] = __fadd2_rn(v[q], f2(bias, bias));
+    float2 delta[NPR];
+    if (softplus) {
+        // softplus(v) = log(1 + e^v): series e - e^2/2 + e^3/3 - e^4/4 for e = e^v < 2^-6
+        // (the SFU log2 has an absolute error near 1), v itself above 15.
+        float2 e[NPR];
+#pragma unroll
+        for (int q = 0; q < NPR; ++q) {
+            const float2 xl = __fmul2_rn(v[q], f2(kLog2e, kLog2e));
+            e[q] = f2(ex2_approx(xl.x), ex2_approx(xl.y));
+        }
+        float2 lg[NPR];
+#pragma unroll
+        for (int q = 0; q < NPR; ++q) {
+            const float2 one_e = __fadd2_rn(e[q], f2(1.f, 1.f));
+            lg[q] = f2(lg2_approx(one_e.x), lg2_approx(one_e.y));
+        }
+        float2 ser[NPR];
+#pragma unroll
+        for (int q = 0; q < NPR; ++q) {
+            float2 s = __ffma2_rn(e[q], f2(-0.25f, -0.25f), f2(0.33333334f, 0.33333334f));
+            s = __ffma2_rn(e[q], s, f2(-0.5f, -0.5f));
+            s = __ffma2_rn(e[q], s, f2(1.f, 1.f));
+            ser[q] = __fmul2_rn(e[q], s);
+        }
+#pragma unroll
+        for (int q = 0; q < NPR; ++q) {
+            const float2 l = __fmul2_rn(lg[q], f2(kLn2, kLn2));
+            delta[q].x = v[q].x > 15.f ? v[q].x : (e[q].x < 0.015625f ? ser[q].x : l.x);
+            delta[q].y = v[q].y > 15.f ? v[q].y : (e[q].y < 0.015625f ? ser[q].y : l.y);
+        }
+    } else {
+#pragma unroll
+        for (int q = 0; q < NPR; ++q) delta[q] = v[q];
+    }
+    float2 u[NPR], dl[NPR];
+#pragma unroll
+    for (int q = 0; q < NPR; ++q) {
+        u[q] = __fmul2_rn(delta[q], xv[q]);
+        dl[q] = __fmul2_rn(delta[q], f2(kLog2e, kLog2e));
+    }
+#pragma unroll
+    for (int q = 0; q < NPR; ++q) {
+        const int t = t0 + 2 * q;
+        rec[t * CH] = t < tlen ? f2(u[q].x, dl[q].x) : f2(0.f, 0.f);
+        rec[(t + 1) * CH] = t + 1 < tlen ? f2(u[q].y, dl[q].y) : f2(0.f, 0.f);
+    }
+}
+
+// ---------------------------------------------------------------- epilogue
+// y for TE steps (rows t0 .. t0+TE-1) of channel c: sum of the four consumer
+// partials, + D x, times silu(z), rounded to T.
+template <typename T>
+__device__ __forceinline__ void epilogue_rows(const float4 *__restrict__ part, const T *__restrict__ sx,
+                                              const T *__restrict__ sz, T *__restrict__ yo, const int t0,
+                                              const float dd, const bool gate) {
+    constexpr int NB = TE / 4;  // blocks of four steps
+    float2 y01[NB], y23[NB];
+#pragma unroll
+    for (int b = 0; b < NB; ++b) {
+        const int blk = t0 / 4 + b;
+        float4 v[CW];
+#pragma unroll
+        for (int w = 0; w < CW; ++w) v[w] = part[(w * (TT / 4) + blk) * CH];
+        float2 lo = __fadd2_rn(f2(v[0].x, v[0].y), f2(v[1].x, v[1].y));
+        float2 hi = __fadd2_rn(f2(v[0].z, v[0].w), f2(v[1].z, v[1].w));
+        const float2 lo2 = __fadd2_rn(f2(v[2].x, v[2].y), f2(v[3].x, v[3].y));
+        const float2 hi2 = __fadd2_rn(f2(v[2].z, v[2].w), f2(v[3].z, v[3].w));
+        lo = __fadd2_rn(lo, lo2);
+        hi = __fadd2_rn(hi, hi2);
+        const int t = t0 + 4 * b;
+        const float2 x01 = f2(Tok<T>::to_f(sx[t * CH]), Tok<T>::to_f(sx[(t + 1) * CH]));
+        const float2 x23 = f2(Tok<T>::to_f(sx[(t + 2) * CH]), Tok<T>::to_f(sx[(t + 3) * CH]));
+        y01[b] = __ffma2_rn(f2(dd, dd), x01, lo);
+        y23[b] = __ffma2_rn(f2(dd, dd), x23, hi);
+    }
+    if (gate) {
+        // silu(z) = z / (1 + e^-z)
+        float2 z01[NB], z23[NB];
+#pragma unroll
+        for (int b = 0; b < NB; ++b) {
+            const int t = t0 + 4 * b;
+            z01[b] = f2(Tok<T>::to_f(sz[t * CH]), Tok<T>::to_f(sz[(t + 1) * CH]));
+            z23[b] = f2(Tok<T>::to_f(sz[(t + 2) * CH]), Tok<T>::to_f(sz[(t + 3) * CH]));
+        }
+        float2 e01[NB], e23[NB];
+#pragma unroll
+        for (int b = 0; b < NB; ++b) {
+            const float2 n01 = __fmul2_rn(z01[b], f2(-kLog2e, -kLog2e));
+            const float2 n23 = __fmul2_rn(z23[b], f2(-kLog2e, -kLog2e));
+            e01[b] = __fadd2_rn(f2(ex2_approx(n01.x), ex2_approx(n01.y)), f2(1.f, 1.f));
+            e23[b] = __fadd2_rn(f2(ex2_approx(n23.x), ex2_approx(n23.y)), f2(1.f, 1.f));
+        }
+#pragma unroll
+        for (int b = 0; b < NB; ++b) {
+            y01[b] = __fmul2_rn(y01[b], __fmul2_rn(z01[b], f2(rcp_approx(e01[b].x), rcp_approx(e01[b].y))));
+            y23[b] = __fmul2_rn(y23[b], __fmul2_rn(z23[b], f2(rcp_approx(e23[b].x), rcp_approx(e23[b].y))));
+        }
+    }
+#pragma unroll
+    for (int b = 0; b < NB; ++b) {
+        const int t = t0 + 4 * b;
+        yo[t * CH] = Tok<T>::from_f(y01[b].x);
+        yo[(t + 1) * CH] = Tok<T>::from_f(y01[b].y);
+        yo[(t + 2) * CH] = Tok<T>::from_f(y23[b].x);
+        yo[(t + 3) * CH] = Tok<T>::from_f(y23[b].y);
     }
 }
 
 // ------------------------------------------------------------------- kernel
 template <typename T>
-__global__ void __launch_bounds__(NTHREADS)
+__global__ void __launch_bounds__(NTHREADS, 2)
     scan_ws_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_dt,
                    const __grid_constant__ CUtensorMap tm_z, const __grid_constant__ CUtensorMap tm_b,
                    const __grid_constant__ CUtensorMap tm_c, const __grid_constant__ CUtensorMap tm_y,
                    const Params p) {
     using S = Layout<T>;
     extern __shared__ __align__(1024) unsigned char smem[];
-    TileMeta *smeta = reinterpret_cast<TileMeta *>(smem + S::smeta_off);  // per TMA stage
+    TileMeta *smeta = reinterpret_cast<TileMeta *>(smem + S::smeta_off);  // per stage
     TileMeta *tmeta = reinterpret_cast<TileMeta *>(smem + S::tmeta_off);  // per record slot
-    uint64_t *bar_tma = reinterpret_cast<uint64_t *>(smem + S::bar_off);
-    uint64_t *bar_rec_full = bar_tma + STAGES;
+    uint64_t *bar_full = reinterpret_cast<uint64_t *>(smem + S::bar_off);
+    uint64_t *bar_sfree = bar_full + STAGES;
+    uint64_t *bar_rec_full = bar_sfree + STAGES;
     uint64_t *bar_rec_free = bar_rec_full + R_REC;
     uint64_t *bar_part_full = bar_rec_free + R_REC;
     uint64_t *bar_part_free = bar_part_full + R_PART;
-    float *dsk = reinterpret_cast<float *>(smem + S::dsk_off);  // D of the tile's channels, per stage
-    auto stage_ptr = [&](int s) { return smem + S::stage_off + size_t(s) * S::stage_bytes; };
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     if (threadIdx.x == 0) {
-        for (int s = 0; s < STAGES; ++s) mbar_init(&bar_tma[s], 1);
+        for (int s = 0; s < STAGES; ++s) {
+            mbar_init(&bar_full[s], 1);
+            mbar_init(&bar_sfree[s], NP + NE);
+        }
         for (int r = 0; r < R_REC; ++r) {
-            mbar_init(&bar_rec_full[r], 32);
-            mbar_init(&bar_rec_free[r], CW * 32);
+            mbar_init(&bar_rec_full[r], NP);
+            mbar_init(&bar_rec_free[r], CW);
         }
         for (int r = 0; r < R_PART; ++r) {
-            mbar_init(&bar_part_full[r], CW * 32);
-            mbar_init(&bar_part_free[r], 32);
+            mbar_init(&bar_part_full[r], CW);
+            mbar_init(&bar_part_free[r], NE);
         }
         fence_mbar_init();
     }
     __syncthreads();
 
-    if (warp == WARP_E) {
-        // ====================================================== E: epilogue + loads
-        const int ntok = p.has_gate ? 3 : 2;
-        const uint32_t tx_bytes = uint32_t(ntok * S::tok_bytes + (p.bc_tma ? 2 * S::bc_bytes : 0));
+    if (warp == WARP_L) {
+        // ================================================================ L: loads
+        const uint32_t tx_bytes = uint32_t((p.has_gate ? 3 : 2) * S::tok_bytes + (p.bc_tma ? 2 * S::bc_bytes : 0));
         if (lane == 0) {
             prefetch_tensormap(&tm_x);
             prefetch_tensormap(&tm_dt);
@@ -254,7 +418,6 @@ __global__ void __launch_bounds__(NTHREADS)
                 prefetch_tensormap(&tm_b);
                 prefetch_tensormap(&tm_c);
             }
-            prefetch_tensormap(&tm_y);
         }
         long long li_g = 0, li_k = 0, li_beg = 0, li_end = 0;
         int li_j = 0, li_n = 0;
@@ -273,7 +436,13 @@ __global__ void __launch_bounds__(NTHREADS)
                 li_j = 0;
             }
         };
-        auto issue = [&](int st) {  // fetch the next tile of the stream into stage st
+        claim();
+        for (int i = 0;; ++i) {
+            const int st = i % STAGES;
+            if (i >= STAGES && !warp_wait(&bar_sfree[st], uint32_t(i / STAGES - 1) & 1u)) {
+                set_timeout(p.status, lane);
+                break;
+            }
             TileMeta m;
             m.g = li_g;
             m.k = li_k;
@@ -284,113 +453,95 @@ __global__ void __launch_bounds__(NTHREADS)
             if (lane == 0) {
                 smeta[st] = m;
                 if (li_ok) {
-                    unsigned char *stage = stage_ptr(st);
+                    unsigned char *stage = smem + S::stage_off + size_t(st) * S::stage_bytes;
                     const int b = int(m.g / p.Dg), d0 = int((m.g % p.Dg) * CH);
-                    mbar_arrive_expect_tx(&bar_tma[st], tx_bytes);
-                    tma_load_3d(stage, &tm_x, &bar_tma[st], d0, m.t0, b);
-                    tma_load_3d(stage + S::tok_bytes, &tm_dt, &bar_tma[st], d0, m.t0, b);
-                    if (p.has_gate) tma_load_3d(stage + 2 * S::tok_bytes, &tm_z, &bar_tma[st], d0, m.t0, b);
+                    mbar_arrive_expect_tx(&bar_full[st], tx_bytes);
+                    tma_load_3d(stage + S::st_x, &tm_x, &bar_full[st], d0, m.t0, b);
+                    tma_load_3d(stage + S::st_dt, &tm_dt, &bar_full[st], d0, m.t0, b);
+                    if (p.has_gate) tma_load_3d(stage + S::st_z, &tm_z, &bar_full[st], d0, m.t0, b);
                     if (p.bc_tma) {
-                        tma_load_3d(stage + 3 * S::tok_bytes, &tm_b, &bar_tma[st], 0, m.t0, b);
-                        tma_load_3d(stage + 3 * S::tok_bytes + S::bc_bytes, &tm_c, &bar_tma[st], 0, m.t0, b);
+                        tma_load_3d(stage + S::st_b, &tm_b, &bar_full[st], 0, m.t0, b);
+                        tma_load_3d(stage + S::st_c, &tm_c, &bar_full[st], 0, m.t0, b);
                     }
                 } else {
-                    mbar_arrive(&bar_tma[st]);  // end of the stream: complete the phase without data
+                    mbar_arrive(&bar_full[st]);  // end of the stream: complete the phase without data
                 }
             }
             __syncwarp();
-            if (li_ok && ++li_j == li_n) claim();
-        };
-
-        claim();
-        for (int s = 0; s < STAGES; ++s) issue(s);
-
-        const int c = lane;  // E lane = channel
+            if (!li_ok) break;
+            if (++li_j == li_n) claim();
+        }
+    } else if (warp >= WARP_E0) {
+        // ================================================================ E: epilogue
+        const int h = warp - WARP_E0;
+        const int c = lane;
+        float dd = 0.f;
         for (int i = 0;; ++i) {
             const int pr = i % R_PART, st = i % STAGES;
             if (!warp_wait(&bar_part_full[pr], uint32_t(i / R_PART) & 1u)) {
-                if (lane == 0) atomicExch(p.status, uint32_t(SSM_ERR_TIMEOUT));
+                set_timeout(p.status, lane);
                 break;
             }
             const TileMeta m = smeta[st];
             if (m.flags & F_END) break;
-            const unsigned char *stage = stage_ptr(st);
-            const T *sx = reinterpret_cast<const T *>(stage);
-            const T *sz = reinterpret_cast<const T *>(stage + 2 * S::tok_bytes);
-            const float4 *part = reinterpret_cast<const float4 *>(smem + S::part_off + pr * S::part_bytes);
-            T *yo = reinterpret_cast<T *>(smem + S::yout_off + (i & 1) * S::yout_bytes);
-            const float dd = dsk[st * CH + c];
-#pragma unroll 2
-            for (int blk = 0; blk < TT / 4; ++blk) {
-                float4 acc = part[(0 * (TT / 4) + blk) * CH + c];
-#pragma unroll
-                for (int w = 1; w < CW; ++w) {
-                    const float4 v = part[(w * (TT / 4) + blk) * CH + c];
-                    const float2 lo = __fadd2_rn(f2(acc.x, acc.y), f2(v.x, v.y));
-                    const float2 hi = __fadd2_rn(f2(acc.z, acc.w), f2(v.z, v.w));
-                    acc = make_float4(lo.x, lo.y, hi.x, hi.y);
-                }
-                const int t = blk * 4;
-                const float2 x01 = f2(Tok<T>::to_f(sx[t * CH + c]), Tok<T>::to_f(sx[(t + 1) * CH + c]));
-                const float2 x23 = f2(Tok<T>::to_f(sx[(t + 2) * CH + c]), Tok<T>::to_f(sx[(t + 3) * CH + c]));
-                float2 y01 = __ffma2_rn(f2(dd, dd), x01, f2(acc.x, acc.y));
-                float2 y23 = __ffma2_rn(f2(dd, dd), x23, f2(acc.z, acc.w));
-                if (p.has_gate) {
-                    const float2 z01 = f2(Tok<T>::to_f(sz[t * CH + c]), Tok<T>::to_f(sz[(t + 1) * CH + c]));
-                    const float2 z23 = f2(Tok<T>::to_f(sz[(t + 2) * CH + c]), Tok<T>::to_f(sz[(t + 3) * CH + c]));
-                    y01 = __fmul2_rn(y01, silu2(z01));
-                    y23 = __fmul2_rn(y23, silu2(z23));
-                }
-                yo[t * CH + c] = Tok<T>::from_f(y01.x);
-                yo[(t + 1) * CH + c] = Tok<T>::from_f(y01.y);
-                yo[(t + 2) * CH + c] = Tok<T>::from_f(y23.x);
-                yo[(t + 3) * CH + c] = Tok<T>::from_f(y23.y);
+            if (!warp_wait(&bar_full[st], uint32_t(i / STAGES) & 1u)) {
+                set_timeout(p.status, lane);
+                break;
             }
-            mbar_arrive(&bar_part_free[pr]);  // the consumers may reuse this partial slot
-            fence_proxy_async_smem();
-            __syncwarp();
-            if (lane == 0) {
+            if (m.flags & F_FIRST) {
+                const int64_t d = (m.g % p.Dg) * CH + c;
+                dd = (d < p.D && p.Dskip) ? __ldg(p.Dskip + d) : 0.f;
+            }
+            const unsigned char *stage = smem + S::stage_off + size_t(st) * S::stage_bytes;
+            const T *sx = reinterpret_cast<const T *>(stage + S::st_x) + c;
+            const T *sz = reinterpret_cast<const T *>(stage + S::st_z) + c;
+            const float4 *part = reinterpret_cast<const float4 *>(smem + S::part_off + pr * S::part_bytes) + c;
+            T *yo = reinterpret_cast<T *>(smem + S::yout_off + (i % YBUF) * S::yout_bytes) + c;
+            epilogue_rows<T>(part, sx, sz, yo, h * TE, dd, p.has_gate != 0);
+            warp_arrive(&bar_part_free[pr]);  // the consumers may reuse this partial slot
+            warp_arrive(&bar_sfree[st]);      // x and z of this stage are no longer needed
+            fence_proxy_async_smem();         // y rows written by this thread -> visible to the TMA store
+            epilogue_sync();
+            if (h == 0 && lane == 0) {
                 const int b = int(m.g / p.Dg), d0 = int((m.g % p.Dg) * CH);
-                tma_store_3d(&tm_y, yo, d0, m.t0, b);
+                tma_store_3d(&tm_y, smem + S::yout_off + (i % YBUF) * S::yout_bytes, d0, m.t0, b);
                 bulk_commit();
-                bulk_wait_read<1>();  // the store issued from the other y buffer has read it
+                bulk_wait_read<1>();  // the store of the previous tile has read its buffer
             }
             __syncwarp();
-            issue(st);  // stage st is no longer needed: refill it with the next tile of the stream
         }
-        if (lane == 0) bulk_wait_read<0>();
-    } else if (warp == WARP_P) {
-        // ============================================================ P: prologue
+        if (h == 0 && lane == 0) bulk_wait_read<0>();
+    } else if (warp >= WARP_P0) {
+        // ================================================================ P: prologue
+        const int h = warp - WARP_P0;
         const T *Bm = static_cast<const T *>(p.Bm);
         const T *Cm = static_cast<const T *>(p.Cm);
-        const int c = lane;  // P lane = channel
-        float bias_c = 0.f, dsk_c = 0.f;
+        const int c = lane;  // P lane = channel (records)
+        float bias_c = 0.f;
         bool struct_item = false;
         for (int i = 0;; ++i) {
             const int r = i % R_REC, st = i % STAGES;
             TileMeta *tm = &tmeta[r];
             if (i >= R_REC && !warp_wait(&bar_rec_free[r], uint32_t(i / R_REC - 1) & 1u)) {
-                if (lane == 0) atomicExch(p.status, uint32_t(SSM_ERR_TIMEOUT));
+                set_timeout(p.status, lane);
                 break;
             }
-            const bool landed = warp_wait(&bar_tma[st], uint32_t(i / STAGES) & 1u);
+            const bool landed = warp_wait(&bar_full[st], uint32_t(i / STAGES) & 1u);
             TileMeta m = smeta[st];
             if (!landed) {
-                if (lane == 0) atomicExch(p.status, uint32_t(SSM_ERR_TIMEOUT));
+                set_timeout(p.status, lane);
                 m.flags = F_END;
             }
             if (m.flags & F_END) {
-                if (lane == 0) *tm = m;
-                __syncwarp();
-                mbar_arrive(&bar_rec_full[r]);
+                if (h == 0 && lane == 0) *tm = m;
+                warp_arrive(&bar_rec_full[r]);
                 break;
             }
             const int64_t b = m.g / p.Dg;
-            const int64_t d = (m.g % p.Dg) * CH + c;
             if (m.flags & F_FIRST) {  // new item: channel parameters and the structure of A
+                const int64_t d = (m.g % p.Dg) * CH + c;
                 const bool ok = d < p.D;
                 bias_c = (ok && p.dt_bias) ? __ldg(p.dt_bias + d) : 0.f;
-                dsk_c = (ok && p.Dskip) ? __ldg(p.Dskip + d) : 0.f;
                 float a[kMaxN];
 #pragma unroll
                 for (int n = 0; n < kMaxN; ++n) a[n] = (ok && n < p.N) ? __ldg(p.A + d * p.N + n) : 0.f;
@@ -401,53 +552,43 @@ __global__ void __launch_bounds__(NTHREADS)
                     if (ok && n < p.N && a[n] != a[0] + float(n) * dl) arith = false;
                 struct_item = p.allow_structured && __all_sync(0xffffffffu, arith);
             }
-            // Records: one per (t, channel), two steps at a time.
-            const unsigned char *stage = stage_ptr(st);
-            const T *sx = reinterpret_cast<const T *>(stage);
-            const T *sdt = reinterpret_cast<const T *>(stage + S::tok_bytes);
-            float2 *rec = reinterpret_cast<float2 *>(smem + S::rec_off + r * S::rec_bytes);
-#pragma unroll 4
-            for (int t = 0; t < TT; t += 2) {
-                const float2 v = __fadd2_rn(f2(Tok<T>::to_f(sdt[t * CH + c]), Tok<T>::to_f(sdt[(t + 1) * CH + c])),
-                                            f2(bias_c, bias_c));
-                const float2 delta = p.softplus ? softplus2(v) : v;
-                const float2 dlg = __fmul2_rn(delta, f2(kLog2e, kLog2e));
-                const float2 u = __fmul2_rn(delta, f2(Tok<T>::to_f(sx[t * CH + c]), Tok<T>::to_f(sx[(t + 1) * CH + c])));
-                // Past the end of the sequence: u = 0 and Delta = 0 give Abar = 1 and no input.
-                rec[t * CH + c] = t < m.tlen ? f2(u.x, dlg.x) : f2(0.f, 0.f);
-                rec[(t + 1) * CH + c] = t + 1 < m.tlen ? f2(u.y, dlg.y) : f2(0.f, 0.f);
-            }
-            // B and C rows widened to float32: row t = [B_0 .. B_15 | C_0 .. C_15]; id =
-            // mq * 32 + lane covers row id / 8 and quarter id % 8 (quarters 0-3 B, 4-7 C).
-            float *bcf = reinterpret_cast<float *>(smem + S::bcf_off + r * S::bcf_bytes);
+            const unsigned char *stage = smem + S::stage_off + size_t(st) * S::stage_bytes;
+            float2 *rec = reinterpret_cast<float2 *>(smem + S::rec_off + r * S::rec_bytes) + c;
+            prologue_rows<T>(reinterpret_cast<const T *>(stage + S::st_x) + c,
+                             reinterpret_cast<const T *>(stage + S::st_dt) + c, rec, h * TP, m.tlen, bias_c,
+                             p.softplus != 0);
+            // B and C rows of this half widened to float32: row t = [B_0 .. B_15 | C_0 .. C_15],
+            // in 16-byte chunks; chunk id = q * 32 + lane covers row h*TP + id / 8 and chunk
+            // id % 8 (0-3: B, 4-7: C), so eight consecutive lanes write one 128-byte row.
+            {
+                float *bcf = reinterpret_cast<float *>(smem + S::bcf_off + r * S::bcf_bytes);
 #pragma unroll
-            for (int mq = 0; mq < TT * 8 / 32; ++mq) {
-                const int id = mq * 32 + lane, t = id >> 3, k = id & 7;
-                const int n0 = (k & 3) * 4;
-                float v[4];
-                if (t >= m.tlen) {
-                    v[0] = v[1] = v[2] = v[3] = 0.f;
-                } else if (p.bc_tma) {
-                    const T *src = reinterpret_cast<const T *>(stage + 3 * S::tok_bytes + (k < 4 ? 0 : S::bc_bytes));
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) v[e] = Tok<T>::to_f(src[t * kMaxN + n0 + e]);
-                } else {
-                    const T *src = k < 4 ? Bm : Cm;
-                    const int64_t tt = m.t0 + t;
-#pragma unroll
-                    for (int e = 0; e < 4; ++e)
-                        v[e] = (n0 + e < p.N) ? Tok<T>::ldg(src + (b * p.L + tt) * p.N + n0 + e) : 0.f;
+                for (int q = 0; q < TP * 8 / 32; ++q) {
+                    const int id = q * 32 + lane, t = h * TP + (id >> 3), j = id & 7;
+                    const int n0 = (j & 3) * 4;
+                    float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+                    if (t < m.tlen) {
+                        if (p.bc_tma) {
+                            v = Tok<T>::quad(reinterpret_cast<const T *>(stage + (j < 4 ? S::st_b : S::st_c)) +
+                                             t * kMaxN + n0);
+                        } else {
+                            const T *src = (j < 4 ? Bm : Cm) + (b * p.L + m.t0 + t) * p.N + n0;
+                            v.x = n0 < p.N ? Tok<T>::ldg(src) : 0.f;
+                            v.y = n0 + 1 < p.N ? Tok<T>::ldg(src + 1) : 0.f;
+                            v.z = n0 + 2 < p.N ? Tok<T>::ldg(src + 2) : 0.f;
+                            v.w = n0 + 3 < p.N ? Tok<T>::ldg(src + 3) : 0.f;
+                        }
+                    }
+                    *reinterpret_cast<float4 *>(bcf + t * 32 + j * 4) = v;
                 }
-                *reinterpret_cast<float4 *>(bcf + t * 32 + k * 4) = make_float4(v[0], v[1], v[2], v[3]);
             }
-            dsk[st * CH + c] = dsk_c;
-            if (lane == 0) {
+            if (h == 0 && lane == 0) {
                 TileMeta mm = m;
                 mm.flags |= struct_item ? F_STRUCT : 0;
                 *tm = mm;
             }
-            __syncwarp();
-            mbar_arrive(&bar_rec_full[r]);
+            warp_arrive(&bar_rec_full[r]);
+            warp_arrive(&bar_sfree[st]);  // x, dt, B, C of this stage read (E still reads x, z)
         }
     } else {
         // ============================================================ consumers
@@ -461,11 +602,11 @@ __global__ void __launch_bounds__(NTHREADS)
             const bool have = warp_wait(&bar_rec_full[r], uint32_t(i / R_REC) & 1u);
             const TileMeta m = tmeta[r];
             if (!have || (m.flags & F_END)) {
-                if (!have && lane == 0) atomicExch(p.status, uint32_t(SSM_ERR_TIMEOUT));
+                if (!have) set_timeout(p.status, lane);
                 // E reads the end marker from its stage. Arrive only once E has released the
                 // slot's previous use: a phase-parity wait cannot tell phase u from u + 2.
                 if (i < R_PART || warp_wait(&bar_part_free[pr], uint32_t(i / R_PART - 1) & 1u))
-                    mbar_arrive(&bar_part_full[pr]);
+                    warp_arrive(&bar_part_full[pr]);
                 break;
             }
             const int64_t b = m.g / p.Dg;
@@ -510,7 +651,7 @@ __global__ void __launch_bounds__(NTHREADS)
                 }
             }
             if (i >= R_PART && !warp_wait(&bar_part_free[pr], uint32_t(i / R_PART - 1) & 1u)) {
-                if (lane == 0) atomicExch(p.status, uint32_t(SSM_ERR_TIMEOUT));
+                set_timeout(p.status, lane);
                 break;
             }
             const float2 *rec = reinterpret_cast<const float2 *>(smem + S::rec_off + r * S::rec_bytes) + c;
@@ -518,8 +659,8 @@ __global__ void __launch_bounds__(NTHREADS)
             float4 *part = reinterpret_cast<float4 *>(smem + S::part_off + pr * S::part_bytes) + w * (TT / 4) * CH + c;
             if (m.flags & F_STRUCT) consume_tile<true>(rec, bc, part, Aq, del, h01, h23);
             else consume_tile<false>(rec, bc, part, Aq, del, h01, h23);
-            mbar_arrive(&bar_rec_free[r]);
-            mbar_arrive(&bar_part_full[pr]);
+            warp_arrive(&bar_rec_free[r]);
+            warp_arrive(&bar_part_full[pr]);
             if (m.flags & F_LAST) {
                 if (m.k == p.K - 1) {
                     if (p.h_last && dvalid) {
