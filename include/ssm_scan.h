@@ -110,9 +110,10 @@ size_t ssm_scan_workspace_size(const ssm_scan_args *args);
  *
  * Where every row of A used by a thread block is an exact arithmetic progression
  * in n (A[d,n] = A[d,0] + n * (A[d,1] - A[d,0]) in float32; the S4D-real
- * initialisation A[d,n] = -(n+1) is one), exp(Delta A[d,n]) for n and n+4 differ
- * by the factor exp(4 Delta (A[d,1] - A[d,0])), and the kernel uses that ratio
- * instead of a fresh exponential. SSM_A_GENERAL turns this off.
+ * initialisation A[d,n] = -(n+1) is one), a thread's four factors exp(Delta A[d,n])
+ * for n = 4w .. 4w+3 follow from two exponentials, exp(Delta A[d,4w]) and the
+ * ratio r = exp(Delta (A[d,1] - A[d,0])), by multiplication. SSM_A_GENERAL turns
+ * this off (one exponential per state and step).
  */
 ssm_status ssm_scan_fwd(const ssm_scan_args *args, void *stream);
 
@@ -123,6 +124,8 @@ ssm_status ssm_scan_fwd(const ssm_scan_args *args, void *stream);
  *   x, dt, z : [B, D] (z may be NULL);  Bm, Cm : [B, N];  A : [D, N];
  *   Dskip, dt_bias : [D] or NULL;  h : [B, D, N] float32, read and overwritten;
  *   y : [B, D] output. No workspace. flags as for the scan.
+ * With dstate == 16, A on 16 bytes and Bm, Cm on four elements, four threads
+ * share a channel (one float4 of h each); otherwise one thread per channel.
  */
 ssm_status ssm_step(int64_t batch, int64_t dim, int64_t dstate, ssm_dtype dtype, uint32_t flags,
                     const void *x, const void *dt, const void *z, const void *Bm, const void *Cm,
