@@ -49,6 +49,8 @@ def parse_args(argv=None):
                     help="time the general exponential path as the headline (flag SSM_A_GENERAL)")
     ap.add_argument("--no-extras", action="store_true",
                     help="skip the e2e, decode, general-A and CPU-baseline legs (profiling runs)")
+    ap.add_argument("--decode-only", action="store_true",
+                    help="run only the recurrent-decode leg (1000 chained steps) and print its line")
     return ap.parse_args(argv)
 
 
@@ -284,6 +286,15 @@ def run_ours(args):
     hbm_peak = peaks["hbm_gbs"] if peaks else FALLBACK_HBM_GBS
     peak_src = "measured" if peaks else "fallback"
 
+    if args.decode_only:
+        line = {"metric": "decode state-updates/s (B·D·N per token step)", "n_gpus": world, "data": "synthetic",
+                "decode": run_decode(ssm, synth, dev, stream, rank, hbm_peak, reps=max(1, args.steps))}
+        if world > 1:
+            dist.barrier()
+            dist.destroy_process_group()
+        if rank == 0:
+            print(json.dumps(line), flush=True)
+        return 0
     inp = synth.scan_inputs(w.batch, w.seqlen, w.dim, w.dstate, w.dtype, seed=rank_seed(w.seed, rank),
                             device=dev, gate=w.gate)
     y = torch.empty_like(inp["x"])
