@@ -103,6 +103,8 @@ def test_decode_workload_sampled(ssm):
     dsel = torch.unique(torch.cat([torch.linspace(0, 5119, 22).round().long(), torch.tensor([1, 5118])]))
     ys_ref, h_ref = _oracle_steps(inp, w.steps, bsel, dsel)
     ys = out[:, bsel.cuda()][:, :, dsel.cuda()].float().cpu().numpy()
-    assert rowwise_rel(ys, ys_ref, axis=2) <= 1e-2
     hs = h[bsel.cuda()][:, dsel.cuda()].cpu().numpy()
-    assert rowwise_rel(hs, h_ref, axis=2) <= 1e-2
+    e_y, e_h = rowwise_rel(ys, ys_ref, axis=2), rowwise_rel(hs, h_ref, axis=2)
+    print(f"\ndecode (8 x {len(dsel)} pairs, 1000 steps): max rel err y {e_y:.3e}, h {e_h:.3e}")
+    assert e_y <= 1e-2
+    assert e_h <= 1e-2
