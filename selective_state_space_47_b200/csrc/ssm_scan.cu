@@ -164,17 +164,24 @@ int sm_count() {
 
 struct ScanPlan {
     int ch = ssm::scan::CH;
+    bool deep = false;
     int64_t G = 0, Dg = 0, K = 0, seg_len = 0, items = 0;
     int grid = 0;
     size_t smem = 0;
 };
 
-void *pick_kernel(ssm_dtype dt) {
-    if (dt == SSM_BF16) return reinterpret_cast<void *>(&ssm::scan::scan_ws_kernel<__nv_bfloat16>);
-    return reinterpret_cast<void *>(&ssm::scan::scan_ws_kernel<float>);
+void *pick_kernel(ssm_dtype dt, bool deep) {
+    using namespace ssm::scan;
+    if (dt == SSM_BF16)
+        return deep ? reinterpret_cast<void *>(&scan_ws_kernel<__nv_bfloat16, Deep>)
+                    : reinterpret_cast<void *>(&scan_ws_kernel<__nv_bfloat16, Shallow>);
+    return deep ? reinterpret_cast<void *>(&scan_ws_kernel<float, Deep>)
+                : reinterpret_cast<void *>(&scan_ws_kernel<float, Shallow>);
 }
-size_t pick_smem(ssm_dtype dt) {
-    return dt == SSM_BF16 ? ssm::scan::Layout<__nv_bfloat16>::total : ssm::scan::Layout<float>::total;
+size_t pick_smem(ssm_dtype dt, bool deep) {
+    using namespace ssm::scan;
+    if (dt == SSM_BF16) return deep ? Layout<__nv_bfloat16, Deep>::total : Layout<__nv_bfloat16, Shallow>::total;
+    return deep ? Layout<float, Deep>::total : Layout<float, Shallow>::total;
 }
 
 // Largest group count over both block shapes: bounds the flag and state arrays.
@@ -186,6 +193,38 @@ size_t ws_total(int64_t Bsz, int64_t D) {
     return ws_carry_off(Bsz, D) + size_t(Bsz) * size_t(round_up(size_t(D), 32)) * kMaxN * 4;
 }
 
+// Blocks per SM of the shallow and deep kernel configurations for a token type, per
+// device (queried once: the attribute calls cost microseconds).
+bool scan_occupancy(ssm_dtype dt, int occ[2]) {
+    constexpr int kDevs = 64;
+    static std::mutex mu;
+    static int cache[kDevs][2][2];
+    static bool have[kDevs][2];
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kDevs) return false;
+    const int ti = dt == SSM_BF16 ? 1 : 0;
+    std::lock_guard<std::mutex> lock(mu);
+    if (!have[dev][ti]) {
+        int optin = 0;
+        if (cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) != cudaSuccess) return false;
+        for (int deep = 0; deep < 2; ++deep) {
+            void *kern = pick_kernel(dt, deep != 0);
+            const size_t smem = pick_smem(dt, deep != 0);
+            int o = 0;
+            if (smem <= size_t(optin)) {
+                if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem)) != cudaSuccess ||
+                    cudaOccupancyMaxActiveBlocksPerMultiprocessor(&o, kern, ssm::scan::NTHREADS, smem) != cudaSuccess)
+                    return false;
+            }
+            cache[dev][ti][deep] = o;
+        }
+        have[dev][ti] = true;
+    }
+    occ[0] = cache[dev][ti][0];
+    occ[1] = cache[dev][ti][1];
+    return occ[0] > 0 || occ[1] > 0;
+}
+
 bool plan_scan(const ssm_scan_args *a, ScanPlan *pl) {
     constexpr int TT = ssm::scan::TT;
     const int sms = sm_count();
@@ -193,15 +232,16 @@ bool plan_scan(const ssm_scan_args *a, ScanPlan *pl) {
     pl->ch = ssm::scan::CH;
     pl->Dg = (a->dim + pl->ch - 1) / pl->ch;
     pl->G = a->batch * pl->Dg;
-    pl->smem = pick_smem(a->dtype);
-    void *kern = pick_kernel(a->dtype);
-    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(pl->smem)) != cudaSuccess)
-        return false;
-    int occ = 0;
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kern, ssm::scan::NTHREADS, pl->smem) != cudaSuccess ||
-        occ <= 0)
-        return false;
-    pl->grid = int(std::min<int64_t>(pl->G, int64_t(occ) * sms));
+    // Shallow rings with two blocks per SM when there are enough channel groups to give
+    // most SMs two (at least 1.25 per SM); otherwise the deep configuration (one block per
+    // SM) if its shared memory fits.
+    int occ[2] = {0, 0};
+    if (!scan_occupancy(a->dtype, occ)) return false;
+    // (measured: the deep rings gain ~8% on 160 groups over 148 SMs and nothing on 192)
+    const bool shallow_fills = occ[0] >= 2 && 4 * pl->G >= 5 * int64_t(sms);
+    pl->deep = occ[1] > 0 && (occ[0] <= 0 || !shallow_fills);
+    pl->smem = pick_smem(a->dtype, pl->deep);
+    pl->grid = int(std::min<int64_t>(pl->G, int64_t(occ[pl->deep ? 1 : 0]) * sms));
     // Segments: about four items per block, between kMinSegTiles and kMaxSegTiles tiles
     // long. Each item start waits for its predecessor's state (a few microseconds), which
     // bounds them from below; dynamic claiming balances the blocks only if items are short
@@ -346,7 +386,7 @@ ssm_status ssm_scan_fwd(const ssm_scan_args *a, void *stream_) {
     p.drop_handoff = (a->flags & SSM_TEST_DROP_HANDOFF) != 0;
     p.bc_tma = bc_tma;
 
-    void *kern = pick_kernel(a->dtype);
+    void *kern = pick_kernel(a->dtype, pl.deep);
     void *args[] = {&tx, &tdt, &tz, &tb, &tc, &ty, &p};
     cudaError_t e = cudaLaunchKernel(kern, dim3(pl.grid), dim3(ssm::scan::NTHREADS), args, pl.smem, stream);
     return e == cudaSuccess ? SSM_OK : SSM_ERR_CUDA;

@@ -61,9 +61,28 @@ constexpr int NTHREADS = (CW + NP + NE + 1) * 32;
 constexpr int TT = 32;                            // time steps per tile
 constexpr int TP = TT / NP;                       // steps per prologue warp and tile
 constexpr int TE = TT / NE;                       // steps per epilogue warp and tile
-constexpr int STAGES = 6;                         // TMA ring depth (tiles)
-constexpr int R_REC = 2;                          // record ring depth
-constexpr int R_PART = 2;                         // partial-sum ring depth
+// Ring depths and blocks per SM. Shallow: 113 KB of shared memory (bf16), two blocks
+// per SM. Deep: rings twice as deep, one block per SM; it decouples the roles further
+// and is the better choice when there are too few channel groups to fill two blocks per
+// SM (the long-context workload has 160 groups for 148 SMs).
+template <int STAGES_, int R_REC_, int R_PART_, int MINB_>
+struct Cfg {
+    static constexpr int STAGES = STAGES_;  // TMA ring depth (tiles)
+    static constexpr int R_REC = R_REC_;    // record ring depth
+    static constexpr int R_PART = R_PART_;  // partial-sum ring depth
+    static constexpr int MINB = MINB_;      // blocks per SM the registers are budgeted for
+};
+#ifndef SSM_DEEP_STAGES
+#define SSM_DEEP_STAGES 8
+#endif
+#ifndef SSM_DEEP_REC
+#define SSM_DEEP_REC 4
+#endif
+#ifndef SSM_DEEP_PART
+#define SSM_DEEP_PART 4
+#endif
+using Shallow = Cfg<6, 2, 2, 2>;
+using Deep = Cfg<SSM_DEEP_STAGES, SSM_DEEP_REC, SSM_DEEP_PART, 1>;
 constexpr int YBUF = 3;                           // y staging buffers for the TMA store
 constexpr int kMaxN = 16;                         // state slots per channel
 constexpr uint64_t kWaitLimitNs = 2000000000ull;  // every device-side wait gives up after 2 s
@@ -95,8 +114,9 @@ struct Params {
     int has_gate, softplus, allow_structured, drop_handoff, bc_tma;
 };
 
-template <typename T>
+template <typename T, typename C>
 struct Layout {
+    static constexpr int STAGES = C::STAGES, R_REC = C::R_REC, R_PART = C::R_PART;
     static constexpr int BOX = TT * CH;           // elements of one token box [TT][CH]
     static constexpr int BCBOX = TT * kMaxN;      // elements of one B or C box [TT][16]
     static constexpr size_t tok_bytes = size_t(BOX) * sizeof(T);
@@ -372,13 +392,14 @@ __device__ __forceinline__ void epilogue_rows(const float4 *__restrict__ part, c
 }
 
 // ------------------------------------------------------------------- kernel
-template <typename T>
-__global__ void __launch_bounds__(NTHREADS, 2)
+template <typename T, typename C>
+__global__ void __launch_bounds__(NTHREADS, C::MINB)
     scan_ws_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_dt,
                    const __grid_constant__ CUtensorMap tm_z, const __grid_constant__ CUtensorMap tm_b,
                    const __grid_constant__ CUtensorMap tm_c, const __grid_constant__ CUtensorMap tm_y,
                    const Params p) {
-    using S = Layout<T>;
+    using S = Layout<T, C>;
+    constexpr int STAGES = C::STAGES, R_REC = C::R_REC, R_PART = C::R_PART;
     extern __shared__ __align__(1024) unsigned char smem[];
     TileMeta *smeta = reinterpret_cast<TileMeta *>(smem + S::smeta_off);  // per stage
     TileMeta *tmeta = reinterpret_cast<TileMeta *>(smem + S::tmeta_off);  // per record slot
