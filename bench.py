@@ -49,6 +49,8 @@ def parse_args(argv=None):
                     help="time the general exponential path as the headline (flag SSM_A_GENERAL)")
     ap.add_argument("--no-extras", action="store_true",
                     help="skip the e2e, decode, general-A and CPU-baseline legs (profiling runs)")
+    ap.add_argument("--seqlen", type=int, default=None,
+                    help="shorten the workload's sequence (profiling captures of a smaller case)")
     ap.add_argument("--decode-only", action="store_true",
                     help="run only the recurrent-decode leg (1000 chained steps) and print its line")
     return ap.parse_args(argv)
@@ -172,15 +174,17 @@ def scan_bytes(w):
 
 
 class W:
-    def __init__(self, name):
+    def __init__(self, name, seqlen=None):
         from selective_state_space_47_b200 import synth
         s = synth.WORKLOADS[name]
         self.name, self.batch, self.seqlen, self.dim, self.dstate = name, s.batch, s.seqlen, s.dim, s.dstate
+        if seqlen:  # shortened sequence for profiling captures (the config line reports it)
+            self.name, self.seqlen = f"{name}@L={seqlen}", seqlen
         self.dtype = s.dtype
         self.dtype_name = "bf16" if str(s.dtype).endswith("bfloat16") else "f32"
         self.gate = s.gate
         self.seed = synth.SEEDS[name]
-        self.updates = s.batch * s.seqlen * s.dim * s.dstate
+        self.updates = s.batch * self.seqlen * s.dim * s.dstate
 
 
 # ------------------------------------------------------------ CPU baseline
@@ -222,7 +226,7 @@ def run_reference(args):
     rank, world, _ = dist_env()
     if rank != 0:
         return 0
-    w = W(args.workload)
+    w = W(args.workload, args.seqlen)
     # Each step is one bounded oracle sample; size it so that the whole run ends in ~2 minutes.
     budget = 120.0 / max(1, args.steps + args.warmup)
     rate, cores, _, _, _ = oracle_sample(w, target_s=min(2.0, budget), max_channels=256)
@@ -281,7 +285,7 @@ def run_ours(args):
     dev = torch.device("cuda", local)
     torch.cuda.set_device(dev)
     stream = torch.cuda.current_stream(dev)
-    w = W(args.workload)
+    w = W(args.workload, args.seqlen)
     peaks = measured_peaks()
     hbm_peak = peaks["hbm_gbs"] if peaks else FALLBACK_HBM_GBS
     peak_src = "measured" if peaks else "fallback"
