@@ -162,6 +162,35 @@ ssm_status ssm_workspace_status(const void *workspace, void *stream);
  */
 ssm_status ssm_scan_fwd_noalloc(const ssm_scan_args *args, void *stream);
 
+/*
+ * The scan with its token tensors in HOST memory, for callers whose inputs arrive from
+ * and whose outputs go back to the host. args->x, dt, z, Bm, Cm and y are host
+ * pointers (page-locked memory lets the copies run asynchronously and overlap; with
+ * pageable memory the copies still work but serialise); A, Dskip, dt_bias, h0, h_last
+ * and workspace are device pointers, as for ssm_scan_fwd. The sequence is processed in
+ * chunks of chunk_len steps through `staging`, caller-owned device memory of at least
+ * ssm_scan_host_staging_size(args, chunk_len) bytes starting on 256 bytes: while chunk
+ * c is scanned on `stream`, chunk c+1 is copied in and the y of chunk c-1 copied out
+ * on two copy streams of the library, so both transfer directions overlap each other
+ * and the kernels. The state passes from chunk to chunk through h0/h_last in the
+ * staging memory, so the result equals ssm_scan_fwd over the whole sequence bit for
+ * bit. Batch rows are strided in host memory ([B, L, ...]); each chunk moves them with
+ * one two-dimensional copy per tensor.
+ *
+ * Ordering: the call enqueues and returns; all of its work is ordered after the work
+ * already on `stream` and before the work enqueued on `stream` later. The host buffers
+ * must stay valid, and y unread, until then. The copy streams and their events are
+ * created on the first call on each device and kept until the process exits (make the
+ * first call before any stream capture); calls from several host threads are
+ * serialised while they enqueue.
+ * Errors: as ssm_scan_fwd; SSM_ERR_INVALID if chunk_len < 1 or staging is NULL or too
+ * small; SSM_ERR_UNSUPPORTED if staging is not 256-byte aligned. There is no
+ * counterpart on the pages: this is the host side of the layer's input and output.
+ */
+size_t ssm_scan_host_staging_size(const ssm_scan_args *args, int64_t chunk_len);
+ssm_status ssm_scan_fwd_host(const ssm_scan_args *args, int64_t chunk_len, void *staging, size_t staging_bytes,
+                             void *stream);
+
 /* Human-readable name of a status code (static storage). */
 const char *ssm_status_string(ssm_status status);
 

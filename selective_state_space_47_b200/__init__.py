@@ -9,6 +9,7 @@ device, the calls raise.
     y = scan_fwd(x, dt, A, B, C, D, z, dt_bias)              # [B, L, D]
     y, h_last = scan_fwd(..., return_last_state=True)         # h_last [B, D, N] fp32
     y = step(x_t, dt_t, A, B_t, C_t, h, D, z_t, dt_bias)     # h [B, D, N] updated in place
+    y = scan_fwd_host(x, dt, A, B, C, D, z, dt_bias)         # x, dt, z, B, C, y in host memory
 """
 import ctypes
 
@@ -17,7 +18,7 @@ import torch
 from . import _native
 from ._native import SSM_A_GENERAL, SSM_DELTA_SOFTPLUS
 
-__all__ = ["scan_fwd", "step", "workspace_size", "workspace_status", "ScanWorkspace"]
+__all__ = ["scan_fwd", "scan_fwd_host", "step", "workspace_size", "workspace_status", "ScanWorkspace"]
 
 _TOKEN_DTYPES = {torch.float32: _native.SSM_F32, torch.bfloat16: _native.SSM_BF16}
 
@@ -131,6 +132,76 @@ def scan_fwd(x, dt, A, B, C, D=None, z=None, dt_bias=None, h0=None, *, delta_sof
     args.workspace = ctypes.c_void_p(ws.data_ptr())
     args.workspace_bytes = ws.numel() * ws.element_size()
     _native.check(_native.lib().ssm_scan_fwd(ctypes.byref(args), _stream_handle(stream)), "ssm_scan_fwd")
+    return (y, h_last) if return_last_state else y
+
+
+def _need_host(t, name, shape, dtype):
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name}: expected shape {tuple(shape)}, got {tuple(t.shape)}")
+    if t.dtype != dtype:
+        raise TypeError(f"{name}: expected {dtype}, got {t.dtype}")
+    if t.device.type != "cpu" or not t.is_contiguous():
+        raise ValueError(f"{name}: must be a contiguous host tensor (page-locked for overlapped copies)")
+
+
+_default_staging = {}
+
+
+def scan_fwd_host(x, dt, A, B, C, D=None, z=None, dt_bias=None, h0=None, *, chunk_len=16384,
+                  delta_softplus=True, general_A=False, return_last_state=False, out=None, h_last=None,
+                  workspace=None, staging=None, stream=None):
+    """Selective scan over host-resident tokens (see include/ssm_scan.h, ssm_scan_fwd_host).
+
+    x, dt, z: [B, L, D] and B, C: [B, L, N] host tensors (page-locked memory lets the
+    copies overlap the scan); the result y is a host tensor too (`out`, or a new
+    page-locked one). A, D, dt_bias, h0 and h_last live on the GPU (A's device). The
+    call is asynchronous on `stream`: synchronise it before reading y.
+    """
+    dev = A.device
+    if x.dtype not in _TOKEN_DTYPES:
+        raise TypeError(f"x: dtype must be float32 or bfloat16, got {x.dtype}")
+    if x.dim() != 3 or A.dim() != 2:
+        raise ValueError("x must be [B, L, D] and A [D, N]")
+    Bsz, L, Dm = x.shape
+    N = A.shape[1]
+    tok = x.dtype
+    _need_host(x, "x", (Bsz, L, Dm), tok)
+    _need_host(dt, "dt", (Bsz, L, Dm), tok)
+    if z is not None:
+        _need_host(z, "z", (Bsz, L, Dm), tok)
+    _need_host(B, "B", (Bsz, L, N), tok)
+    _need_host(C, "C", (Bsz, L, N), tok)
+    _need(A, "A", (Dm, N), torch.float32, dev)
+    if D is not None:
+        _need(D, "D", (Dm,), torch.float32, dev)
+    if dt_bias is not None:
+        _need(dt_bias, "dt_bias", (Dm,), torch.float32, dev)
+    if h0 is not None:
+        _need(h0, "h0", (Bsz, Dm, N), torch.float32, dev)
+    y = torch.empty(x.shape, dtype=tok, pin_memory=True) if out is None else out
+    _need_host(y, "out", (Bsz, L, Dm), tok)
+    if return_last_state and h_last is None:
+        h_last = torch.empty((Bsz, Dm, N), dtype=torch.float32, device=dev)
+    if h_last is not None:
+        _need(h_last, "h_last", (Bsz, Dm, N), torch.float32, dev)
+    args = _scan_args(x, dt, A, B, C, D, z, dt_bias, h0, y, h_last, _flags(delta_softplus, general_A))
+    lib = _native.lib()
+    key = (dev, torch.cuda.current_stream(dev).cuda_stream if stream is None else stream.cuda_stream)
+    nbytes = int(lib.ssm_scan_workspace_size(ctypes.byref(args)))
+    if workspace is None:
+        workspace = _default_ws.setdefault(key, ScanWorkspace())
+    ws = workspace.get(nbytes, dev) if isinstance(workspace, ScanWorkspace) else workspace
+    args.workspace = ctypes.c_void_p(ws.data_ptr())
+    args.workspace_bytes = ws.numel() * ws.element_size()
+    sbytes = int(lib.ssm_scan_host_staging_size(ctypes.byref(args), int(chunk_len)))
+    if staging is None:
+        staging = _default_staging.setdefault(key, ScanWorkspace())
+    st = staging.get(sbytes, dev) if isinstance(staging, ScanWorkspace) else staging
+    _native.check(lib.ssm_scan_fwd_host(ctypes.byref(args), int(chunk_len), ctypes.c_void_p(st.data_ptr()),
+                                        st.numel() * st.element_size(), _stream_handle(stream)),
+                  "ssm_scan_fwd_host")
     return (y, h_last) if return_last_state else y
 
 

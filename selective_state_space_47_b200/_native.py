@@ -13,7 +13,7 @@ SSM_TEST_DROP_HANDOFF = 0x80000000
 
 # Every symbol the header declares (checked by the CPU test suite).
 EXPORTS = ("ssm_scan_workspace_size", "ssm_scan_fwd", "ssm_step", "ssm_workspace_status",
-           "ssm_status_string", "ssm_scan_fwd_noalloc")
+           "ssm_status_string", "ssm_scan_fwd_noalloc", "ssm_scan_host_staging_size", "ssm_scan_fwd_host")
 
 
 class ScanArgs(ctypes.Structure):
@@ -46,6 +46,10 @@ def lib():
         L.ssm_scan_fwd.restype = ctypes.c_int
         L.ssm_scan_fwd_noalloc.argtypes = [ctypes.POINTER(ScanArgs), vp]
         L.ssm_scan_fwd_noalloc.restype = ctypes.c_int
+        L.ssm_scan_host_staging_size.argtypes = [ctypes.POINTER(ScanArgs), i64]
+        L.ssm_scan_host_staging_size.restype = ctypes.c_size_t
+        L.ssm_scan_fwd_host.argtypes = [ctypes.POINTER(ScanArgs), i64, vp, ctypes.c_size_t, vp]
+        L.ssm_scan_fwd_host.restype = ctypes.c_int
         L.ssm_step.argtypes = [i64, i64, i64, ctypes.c_int, ctypes.c_uint32] + [vp] * 10 + [vp]
         L.ssm_step.restype = ctypes.c_int
         L.ssm_workspace_status.argtypes = [vp, vp]

@@ -139,3 +139,25 @@ def test_python_binding_refuses_cpu_tensors():
     x = torch.zeros(1, 4, 8)
     with pytest.raises(ValueError):
         ssm.scan_fwd(x, x, torch.zeros(8, 16), torch.zeros(1, 4, 16), torch.zeros(1, 4, 16))
+
+
+def test_host_scan_staging_size_and_argument_checks(lib):
+    """ssm_scan_fwd_host: staging size arithmetic and the checks made before any CUDA call."""
+    a = _args()
+    a.batch, a.seqlen, a.dim, a.dstate = 3, 1000, 64, 16
+    up = lambda v: (v + 255) // 256 * 256
+    Lc = 256
+    tok, bc = up(3 * Lc * 64 * 2), up(3 * Lc * 16 * 2)
+    carry = up(3 * 64 * 16 * 4)
+    assert lib.ssm_scan_host_staging_size(ctypes.byref(a), Lc) == 2 * (4 * tok + 2 * bc) + 2 * carry
+    # chunks longer than the sequence are sized for the sequence
+    assert lib.ssm_scan_host_staging_size(ctypes.byref(a), 10**6) == lib.ssm_scan_host_staging_size(
+        ctypes.byref(a), 1000)
+    assert lib.ssm_scan_host_staging_size(ctypes.byref(a), 0) == 0
+    need = lib.ssm_scan_host_staging_size(ctypes.byref(a), Lc)
+    fake = ctypes.c_void_p(1 << 20)  # never dereferenced: every case below fails first
+    assert lib.ssm_scan_fwd_host(ctypes.byref(a), 0, fake, need, None) == _native.SSM_ERR_INVALID
+    assert lib.ssm_scan_fwd_host(ctypes.byref(a), Lc, None, need, None) == _native.SSM_ERR_INVALID
+    assert lib.ssm_scan_fwd_host(ctypes.byref(a), Lc, ctypes.c_void_p((1 << 20) + 16), need, None) == \
+        _native.SSM_ERR_UNSUPPORTED
+    assert lib.ssm_scan_fwd_host(ctypes.byref(a), Lc, fake, need - 1, None) == _native.SSM_ERR_INVALID
