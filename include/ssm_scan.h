@@ -124,8 +124,8 @@ ssm_status ssm_scan_fwd(const ssm_scan_args *args, void *stream);
  *   x, dt, z : [B, D] (z may be NULL);  Bm, Cm : [B, N];  A : [D, N];
  *   Dskip, dt_bias : [D] or NULL;  h : [B, D, N] float32, read and overwritten;
  *   y : [B, D] output. No workspace. flags as for the scan.
- * With dstate == 16, A on 16 bytes and Bm, Cm on four elements, four threads
- * share a channel (one float4 of h each); otherwise one thread per channel.
+ * With dstate == 16, A on 16 bytes and Bm, Cm on four elements, two threads
+ * share a channel (two float4 of h each); otherwise one thread per channel.
  */
 ssm_status ssm_step(int64_t batch, int64_t dim, int64_t dstate, ssm_dtype dtype, uint32_t flags,
                     const void *x, const void *dt, const void *z, const void *Bm, const void *Cm,

@@ -79,20 +79,22 @@ __global__ void __launch_bounds__(128)
     y[ch] = Tok<T>::from_f(yv);
 }
 
-// One-token step with N = 16: four threads per channel, thread q owning states 4q ..
-// 4q+3 as one float4, so that each load and store instruction of a warp covers 512
-// contiguous bytes of h; the readout is summed over the four threads with two
-// butterfly shuffles. Requires 16-byte aligned h and A rows and 4-element aligned B, C.
+// One-token step with N = 16: two threads per channel, thread q owning states 8q ..
+// 8q+7 as two float4, so that a warp's loads and stores of h cover 1 KB of contiguous
+// state (each 32-byte sector is used whole by the pair of loads); the per-channel
+// work (softplus, gate) is repeated by only two threads, and the readout is summed
+// with one butterfly shuffle. Requires 16-byte aligned h and A rows and 4-element
+// aligned B, C rows.
 template <typename T>
 __global__ void __launch_bounds__(256)
-    step_quad_kernel(int64_t Bsz, int64_t D, int softplus, const T *__restrict__ x, const T *__restrict__ dt,
+    step_pair_kernel(int64_t Bsz, int64_t D, int softplus, const T *__restrict__ x, const T *__restrict__ dt,
                      const T *__restrict__ z, const T *__restrict__ Bm, const T *__restrict__ Cm,
                      const float *__restrict__ A, const float *__restrict__ Dskip, const float *__restrict__ dt_bias,
                      float *__restrict__ h, T *__restrict__ y) {
     const int64_t gid = int64_t(blockIdx.x) * blockDim.x + threadIdx.x;
-    const int64_t ch = gid >> 2;
-    const int q = int(gid & 3);
-    const bool valid = ch < Bsz * D;  // all four threads of a channel agree
+    const int64_t ch = gid >> 1;
+    const int q = int(gid & 1);
+    const bool valid = ch < Bsz * D;  // both threads of a channel agree
     const int64_t chv = valid ? ch : 0;
     const int64_t b = chv / D, d = chv % D;
     float yv = 0.f, xv = 0.f;
@@ -101,20 +103,25 @@ __global__ void __launch_bounds__(256)
         const float v = Tok<T>::ldg(dt + ch) + (dt_bias ? __ldg(dt_bias + d) : 0.f);
         const float delta = softplus ? softplus_f(v) : v;
         const float dl = delta * kLog2e, u = delta * xv;
-        float4 *hp = reinterpret_cast<float4 *>(h + ch * kMaxN) + q;
-        float4 hv = *hp;
-        const float4 av = __ldg(reinterpret_cast<const float4 *>(A + d * kMaxN) + q);
-        const float4 bv = Tok<T>::quad(Bm + b * kMaxN + 4 * q);
-        const float4 cv = Tok<T>::quad(Cm + b * kMaxN + 4 * q);
-        hv.x = fmaf(ex2_approx(dl * av.x), hv.x, u * bv.x);
-        hv.y = fmaf(ex2_approx(dl * av.y), hv.y, u * bv.y);
-        hv.z = fmaf(ex2_approx(dl * av.z), hv.z, u * bv.z);
-        hv.w = fmaf(ex2_approx(dl * av.w), hv.w, u * bv.w);
-        *hp = hv;
-        yv = fmaf(cv.x, hv.x, fmaf(cv.y, hv.y, fmaf(cv.z, hv.z, cv.w * hv.w)));
+        float4 *hp = reinterpret_cast<float4 *>(h + ch * kMaxN) + 2 * q;
+        float4 hv[2] = {hp[0], hp[1]};
+        const float4 *ap = reinterpret_cast<const float4 *>(A + d * kMaxN) + 2 * q;
+        const float4 av[2] = {__ldg(ap), __ldg(ap + 1)};
+        const float4 bv[2] = {Tok<T>::quad(Bm + b * kMaxN + 8 * q), Tok<T>::quad(Bm + b * kMaxN + 8 * q + 4)};
+        const float4 cv[2] = {Tok<T>::quad(Cm + b * kMaxN + 8 * q), Tok<T>::quad(Cm + b * kMaxN + 8 * q + 4)};
+#pragma unroll
+        for (int i = 0; i < 2; ++i) {
+            hv[i].x = fmaf(ex2_approx(dl * av[i].x), hv[i].x, u * bv[i].x);
+            hv[i].y = fmaf(ex2_approx(dl * av[i].y), hv[i].y, u * bv[i].y);
+            hv[i].z = fmaf(ex2_approx(dl * av[i].z), hv[i].z, u * bv[i].z);
+            hv[i].w = fmaf(ex2_approx(dl * av[i].w), hv[i].w, u * bv[i].w);
+        }
+        hp[0] = hv[0];
+        hp[1] = hv[1];
+        yv = fmaf(cv[0].x, hv[0].x, fmaf(cv[0].y, hv[0].y, fmaf(cv[0].z, hv[0].z, cv[0].w * hv[0].w)));
+        yv += fmaf(cv[1].x, hv[1].x, fmaf(cv[1].y, hv[1].y, fmaf(cv[1].z, hv[1].z, cv[1].w * hv[1].w)));
     }
     yv += __shfl_xor_sync(0xffffffffu, yv, 1);
-    yv += __shfl_xor_sync(0xffffffffu, yv, 2);
     if (valid && q == 0) {
         yv = fmaf(Dskip ? __ldg(Dskip + d) : 0.f, xv, yv);
         if (z) yv *= silu_f(Tok<T>::ldg(z + ch));
@@ -410,16 +417,16 @@ ssm_status ssm_step(int64_t batch, int64_t dim, int64_t dstate, ssm_dtype dtype,
     cudaStream_t stream = static_cast<cudaStream_t>(stream_);
     const int64_t nch = batch * dim;
     const int sp = (flags & SSM_DELTA_SOFTPLUS) != 0;
-    // Four threads per channel when the state rows are whole float4 rows and B, C rows
+    // Two threads per channel when the state rows are whole float4 rows and B, C rows
     // can be read four elements at a time; one thread per channel otherwise.
-    const bool quad = dstate == kMaxN && aligned(A, 16) && aligned(Bm, 4 * es) && aligned(Cm, 4 * es);
-    const int threads = quad ? 256 : 128;
-    const int64_t blocks = ((quad ? 4 : 1) * nch + threads - 1) / threads;
+    const bool pair = dstate == kMaxN && aligned(A, 16) && aligned(Bm, 4 * es) && aligned(Cm, 4 * es);
+    const int threads = pair ? 256 : 128;
+    const int64_t blocks = ((pair ? 2 : 1) * nch + threads - 1) / threads;
     if (blocks > INT32_MAX) return SSM_ERR_UNSUPPORTED;
     if (dtype == SSM_BF16) {
         using T = __nv_bfloat16;
-        if (quad)
-            step_quad_kernel<T><<<unsigned(blocks), threads, 0, stream>>>(
+        if (pair)
+            step_pair_kernel<T><<<unsigned(blocks), threads, 0, stream>>>(
                 batch, dim, sp, static_cast<const T *>(x), static_cast<const T *>(dt), static_cast<const T *>(z),
                 static_cast<const T *>(Bm), static_cast<const T *>(Cm), A, Dskip, dt_bias, h, static_cast<T *>(y));
         else
@@ -428,8 +435,8 @@ ssm_status ssm_step(int64_t batch, int64_t dim, int64_t dstate, ssm_dtype dtype,
                 static_cast<const T *>(z), static_cast<const T *>(Bm), static_cast<const T *>(Cm), A, Dskip,
                 dt_bias, h, static_cast<T *>(y));
     } else {
-        if (quad)
-            step_quad_kernel<float><<<unsigned(blocks), threads, 0, stream>>>(
+        if (pair)
+            step_pair_kernel<float><<<unsigned(blocks), threads, 0, stream>>>(
                 batch, dim, sp, static_cast<const float *>(x), static_cast<const float *>(dt),
                 static_cast<const float *>(z), static_cast<const float *>(Bm), static_cast<const float *>(Cm), A,
                 Dskip, dt_bias, h, static_cast<float *>(y));
