@@ -61,6 +61,11 @@ enum {
     SSM_DELTA_SOFTPLUS = 1u, /* Delta = softplus(dt + dt_bias); without it Delta = dt + dt_bias */
     SSM_A_GENERAL = 2u,      /* evaluate every exp(Delta A[d,n]) on its own, even where a row of A
                                 is an arithmetic progression in n (see ssm_scan_fwd) */
+    SSM_EXACT_ZOH = 4u,      /* exact zero-order hold for the input: Bbar = (exp(Delta A) - 1) / A * B
+                                (Delta B where A[d,n] = 0) instead of Delta B; the form under which
+                                the Mamba summary's Theorem 1 (a gated RNN for N = 1) is exact. The
+                                kernels evaluate (exp(z) - 1) / z, z = Delta A, by a series for
+                                |z| < 1/16, where the subtraction would lose relative precision */
     SSM_TEST_DROP_HANDOFF = 0x80000000u /* fault-injection hook for tests: the first time segment of
                                 channel group 0 does not publish its state, so its successor's
                                 bounded wait runs out; ssm_workspace_status() then reports

@@ -16,7 +16,7 @@ import ctypes
 import torch
 
 from . import _native
-from ._native import SSM_A_GENERAL, SSM_DELTA_SOFTPLUS
+from ._native import SSM_A_GENERAL, SSM_DELTA_SOFTPLUS, SSM_EXACT_ZOH
 
 __all__ = ["scan_fwd", "scan_fwd_host", "step", "workspace_size", "workspace_status", "ScanWorkspace"]
 
@@ -45,8 +45,9 @@ def _need(t, name, shape, dtype, device):
         raise ValueError(f"{name}: must be contiguous")
 
 
-def _flags(delta_softplus, general_A):
-    return (SSM_DELTA_SOFTPLUS if delta_softplus else 0) | (SSM_A_GENERAL if general_A else 0)
+def _flags(delta_softplus, general_A, exact_zoh=False):
+    return ((SSM_DELTA_SOFTPLUS if delta_softplus else 0) | (SSM_A_GENERAL if general_A else 0)
+            | (SSM_EXACT_ZOH if exact_zoh else 0))
 
 
 def _scan_args(x, dt, A, B, C, D, z, dt_bias, h0, y, h_last, flags):
@@ -86,13 +87,14 @@ _default_ws = {}
 
 
 def scan_fwd(x, dt, A, B, C, D=None, z=None, dt_bias=None, h0=None, *, delta_softplus=True,
-             general_A=False, return_last_state=False, out=None, h_last=None, workspace=None,
+             general_A=False, exact_zoh=False, return_last_state=False, out=None, h_last=None, workspace=None,
              stream=None):
     """Selective scan forward over whole sequences (see include/ssm_scan.h, ssm_scan_fwd).
 
     x, dt, z: [B, L, D] float32 or bfloat16; B, C: [B, L, N] same dtype; A: [D, N]
     float32; D, dt_bias: [D] float32; h0: [B, D, N] float32. Returns y (same dtype
-    as x) and, with return_last_state, the final state [B, D, N] float32.
+    as x) and, with return_last_state, the final state [B, D, N] float32. exact_zoh:
+    Bbar = (exp(Delta A) - 1) / A B instead of Delta B.
     """
     dev = x.device
     if x.dtype not in _TOKEN_DTYPES:
@@ -121,7 +123,7 @@ def scan_fwd(x, dt, A, B, C, D=None, z=None, dt_bias=None, h0=None, *, delta_sof
         h_last = torch.empty((Bsz, Dm, N), dtype=torch.float32, device=dev)
     if h_last is not None:
         _need(h_last, "h_last", (Bsz, Dm, N), torch.float32, dev)
-    args = _scan_args(x, dt, A, B, C, D, z, dt_bias, h0, y, h_last, _flags(delta_softplus, general_A))
+    args = _scan_args(x, dt, A, B, C, D, z, dt_bias, h0, y, h_last, _flags(delta_softplus, general_A, exact_zoh))
     nbytes = int(_native.lib().ssm_scan_workspace_size(ctypes.byref(args)))
     if workspace is None:
         key = (dev, torch.cuda.current_stream(dev).cuda_stream if stream is None else stream.cuda_stream)
@@ -150,8 +152,8 @@ _default_staging = {}
 
 
 def scan_fwd_host(x, dt, A, B, C, D=None, z=None, dt_bias=None, h0=None, *, chunk_len=16384,
-                  delta_softplus=True, general_A=False, return_last_state=False, out=None, h_last=None,
-                  workspace=None, staging=None, stream=None):
+                  delta_softplus=True, general_A=False, exact_zoh=False, return_last_state=False, out=None,
+                  h_last=None, workspace=None, staging=None, stream=None):
     """Selective scan over host-resident tokens (see include/ssm_scan.h, ssm_scan_fwd_host).
 
     x, dt, z: [B, L, D] and B, C: [B, L, N] host tensors (page-locked memory lets the
@@ -186,7 +188,7 @@ def scan_fwd_host(x, dt, A, B, C, D=None, z=None, dt_bias=None, h0=None, *, chun
         h_last = torch.empty((Bsz, Dm, N), dtype=torch.float32, device=dev)
     if h_last is not None:
         _need(h_last, "h_last", (Bsz, Dm, N), torch.float32, dev)
-    args = _scan_args(x, dt, A, B, C, D, z, dt_bias, h0, y, h_last, _flags(delta_softplus, general_A))
+    args = _scan_args(x, dt, A, B, C, D, z, dt_bias, h0, y, h_last, _flags(delta_softplus, general_A, exact_zoh))
     lib = _native.lib()
     key = (dev, torch.cuda.current_stream(dev).cuda_stream if stream is None else stream.cuda_stream)
     nbytes = int(lib.ssm_scan_workspace_size(ctypes.byref(args)))
@@ -212,7 +214,7 @@ def workspace_status(workspace, stream=None):
 
 
 def step(x, dt, A, B, C, h, D=None, z=None, dt_bias=None, *, delta_softplus=True, general_A=False,
-         out=None, stream=None):
+         exact_zoh=False, out=None, stream=None):
     """One recurrent decode step (see include/ssm_scan.h, ssm_step); h is updated in place.
 
     x, dt, z: [B, D]; B, C: [B, N]; A: [D, N]; h: [B, D, N] float32. Returns y [B, D].
@@ -237,7 +239,7 @@ def step(x, dt, A, B, C, h, D=None, z=None, dt_bias=None, *, delta_softplus=True
         _need(dt_bias, "dt_bias", (Dm,), torch.float32, dev)
     y = torch.empty_like(x) if out is None else out
     _need(y, "out", (Bsz, Dm), tok, dev)
-    rc = _native.lib().ssm_step(Bsz, Dm, N, _TOKEN_DTYPES[tok], _flags(delta_softplus, general_A),
+    rc = _native.lib().ssm_step(Bsz, Dm, N, _TOKEN_DTYPES[tok], _flags(delta_softplus, general_A, exact_zoh),
                                 _ptr(x), _ptr(dt), _ptr(z), _ptr(B), _ptr(C), _ptr(A), _ptr(D),
                                 _ptr(dt_bias), _ptr(h), _ptr(y), _stream_handle(stream))
     _native.check(rc, "ssm_step")

@@ -37,8 +37,17 @@ constexpr size_t kWsHeader = 256;
 
 inline size_t round_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 
+// Exact zero-order hold: Bbar / B per unit input = (Abar - 1) / A, by the series
+// Delta (1 + z/2 + z^2/6 + z^3/24 + z^4/120), z = Delta A, below |z| = 1/16.
+__device__ __forceinline__ float zoh_w(const float delta, const float A, const float abar) {
+    const float z = delta * A;
+    if (fabsf(z) < 0.0625f)
+        return delta * fmaf(z, fmaf(z, fmaf(z, fmaf(z, 1.f / 120.f, 1.f / 24.f), 1.f / 6.f), 0.5f), 1.f);
+    return __fdividef(abar - 1.f, A);
+}
+
 // ------------------------------------------------------------- step kernel
-template <typename T>
+template <typename T, bool ZOH>
 __global__ void __launch_bounds__(128)
     step_kernel(int64_t Bsz, int64_t D, int N, int softplus, const T *__restrict__ x, const T *__restrict__ dt,
                 const T *__restrict__ z, const T *__restrict__ Bm, const T *__restrict__ Cm,
@@ -60,16 +69,18 @@ __global__ void __launch_bounds__(128)
         float *hs = reinterpret_cast<float *>(hv);
 #pragma unroll
         for (int n = 0; n < kMaxN; ++n) {
-            const float a = ex2_approx(dl * __ldg(A + d * kMaxN + n));
-            hs[n] = fmaf(a, hs[n], u * Tok<T>::ldg(Bm + b * kMaxN + n));
+            const float an = __ldg(A + d * kMaxN + n), a = ex2_approx(dl * an);
+            const float bx = ZOH ? xv * zoh_w(delta, an, a) : u;
+            hs[n] = fmaf(a, hs[n], bx * Tok<T>::ldg(Bm + b * kMaxN + n));
             yv = fmaf(Tok<T>::ldg(Cm + b * kMaxN + n), hs[n], yv);
         }
 #pragma unroll
         for (int i = 0; i < 4; ++i) reinterpret_cast<float4 *>(hp)[i] = hv[i];
     } else {
         for (int n = 0; n < N; ++n) {
-            const float a = ex2_approx(dl * __ldg(A + d * N + n));
-            const float hn = fmaf(a, hp[n], u * Tok<T>::ldg(Bm + b * N + n));
+            const float an = __ldg(A + d * N + n), a = ex2_approx(dl * an);
+            const float bx = ZOH ? xv * zoh_w(delta, an, a) : u;
+            const float hn = fmaf(a, hp[n], bx * Tok<T>::ldg(Bm + b * N + n));
             hp[n] = hn;
             yv = fmaf(Tok<T>::ldg(Cm + b * N + n), hn, yv);
         }
@@ -85,7 +96,7 @@ __global__ void __launch_bounds__(128)
 // work (softplus, gate) is repeated by only two threads, and the readout is summed
 // with one butterfly shuffle. Requires 16-byte aligned h and A rows and 4-element
 // aligned B, C rows.
-template <typename T>
+template <typename T, bool ZOH>
 __global__ void __launch_bounds__(256)
     step_pair_kernel(int64_t Bsz, int64_t D, int softplus, const T *__restrict__ x, const T *__restrict__ dt,
                      const T *__restrict__ z, const T *__restrict__ Bm, const T *__restrict__ Cm,
@@ -109,12 +120,24 @@ __global__ void __launch_bounds__(256)
         const float4 av[2] = {__ldg(ap), __ldg(ap + 1)};
         const float4 bv[2] = {Tok<T>::quad(Bm + b * kMaxN + 8 * q), Tok<T>::quad(Bm + b * kMaxN + 8 * q + 4)};
         const float4 cv[2] = {Tok<T>::quad(Cm + b * kMaxN + 8 * q), Tok<T>::quad(Cm + b * kMaxN + 8 * q + 4)};
+        if (ZOH) {
 #pragma unroll
-        for (int i = 0; i < 2; ++i) {
-            hv[i].x = fmaf(ex2_approx(dl * av[i].x), hv[i].x, u * bv[i].x);
-            hv[i].y = fmaf(ex2_approx(dl * av[i].y), hv[i].y, u * bv[i].y);
-            hv[i].z = fmaf(ex2_approx(dl * av[i].z), hv[i].z, u * bv[i].z);
-            hv[i].w = fmaf(ex2_approx(dl * av[i].w), hv[i].w, u * bv[i].w);
+            for (int i = 0; i < 2; ++i) {
+                const float a0 = ex2_approx(dl * av[i].x), a1 = ex2_approx(dl * av[i].y);
+                const float a2 = ex2_approx(dl * av[i].z), a3 = ex2_approx(dl * av[i].w);
+                hv[i].x = fmaf(a0, hv[i].x, xv * zoh_w(delta, av[i].x, a0) * bv[i].x);
+                hv[i].y = fmaf(a1, hv[i].y, xv * zoh_w(delta, av[i].y, a1) * bv[i].y);
+                hv[i].z = fmaf(a2, hv[i].z, xv * zoh_w(delta, av[i].z, a2) * bv[i].z);
+                hv[i].w = fmaf(a3, hv[i].w, xv * zoh_w(delta, av[i].w, a3) * bv[i].w);
+            }
+        } else {
+#pragma unroll
+            for (int i = 0; i < 2; ++i) {
+                hv[i].x = fmaf(ex2_approx(dl * av[i].x), hv[i].x, u * bv[i].x);
+                hv[i].y = fmaf(ex2_approx(dl * av[i].y), hv[i].y, u * bv[i].y);
+                hv[i].z = fmaf(ex2_approx(dl * av[i].z), hv[i].z, u * bv[i].z);
+                hv[i].w = fmaf(ex2_approx(dl * av[i].w), hv[i].w, u * bv[i].w);
+            }
         }
         hp[0] = hv[0];
         hp[1] = hv[1];
@@ -177,13 +200,19 @@ struct ScanPlan {
     size_t smem = 0;
 };
 
-void *pick_kernel(ssm_dtype dt, bool deep) {
+template <bool ZOH>
+void *pick_kernel_t(ssm_dtype dt, bool deep) {
     using namespace ssm::scan;
     if (dt == SSM_BF16)
-        return deep ? reinterpret_cast<void *>(&scan_ws_kernel<__nv_bfloat16, Deep>)
-                    : reinterpret_cast<void *>(&scan_ws_kernel<__nv_bfloat16, Shallow>);
-    return deep ? reinterpret_cast<void *>(&scan_ws_kernel<float, Deep>)
-                : reinterpret_cast<void *>(&scan_ws_kernel<float, Shallow>);
+        return deep ? reinterpret_cast<void *>(&scan_ws_kernel<__nv_bfloat16, Deep, ZOH>)
+                    : reinterpret_cast<void *>(&scan_ws_kernel<__nv_bfloat16, Shallow, ZOH>);
+    return deep ? reinterpret_cast<void *>(&scan_ws_kernel<float, Deep, ZOH>)
+                : reinterpret_cast<void *>(&scan_ws_kernel<float, Shallow, ZOH>);
+}
+// The exact zero-order hold is a separate instantiation, so the default kernel carries
+// none of its code.
+void *pick_kernel(ssm_dtype dt, bool deep, bool zoh = false) {
+    return zoh ? pick_kernel_t<true>(dt, deep) : pick_kernel_t<false>(dt, deep);
 }
 size_t pick_smem(ssm_dtype dt, bool deep) {
     using namespace ssm::scan;
@@ -216,10 +245,13 @@ bool scan_occupancy(ssm_dtype dt, int occ[2]) {
         if (cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) != cudaSuccess) return false;
         for (int deep = 0; deep < 2; ++deep) {
             void *kern = pick_kernel(dt, deep != 0);
+            void *kern_zoh = pick_kernel(dt, deep != 0, true);  // same shape and register budget
             const size_t smem = pick_smem(dt, deep != 0);
             int o = 0;
             if (smem <= size_t(optin)) {
                 if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem)) != cudaSuccess ||
+                    cudaFuncSetAttribute(kern_zoh, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem)) !=
+                        cudaSuccess ||
                     cudaOccupancyMaxActiveBlocksPerMultiprocessor(&o, kern, ssm::scan::NTHREADS, smem) != cudaSuccess)
                     return false;
             }
@@ -266,7 +298,8 @@ bool plan_scan(const ssm_scan_args *a, ScanPlan *pl) {
 ssm_status check_common(int64_t Bsz, int64_t D, int64_t N, ssm_dtype dt, uint32_t flags) {
     if (Bsz < 0 || D < 0 || N < 1) return SSM_ERR_INVALID;
     if (dt != SSM_F32 && dt != SSM_BF16) return SSM_ERR_INVALID;
-    if (flags & ~uint32_t(SSM_DELTA_SOFTPLUS | SSM_A_GENERAL | SSM_TEST_DROP_HANDOFF)) return SSM_ERR_INVALID;
+    if (flags & ~uint32_t(SSM_DELTA_SOFTPLUS | SSM_A_GENERAL | SSM_EXACT_ZOH | SSM_TEST_DROP_HANDOFF))
+        return SSM_ERR_INVALID;
     if (N > kMaxN) return SSM_ERR_UNSUPPORTED;
     if (D % (dt == SSM_BF16 ? 8 : 4) != 0) return SSM_ERR_UNSUPPORTED;
     return SSM_OK;
@@ -324,6 +357,21 @@ unsigned char *static_scratch() {
 }  // namespace
 
 // ======================================================================= C ABI
+template <typename T, bool ZOH>
+void launch_step(bool pair, unsigned grid, int threads, cudaStream_t stream, int64_t batch, int64_t dim, int N,
+                 int sp, const void *x, const void *dt, const void *z, const void *Bm, const void *Cm,
+                 const float *A, const float *Dskip, const float *dt_bias, float *h, void *y) {
+    if (pair)
+        step_pair_kernel<T, ZOH><<<grid, threads, 0, stream>>>(
+            batch, dim, sp, static_cast<const T *>(x), static_cast<const T *>(dt), static_cast<const T *>(z),
+            static_cast<const T *>(Bm), static_cast<const T *>(Cm), A, Dskip, dt_bias, h, static_cast<T *>(y));
+    else
+        step_kernel<T, ZOH><<<grid, threads, 0, stream>>>(
+            batch, dim, N, sp, static_cast<const T *>(x), static_cast<const T *>(dt), static_cast<const T *>(z),
+            static_cast<const T *>(Bm), static_cast<const T *>(Cm), A, Dskip, dt_bias, h, static_cast<T *>(y));
+}
+
+
 extern "C" {
 
 size_t ssm_scan_workspace_size(const ssm_scan_args *a) {
@@ -393,7 +441,7 @@ ssm_status ssm_scan_fwd(const ssm_scan_args *a, void *stream_) {
     p.drop_handoff = (a->flags & SSM_TEST_DROP_HANDOFF) != 0;
     p.bc_tma = bc_tma;
 
-    void *kern = pick_kernel(a->dtype, pl.deep);
+    void *kern = pick_kernel(a->dtype, pl.deep, (a->flags & SSM_EXACT_ZOH) != 0);
     void *args[] = {&tx, &tdt, &tz, &tb, &tc, &ty, &p};
     cudaError_t e = cudaLaunchKernel(kern, dim3(pl.grid), dim3(ssm::scan::NTHREADS), args, pl.smem, stream);
     return e == cudaSuccess ? SSM_OK : SSM_ERR_CUDA;
@@ -417,34 +465,28 @@ ssm_status ssm_step(int64_t batch, int64_t dim, int64_t dstate, ssm_dtype dtype,
     cudaStream_t stream = static_cast<cudaStream_t>(stream_);
     const int64_t nch = batch * dim;
     const int sp = (flags & SSM_DELTA_SOFTPLUS) != 0;
+    const int zoh = (flags & SSM_EXACT_ZOH) != 0;
     // Two threads per channel when the state rows are whole float4 rows and B, C rows
     // can be read four elements at a time; one thread per channel otherwise.
     const bool pair = dstate == kMaxN && aligned(A, 16) && aligned(Bm, 4 * es) && aligned(Cm, 4 * es);
     const int threads = pair ? 256 : 128;
     const int64_t blocks = ((pair ? 2 : 1) * nch + threads - 1) / threads;
     if (blocks > INT32_MAX) return SSM_ERR_UNSUPPORTED;
+    const unsigned grid = unsigned(blocks);
     if (dtype == SSM_BF16) {
-        using T = __nv_bfloat16;
-        if (pair)
-            step_pair_kernel<T><<<unsigned(blocks), threads, 0, stream>>>(
-                batch, dim, sp, static_cast<const T *>(x), static_cast<const T *>(dt), static_cast<const T *>(z),
-                static_cast<const T *>(Bm), static_cast<const T *>(Cm), A, Dskip, dt_bias, h, static_cast<T *>(y));
+        if (zoh)
+            launch_step<__nv_bfloat16, true>(pair, grid, threads, stream, batch, dim, int(dstate), sp, x, dt, z, Bm,
+                                             Cm, A, Dskip, dt_bias, h, y);
         else
-            step_kernel<T><<<unsigned(blocks), threads, 0, stream>>>(
-                batch, dim, int(dstate), sp, static_cast<const T *>(x), static_cast<const T *>(dt),
-                static_cast<const T *>(z), static_cast<const T *>(Bm), static_cast<const T *>(Cm), A, Dskip,
-                dt_bias, h, static_cast<T *>(y));
+            launch_step<__nv_bfloat16, false>(pair, grid, threads, stream, batch, dim, int(dstate), sp, x, dt, z,
+                                              Bm, Cm, A, Dskip, dt_bias, h, y);
     } else {
-        if (pair)
-            step_pair_kernel<float><<<unsigned(blocks), threads, 0, stream>>>(
-                batch, dim, sp, static_cast<const float *>(x), static_cast<const float *>(dt),
-                static_cast<const float *>(z), static_cast<const float *>(Bm), static_cast<const float *>(Cm), A,
-                Dskip, dt_bias, h, static_cast<float *>(y));
+        if (zoh)
+            launch_step<float, true>(pair, grid, threads, stream, batch, dim, int(dstate), sp, x, dt, z, Bm, Cm, A,
+                                     Dskip, dt_bias, h, y);
         else
-            step_kernel<float><<<unsigned(blocks), threads, 0, stream>>>(
-                batch, dim, int(dstate), sp, static_cast<const float *>(x), static_cast<const float *>(dt),
-                static_cast<const float *>(z), static_cast<const float *>(Bm), static_cast<const float *>(Cm), A,
-                Dskip, dt_bias, h, static_cast<float *>(y));
+            launch_step<float, false>(pair, grid, threads, stream, batch, dim, int(dstate), sp, x, dt, z, Bm, Cm, A,
+                                      Dskip, dt_bias, h, y);
     }
     return cudaGetLastError() == cudaSuccess ? SSM_OK : SSM_ERR_CUDA;
 }

@@ -193,16 +193,31 @@ __device__ __forceinline__ void set_timeout(uint32_t *status, int lane) {
     if (lane == 0) atomicExch(status, uint32_t(SSM_ERR_TIMEOUT));
 }
 
+// Exact zero-order hold for two states: w = Bbar / B per unit input = (Abar - 1) / A,
+// with z = Delta A; below |z| = 1/16 the series Delta (1 + z/2 + z^2/6 + z^3/24 +
+// z^4/120) (truncation below 2e-9 relative), where Abar - 1 would lose precision.
+// a: Abar; ia: 1/A (0 where A = 0, where the series gives Delta).
+__device__ __forceinline__ float2 zoh_weight(const float2 z, const float2 a, const float2 ia, const float delta) {
+    float2 q = __ffma2_rn(z, f2(1.f / 120.f, 1.f / 120.f), f2(1.f / 24.f, 1.f / 24.f));
+    q = __ffma2_rn(z, q, f2(1.f / 6.f, 1.f / 6.f));
+    q = __ffma2_rn(z, q, f2(0.5f, 0.5f));
+    q = __ffma2_rn(z, q, f2(1.f, 1.f));
+    const float2 ser = __fmul2_rn(f2(delta, delta), q);
+    const float2 dir = __fmul2_rn(__fadd2_rn(a, f2(-1.f, -1.f)), ia);
+    return f2(fabsf(z.x) < 0.0625f ? ser.x : dir.x, fabsf(z.y) < 0.0625f ? ser.y : dir.y);
+}
+
 // ---------------------------------------------------------------- consumers
 // TT steps of one tile for one lane (its channel, the warp's four states), in
 // blocks of four steps. rec: this lane's records (stride CH float2 per step); bc: B
 // of the warp's states (stride 32 floats per step; C at +16); part: this lane's
 // partials (stride CH float4 per block of four steps). Aq: A[c][4w .. 4w+3]; del:
-// A[c][1] - A[c][0].
-template <bool STRUCT>
+// A[c][1] - A[c][0]; ZOH (exact zero-order hold): zA = A ln 2 and iA = 1/A of the
+// four states, and the records carry x in place of Delta x.
+template <bool STRUCT, bool ZOH>
 __device__ __forceinline__ void consume_tile(const float2 *__restrict__ rec, const float *__restrict__ bc,
                                              float4 *__restrict__ part, const float4 Aq, const float del,
-                                             float2 &h01, float2 &h23) {
+                                             const float4 zA, const float4 iA, float2 &h01, float2 &h23) {
     constexpr int S = 4;
 #pragma unroll 2
     for (int t0 = 0; t0 < TT; t0 += S) {
@@ -248,6 +263,16 @@ __device__ __forceinline__ void consume_tile(const float2 *__restrict__ rec, con
             ub01[s] = __fmul2_rn(f2(p[s].x, p[s].x), f2(b4[s].x, b4[s].y));
             ub23[s] = __fmul2_rn(f2(p[s].x, p[s].x), f2(b4[s].z, b4[s].w));
         }
+        if (ZOH) {  // the record carries x; Bbar x = B x (Abar - 1) / A
+#pragma unroll
+            for (int s = 0; s < S; ++s) {
+                const float delta = p[s].y * kLn2;
+                const float2 z01 = __fmul2_rn(f2(p[s].y, p[s].y), f2(zA.x, zA.y));
+                const float2 z23 = __fmul2_rn(f2(p[s].y, p[s].y), f2(zA.z, zA.w));
+                ub01[s] = __fmul2_rn(ub01[s], zoh_weight(z01, a01[s], f2(iA.x, iA.y), delta));
+                ub23[s] = __fmul2_rn(ub23[s], zoh_weight(z23, a23[s], f2(iA.z, iA.w), delta));
+            }
+        }
         float2 g01[S], g23[S];
 #pragma unroll
         for (int s = 0; s < S; ++s) {
@@ -268,12 +293,13 @@ __device__ __forceinline__ void consume_tile(const float2 *__restrict__ rec, con
 
 // ---------------------------------------------------------------- prologue
 // Records of TP steps (rows t0 .. t0+TP-1 of a tile) for channel c: (u = Delta x,
-// Delta log2 e), with Delta = softplus(dt + bias) (or dt + bias). Rows at or past tlen
-// get (0, 0): Abar = 1, no input.
+// Delta log2 e), with Delta = softplus(dt + bias) (or dt + bias); with `zoh` (exact
+// zero-order hold) u = x, the consumers apply the weight. Rows at or past tlen get
+// (0, 0): Abar = 1, no input.
 template <typename T>
 __device__ __forceinline__ void prologue_rows(const T *__restrict__ sx, const T *__restrict__ sdt,
                                               float2 *__restrict__ rec, const int t0, const int tlen,
-                                              const float bias, const bool softplus) {
+                                              const float bias, const bool softplus, const bool zoh) {
     constexpr int NPR = TP / 2;  // pairs of steps
     float2 v[NPR], xv[NPR];
 #pragma unroll
@@ -293,7 +319,7 @@ __device__ __forceinline__ void prologue_rows(const T *__restrict__ sx, const T 
     float2 u[NPR], dl[NPR];
 #pragma unroll
     for (int q = 0; q < NPR; ++q) {
-        u[q] = __fmul2_rn(delta[q], xv[q]);
+        u[q] = zoh ? xv[q] : __fmul2_rn(delta[q], xv[q]);
         dl[q] = __fmul2_rn(delta[q], f2(kLog2e, kLog2e));
     }
 #pragma unroll
@@ -357,7 +383,7 @@ __device__ __forceinline__ void epilogue_rows(const float4 *__restrict__ part, c
 }
 
 // ------------------------------------------------------------------- kernel
-template <typename T, typename C>
+template <typename T, typename C, bool ZOH>
 __global__ void __launch_bounds__(NTHREADS, C::MINB)
     scan_ws_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_dt,
                    const __grid_constant__ CUtensorMap tm_z, const __grid_constant__ CUtensorMap tm_b,
@@ -542,7 +568,7 @@ __global__ void __launch_bounds__(NTHREADS, C::MINB)
             float2 *rec = reinterpret_cast<float2 *>(smem + S::rec_off + r * S::rec_bytes) + c;
             prologue_rows<T>(reinterpret_cast<const T *>(stage + S::st_x) + c,
                              reinterpret_cast<const T *>(stage + S::st_dt) + c, rec, h * TP, m.tlen, bias_c,
-                             p.softplus != 0);
+                             p.softplus != 0, ZOH);
             // B and C rows of this half widened to float32: row t = [B_0 .. B_15 | C_0 .. C_15],
             // in 16-byte chunks; chunk id = q * 32 + lane covers row h*TP + id / 8 and chunk
             // id % 8 (0-3: B, 4-7: C), so eight consecutive lanes write one 128-byte row.
@@ -581,7 +607,7 @@ __global__ void __launch_bounds__(NTHREADS, C::MINB)
         const int c = lane;  // channel within the group
         const int w = warp;  // states 4w .. 4w+3
         float2 h01 = f2(0.f, 0.f), h23 = f2(0.f, 0.f);
-        float4 Aq = make_float4(0.f, 0.f, 0.f, 0.f);
+        float4 Aq = make_float4(0.f, 0.f, 0.f, 0.f), zA = Aq, iA = Aq;
         float del = 0.f;
         for (int i = 0;; ++i) {
             const int r = i % R_REC, pr = i % R_PART;
@@ -606,6 +632,11 @@ __global__ void __launch_bounds__(NTHREADS, C::MINB)
                     a[j] = (dvalid && n < p.N) ? __ldg(p.A + d * p.N + n) : 0.f;
                 }
                 Aq = make_float4(a[0], a[1], a[2], a[3]);
+                if (ZOH) {
+                    zA = make_float4(a[0] * kLn2, a[1] * kLn2, a[2] * kLn2, a[3] * kLn2);
+                    iA = make_float4(a[0] != 0.f ? 1.f / a[0] : 0.f, a[1] != 0.f ? 1.f / a[1] : 0.f,
+                                     a[2] != 0.f ? 1.f / a[2] : 0.f, a[3] != 0.f ? 1.f / a[3] : 0.f);
+                }
                 del = (dvalid && p.N >= 2) ? __ldg(p.A + d * p.N + 1) - __ldg(p.A + d * p.N) : 0.f;
                 if (m.k == 0) {
                     float hv[4];
@@ -643,8 +674,8 @@ __global__ void __launch_bounds__(NTHREADS, C::MINB)
             const float2 *rec = reinterpret_cast<const float2 *>(smem + S::rec_off + r * S::rec_bytes) + c;
             const float *bc = reinterpret_cast<const float *>(smem + S::bcf_off + r * S::bcf_bytes) + 4 * w;
             float4 *part = reinterpret_cast<float4 *>(smem + S::part_off + pr * S::part_bytes) + w * (TT / 4) * CH + c;
-            if (m.flags & F_STRUCT) consume_tile<true>(rec, bc, part, Aq, del, h01, h23);
-            else consume_tile<false>(rec, bc, part, Aq, del, h01, h23);
+            if (m.flags & F_STRUCT) consume_tile<true, ZOH>(rec, bc, part, Aq, del, zA, iA, h01, h23);
+            else consume_tile<false, ZOH>(rec, bc, part, Aq, del, zA, iA, h01, h23);
             warp_arrive(&bar_rec_free[r]);
             warp_arrive(&bar_part_full[pr]);
             if (m.flags & F_LAST) {

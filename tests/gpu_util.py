@@ -18,7 +18,7 @@ def f32np(t):
     return None if t is None else t.detach().cpu().float().numpy()
 
 
-def oracle_scan(inp, delta_softplus=True, sel=None):
+def oracle_scan(inp, delta_softplus=True, sel=None, exact_zoh=False):
     """Run the float64 oracle on exactly the tensors the GPU saw (optionally a channel subset)."""
     def tok(name):
         t = inp[name]
@@ -39,7 +39,7 @@ def oracle_scan(inp, delta_softplus=True, sel=None):
         h0 = h0[:, sel]
     return oracle.scan(tok("x"), tok("dt"), par("A"), storage(inp["B"]), storage(inp["C"]),
                        D=par("D"), z=tok("z"), dt_bias=par("dt_bias"), h0=f32np(h0),
-                       dtype=dtype_name(inp["x"]), delta_softplus=delta_softplus)
+                       dtype=dtype_name(inp["x"]), delta_softplus=delta_softplus, exact_zoh=exact_zoh)
 
 
 def rowwise_rel(got, ref, axis):
