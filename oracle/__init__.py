@@ -24,6 +24,8 @@ def _open(path):
     vp, i64, c_int, c_uint = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.c_uint
     lib.oracle_scan_f64.argtypes = [i64, i64, i64, i64, c_int, c_uint] + [vp] * 11 + [c_int]
     lib.oracle_scan_f64.restype = c_int
+    lib.oracle_scan_conv_f64.argtypes = [i64, i64, i64, i64, c_int, c_uint] + [vp] * 14 + [c_int]
+    lib.oracle_scan_conv_f64.restype = c_int
     lib.oracle_step_f64.argtypes = [i64, i64, i64, c_int, c_uint] + [vp] * 10 + [c_int]
     lib.oracle_step_f64.restype = c_int
     return lib
@@ -63,9 +65,10 @@ class Oracle:
         self.lib = _open(self.path)
 
     def scan(self, x, dt, A, B, C, D=None, z=None, dt_bias=None, h0=None, dtype="f32",
-             delta_softplus=True, exact_zoh=False, nthreads=None):
+             delta_softplus=True, exact_zoh=False, nthreads=None, conv_w=None, conv_b=None,
+             conv_x0=None):
         return _scan(self.lib, x, dt, A, B, C, D, z, dt_bias, h0, dtype, delta_softplus,
-                     exact_zoh, nthreads)
+                     exact_zoh, nthreads, conv_w, conv_b, conv_x0)
 
     def step(self, x, dt, A, B, C, h, D=None, z=None, dt_bias=None, dtype="f32",
              delta_softplus=True, exact_zoh=False, nthreads=None):
@@ -94,11 +97,15 @@ def step(*args, **kw):
 
 
 def _scan(lib, x, dt, A, B, C, D=None, z=None, dt_bias=None, h0=None, dtype="f32",
-          delta_softplus=True, exact_zoh=False, nthreads=None):
+          delta_softplus=True, exact_zoh=False, nthreads=None, conv_w=None, conv_b=None,
+          conv_x0=None):
     """Selective scan over a whole sequence.
 
     x, dt, z: [Bsz, L, Dm]; B, C: [Bsz, L, N]; A: [Dm, N]; D, dt_bias: [Dm];
     h0: [Bsz, Dm, N] (float32) or None for a zero initial state.
+    conv_w: [Dm, 4] (float32) puts the block's causal convolution and SiLU in front of
+    the SSM (its input becomes silu(conv_b + sum_k conv_w[:, k] x_{t-3+k})); conv_b: [Dm]
+    or None; conv_x0: [Bsz, 3, Dm] tokens before t = 0 (x's storage type) or None (zeros).
     Returns (y [Bsz, L, Dm] float64, h_last [Bsz, Dm, N] float64).
     """
     Bsz, L, Dm = np.shape(x)
@@ -115,12 +122,21 @@ def _scan(lib, x, dt, A, B, C, D=None, z=None, dt_bias=None, h0=None, dtype="f32
     y = np.empty((Bsz, L, Dm), dtype=np.float64)
     h_last = np.empty((Bsz, Dm, N), dtype=np.float64)
     flags = (DELTA_SOFTPLUS if delta_softplus else 0) | (EXACT_ZOH if exact_zoh else 0)
-    rc = lib.oracle_scan_f64(Bsz, L, Dm, N, 0 if dtype == "f32" else 1, flags,
-                             _ptr(x), _ptr(dt), _ptr(z), _ptr(B), _ptr(C), _ptr(A), _ptr(D),
-                             _ptr(dt_bias), _ptr(h0), _ptr(y), _ptr(h_last),
-                             default_threads() if nthreads is None else nthreads)
+    nt = default_threads() if nthreads is None else nthreads
+    common = (Bsz, L, Dm, N, 0 if dtype == "f32" else 1, flags, _ptr(x), _ptr(dt), _ptr(z), _ptr(B),
+              _ptr(C), _ptr(A), _ptr(D), _ptr(dt_bias), _ptr(h0))
+    if conv_w is None:
+        if conv_b is not None or conv_x0 is not None:
+            raise ValueError("conv_b and conv_x0 need conv_w")
+        rc = lib.oracle_scan_f64(*common, _ptr(y), _ptr(h_last), nt)
+    else:
+        conv_w = _f32(conv_w, (Dm, 4), "conv_w")
+        conv_b = _f32(conv_b, (Dm,), "conv_b")
+        conv_x0 = None if conv_x0 is None else _tok(conv_x0, dtype, (Bsz, 3, Dm), "conv_x0")
+        rc = lib.oracle_scan_conv_f64(*common, _ptr(conv_w), _ptr(conv_b), _ptr(conv_x0), _ptr(y),
+                                      _ptr(h_last), nt)
     if rc != 0:
-        raise ValueError("oracle_scan_f64 rejected its arguments")
+        raise ValueError("oracle scan rejected its arguments")
     return y, h_last
 
 

@@ -24,6 +24,14 @@
  *       [Mamba summary, block-architecture paragraph (gate branch: SiLU, multiply)]
  *   recurrent decode  one token: the same update with the state carried in place
  *       [SSM blog (shakilmahmud.com), section 3 "dual form": recurrence at O(1)]
+ *   short convolution (optional, oracle_scan_conv_f64) the block's main branch runs
+ *                     a short causal convolution (kernel width 4) and SiLU before the
+ *                     selective SSM; the SSM's input, in Bbar x and in D x, is then
+ *                     u_t = silu(conv_b + sum_{k=0..3} conv_w[d,k] x_{t-3+k}), one
+ *                     filter per channel, x_tau for tau < 0 taken from conv_x0 (the
+ *                     three tokens before the sequence, oldest first) or 0
+ *       [Mamba summary, block-architecture paragraph: projection, 1-D convolution of
+ *        kernel size 4, SiLU, selective SSM]
  *
  * Inputs are read in their storage type (float32, or bfloat16 given as raw
  * 16-bit patterns) and widened exactly to double, so a comparison measures the
@@ -32,6 +40,7 @@
  * Layouts (all row-major, contiguous):
  *   x, dt, z : [Bsz, L, Dm]     B, C : [Bsz, L, N]
  *   A : [Dm, N]   Dskip, dt_bias : [Dm]   h0, h_last : [Bsz, Dm, N]
+ *   conv_w : [Dm, 4]   conv_b : [Dm]   conv_x0 : [Bsz, 3, Dm] (storage type of x)
  *   y (double) : [Bsz, L, Dm]
  */
 #include <math.h>
@@ -41,6 +50,7 @@
 
 #define ORACLE_DELTA_SOFTPLUS 1u /* Delta = softplus(dt + dt_bias); else Delta = dt + dt_bias */
 #define ORACLE_EXACT_ZOH 2u      /* Bbar = (exp(Delta A) - 1) / A * B instead of Delta * B */
+#define ORACLE_CONV_K 4          /* width of the short causal convolution */
 
 /* Widen element i of a float32 (dtype 0) or bfloat16 (dtype 1) array to double. */
 static double widen(const void *p, int dtype, int64_t i) {
@@ -67,7 +77,25 @@ typedef struct {
     double *y, *h_last;
     const double *h0_f64; /* optional double initial state (used by the decode oracle) */
     int64_t ch_begin, ch_end; /* channel range [begin, end) over b * Dm + d */
+    const float *conv_w, *conv_b; /* optional short convolution: [Dm, 4] taps, [Dm] bias */
+    const void *conv_x0;          /* [Bsz, 3, Dm] tokens before t = 0, or NULL for zeros */
 } scan_job;
+
+/* Raw input token x_tau of channel (b, d); tau in [-3, 0) reads conv_x0, else 0. */
+static double raw_token(const scan_job *J, int64_t b, int64_t tau, int64_t d) {
+    if (tau >= 0) return widen(J->x, J->dtype, (b * J->L + tau) * J->Dm + d);
+    if (J->conv_x0) return widen(J->conv_x0, J->dtype, (b * (ORACLE_CONV_K - 1) + (tau + ORACLE_CONV_K - 1)) * J->Dm + d);
+    return 0.0;
+}
+
+/* The SSM's input at step t after the block's causal convolution and SiLU:
+   v = conv_b[d] + sum_k conv_w[d,k] x_{t-3+k} (tap 3 meets the current token), u = v sigma(v). */
+static double conv_silu(const scan_job *J, int64_t b, int64_t t, int64_t d) {
+    double v = J->conv_b ? (double)J->conv_b[d] : 0.0;
+    for (int k = 0; k < ORACLE_CONV_K; k++)
+        v += (double)J->conv_w[d * ORACLE_CONV_K + k] * raw_token(J, b, t - (ORACLE_CONV_K - 1) + k, d);
+    return v * sigmoid(v);
+}
 
 /* One channel (b, d): the whole sequence, in time order. */
 static void scan_channel(const scan_job *J, int64_t b, int64_t d, double *h) {
@@ -83,7 +111,7 @@ static void scan_channel(const scan_job *J, int64_t b, int64_t d, double *h) {
         const int64_t bc = (b * L + t) * N;            /* row of B_t and C_t      */
         const double v = widen(J->dt, J->dtype, i) + bias;
         const double delta = (J->flags & ORACLE_DELTA_SOFTPLUS) ? softplus(v) : v;
-        const double xv = widen(J->x, J->dtype, i);
+        const double xv = J->conv_w ? conv_silu(J, b, t, d) : widen(J->x, J->dtype, i);
         double y = 0.0;
         for (int64_t n = 0; n < N; n++) {
             const double a = (double)J->A[d * N + n];
@@ -114,6 +142,31 @@ static void *scan_worker(void *arg) {
     return NULL;
 }
 
+/* Run `base` over all its channels, split over `nthreads` POSIX threads
+   (nthreads <= 1 runs on the calling thread). */
+static void run_jobs(const scan_job *base, int nthreads) {
+    const int64_t nch = base->ch_end - base->ch_begin;
+    if (nthreads <= 1 || nch < 2) {
+        scan_worker((void *)base);
+        return;
+    }
+    if (nthreads > 512) nthreads = 512;
+    if (nthreads > nch) nthreads = (int)nch;
+    pthread_t tid[512];
+    scan_job jobs[512];
+    for (int k = 0; k < nthreads; k++) {
+        jobs[k] = *base;
+        jobs[k].ch_begin = base->ch_begin + nch * k / nthreads;
+        jobs[k].ch_end = base->ch_begin + nch * (k + 1) / nthreads;
+        if (pthread_create(&tid[k], NULL, scan_worker, &jobs[k]) != 0) {
+            scan_worker(&jobs[k]); /* run inline if a thread cannot be started */
+            tid[k] = 0;
+        }
+    }
+    for (int k = 0; k < nthreads; k++)
+        if (tid[k]) pthread_join(tid[k], NULL);
+}
+
 /*
  * Full-sequence scan. Returns 0 on success, -1 on invalid arguments.
  * Channels (b, d) are independent and are split over `nthreads` POSIX threads
@@ -126,27 +179,27 @@ int oracle_scan_f64(int64_t Bsz, int64_t L, int64_t Dm, int64_t N, int dtype, un
     if (Bsz < 0 || L < 0 || Dm < 0 || N < 1 || N > 256 || (dtype != 0 && dtype != 1)) return -1;
     if (!x || !dt || !Bm || !Cm || !A || !y) return -1;
     scan_job base = {Bsz, L, Dm, N, dtype, flags, x, dt, z, Bm, Cm, A, Dskip, dt_bias, h0,
-                     y, h_last, NULL, 0, Bsz * Dm};
-    const int64_t nch = Bsz * Dm;
-    if (nthreads <= 1 || nch < 2) {
-        scan_worker(&base);
-        return 0;
-    }
-    if (nthreads > 512) nthreads = 512;
-    if (nthreads > nch) nthreads = (int)nch;
-    pthread_t tid[512];
-    scan_job jobs[512];
-    for (int k = 0; k < nthreads; k++) {
-        jobs[k] = base;
-        jobs[k].ch_begin = nch * k / nthreads;
-        jobs[k].ch_end = nch * (k + 1) / nthreads;
-        if (pthread_create(&tid[k], NULL, scan_worker, &jobs[k]) != 0) {
-            scan_worker(&jobs[k]); /* run inline if a thread cannot be started */
-            tid[k] = 0;
-        }
-    }
-    for (int k = 0; k < nthreads; k++)
-        if (tid[k]) pthread_join(tid[k], NULL);
+                     y, h_last, NULL, 0, Bsz * Dm, NULL, NULL, NULL};
+    run_jobs(&base, nthreads);
+    return 0;
+}
+
+/*
+ * The scan behind the block's short causal convolution and SiLU: as oracle_scan_f64,
+ * with the SSM's input u_t = silu(conv_b + sum_k conv_w[d,k] x_{t-3+k}) (conv_w
+ * [Dm, 4] required; conv_b [Dm] or NULL; conv_x0 [Bsz, 3, Dm] in x's storage type, or
+ * NULL for zero tokens before t = 0).
+ */
+int oracle_scan_conv_f64(int64_t Bsz, int64_t L, int64_t Dm, int64_t N, int dtype, unsigned flags,
+                         const void *x, const void *dt, const void *z, const void *Bm, const void *Cm,
+                         const float *A, const float *Dskip, const float *dt_bias, const float *h0,
+                         const float *conv_w, const float *conv_b, const void *conv_x0,
+                         double *y, double *h_last, int nthreads) {
+    if (Bsz < 0 || L < 0 || Dm < 0 || N < 1 || N > 256 || (dtype != 0 && dtype != 1)) return -1;
+    if (!x || !dt || !Bm || !Cm || !A || !y || !conv_w) return -1;
+    scan_job base = {Bsz, L, Dm, N, dtype, flags, x, dt, z, Bm, Cm, A, Dskip, dt_bias, h0,
+                     y, h_last, NULL, 0, Bsz * Dm, conv_w, conv_b, conv_x0};
+    run_jobs(&base, nthreads);
     return 0;
 }
 
@@ -163,26 +216,7 @@ int oracle_step_f64(int64_t Bsz, int64_t Dm, int64_t N, int dtype, unsigned flag
     if (!x || !dt || !Bm || !Cm || !A || !h || !y) return -1;
     /* A step is the scan with L = 1, started from h and writing its end state to h. */
     scan_job base = {Bsz, 1, Dm, N, dtype, flags, x, dt, z, Bm, Cm, A, Dskip, dt_bias, NULL,
-                     y, h, h, 0, Bsz * Dm};
-    const int64_t nch = Bsz * Dm;
-    if (nthreads <= 1 || nch < 2) {
-        scan_worker(&base);
-        return 0;
-    }
-    if (nthreads > 512) nthreads = 512;
-    if (nthreads > nch) nthreads = (int)nch;
-    pthread_t tid[512];
-    scan_job jobs[512];
-    for (int k = 0; k < nthreads; k++) {
-        jobs[k] = base;
-        jobs[k].ch_begin = nch * k / nthreads;
-        jobs[k].ch_end = nch * (k + 1) / nthreads;
-        if (pthread_create(&tid[k], NULL, scan_worker, &jobs[k]) != 0) {
-            scan_worker(&jobs[k]);
-            tid[k] = 0;
-        }
-    }
-    for (int k = 0; k < nthreads; k++)
-        if (tid[k]) pthread_join(tid[k], NULL);
+                     y, h, h, 0, Bsz * Dm, NULL, NULL, NULL};
+    run_jobs(&base, nthreads);
     return 0;
 }

@@ -373,3 +373,58 @@ def pin_lti_convolution_bf16(orc):
 
 
 ALL_PINS.append(pin_lti_convolution_bf16)
+
+
+def pin_conv_front_end(orc, dtype=DT_F32, seed=12, with_bias=True):
+    """The block's short convolution in front of the SSM equals the SSM run on its output.
+
+    [Mamba summary (azimuth.plus), block-architecture paragraph: main branch = projection,
+    1-D convolution (kernel size 4), SiLU, selective SSM]. Expected input of the SSM:
+    u = silu(v), v_t = conv_b + sum_k conv_w[k] x_{t-3+k}, computed per channel by numpy's
+    cross-correlation over the sequence prefixed with conv_x0 (or three zeros); the oracle
+    without the convolution is then run on u (stored as float32) with every other input
+    unchanged, so the comparison carries only u's float32 rounding (~1e-7 relative).
+    Checks: the taps' order and causality, the bias, the SiLU, the three tokens before
+    t = 0 in both storage types, and that u feeds both Bbar x and D x.
+    """
+    rng = _rng(seed)
+    Bsz, L, Dm, N = 2, 29, 5, 3
+    xf = rng.standard_normal((Bsz, L, Dm)).astype(np.float32)
+    x0f = rng.standard_normal((Bsz, 3, Dm)).astype(np.float32)
+    toks = [rng.standard_normal((Bsz, L, Dm)).astype(np.float32) for _ in range(2)]  # dt, z
+    BC = [rng.standard_normal((Bsz, L, N)).astype(np.float32) for _ in range(2)]
+    A = (-0.2 - rng.random((Dm, N)) * 2.0).astype(np.float32)
+    D = rng.standard_normal(Dm).astype(np.float32)
+    bias = rng.standard_normal(Dm).astype(np.float32) * 0.5
+    w = (rng.standard_normal((Dm, 4)) * 0.7).astype(np.float32)
+    cb = (rng.standard_normal(Dm) * 0.3).astype(np.float32) if with_bias else None
+    if dtype == "bf16":
+        st = _bf16_bits
+        val = _bf16_value
+    else:
+        st = lambda a: a
+        val = lambda a: a.astype(np.float64)
+    x, x0, dt, z, Bm, Cm = (st(a) for a in (xf, x0f, toks[0], toks[1], BC[0], BC[1]))
+    for prefix in (x0, None):
+        pre = val(prefix) if prefix is not None else np.zeros((Bsz, 3, Dm))
+        seq = np.concatenate([pre, val(x)], axis=1)  # [Bsz, 3 + L, Dm]
+        v = np.empty((Bsz, L, Dm))
+        for b in range(Bsz):
+            for d in range(Dm):
+                v[b, :, d] = np.correlate(seq[b, :, d], w[d].astype(np.float64), mode="valid")
+        if cb is not None:
+            v += cb.astype(np.float64)
+        u = (v * _sigma(v)).astype(np.float32)
+        f32 = lambda a: val(a).astype(np.float32)  # exact: every stored value is a float32
+        y_ref, h_ref = orc.scan(u, f32(dt), A, f32(Bm), f32(Cm), D=D, z=f32(z), dt_bias=bias, dtype=DT_F32)
+        y, h = orc.scan(x, dt, A, Bm, Cm, D=D, z=z, dt_bias=bias, dtype=dtype, conv_w=w, conv_b=cb,
+                        conv_x0=prefix)
+        assert _rel(y - y_ref, y_ref) < 1e-5, "convolution front end: y"
+        assert _rel(h - h_ref, h_ref) < 1e-5, "convolution front end: final state"
+
+
+def pin_conv_front_end_bf16(orc):
+    pin_conv_front_end(orc, dtype="bf16", seed=13, with_bias=False)
+
+
+ALL_PINS += [pin_conv_front_end, pin_conv_front_end_bf16]

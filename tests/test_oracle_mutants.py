@@ -41,6 +41,14 @@ MUTANTS = {
     "sigmoid_sign": ("static double sigmoid(double v) { return 1.0 / (1.0 + exp(-v)); }",
                      "static double sigmoid(double v) { return 1.0 / (1.0 + exp(v)); }"),
     "delta_times_A_squared": ("const double abar = exp(delta * a);", "const double abar = exp(delta * a * a);"),
+    "conv_taps_reversed": ("J->conv_w[d * ORACLE_CONV_K + k]", "J->conv_w[d * ORACLE_CONV_K + (ORACLE_CONV_K - 1 - k)]"),
+    "conv_bias_dropped": ("double v = J->conv_b ? (double)J->conv_b[d] : 0.0;", "double v = 0.0;"),
+    "conv_without_silu": ("return v * sigmoid(v);", "return v;"),
+    "conv_x0_ignored": ("if (J->conv_x0) return", "if (0) return"),
+    "conv_x0_rows_reversed": ("(tau + ORACLE_CONV_K - 1)", "(-1 - tau)"),
+    "conv_reads_next_token": ("t - (ORACLE_CONV_K - 1) + k", "t - (ORACLE_CONV_K - 2) + k"),
+    "conv_skip_uses_raw_x": ("y += dskip * xv;", "y += dskip * widen(J->x, J->dtype, i);"),
+    "conv_update_uses_raw_x": ("h[n] = abar * h[n] + bbar * xv;", "h[n] = abar * h[n] + bbar * widen(J->x, J->dtype, i);"),
 }
 
 
