@@ -47,6 +47,8 @@ def parse_args(argv=None):
                     choices=["long_context", "mid_layer", "small_layer", "tiny_f32"])
     ap.add_argument("--general-A", action="store_true",
                     help="time the general exponential path as the headline (flag SSM_A_GENERAL)")
+    ap.add_argument("--conv", action="store_true",
+                    help="time the scan with the block's short convolution fused in front as the headline")
     ap.add_argument("--no-extras", action="store_true",
                     help="skip the e2e, decode, general-A and CPU-baseline legs (profiling runs)")
     ap.add_argument("--seqlen", type=int, default=None,
@@ -303,10 +305,12 @@ def run_ours(args):
                             device=dev, gate=w.gate)
     y = torch.empty_like(inp["x"])
     ws = ssm.ScanWorkspace()
+    conv = synth.conv_params(w.dim, w.batch, w.dtype, seed=rank_seed(w.seed + 5, rank), device=dev)
+    head_conv = conv if args.conv else {}
 
     def scan_step(general=args.general_A):
         ssm.scan_fwd(inp["x"], inp["dt"], inp["A"], inp["B"], inp["C"], inp["D"], inp["z"], inp["dt_bias"],
-                     out=y, workspace=ws, general_A=general)
+                     out=y, workspace=ws, general_A=general, **head_conv)
 
     for _ in range(args.warmup):
         scan_step()
@@ -331,14 +335,14 @@ def run_ours(args):
     per_launch_ms = ms / args.steps
     nbytes = scan_bytes(w)
     achieved = nbytes / (per_launch_ms / 1e3) / 1e9
-    path = "general" if args.general_A else "auto"
+    path = ("general" if args.general_A else "auto") + ("+conv" if args.conv else "")
 
     line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_max / args.steps, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
             "config": {"workload": w.name, "batch": w.batch, "seqlen": w.seqlen, "dim": w.dim,
                        "dstate": w.dstate, "io": w.dtype_name, "state": "f32", "gate": w.gate,
-                       "A": "S4D-real A[d,n] = -(n+1)", "exp_path": path,
+                       "A": "S4D-real A[d,n] = -(n+1)", "exp_path": path, "conv1d": bool(args.conv),
                        "l2": f"no flush: {nbytes / 1e9:.2f} GB moved per step > 126 MB L2",
                        "parallelism": f"replicas x{world}" if world > 1 else "single GPU"},
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
@@ -350,7 +354,7 @@ def run_ours(args):
 
     if not args.no_extras:
         # General-exponential path on the same inputs (no use of A's structure).
-        if not args.general_A:
+        if not args.general_A and not args.conv:
             gsteps = max(3, args.steps // 5)
             scan_step(True)
             gms = time_region(lambda: scan_step(True), gsteps, stream) / gsteps
@@ -359,6 +363,26 @@ def run_ours(args):
                                  "roofline_frac": gach / hbm_peak, "achieved_GBs": gach,
                                  "traffic": recorded_traffic(w.name, "general")}
             line["gpu_launches"] += gsteps
+        # The block's short causal convolution and SiLU fused in front of the scan (same
+        # tokens): what the fusion costs over the plain scan, against what a separate
+        # convolution pass would move through HBM (read x, write its output) at the peak.
+        if not args.conv:
+            def conv_step():
+                ssm.scan_fwd(inp["x"], inp["dt"], inp["A"], inp["B"], inp["C"], inp["D"], inp["z"], inp["dt_bias"],
+                             out=y, workspace=ws, **conv)
+
+            csteps = max(3, args.steps // 5)
+            conv_step()
+            if ssm.workspace_status(ws) != 0:
+                raise RuntimeError("device-side status of the fused-convolution scan is not SSM_OK")
+            cms = time_region(conv_step, csteps, stream) / csteps
+            es = 2 if w.dtype == torch.bfloat16 else 4
+            sep = 2 * w.batch * w.seqlen * w.dim * es
+            line["conv1d_fused"] = {"value": w.updates / (cms / 1e3), "unit": UNIT, "ms_per_step": cms,
+                                    "extra_ms_over_scan": cms - per_launch_ms,
+                                    "separate_pass_ms_at_hbm_peak": sep / (hbm_peak * 1e9) * 1e3,
+                                    "kernel": "scan_ws_kernel (short-convolution instantiation)"}
+            line["gpu_launches"] += csteps
         # End to end through the public API: pinned host inputs in, result back each step.
         names = ["x", "dt", "z", "B", "C"] if w.gate else ["x", "dt", "B", "C"]
         host = {k: torch.empty(inp[k].shape, dtype=inp[k].dtype, pin_memory=True) for k in names}
@@ -377,7 +401,7 @@ def run_ours(args):
             # with each other and with the scans.
             ssm.scan_fwd_host(host["x"], host["dt"], inp["A"], host["B"], host["C"], inp["D"], host.get("z"),
                               inp["dt_bias"], out=y_host, chunk_len=chunk, workspace=ws, staging=staging,
-                              general_A=args.general_A)
+                              general_A=args.general_A, **head_conv)
 
         esteps = max(2, min(5, args.steps))
         e2e_step()

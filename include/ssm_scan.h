@@ -90,6 +90,11 @@ typedef struct {
     float *h_last;           /* [B, D, N] final state out (float32), or NULL         */
     void *workspace;         /* device scratch of ssm_scan_workspace_size() bytes    */
     size_t workspace_bytes;
+    /* The block's short causal convolution in front of the scan (optional, see ssm_scan_fwd) */
+    const float *conv_w;     /* [D, 4] depthwise taps, oldest token first, float32 on 16 bytes; NULL: none */
+    const float *conv_b;     /* [D] convolution bias, or NULL for 0 (needs conv_w)    */
+    const void *conv_x0;     /* [B, 3, D] the three tokens before t = 0, oldest first, dtype of x;
+                                NULL for zeros (needs conv_w)                         */
 } ssm_scan_args;
 
 /*
@@ -119,6 +124,17 @@ size_t ssm_scan_workspace_size(const ssm_scan_args *args);
  * for n = 4w .. 4w+3 follow from two exponentials, exp(Delta A[d,4w]) and the
  * ratio r = exp(Delta (A[d,1] - A[d,0])), by multiplication. SSM_A_GENERAL turns
  * this off (one exponential per state and step).
+ *
+ * Short convolution (conv_w not NULL): the Mamba block's main branch runs a causal
+ * 1-D convolution of kernel size 4 and SiLU before the selective SSM (Mamba summary,
+ * block-architecture paragraph). The scan then reads, per channel d,
+ *   u_t = silu(conv_b[d] + sum_{k=0..3} conv_w[d,k] x_{t-3+k})
+ * (x_{t} for t < 0 from conv_x0, or 0) and uses u_t wherever x_t appears above (Bbar_t
+ * u_t and D u_t). The convolution runs inside the scan kernel on the tiles it loads
+ * anyway, in float32: x crosses HBM once and u is never stored. The y, h_last and
+ * chunking rules are unchanged; to continue a sequence in a later call, pass its last
+ * three tokens as conv_x0 and its h_last as h0. Errors: SSM_ERR_INVALID for conv_b or
+ * conv_x0 without conv_w; SSM_ERR_UNSUPPORTED for conv_w not on 16 bytes.
  */
 ssm_status ssm_scan_fwd(const ssm_scan_args *args, void *stream);
 
@@ -180,7 +196,9 @@ ssm_status ssm_scan_fwd_noalloc(const ssm_scan_args *args, void *stream);
  * and the kernels. The state passes from chunk to chunk through h0/h_last in the
  * staging memory, so the result equals ssm_scan_fwd over the whole sequence bit for
  * bit. Batch rows are strided in host memory ([B, L, ...]); each chunk moves them with
- * one two-dimensional copy per tensor.
+ * one two-dimensional copy per tensor. With the short convolution (conv_w, conv_b and
+ * conv_x0 device pointers), every chunk after the first also copies in the three host
+ * tokens before it as its prefix; the staging size then includes room for them.
  *
  * Ordering: the call enqueues and returns; all of its work is ordered after the work
  * already on `stream` and before the work enqueued on `stream` later. The host buffers

@@ -50,7 +50,20 @@ def _flags(delta_softplus, general_A, exact_zoh=False):
             | (SSM_EXACT_ZOH if exact_zoh else 0))
 
 
-def _scan_args(x, dt, A, B, C, D, z, dt_bias, h0, y, h_last, flags):
+def _need_conv(conv_w, conv_b, conv_x0, Bsz, Dm, tok, dev):
+    """Check the optional short-convolution arguments (taps [D, 4], bias [D], prefix [B, 3, D])."""
+    if conv_w is None:
+        if conv_b is not None or conv_x0 is not None:
+            raise ValueError("conv_b and conv_x0 need conv_w")
+        return
+    _need(conv_w, "conv_w", (Dm, 4), torch.float32, dev)
+    if conv_b is not None:
+        _need(conv_b, "conv_b", (Dm,), torch.float32, dev)
+    if conv_x0 is not None:
+        _need(conv_x0, "conv_x0", (Bsz, 3, Dm), tok, dev)
+
+
+def _scan_args(x, dt, A, B, C, D, z, dt_bias, h0, y, h_last, flags, conv_w=None, conv_b=None, conv_x0=None):
     a = _native.ScanArgs()
     a.batch, a.seqlen, a.dim = x.shape
     a.dstate = A.shape[1]
@@ -59,6 +72,7 @@ def _scan_args(x, dt, A, B, C, D, z, dt_bias, h0, y, h_last, flags):
     a.x, a.dt, a.z, a.Bm, a.Cm = (_ptr(t) for t in (x, dt, z, B, C))
     a.A, a.Dskip, a.dt_bias, a.h0 = (_ptr(t) for t in (A, D, dt_bias, h0))
     a.y, a.h_last = _ptr(y), _ptr(h_last)
+    a.conv_w, a.conv_b, a.conv_x0 = (_ptr(t) for t in (conv_w, conv_b, conv_x0))
     return a
 
 
@@ -88,13 +102,15 @@ _default_ws = {}
 
 def scan_fwd(x, dt, A, B, C, D=None, z=None, dt_bias=None, h0=None, *, delta_softplus=True,
              general_A=False, exact_zoh=False, return_last_state=False, out=None, h_last=None, workspace=None,
-             stream=None):
+             stream=None, conv_w=None, conv_b=None, conv_x0=None):
     """Selective scan forward over whole sequences (see include/ssm_scan.h, ssm_scan_fwd).
 
     x, dt, z: [B, L, D] float32 or bfloat16; B, C: [B, L, N] same dtype; A: [D, N]
     float32; D, dt_bias: [D] float32; h0: [B, D, N] float32. Returns y (same dtype
     as x) and, with return_last_state, the final state [B, D, N] float32. exact_zoh:
-    Bbar = (exp(Delta A) - 1) / A B instead of Delta B.
+    Bbar = (exp(Delta A) - 1) / A B instead of Delta B. conv_w [D, 4] float32 (with
+    conv_b [D] and conv_x0 [B, 3, D], the tokens before t = 0, both optional) runs the
+    block's causal convolution and SiLU on x inside the scan kernel.
     """
     dev = x.device
     if x.dtype not in _TOKEN_DTYPES:
@@ -123,7 +139,9 @@ def scan_fwd(x, dt, A, B, C, D=None, z=None, dt_bias=None, h0=None, *, delta_sof
         h_last = torch.empty((Bsz, Dm, N), dtype=torch.float32, device=dev)
     if h_last is not None:
         _need(h_last, "h_last", (Bsz, Dm, N), torch.float32, dev)
-    args = _scan_args(x, dt, A, B, C, D, z, dt_bias, h0, y, h_last, _flags(delta_softplus, general_A, exact_zoh))
+    _need_conv(conv_w, conv_b, conv_x0, Bsz, Dm, tok, dev)
+    args = _scan_args(x, dt, A, B, C, D, z, dt_bias, h0, y, h_last, _flags(delta_softplus, general_A, exact_zoh),
+                      conv_w, conv_b, conv_x0)
     nbytes = int(_native.lib().ssm_scan_workspace_size(ctypes.byref(args)))
     if workspace is None:
         key = (dev, torch.cuda.current_stream(dev).cuda_stream if stream is None else stream.cuda_stream)
@@ -153,13 +171,15 @@ _default_staging = {}
 
 def scan_fwd_host(x, dt, A, B, C, D=None, z=None, dt_bias=None, h0=None, *, chunk_len=16384,
                   delta_softplus=True, general_A=False, exact_zoh=False, return_last_state=False, out=None,
-                  h_last=None, workspace=None, staging=None, stream=None):
+                  h_last=None, workspace=None, staging=None, stream=None, conv_w=None, conv_b=None,
+                  conv_x0=None):
     """Selective scan over host-resident tokens (see include/ssm_scan.h, ssm_scan_fwd_host).
 
     x, dt, z: [B, L, D] and B, C: [B, L, N] host tensors (page-locked memory lets the
     copies overlap the scan); the result y is a host tensor too (`out`, or a new
-    page-locked one). A, D, dt_bias, h0 and h_last live on the GPU (A's device). The
-    call is asynchronous on `stream`: synchronise it before reading y.
+    page-locked one). A, D, dt_bias, h0, h_last and the optional short convolution's
+    conv_w, conv_b, conv_x0 live on the GPU (A's device). The call is asynchronous on
+    `stream`: synchronise it before reading y.
     """
     dev = A.device
     if x.dtype not in _TOKEN_DTYPES:
@@ -188,7 +208,9 @@ def scan_fwd_host(x, dt, A, B, C, D=None, z=None, dt_bias=None, h0=None, *, chun
         h_last = torch.empty((Bsz, Dm, N), dtype=torch.float32, device=dev)
     if h_last is not None:
         _need(h_last, "h_last", (Bsz, Dm, N), torch.float32, dev)
-    args = _scan_args(x, dt, A, B, C, D, z, dt_bias, h0, y, h_last, _flags(delta_softplus, general_A, exact_zoh))
+    _need_conv(conv_w, conv_b, conv_x0, Bsz, Dm, tok, dev)
+    args = _scan_args(x, dt, A, B, C, D, z, dt_bias, h0, y, h_last, _flags(delta_softplus, general_A, exact_zoh),
+                      conv_w, conv_b, conv_x0)
     lib = _native.lib()
     key = (dev, torch.cuda.current_stream(dev).cuda_stream if stream is None else stream.cuda_stream)
     nbytes = int(lib.ssm_scan_workspace_size(ctypes.byref(args)))

@@ -26,6 +26,7 @@ class ScanArgs(ctypes.Structure):
         ("Dskip", ctypes.c_void_p), ("dt_bias", ctypes.c_void_p), ("h0", ctypes.c_void_p),
         ("y", ctypes.c_void_p), ("h_last", ctypes.c_void_p), ("workspace", ctypes.c_void_p),
         ("workspace_bytes", ctypes.c_size_t),
+        ("conv_w", ctypes.c_void_p), ("conv_b", ctypes.c_void_p), ("conv_x0", ctypes.c_void_p),
     ]
 
 

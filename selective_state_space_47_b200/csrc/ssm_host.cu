@@ -14,10 +14,11 @@ namespace {
 inline size_t up256(size_t v) { return (v + 255) / 256 * 256; }
 
 // Staging layout for chunks of Lc steps: two buffers, each x | dt | z | y (B x Lc x D
-// tokens) and B | C (B x Lc x N tokens), then two carried states [B, D, N] float32.
+// tokens), B | C (B x Lc x N tokens) and, with the short convolution, the three tokens
+// before the chunk (B x 3 x D); then two carried states [B, D, N] float32.
 struct Staging {
-    size_t tok, bc, buf, carry, total;
-    size_t off_x, off_dt, off_z, off_y, off_b, off_c, off_carry;
+    size_t tok, bc, x0, buf, carry, total;
+    size_t off_x, off_dt, off_z, off_y, off_b, off_c, off_x0, off_carry;
 };
 
 Staging staging_layout(const ssm_scan_args *a, int64_t Lc) {
@@ -31,7 +32,9 @@ Staging staging_layout(const ssm_scan_args *a, int64_t Lc) {
     s.off_y = 3 * s.tok;
     s.off_b = 4 * s.tok;
     s.off_c = 4 * s.tok + s.bc;
-    s.buf = 4 * s.tok + 2 * s.bc;
+    s.x0 = a->conv_w ? up256(size_t(a->batch) * 3 * size_t(a->dim) * es) : 0;
+    s.off_x0 = 4 * s.tok + 2 * s.bc;
+    s.buf = 4 * s.tok + 2 * s.bc + s.x0;
     s.carry = up256(size_t(a->batch) * size_t(a->dim) * size_t(a->dstate) * 4);
     s.off_carry = 2 * s.buf;
     s.total = 2 * s.buf + 2 * s.carry;
@@ -77,6 +80,33 @@ cudaError_t copy_rows(void *dst, const void *src, const ssm_scan_args *a, int64_
                                  size_t(a->batch), cudaMemcpyHostToDevice, st);
     return cudaMemcpy2DAsync(static_cast<unsigned char *>(dst) + host_off, host_pitch, src, width, width,
                              size_t(a->batch), cudaMemcpyDeviceToHost, st);
+}
+
+// The three tokens before step t0 ([B, 3, D], oldest first), the short convolution's
+// prefix for a chunk that starts at t0 > 0: rows t0-3 .. t0-1 of the host x, and before
+// t = 0 the caller's device prefix (or zeros).
+cudaError_t copy_prefix(void *dst, const ssm_scan_args *a, int64_t t0, cudaStream_t st) {
+    const size_t es = a->dtype == SSM_BF16 ? 2 : 4;
+    const size_t row = size_t(a->dim) * es, pitch = 3 * row, host_pitch = size_t(a->seqlen) * row;
+    const unsigned char *x = static_cast<const unsigned char *>(a->x);
+    if (t0 >= 3)
+        return cudaMemcpy2DAsync(dst, pitch, x + size_t(t0 - 3) * row, host_pitch, pitch, size_t(a->batch),
+                                 cudaMemcpyHostToDevice, st);
+    for (int r = 0; r < 3; ++r) {  // chunks shorter than three steps
+        unsigned char *d = static_cast<unsigned char *>(dst) + r * row;
+        const int64_t tau = t0 - 3 + r;
+        cudaError_t e;
+        if (tau >= 0)
+            e = cudaMemcpy2DAsync(d, pitch, x + size_t(tau) * row, host_pitch, row, size_t(a->batch),
+                                  cudaMemcpyHostToDevice, st);
+        else if (a->conv_x0)
+            e = cudaMemcpy2DAsync(d, pitch, static_cast<const unsigned char *>(a->conv_x0) + size_t(tau + 3) * row,
+                                  pitch, row, size_t(a->batch), cudaMemcpyDeviceToDevice, st);
+        else
+            e = cudaMemset2DAsync(d, pitch, 0, row, size_t(a->batch), st);
+        if (e != cudaSuccess) return e;
+    }
+    return cudaSuccess;
 }
 
 }  // namespace
@@ -129,6 +159,7 @@ ssm_status ssm_scan_fwd_host(const ssm_scan_args *a, int64_t chunk_len, void *st
         if (a->z) SSM_CK(copy_rows(buf + s.off_z, a->z, a, a->dim, t0, n, true, e.in));
         SSM_CK(copy_rows(buf + s.off_b, a->Bm, a, a->dstate, t0, n, true, e.in));
         SSM_CK(copy_rows(buf + s.off_c, a->Cm, a, a->dstate, t0, n, true, e.in));
+        if (a->conv_w && c > 0) SSM_CK(copy_prefix(buf + s.off_x0, a, t0, e.in));
         SSM_CK(cudaEventRecord(e.ev_in[k], e.in));
         // Scan chunk c once its inputs are in and the y of chunk c-2 has left this buffer.
         SSM_CK(cudaStreamWaitEvent(stream, e.ev_in[k], 0));
@@ -143,6 +174,7 @@ ssm_status ssm_scan_fwd_host(const ssm_scan_args *a, int64_t chunk_len, void *st
         b.y = buf + s.off_y;
         b.h0 = c == 0 ? a->h0 : carry[(c - 1) & 1];
         b.h_last = c == nc - 1 ? a->h_last : carry[c & 1];
+        if (a->conv_w) b.conv_x0 = c == 0 ? a->conv_x0 : buf + s.off_x0;
         const ssm_status st = ssm_scan_fwd(&b, stream);
         if (st != SSM_OK) return st;
         SSM_CK(cudaEventRecord(e.ev_scan[k], stream));

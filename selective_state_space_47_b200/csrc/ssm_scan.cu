@@ -166,15 +166,15 @@ PFN_cuTensorMapEncodeTiled_v12000 get_encode_fn() {
     return fn;
 }
 
-// A [B, L, inner] tensor as a 3-D TMA map with a [box_inner x TT x 1] box.
+// A [B, L, inner] tensor as a 3-D TMA map with a [box_inner x box_rows x 1] box.
 bool make_map_3d(CUtensorMap *m, const void *ptr, ssm_dtype dt, int64_t Bsz, int64_t L, int64_t inner,
-                 int box_inner) {
+                 int box_inner, int box_rows = ssm::scan::TT) {
     auto enc = get_encode_fn();
     if (!enc) return false;
     const size_t es = dt == SSM_BF16 ? 2 : 4;
     cuuint64_t dims[3] = {cuuint64_t(inner), cuuint64_t(L), cuuint64_t(Bsz)};
     cuuint64_t strides[2] = {cuuint64_t(inner * es), cuuint64_t(L * inner * es)};
-    cuuint32_t box[3] = {cuuint32_t(box_inner), cuuint32_t(ssm::scan::TT), 1};
+    cuuint32_t box[3] = {cuuint32_t(box_inner), cuuint32_t(box_rows), 1};
     cuuint32_t estr[3] = {1, 1, 1};
     CUresult r = enc(m, dt == SSM_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3,
                      const_cast<void *>(ptr), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
@@ -200,24 +200,30 @@ struct ScanPlan {
     size_t smem = 0;
 };
 
-template <bool ZOH>
+template <bool ZOH, bool CONV>
 void *pick_kernel_t(ssm_dtype dt, bool deep) {
     using namespace ssm::scan;
     if (dt == SSM_BF16)
-        return deep ? reinterpret_cast<void *>(&scan_ws_kernel<__nv_bfloat16, Deep, ZOH>)
-                    : reinterpret_cast<void *>(&scan_ws_kernel<__nv_bfloat16, Shallow, ZOH>);
-    return deep ? reinterpret_cast<void *>(&scan_ws_kernel<float, Deep, ZOH>)
-                : reinterpret_cast<void *>(&scan_ws_kernel<float, Shallow, ZOH>);
+        return deep ? reinterpret_cast<void *>(&scan_ws_kernel<__nv_bfloat16, Deep, ZOH, CONV>)
+                    : reinterpret_cast<void *>(&scan_ws_kernel<__nv_bfloat16, Shallow, ZOH, CONV>);
+    return deep ? reinterpret_cast<void *>(&scan_ws_kernel<float, Deep, ZOH, CONV>)
+                : reinterpret_cast<void *>(&scan_ws_kernel<float, Shallow, ZOH, CONV>);
 }
-// The exact zero-order hold is a separate instantiation, so the default kernel carries
-// none of its code.
-void *pick_kernel(ssm_dtype dt, bool deep, bool zoh = false) {
-    return zoh ? pick_kernel_t<true>(dt, deep) : pick_kernel_t<false>(dt, deep);
+// The exact zero-order hold and the short convolution are separate instantiations, so
+// the default kernel carries none of their code.
+void *pick_kernel(ssm_dtype dt, bool deep, bool zoh, bool conv) {
+    if (conv) return zoh ? pick_kernel_t<true, true>(dt, deep) : pick_kernel_t<false, true>(dt, deep);
+    return zoh ? pick_kernel_t<true, false>(dt, deep) : pick_kernel_t<false, false>(dt, deep);
 }
-size_t pick_smem(ssm_dtype dt, bool deep) {
+template <bool CONV>
+size_t pick_smem_t(ssm_dtype dt, bool deep) {
     using namespace ssm::scan;
-    if (dt == SSM_BF16) return deep ? Layout<__nv_bfloat16, Deep>::total : Layout<__nv_bfloat16, Shallow>::total;
-    return deep ? Layout<float, Deep>::total : Layout<float, Shallow>::total;
+    if (dt == SSM_BF16)
+        return deep ? Layout<__nv_bfloat16, Deep, CONV>::total : Layout<__nv_bfloat16, Shallow, CONV>::total;
+    return deep ? Layout<float, Deep, CONV>::total : Layout<float, Shallow, CONV>::total;
+}
+size_t pick_smem(ssm_dtype dt, bool deep, bool conv) {
+    return conv ? pick_smem_t<true>(dt, deep) : pick_smem_t<false>(dt, deep);
 }
 
 // Largest group count over both block shapes: bounds the flag and state arrays.
@@ -229,24 +235,25 @@ size_t ws_total(int64_t Bsz, int64_t D) {
     return ws_carry_off(Bsz, D) + size_t(Bsz) * size_t(round_up(size_t(D), 32)) * kMaxN * 4;
 }
 
-// Blocks per SM of the shallow and deep kernel configurations for a token type, per
-// device (queried once: the attribute calls cost microseconds).
-bool scan_occupancy(ssm_dtype dt, int occ[2]) {
+// Blocks per SM of the shallow and deep kernel configurations for a token type, with or
+// without the short convolution, per device (queried once: the attribute calls cost
+// microseconds).
+bool scan_occupancy(ssm_dtype dt, bool conv, int occ[2]) {
     constexpr int kDevs = 64;
     static std::mutex mu;
-    static int cache[kDevs][2][2];
-    static bool have[kDevs][2];
+    static int cache[kDevs][2][2][2];
+    static bool have[kDevs][2][2];
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kDevs) return false;
-    const int ti = dt == SSM_BF16 ? 1 : 0;
+    const int ti = dt == SSM_BF16 ? 1 : 0, ci = conv ? 1 : 0;
     std::lock_guard<std::mutex> lock(mu);
-    if (!have[dev][ti]) {
+    if (!have[dev][ti][ci]) {
         int optin = 0;
         if (cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) != cudaSuccess) return false;
         for (int deep = 0; deep < 2; ++deep) {
-            void *kern = pick_kernel(dt, deep != 0);
-            void *kern_zoh = pick_kernel(dt, deep != 0, true);  // same shape and register budget
-            const size_t smem = pick_smem(dt, deep != 0);
+            void *kern = pick_kernel(dt, deep != 0, false, conv);
+            void *kern_zoh = pick_kernel(dt, deep != 0, true, conv);  // same shape and register budget
+            const size_t smem = pick_smem(dt, deep != 0, conv);
             int o = 0;
             if (smem <= size_t(optin)) {
                 if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem)) != cudaSuccess ||
@@ -255,12 +262,12 @@ bool scan_occupancy(ssm_dtype dt, int occ[2]) {
                     cudaOccupancyMaxActiveBlocksPerMultiprocessor(&o, kern, ssm::scan::NTHREADS, smem) != cudaSuccess)
                     return false;
             }
-            cache[dev][ti][deep] = o;
+            cache[dev][ti][ci][deep] = o;
         }
-        have[dev][ti] = true;
+        have[dev][ti][ci] = true;
     }
-    occ[0] = cache[dev][ti][0];
-    occ[1] = cache[dev][ti][1];
+    occ[0] = cache[dev][ti][ci][0];
+    occ[1] = cache[dev][ti][ci][1];
     return occ[0] > 0 || occ[1] > 0;
 }
 
@@ -275,11 +282,12 @@ bool plan_scan(const ssm_scan_args *a, ScanPlan *pl) {
     // most SMs two (at least 1.25 per SM); otherwise the deep configuration (one block per
     // SM) if its shared memory fits.
     int occ[2] = {0, 0};
-    if (!scan_occupancy(a->dtype, occ)) return false;
+    const bool conv = a->conv_w != nullptr;
+    if (!scan_occupancy(a->dtype, conv, occ)) return false;
     // (measured: the deep rings gain ~8% on 160 groups over 148 SMs and nothing on 192)
     const bool shallow_fills = occ[0] >= 2 && 4 * pl->G >= 5 * int64_t(sms);
     pl->deep = occ[1] > 0 && (occ[0] <= 0 || !shallow_fills);
-    pl->smem = pick_smem(a->dtype, pl->deep);
+    pl->smem = pick_smem(a->dtype, pl->deep, conv);
     pl->grid = int(std::min<int64_t>(pl->G, int64_t(occ[pl->deep ? 1 : 0]) * sms));
     // Segments: about four items per block, between kMinSegTiles and kMaxSegTiles tiles
     // long. Each item start waits for its predecessor's state (a few microseconds), which
@@ -321,9 +329,13 @@ ssm_status validate_scan(const ssm_scan_args *a) {
     const void *pes[] = {a->Bm, a->Cm};
     for (const void *p : pes)
         if (p && !aligned(p, es)) return SSM_ERR_UNSUPPORTED;
-    const void *p4[] = {a->A, a->Dskip, a->dt_bias, a->h0, a->h_last};
+    const void *p4[] = {a->A, a->Dskip, a->dt_bias, a->h0, a->h_last, a->conv_b};
     for (const void *p : p4)
         if (p && !aligned(p, 4)) return SSM_ERR_UNSUPPORTED;
+    // The short convolution: taps read as one float4 per channel; bias and prefix only with taps.
+    if (!a->conv_w && (a->conv_b || a->conv_x0)) return SSM_ERR_INVALID;
+    if (a->conv_w && !aligned(a->conv_w, 16)) return SSM_ERR_UNSUPPORTED;
+    if (a->conv_x0 && !aligned(a->conv_x0, es)) return SSM_ERR_UNSUPPORTED;
     if (work && (!a->workspace || a->workspace_bytes < ws_total(a->batch, a->dim))) return SSM_ERR_INVALID;
     return SSM_OK;
 }
@@ -400,7 +412,10 @@ ssm_status ssm_scan_fwd(const ssm_scan_args *a, void *stream_) {
     const int es = a->dtype == SSM_BF16 ? 2 : 4;
     const bool bc_tma = (a->dstate * es) % 16 == 0 && aligned(a->Bm, 16) && aligned(a->Cm, 16);
     CUtensorMap tx, tdt, tz, ty, tb, tc;
-    if (!make_map_3d(&tx, a->x, a->dtype, a->batch, a->seqlen, a->dim, pl.ch) ||
+    const bool conv = a->conv_w != nullptr;
+    // With the short convolution the x box carries the three rows before its tile.
+    const int x_rows = ssm::scan::TT + (conv ? ssm::scan::KCONV - 1 : 0);
+    if (!make_map_3d(&tx, a->x, a->dtype, a->batch, a->seqlen, a->dim, pl.ch, x_rows) ||
         !make_map_3d(&tdt, a->dt, a->dtype, a->batch, a->seqlen, a->dim, pl.ch) ||
         !make_map_3d(&tz, a->z ? a->z : a->x, a->dtype, a->batch, a->seqlen, a->dim, pl.ch) ||
         !make_map_3d(&ty, a->y, a->dtype, a->batch, a->seqlen, a->dim, pl.ch))
@@ -435,13 +450,16 @@ ssm_status ssm_scan_fwd(const ssm_scan_args *a, void *stream_) {
     p.status = reinterpret_cast<uint32_t *>(ws + 4);
     p.flags = reinterpret_cast<uint32_t *>(ws + ws_flags_off());
     p.carry = reinterpret_cast<float *>(ws + ws_carry_off(a->batch, a->dim));
+    p.conv_w = a->conv_w;
+    p.conv_b = a->conv_b;
+    p.conv_x0 = a->conv_x0;
     p.has_gate = a->z != nullptr;
     p.softplus = (a->flags & SSM_DELTA_SOFTPLUS) != 0;
     p.allow_structured = (a->flags & SSM_A_GENERAL) == 0;
     p.drop_handoff = (a->flags & SSM_TEST_DROP_HANDOFF) != 0;
     p.bc_tma = bc_tma;
 
-    void *kern = pick_kernel(a->dtype, pl.deep, (a->flags & SSM_EXACT_ZOH) != 0);
+    void *kern = pick_kernel(a->dtype, pl.deep, (a->flags & SSM_EXACT_ZOH) != 0, conv);
     void *args[] = {&tx, &tdt, &tz, &tb, &tc, &ty, &p};
     cudaError_t e = cudaLaunchKernel(kern, dim3(pl.grid), dim3(ssm::scan::NTHREADS), args, pl.smem, stream);
     return e == cudaSuccess ? SSM_OK : SSM_ERR_CUDA;

@@ -39,6 +39,13 @@
 // blocks, an item (group g, segment k) starts from the state its predecessor (g,
 // k-1) published in the workspace.
 //
+// Short convolution (the CONV instantiations): the block's causal depthwise conv1d of
+// width 4 and SiLU in front of the SSM, u_t = silu(cb + sum_k w_k x_{t-3+k}) (Mamba
+// summary, block-architecture paragraph). The x box of every stage carries the three
+// rows before the tile (TMA fills rows before t = 0 with zeros, or the prologue and
+// epilogue take them from the caller's prefix), and both P and E evaluate u from it:
+// P for Delta u, E for D u. Nothing else changes, and x still crosses HBM once.
+//
 // Exponentials: Abar_n = 2^(Delta log2 e * A[d,n]) on the SFU (ex2.approx). Where
 // every row of A in the block is an arithmetic progression in n (A[d,n] = A[d,0] +
 // n (A[d,1] - A[d,0]); the S4D-real rows A[d,n] = -(n+1) are one), a lane's four
@@ -62,6 +69,7 @@ constexpr int NTHREADS = (CW + NP + NE + 1) * 32;
 constexpr int TT = 32;                            // time steps per tile
 constexpr int TP = TT / NP;                       // steps per prologue warp and tile
 constexpr int TE = TT / NE;                       // steps per epilogue warp and tile
+constexpr int KCONV = 4;                          // width of the short causal convolution
 // Ring depths and blocks per SM. Shallow: 113 KB of shared memory (bf16), two blocks
 // per SM. Deep: rings twice as deep, one block per SM; it decouples the roles further
 // and is the better choice when there are too few channel groups to fill two blocks per
@@ -112,20 +120,26 @@ struct Params {
     uint32_t *status;
     uint32_t *flags;
     float *carry;
+    const float *conv_w;  // [D, 4] taps of the short convolution (CONV instantiations)
+    const float *conv_b;  // [D] or null
+    const void *conv_x0;  // [B, 3, D] tokens before t = 0, or null for zeros
     int has_gate, softplus, allow_structured, drop_handoff, bc_tma;
 };
 
-template <typename T, typename C>
+template <typename T, typename C, bool CONV = false>
 struct Layout {
     static constexpr int STAGES = C::STAGES, R_REC = C::R_REC, R_PART = C::R_PART;
     static constexpr int BOX = TT * CH;           // elements of one token box [TT][CH]
     static constexpr int BCBOX = TT * kMaxN;      // elements of one B or C box [TT][16]
+    static constexpr int HALO = CONV ? KCONV - 1 : 0;  // rows of x before the tile in its box
     static constexpr size_t tok_bytes = size_t(BOX) * sizeof(T);
     static constexpr size_t bc_bytes = size_t(BCBOX) * sizeof(T);
-    // stage: x | dt | z | B | C
-    static constexpr size_t st_x = 0, st_dt = tok_bytes, st_z = 2 * tok_bytes, st_b = 3 * tok_bytes,
-                            st_c = 3 * tok_bytes + bc_bytes;
-    static constexpr size_t stage_bytes = 3 * tok_bytes + 2 * bc_bytes;
+    static constexpr size_t xbox_bytes = size_t(TT + HALO) * CH * sizeof(T);  // what one x box delivers
+    static constexpr size_t x_bytes = (xbox_bytes + 127) / 128 * 128;
+    // stage: x (with its halo rows) | dt | z | B | C
+    static constexpr size_t st_x = 0, st_dt = x_bytes, st_z = x_bytes + tok_bytes, st_b = x_bytes + 2 * tok_bytes,
+                            st_c = x_bytes + 2 * tok_bytes + bc_bytes;
+    static constexpr size_t stage_bytes = x_bytes + 2 * tok_bytes + 2 * bc_bytes;
     static constexpr size_t stage_off = 0;
     static constexpr size_t rec_off = stage_off + STAGES * stage_bytes;
     static constexpr size_t rec_bytes = size_t(BOX) * 8;            // float2 (u, Delta log2 e) per (t, c)
@@ -291,23 +305,71 @@ __device__ __forceinline__ void consume_tile(const float2 *__restrict__ rec, con
     }
 }
 
+// ------------------------------------------------------ short convolution
+// u for rows t0 .. t0+2*NPR-1 of a tile, as pairs: u_t = silu(cb + w.x x_{t-3} + w.y
+// x_{t-2} + w.z x_{t-1} + w.w x_t). sx points at row 0 of the tile; the three rows before
+// it are the box's halo. With use_x0 (the sequence's first rows, t0 = 0) the caller's
+// prefix x0 replaces the halo rows, which TMA filled with zeros.
+template <typename T, int NPR>
+__device__ __forceinline__ void conv_silu_rows(const T *__restrict__ sx, const int t0, const float4 w, const float cb,
+                                               const bool use_x0, const float3 x0, float2 (&u)[NPR]) {
+    constexpr int NR = 2 * NPR + KCONV - 1;
+    float r[NR];
+#pragma unroll
+    for (int j = 0; j < NR; ++j) r[j] = Tok<T>::to_f(sx[(t0 - (KCONV - 1) + j) * CH]);
+    if (use_x0) {
+        r[0] = x0.x;
+        r[1] = x0.y;
+        r[2] = x0.z;
+    }
+#pragma unroll
+    for (int q = 0; q < NPR; ++q) {
+        float2 v = __ffma2_rn(f2(w.x, w.x), f2(r[2 * q], r[2 * q + 1]), f2(cb, cb));
+        v = __ffma2_rn(f2(w.y, w.y), f2(r[2 * q + 1], r[2 * q + 2]), v);
+        v = __ffma2_rn(f2(w.z, w.z), f2(r[2 * q + 2], r[2 * q + 3]), v);
+        v = __ffma2_rn(f2(w.w, w.w), f2(r[2 * q + 3], r[2 * q + 4]), v);
+        u[q] = f2(silu_f(v.x), silu_f(v.y));  // per value, as softplus and the gate
+    }
+}
+
+// Taps and bias of the short convolution for channel d (zeros past the last channel).
+__device__ __forceinline__ void load_conv(const Params &p, const int64_t d, float4 &w, float &b) {
+    const bool ok = d < p.D;
+    w = ok ? __ldg(reinterpret_cast<const float4 *>(p.conv_w) + d) : make_float4(0.f, 0.f, 0.f, 0.f);
+    b = (ok && p.conv_b) ? __ldg(p.conv_b + d) : 0.f;
+}
+
+// The caller's three tokens before t = 0 for lane c of group g, oldest first; false
+// (the halo keeps TMA's zeros) without a prefix or past the last channel.
+template <typename T>
+__device__ __forceinline__ bool conv_prefix(const Params &p, const long long g, const int c, float3 &x0) {
+    const int64_t b = g / p.Dg, d = (g % p.Dg) * CH + c;
+    if (!p.conv_x0 || d >= p.D) return false;
+    const T *src = static_cast<const T *>(p.conv_x0) + b * (KCONV - 1) * p.D + d;
+    x0 = make_float3(Tok<T>::ldg(src), Tok<T>::ldg(src + p.D), Tok<T>::ldg(src + 2 * p.D));
+    return true;
+}
+
 // ---------------------------------------------------------------- prologue
 // Records of TP steps (rows t0 .. t0+TP-1 of a tile) for channel c: (u = Delta x,
 // Delta log2 e), with Delta = softplus(dt + bias) (or dt + bias); with `zoh` (exact
 // zero-order hold) u = x, the consumers apply the weight. Rows at or past tlen get
-// (0, 0): Abar = 1, no input.
-template <typename T>
+// (0, 0): Abar = 1, no input. CONV: x is the short convolution's output (cw, cb, and
+// use_x0 / x0 as for conv_silu_rows).
+template <typename T, bool CONV>
 __device__ __forceinline__ void prologue_rows(const T *__restrict__ sx, const T *__restrict__ sdt,
                                               float2 *__restrict__ rec, const int t0, const int tlen,
-                                              const float bias, const bool softplus, const bool zoh) {
+                                              const float bias, const bool softplus, const bool zoh,
+                                              const float4 cw, const float cb, const bool use_x0, const float3 x0) {
     constexpr int NPR = TP / 2;  // pairs of steps
     float2 v[NPR], xv[NPR];
 #pragma unroll
     for (int q = 0; q < NPR; ++q) {
         const int t = t0 + 2 * q;
         v[q] = f2(Tok<T>::to_f(sdt[t * CH]), Tok<T>::to_f(sdt[(t + 1) * CH]));
-        xv[q] = f2(Tok<T>::to_f(sx[t * CH]), Tok<T>::to_f(sx[(t + 1) * CH]));
+        if (!CONV) xv[q] = f2(Tok<T>::to_f(sx[t * CH]), Tok<T>::to_f(sx[(t + 1) * CH]));
     }
+    if (CONV) conv_silu_rows<T, NPR>(sx, t0, cw, cb, use_x0, x0, xv);
 #pragma unroll
     for (int q = 0; q < NPR; ++q) v[q] = __fadd2_rn(v[q], f2(bias, bias));
     // softplus per value (measured: 1.8x faster here than the same arithmetic staged
@@ -332,13 +394,17 @@ __device__ __forceinline__ void prologue_rows(const T *__restrict__ sx, const T 
 
 // ---------------------------------------------------------------- epilogue
 // y for TE steps (rows t0 .. t0+TE-1) of channel c: sum of the four consumer
-// partials, + D x, times silu(z), rounded to T.
-template <typename T>
+// partials, + D x, times silu(z), rounded to T. CONV: x is the short convolution's
+// output, recomputed here from the stage (as in the prologue).
+template <typename T, bool CONV>
 __device__ __forceinline__ void epilogue_rows(const float4 *__restrict__ part, const T *__restrict__ sx,
                                               const T *__restrict__ sz, T *__restrict__ yo, const int t0,
-                                              const float dd, const bool gate) {
+                                              const float dd, const bool gate, const float4 cw, const float cb,
+                                              const bool use_x0, const float3 x0) {
     constexpr int NB = TE / 4;  // blocks of four steps
     float2 y01[NB], y23[NB];
+    float2 xc[CONV ? TE / 2 : 1];
+    if constexpr (CONV) conv_silu_rows<T, TE / 2>(sx, t0, cw, cb, use_x0, x0, xc);
 #pragma unroll
     for (int b = 0; b < NB; ++b) {
         const int blk = t0 / 4 + b;
@@ -352,8 +418,9 @@ __device__ __forceinline__ void epilogue_rows(const float4 *__restrict__ part, c
         lo = __fadd2_rn(lo, lo2);
         hi = __fadd2_rn(hi, hi2);
         const int t = t0 + 4 * b;
-        const float2 x01 = f2(Tok<T>::to_f(sx[t * CH]), Tok<T>::to_f(sx[(t + 1) * CH]));
-        const float2 x23 = f2(Tok<T>::to_f(sx[(t + 2) * CH]), Tok<T>::to_f(sx[(t + 3) * CH]));
+        const float2 x01 = CONV ? xc[2 * b] : f2(Tok<T>::to_f(sx[t * CH]), Tok<T>::to_f(sx[(t + 1) * CH]));
+        const float2 x23 =
+            CONV ? xc[2 * b + 1] : f2(Tok<T>::to_f(sx[(t + 2) * CH]), Tok<T>::to_f(sx[(t + 3) * CH]));
         y01[b] = __ffma2_rn(f2(dd, dd), x01, lo);
         y23[b] = __ffma2_rn(f2(dd, dd), x23, hi);
     }
@@ -383,13 +450,13 @@ __device__ __forceinline__ void epilogue_rows(const float4 *__restrict__ part, c
 }
 
 // ------------------------------------------------------------------- kernel
-template <typename T, typename C, bool ZOH>
+template <typename T, typename C, bool ZOH, bool CONV>
 __global__ void __launch_bounds__(NTHREADS, C::MINB)
     scan_ws_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_dt,
                    const __grid_constant__ CUtensorMap tm_z, const __grid_constant__ CUtensorMap tm_b,
                    const __grid_constant__ CUtensorMap tm_c, const __grid_constant__ CUtensorMap tm_y,
                    const Params p) {
-    using S = Layout<T, C>;
+    using S = Layout<T, C, CONV>;
     constexpr int STAGES = C::STAGES, R_REC = C::R_REC, R_PART = C::R_PART;
     extern __shared__ __align__(1024) unsigned char smem[];
     TileMeta *smeta = reinterpret_cast<TileMeta *>(smem + S::smeta_off);  // per stage
@@ -421,7 +488,8 @@ __global__ void __launch_bounds__(NTHREADS, C::MINB)
 
     if (warp == WARP_L) {
         // ================================================================ L: loads
-        const uint32_t tx_bytes = uint32_t((p.has_gate ? 3 : 2) * S::tok_bytes + (p.bc_tma ? 2 * S::bc_bytes : 0));
+        const uint32_t tx_bytes =
+            uint32_t(S::xbox_bytes + (p.has_gate ? 2 : 1) * S::tok_bytes + (p.bc_tma ? 2 * S::bc_bytes : 0));
         if (lane == 0) {
             prefetch_tensormap(&tm_x);
             prefetch_tensormap(&tm_dt);
@@ -468,7 +536,8 @@ __global__ void __launch_bounds__(NTHREADS, C::MINB)
                     unsigned char *stage = smem + S::stage_off + size_t(st) * S::stage_bytes;
                     const int b = int(m.g / p.Dg), d0 = int((m.g % p.Dg) * CH);
                     mbar_arrive_expect_tx(&bar_full[st], tx_bytes);
-                    tma_load_3d(stage + S::st_x, &tm_x, &bar_full[st], d0, m.t0, b);
+                    // CONV: the box starts HALO rows early (before t = 0 TMA reads zeros)
+                    tma_load_3d(stage + S::st_x, &tm_x, &bar_full[st], d0, m.t0 - S::HALO, b);
                     tma_load_3d(stage + S::st_dt, &tm_dt, &bar_full[st], d0, m.t0, b);
                     if (p.has_gate) tma_load_3d(stage + S::st_z, &tm_z, &bar_full[st], d0, m.t0, b);
                     if (p.bc_tma) {
@@ -487,7 +556,8 @@ __global__ void __launch_bounds__(NTHREADS, C::MINB)
         // ================================================================ E: epilogue
         const int h = warp - WARP_E0;
         const int c = lane;
-        float dd = 0.f;
+        float dd = 0.f, cb = 0.f;
+        float4 cw = make_float4(0.f, 0.f, 0.f, 0.f);
         for (int i = 0;; ++i) {
             const int pr = i % R_PART, st = i % STAGES;
             if (!warp_wait(&bar_part_full[pr], uint32_t(i / R_PART) & 1u)) {
@@ -503,13 +573,16 @@ __global__ void __launch_bounds__(NTHREADS, C::MINB)
             if (m.flags & F_FIRST) {
                 const int64_t d = (m.g % p.Dg) * CH + c;
                 dd = (d < p.D && p.Dskip) ? __ldg(p.Dskip + d) : 0.f;
+                if (CONV) load_conv(p, d, cw, cb);
             }
+            float3 x0 = make_float3(0.f, 0.f, 0.f);
+            const bool use_x0 = CONV && h == 0 && m.t0 == 0 && conv_prefix<T>(p, m.g, c, x0);
             const unsigned char *stage = smem + S::stage_off + size_t(st) * S::stage_bytes;
-            const T *sx = reinterpret_cast<const T *>(stage + S::st_x) + c;
+            const T *sx = reinterpret_cast<const T *>(stage + S::st_x) + S::HALO * CH + c;
             const T *sz = reinterpret_cast<const T *>(stage + S::st_z) + c;
             const float4 *part = reinterpret_cast<const float4 *>(smem + S::part_off + pr * S::part_bytes) + c;
             T *yo = reinterpret_cast<T *>(smem + S::yout_off + (i % YBUF) * S::yout_bytes) + c;
-            epilogue_rows<T>(part, sx, sz, yo, h * TE, dd, p.has_gate != 0);
+            epilogue_rows<T, CONV>(part, sx, sz, yo, h * TE, dd, p.has_gate != 0, cw, cb, use_x0, x0);
             warp_arrive(&bar_part_free[pr]);  // the consumers may reuse this partial slot
             warp_arrive(&bar_sfree[st]);      // x and z of this stage are no longer needed
             fence_proxy_async_smem();         // y rows written by this thread -> visible to the TMA store
@@ -529,7 +602,8 @@ __global__ void __launch_bounds__(NTHREADS, C::MINB)
         const T *Bm = static_cast<const T *>(p.Bm);
         const T *Cm = static_cast<const T *>(p.Cm);
         const int c = lane;  // P lane = channel (records)
-        float bias_c = 0.f;
+        float bias_c = 0.f, cb = 0.f;
+        float4 cw = make_float4(0.f, 0.f, 0.f, 0.f);
         bool struct_item = false;
         for (int i = 0;; ++i) {
             const int r = i % R_REC, st = i % STAGES;
@@ -554,6 +628,7 @@ __global__ void __launch_bounds__(NTHREADS, C::MINB)
                 const int64_t d = (m.g % p.Dg) * CH + c;
                 const bool ok = d < p.D;
                 bias_c = (ok && p.dt_bias) ? __ldg(p.dt_bias + d) : 0.f;
+                if (CONV) load_conv(p, d, cw, cb);
                 float a[kMaxN];
 #pragma unroll
                 for (int n = 0; n < kMaxN; ++n) a[n] = (ok && n < p.N) ? __ldg(p.A + d * p.N + n) : 0.f;
@@ -566,9 +641,11 @@ __global__ void __launch_bounds__(NTHREADS, C::MINB)
             }
             const unsigned char *stage = smem + S::stage_off + size_t(st) * S::stage_bytes;
             float2 *rec = reinterpret_cast<float2 *>(smem + S::rec_off + r * S::rec_bytes) + c;
-            prologue_rows<T>(reinterpret_cast<const T *>(stage + S::st_x) + c,
-                             reinterpret_cast<const T *>(stage + S::st_dt) + c, rec, h * TP, m.tlen, bias_c,
-                             p.softplus != 0, ZOH);
+            float3 x0 = make_float3(0.f, 0.f, 0.f);
+            const bool use_x0 = CONV && h == 0 && m.t0 == 0 && conv_prefix<T>(p, m.g, c, x0);
+            prologue_rows<T, CONV>(reinterpret_cast<const T *>(stage + S::st_x) + S::HALO * CH + c,
+                                   reinterpret_cast<const T *>(stage + S::st_dt) + c, rec, h * TP, m.tlen, bias_c,
+                                   p.softplus != 0, ZOH, cw, cb, use_x0, x0);
             // B and C rows of this half widened to float32: row t = [B_0 .. B_15 | C_0 .. C_15],
             // in 16-byte chunks; chunk id = q * 32 + lane covers row h*TP + id / 8 and chunk
             // id % 8 (0-3: B, 4-7: C), so eight consecutive lanes write one 128-byte row.

@@ -112,6 +112,19 @@ def step_inputs(batch, dim, dstate, steps, dtype=torch.bfloat16, seed=SEED_BASE 
     return dict(h=h, x=x, dt=dt, z=z, B=Bm, C=Cm, A=A, D=Dskip, dt_bias=dt_bias)
 
 
+def conv_params(dim, batch, dtype=torch.bfloat16, seed=SEED_BASE + 5, device="cpu", bias=True, prefix=True):
+    """The block's short convolution: taps conv_w [D, 4] and bias conv_b [D] (float32,
+    uniform in [-1/2, 1/2], the default initialisation of a depthwise Conv1d with fan-in
+    4), and conv_x0 [B, 3, D], the three tokens before t = 0, ~ N(0, 1) in the token
+    dtype. bias / prefix False give None for those."""
+    g = _gen(seed + 104729, "cpu")
+    w = torch.rand((dim, 4), generator=g, dtype=torch.float32) - 0.5
+    b = torch.rand((dim,), generator=g, dtype=torch.float32) - 0.5
+    x0 = _normal((batch, 3, dim), g, "cpu", dtype)
+    return dict(conv_w=w.to(device), conv_b=b.to(device) if bias else None,
+                conv_x0=x0.to(device) if prefix else None)
+
+
 def to_numpy_storage(t):
     """A token tensor as numpy in its storage form: float32, or uint16 bfloat16 bit patterns."""
     if t is None:

@@ -18,8 +18,9 @@ def f32np(t):
     return None if t is None else t.detach().cpu().float().numpy()
 
 
-def oracle_scan(inp, delta_softplus=True, sel=None, exact_zoh=False):
-    """Run the float64 oracle on exactly the tensors the GPU saw (optionally a channel subset)."""
+def oracle_scan(inp, delta_softplus=True, sel=None, exact_zoh=False, conv=None):
+    """Run the float64 oracle on exactly the tensors the GPU saw (optionally a channel subset).
+    conv: the short convolution's conv_w / conv_b / conv_x0 tensors (no channel subset)."""
     def tok(name):
         t = inp[name]
         if t is None:
@@ -37,9 +38,14 @@ def oracle_scan(inp, delta_softplus=True, sel=None, exact_zoh=False):
     h0 = inp.get("h0")
     if h0 is not None and sel is not None:
         h0 = h0[:, sel]
+    kw = {}
+    if conv is not None:
+        assert sel is None
+        kw = dict(conv_w=f32np(conv["conv_w"]), conv_b=f32np(conv.get("conv_b")),
+                  conv_x0=storage(conv.get("conv_x0")))
     return oracle.scan(tok("x"), tok("dt"), par("A"), storage(inp["B"]), storage(inp["C"]),
                        D=par("D"), z=tok("z"), dt_bias=par("dt_bias"), h0=f32np(h0),
-                       dtype=dtype_name(inp["x"]), delta_softplus=delta_softplus, exact_zoh=exact_zoh)
+                       dtype=dtype_name(inp["x"]), delta_softplus=delta_softplus, exact_zoh=exact_zoh, **kw)
 
 
 def rowwise_rel(got, ref, axis):

@@ -36,6 +36,20 @@ def test_header_and_exports_agree(lib):
         assert hasattr(lib, name)
 
 
+def test_args_struct_layout_matches_binding(tmp_path):
+    """The ctypes mirror of ssm_scan_args has the C compiler's field offsets and size."""
+    names = [f[0] for f in _native.ScanArgs._fields_]
+    src = tmp_path / "layout.c"
+    body = "".join(f'printf("%zu\\n", offsetof(ssm_scan_args, {n}));' for n in names)
+    src.write_text('#include <stddef.h>\n#include <stdio.h>\n#include "ssm_scan.h"\n'
+                   f'int main(void){{ {body} printf("%zu\\n", sizeof(ssm_scan_args)); return 0; }}\n')
+    exe = tmp_path / "layout"
+    subprocess.check_call(["gcc", "-std=c99", "-I", os.path.join(ROOT, "include"), "-o", str(exe), str(src)])
+    got = [int(v) for v in subprocess.check_output([str(exe)]).decode().split()]
+    want = [getattr(_native.ScanArgs, n).offset for n in names] + [ctypes.sizeof(_native.ScanArgs)]
+    assert got == want
+
+
 def test_header_compiles_as_c(tmp_path):
     src = tmp_path / "use.c"
     src.write_text('#include "ssm_scan.h"\nint main(void){ ssm_scan_args a = {0}; (void)a;'
@@ -100,6 +114,11 @@ def test_workspace_size(lib):
     (dict(workspace=(1 << 20) + 8), _native.SSM_ERR_UNSUPPORTED),
     (dict(workspace=None), _native.SSM_ERR_INVALID),
     (dict(workspace_bytes=100), _native.SSM_ERR_INVALID),
+    (dict(conv_b=1 << 30), _native.SSM_ERR_INVALID),                         # bias without taps
+    (dict(conv_x0=1 << 30), _native.SSM_ERR_INVALID),                        # prefix without taps
+    (dict(conv_w=(1 << 30) + 4), _native.SSM_ERR_UNSUPPORTED),               # taps: one float4 per channel
+    (dict(conv_w=1 << 30, conv_x0=(1 << 30) + 1), _native.SSM_ERR_UNSUPPORTED),  # bf16 prefix on 2 bytes
+    (dict(conv_w=1 << 30, conv_b=(1 << 30) + 2), _native.SSM_ERR_UNSUPPORTED),
 ])
 def test_scan_rejects_on_host(lib, bad, code):
     a = _args(**bad)
@@ -161,3 +180,7 @@ def test_host_scan_staging_size_and_argument_checks(lib):
     assert lib.ssm_scan_fwd_host(ctypes.byref(a), Lc, ctypes.c_void_p((1 << 20) + 16), need, None) == \
         _native.SSM_ERR_UNSUPPORTED
     assert lib.ssm_scan_fwd_host(ctypes.byref(a), Lc, fake, need - 1, None) == _native.SSM_ERR_INVALID
+    # with the short convolution each buffer also holds the three tokens before its chunk
+    a.conv_w = 1 << 30
+    assert lib.ssm_scan_host_staging_size(ctypes.byref(a), Lc) == 2 * (4 * tok + 2 * bc + up(3 * 3 * 64 * 2)) + \
+        2 * carry
