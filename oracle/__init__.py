@@ -28,6 +28,8 @@ def _open(path):
     lib.oracle_scan_conv_f64.restype = c_int
     lib.oracle_step_f64.argtypes = [i64, i64, i64, c_int, c_uint] + [vp] * 10 + [c_int]
     lib.oracle_step_f64.restype = c_int
+    lib.oracle_step_conv_f64.argtypes = [i64, i64, i64, c_int, c_uint] + [vp] * 13 + [c_int]
+    lib.oracle_step_conv_f64.restype = c_int
     return lib
 
 
@@ -71,9 +73,10 @@ class Oracle:
                      exact_zoh, nthreads, conv_w, conv_b, conv_x0)
 
     def step(self, x, dt, A, B, C, h, D=None, z=None, dt_bias=None, dtype="f32",
-             delta_softplus=True, exact_zoh=False, nthreads=None):
+             delta_softplus=True, exact_zoh=False, nthreads=None, conv_w=None, conv_b=None,
+             conv_state=None):
         return _step(self.lib, x, dt, A, B, C, h, D, z, dt_bias, dtype, delta_softplus,
-                     exact_zoh, nthreads)
+                     exact_zoh, nthreads, conv_w, conv_b, conv_state)
 
 
 _default = None
@@ -141,9 +144,13 @@ def _scan(lib, x, dt, A, B, C, D=None, z=None, dt_bias=None, h0=None, dtype="f32
 
 
 def _step(lib, x, dt, A, B, C, h, D=None, z=None, dt_bias=None, dtype="f32",
-          delta_softplus=True, exact_zoh=False, nthreads=None):
+          delta_softplus=True, exact_zoh=False, nthreads=None, conv_w=None, conv_b=None,
+          conv_state=None):
     """One recurrent decode step. x, dt, z: [Bsz, Dm]; B, C: [Bsz, N];
-    h: float64 [Bsz, Dm, N], updated in place. Returns y [Bsz, Dm] float64."""
+    h: float64 [Bsz, Dm, N], updated in place. Returns y [Bsz, Dm] float64.
+    conv_w [Dm, 4] (float32) puts the block's causal convolution and SiLU in front: the
+    three previous tokens come from conv_state [Bsz, 3, Dm] (x's storage type, oldest
+    first), which is then shifted in place to end with x; conv_b [Dm] or None."""
     Bsz, Dm = np.shape(x)
     N = np.shape(A)[1]
     x = _tok(x, dtype, (Bsz, Dm), "x")
@@ -159,10 +166,25 @@ def _step(lib, x, dt, A, B, C, h, D=None, z=None, dt_bias=None, dtype="f32",
         raise ValueError("h must be a C-contiguous float64 array of shape [Bsz, Dm, N]")
     y = np.empty((Bsz, Dm), dtype=np.float64)
     flags = (DELTA_SOFTPLUS if delta_softplus else 0) | (EXACT_ZOH if exact_zoh else 0)
-    rc = lib.oracle_step_f64(Bsz, Dm, N, 0 if dtype == "f32" else 1, flags,
-                             _ptr(x), _ptr(dt), _ptr(z), _ptr(B), _ptr(C), _ptr(A), _ptr(D),
-                             _ptr(dt_bias), _ptr(h), _ptr(y),
-                             default_threads() if nthreads is None else nthreads)
+    nt = default_threads() if nthreads is None else nthreads
+    common = (Bsz, Dm, N, 0 if dtype == "f32" else 1, flags, _ptr(x), _ptr(dt), _ptr(z), _ptr(B), _ptr(C),
+              _ptr(A), _ptr(D), _ptr(dt_bias))
+    if conv_w is None:
+        if conv_b is not None or conv_state is not None:
+            raise ValueError("conv_b and conv_state need conv_w")
+        rc = lib.oracle_step_f64(*common, _ptr(h), _ptr(y), nt)
+    else:
+        want = np.float32 if dtype == "f32" else np.uint16
+        if not (isinstance(conv_state, np.ndarray) and conv_state.dtype == want
+                and conv_state.shape == (Bsz, 3, Dm) and conv_state.flags.c_contiguous):
+            raise ValueError(f"conv_state must be a C-contiguous {want.__name__} array of shape [Bsz, 3, Dm]")
+        conv_w = _f32(conv_w, (Dm, 4), "conv_w")
+        conv_b = _f32(conv_b, (Dm,), "conv_b")
+        rc = lib.oracle_step_conv_f64(*common, _ptr(conv_w), _ptr(conv_b), _ptr(conv_state), _ptr(h),
+                                      _ptr(y), nt)
+        if rc == 0:  # the window moves by one token (bookkeeping, no arithmetic)
+            conv_state[:, :2] = conv_state[:, 1:].copy()
+            conv_state[:, 2] = x
     if rc != 0:
-        raise ValueError("oracle_step_f64 rejected its arguments")
+        raise ValueError("oracle step rejected its arguments")
     return y

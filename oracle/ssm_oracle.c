@@ -220,3 +220,22 @@ int oracle_step_f64(int64_t Bsz, int64_t Dm, int64_t N, int dtype, unsigned flag
     run_jobs(&base, nthreads);
     return 0;
 }
+
+/*
+ * One decode step behind the block's short convolution: oracle_step_f64 with the SSM's
+ * input u = silu(conv_b + sum_k conv_w[d,k] x_{t-3+k}), the three previous tokens read
+ * from conv_state ([Bsz, 3, Dm], x's storage type, oldest first). The state itself is
+ * left as it is (the caller shifts in the new token).
+ */
+int oracle_step_conv_f64(int64_t Bsz, int64_t Dm, int64_t N, int dtype, unsigned flags,
+                         const void *x, const void *dt, const void *z, const void *Bm, const void *Cm,
+                         const float *A, const float *Dskip, const float *dt_bias,
+                         const float *conv_w, const float *conv_b, const void *conv_state,
+                         double *h, double *y, int nthreads) {
+    if (Bsz < 0 || Dm < 0 || N < 1 || N > 256 || (dtype != 0 && dtype != 1)) return -1;
+    if (!x || !dt || !Bm || !Cm || !A || !h || !y || !conv_w || !conv_state) return -1;
+    scan_job base = {Bsz, 1, Dm, N, dtype, flags, x, dt, z, Bm, Cm, A, Dskip, dt_bias, NULL,
+                     y, h, h, 0, Bsz * Dm, conv_w, conv_b, conv_state};
+    run_jobs(&base, nthreads);
+    return 0;
+}

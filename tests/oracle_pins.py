@@ -427,4 +427,34 @@ def pin_conv_front_end_bf16(orc):
     pin_conv_front_end(orc, dtype="bf16", seed=13, with_bias=False)
 
 
-ALL_PINS += [pin_conv_front_end, pin_conv_front_end_bf16]
+def pin_conv_step_matches_conv_scan(orc, seed=14):
+    """Decode behind the short convolution: L chained steps, each reading the three previous
+    tokens from a rolling window that starts as the scan's prefix, equal one scan with the
+    convolution (itself pinned to numpy's cross-correlation above); the window ends as the
+    last three tokens. [SSM blog (shakilmahmud.com), section 3: recurrence at inference;
+    Mamba summary, block-architecture paragraph]."""
+    rng = _rng(seed)
+    Bsz, L, Dm, N = 2, 9, 3, 4
+    x = rng.standard_normal((Bsz, L, Dm)).astype(np.float32)
+    dt = (0.5 * rng.standard_normal((Bsz, L, Dm))).astype(np.float32)
+    z = rng.standard_normal((Bsz, L, Dm)).astype(np.float32)
+    Bm = rng.standard_normal((Bsz, L, N)).astype(np.float32)
+    Cm = rng.standard_normal((Bsz, L, N)).astype(np.float32)
+    A = (-rng.uniform(0.5, 4.0, (Dm, N))).astype(np.float32)
+    Dskip = rng.standard_normal(Dm).astype(np.float32)
+    bias = rng.uniform(-3, 0, Dm).astype(np.float32)
+    w = (rng.standard_normal((Dm, 4)) * 0.7).astype(np.float32)
+    cb = (rng.standard_normal(Dm) * 0.3).astype(np.float32)
+    x0 = rng.standard_normal((Bsz, 3, Dm)).astype(np.float32)
+    y, hL = orc.scan(x, dt, A, Bm, Cm, D=Dskip, z=z, dt_bias=bias, conv_w=w, conv_b=cb, conv_x0=x0)
+    h = np.zeros((Bsz, Dm, N))
+    window = x0.copy()
+    for t in range(L):
+        yt = orc.step(x[:, t], dt[:, t], A, Bm[:, t], Cm[:, t], h, D=Dskip, z=z[:, t], dt_bias=bias,
+                      conv_w=w, conv_b=cb, conv_state=window)
+        assert _rel(yt - y[:, t], y[:, t]) < 1e-14, f"convolution step {t} differs from the scan"
+    assert _rel(h - hL, hL) < 1e-14
+    assert np.array_equal(window, x[:, L - 3:]), "the window must end as the last three tokens"
+
+
+ALL_PINS += [pin_conv_front_end, pin_conv_front_end_bf16, pin_conv_step_matches_conv_scan]

@@ -49,6 +49,8 @@ MUTANTS = {
     "conv_reads_next_token": ("t - (ORACLE_CONV_K - 1) + k", "t - (ORACLE_CONV_K - 2) + k"),
     "conv_skip_uses_raw_x": ("y += dskip * xv;", "y += dskip * widen(J->x, J->dtype, i);"),
     "conv_update_uses_raw_x": ("h[n] = abar * h[n] + bbar * xv;", "h[n] = abar * h[n] + bbar * widen(J->x, J->dtype, i);"),
+    "conv_step_ignores_window": ("y, h, h, 0, Bsz * Dm, conv_w, conv_b, conv_state};",
+                                 "y, h, h, 0, Bsz * Dm, conv_w, conv_b, NULL};"),
 }
 
 
