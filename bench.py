@@ -294,7 +294,8 @@ def run_ours(args):
 
     if args.decode_only:
         line = {"metric": "decode state-updates/s (B·D·N per token step)", "n_gpus": world, "data": "synthetic",
-                "decode": run_decode(ssm, synth, dev, stream, rank, hbm_peak, reps=max(1, args.steps))}
+                "decode": run_decode(ssm, synth, dev, stream, rank, hbm_peak, reps=max(1, args.steps),
+                                     conv=args.conv)}
         if world > 1:
             dist.barrier()
             dist.destroy_process_group()
@@ -417,6 +418,8 @@ def run_ours(args):
         # Recurrent decode (one-token step): 1000 chained steps in one CUDA graph.
         line["decode"] = run_decode(ssm, synth, dev, stream, rank, hbm_peak)
         line["gpu_launches"] += line["decode"]["launches"]
+        line["decode_conv1d"] = run_decode(ssm, synth, dev, stream, rank, hbm_peak, conv=True)
+        line["gpu_launches"] += line["decode_conv1d"]["launches"]
         # CPU baseline (rank 0, single GPU only).
         if rank == 0 and world == 1:
             rate, cores, desc, sec, upd = oracle_sample(w, max_channels=1024)
@@ -430,18 +433,24 @@ def run_ours(args):
     return 0
 
 
-def run_decode(ssm, synth, dev, stream, rank, hbm_peak, reps=3):
+def run_decode(ssm, synth, dev, stream, rank, hbm_peak, reps=3, conv=False):
+    """1000 chained decode steps in one CUDA graph; conv: behind the block's short
+    convolution (ssm_step_conv, its [B, 3, D] window read and moved on every step)."""
     import torch
     s = synth.WORKLOADS["decode"]
     inp = synth.step_inputs(s.batch, s.dim, s.dstate, s.steps, s.dtype,
                             seed=rank_seed(synth.SEEDS["decode"], rank), device=dev)
     h = inp["h"].clone()
     out = torch.empty((s.steps, s.batch, s.dim), dtype=s.dtype, device=dev)
+    cv = {}
+    if conv:
+        c = synth.conv_params(s.dim, s.batch, s.dtype, seed=rank_seed(synth.SEEDS["decode"] + 5, rank), device=dev)
+        cv = dict(conv_w=c["conv_w"], conv_b=c["conv_b"], conv_state=c["conv_x0"])
 
     def steps():
         for t in range(s.steps):
             ssm.step(inp["x"][t], inp["dt"][t], inp["A"], inp["B"][t], inp["C"][t], h, inp["D"],
-                     inp["z"][t], inp["dt_bias"], out=out[t])
+                     inp["z"][t], inp["dt_bias"], out=out[t], **cv)
 
     side = torch.cuda.Stream(dev)
     side.wait_stream(stream)
@@ -457,9 +466,12 @@ def run_decode(ssm, synth, dev, stream, rank, hbm_peak, reps=3):
     ms = time_region(g.replay, reps, stream) / reps
     upd = s.batch * s.dim * s.dstate * s.steps
     per_step_bytes = 2 * s.batch * s.dim * s.dstate * 4 + 4 * s.batch * s.dim * 2 + 2 * s.batch * s.dstate * 2
+    if conv:  # the window: three tokens read and written per channel
+        per_step_bytes += 2 * 3 * s.batch * s.dim * 2
     gbs = per_step_bytes * s.steps / (ms / 1e3) / 1e9
     del g
-    return {"workload": "decode B=256 D=5120 N=16, 1000 chained steps in one CUDA graph",
+    return {"workload": "decode B=256 D=5120 N=16, 1000 chained steps in one CUDA graph"
+                        + (", behind the short convolution" if conv else ""),
             "value": upd / (ms / 1e3), "unit": UNIT, "ms_per_1000_steps": ms,
             "us_per_step": 1e3 * ms / s.steps, "algorithmic_GBs": gbs, "hbm_frac": gbs / hbm_peak,
             "note": "the 84 MB state h stays in the 126 MB L2 across chained steps",

@@ -154,6 +154,22 @@ ssm_status ssm_step(int64_t batch, int64_t dim, int64_t dstate, ssm_dtype dtype,
                     void *stream);
 
 /*
+ * ssm_step behind the Mamba block's short causal convolution (kernel size 4) and SiLU
+ * (Mamba summary, block-architecture paragraph), the decode form of the scan's conv_w:
+ * the SSM's input is u = silu(conv_b[d] + conv_w[d,0] s0 + conv_w[d,1] s1 +
+ * conv_w[d,2] s2 + conv_w[d,3] x), where s0, s1, s2 are the three previous tokens of
+ * the window conv_state ([B, 3, D], dtype of x, oldest first: the layout of the scan's
+ * conv_x0, so the last three tokens of a prefill start the decode). conv_state is then
+ * moved on by one token in place, to (s1, s2, x). conv_w [D, 4] float32 on 16 bytes;
+ * conv_b [D] or NULL; conv_state must not alias any other argument. Errors as
+ * ssm_step; SSM_ERR_INVALID if conv_w or conv_state is NULL.
+ */
+ssm_status ssm_step_conv(int64_t batch, int64_t dim, int64_t dstate, ssm_dtype dtype, uint32_t flags,
+                         const void *x, const void *dt, const void *z, const void *Bm, const void *Cm,
+                         const float *A, const float *Dskip, const float *dt_bias, const float *conv_w,
+                         const float *conv_b, void *conv_state, float *h, void *y, void *stream);
+
+/*
  * Synchronises `stream` and returns the device-side status of the last scan
  * that used `workspace`: SSM_OK, or SSM_ERR_TIMEOUT if a segment gave up
  * waiting for its predecessor's state (its outputs are then incomplete).

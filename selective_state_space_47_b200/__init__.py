@@ -236,10 +236,13 @@ def workspace_status(workspace, stream=None):
 
 
 def step(x, dt, A, B, C, h, D=None, z=None, dt_bias=None, *, delta_softplus=True, general_A=False,
-         exact_zoh=False, out=None, stream=None):
+         exact_zoh=False, out=None, stream=None, conv_w=None, conv_b=None, conv_state=None):
     """One recurrent decode step (see include/ssm_scan.h, ssm_step); h is updated in place.
 
     x, dt, z: [B, D]; B, C: [B, N]; A: [D, N]; h: [B, D, N] float32. Returns y [B, D].
+    conv_w [D, 4] float32 with conv_state [B, 3, D] (x's dtype: the three previous
+    tokens, oldest first, moved on by one token in place) and optional conv_b [D]: the
+    block's short convolution and SiLU in front (ssm_step_conv).
     """
     dev = x.device
     if x.dtype not in _TOKEN_DTYPES:
@@ -261,8 +264,22 @@ def step(x, dt, A, B, C, h, D=None, z=None, dt_bias=None, *, delta_softplus=True
         _need(dt_bias, "dt_bias", (Dm,), torch.float32, dev)
     y = torch.empty_like(x) if out is None else out
     _need(y, "out", (Bsz, Dm), tok, dev)
-    rc = _native.lib().ssm_step(Bsz, Dm, N, _TOKEN_DTYPES[tok], _flags(delta_softplus, general_A, exact_zoh),
-                                _ptr(x), _ptr(dt), _ptr(z), _ptr(B), _ptr(C), _ptr(A), _ptr(D),
-                                _ptr(dt_bias), _ptr(h), _ptr(y), _stream_handle(stream))
-    _native.check(rc, "ssm_step")
+    flags = _flags(delta_softplus, general_A, exact_zoh)
+    common = (Bsz, Dm, N, _TOKEN_DTYPES[tok], flags, _ptr(x), _ptr(dt), _ptr(z), _ptr(B), _ptr(C), _ptr(A),
+              _ptr(D), _ptr(dt_bias))
+    if conv_w is None:
+        if conv_b is not None or conv_state is not None:
+            raise ValueError("conv_b and conv_state need conv_w")
+        rc = _native.lib().ssm_step(*common, _ptr(h), _ptr(y), _stream_handle(stream))
+        _native.check(rc, "ssm_step")
+        return y
+    _need(conv_w, "conv_w", (Dm, 4), torch.float32, dev)
+    if conv_b is not None:
+        _need(conv_b, "conv_b", (Dm,), torch.float32, dev)
+    if conv_state is None:
+        raise ValueError("conv_state [B, 3, D] is required with conv_w")
+    _need(conv_state, "conv_state", (Bsz, 3, Dm), tok, dev)
+    rc = _native.lib().ssm_step_conv(*common, _ptr(conv_w), _ptr(conv_b), _ptr(conv_state), _ptr(h), _ptr(y),
+                                     _stream_handle(stream))
+    _native.check(rc, "ssm_step_conv")
     return y

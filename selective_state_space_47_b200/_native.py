@@ -13,7 +13,7 @@ SSM_EXACT_ZOH = 4
 SSM_TEST_DROP_HANDOFF = 0x80000000
 
 # Every symbol the header declares (checked by the CPU test suite).
-EXPORTS = ("ssm_scan_workspace_size", "ssm_scan_fwd", "ssm_step", "ssm_workspace_status",
+EXPORTS = ("ssm_scan_workspace_size", "ssm_scan_fwd", "ssm_step", "ssm_step_conv", "ssm_workspace_status",
            "ssm_status_string", "ssm_scan_fwd_noalloc", "ssm_scan_host_staging_size", "ssm_scan_fwd_host")
 
 
@@ -54,6 +54,8 @@ def lib():
         L.ssm_scan_fwd_host.restype = ctypes.c_int
         L.ssm_step.argtypes = [i64, i64, i64, ctypes.c_int, ctypes.c_uint32] + [vp] * 10 + [vp]
         L.ssm_step.restype = ctypes.c_int
+        L.ssm_step_conv.argtypes = [i64, i64, i64, ctypes.c_int, ctypes.c_uint32] + [vp] * 13 + [vp]
+        L.ssm_step_conv.restype = ctypes.c_int
         L.ssm_workspace_status.argtypes = [vp, vp]
         L.ssm_workspace_status.restype = ctypes.c_int
         L.ssm_status_string.argtypes = [ctypes.c_int]

@@ -46,17 +46,46 @@ __device__ __forceinline__ float zoh_w(const float delta, const float A, const f
     return __fdividef(abar - 1.f, A);
 }
 
+// The short convolution at one decode step for channel d: u = silu(cb + w.x s0 + w.y s1 +
+// w.z s2 + w.w x), s = the three previous tokens of the window (conv_state [B, 3, D],
+// oldest first; s points at s0, the others follow at stride D). The same fused
+// multiply-adds in the same order as the scan kernel's.
+template <typename T>
+__device__ __forceinline__ float conv_u(const float xv, const T *s, const int64_t D, const float4 w, const float cb) {
+    float v = fmaf(w.x, Tok<T>::to_f(s[0]), cb);
+    v = fmaf(w.y, Tok<T>::to_f(s[D]), v);
+    v = fmaf(w.z, Tok<T>::to_f(s[2 * D]), v);
+    v = fmaf(w.w, xv, v);
+    return silu_f(v);
+}
+
+// Taps ([D, 4], one float4 per channel) and bias of channel d.
+__device__ __forceinline__ float4 conv_taps(const float *w, const int64_t d) {
+    return __ldg(reinterpret_cast<const float4 *>(w) + d);
+}
+
 // ------------------------------------------------------------- step kernel
-template <typename T, bool ZOH>
+// CONV: the SSM's input is the short convolution's u; the window conv_state moves by one
+// token (s0, s1, s2) -> (s1, s2, x).
+template <typename T, bool ZOH, bool CONV>
 __global__ void __launch_bounds__(128)
     step_kernel(int64_t Bsz, int64_t D, int N, int softplus, const T *__restrict__ x, const T *__restrict__ dt,
                 const T *__restrict__ z, const T *__restrict__ Bm, const T *__restrict__ Cm,
                 const float *__restrict__ A, const float *__restrict__ Dskip, const float *__restrict__ dt_bias,
-                float *__restrict__ h, T *__restrict__ y) {
+                float *__restrict__ h, T *__restrict__ y, const float *__restrict__ conv_w,
+                const float *__restrict__ conv_b, T *__restrict__ conv_state) {
     const int64_t ch = int64_t(blockIdx.x) * blockDim.x + threadIdx.x;
     if (ch >= Bsz * D) return;
     const int64_t b = ch / D, d = ch % D;
-    const float xv = Tok<T>::ldg(x + ch);
+    float xv = Tok<T>::ldg(x + ch);
+    if (CONV) {
+        T *s = conv_state + b * 3 * D + d;
+        const T s1 = s[D], s2 = s[2 * D];
+        xv = conv_u<T>(xv, s, D, conv_taps(conv_w, d), conv_b ? __ldg(conv_b + d) : 0.f);
+        s[0] = s1;
+        s[D] = s2;
+        s[2 * D] = x[ch];
+    }
     const float v = Tok<T>::ldg(dt + ch) + (dt_bias ? __ldg(dt_bias + d) : 0.f);
     const float delta = softplus ? softplus_f(v) : v;
     const float dl = delta * kLog2e, u = delta * xv;
@@ -96,12 +125,15 @@ __global__ void __launch_bounds__(128)
 // work (softplus, gate) is repeated by only two threads, and the readout is summed
 // with one butterfly shuffle. Requires 16-byte aligned h and A rows and 4-element
 // aligned B, C rows.
-template <typename T, bool ZOH>
+// CONV as for step_kernel: both threads of a channel form u; the first moves the window
+// once both have read it (after the warp-wide shuffle).
+template <typename T, bool ZOH, bool CONV>
 __global__ void __launch_bounds__(256)
     step_pair_kernel(int64_t Bsz, int64_t D, int softplus, const T *__restrict__ x, const T *__restrict__ dt,
                      const T *__restrict__ z, const T *__restrict__ Bm, const T *__restrict__ Cm,
                      const float *__restrict__ A, const float *__restrict__ Dskip, const float *__restrict__ dt_bias,
-                     float *__restrict__ h, T *__restrict__ y) {
+                     float *__restrict__ h, T *__restrict__ y, const float *__restrict__ conv_w,
+                     const float *__restrict__ conv_b, T *__restrict__ conv_state) {
     const int64_t gid = int64_t(blockIdx.x) * blockDim.x + threadIdx.x;
     const int64_t ch = gid >> 1;
     const int q = int(gid & 1);
@@ -109,8 +141,15 @@ __global__ void __launch_bounds__(256)
     const int64_t chv = valid ? ch : 0;
     const int64_t b = chv / D, d = chv % D;
     float yv = 0.f, xv = 0.f;
+    T s1{}, s2{};  // CONV: the window's next first two tokens
     if (valid) {
         xv = Tok<T>::ldg(x + ch);
+        if (CONV) {
+            const T *s = conv_state + b * 3 * D + d;
+            s1 = s[D];
+            s2 = s[2 * D];
+            xv = conv_u<T>(xv, s, D, conv_taps(conv_w, d), conv_b ? __ldg(conv_b + d) : 0.f);
+        }
         const float v = Tok<T>::ldg(dt + ch) + (dt_bias ? __ldg(dt_bias + d) : 0.f);
         const float delta = softplus ? softplus_f(v) : v;
         const float dl = delta * kLog2e, u = delta * xv;
@@ -149,6 +188,12 @@ __global__ void __launch_bounds__(256)
         yv = fmaf(Dskip ? __ldg(Dskip + d) : 0.f, xv, yv);
         if (z) yv *= silu_f(Tok<T>::ldg(z + ch));
         y[ch] = Tok<T>::from_f(yv);
+        if (CONV) {
+            T *s = conv_state + b * 3 * D + d;
+            s[0] = s1;
+            s[D] = s2;
+            s[2 * D] = x[ch];
+        }
     }
 }
 
@@ -369,20 +414,90 @@ unsigned char *static_scratch() {
 }  // namespace
 
 // ======================================================================= C ABI
-template <typename T, bool ZOH>
+namespace {
+
+template <typename T, bool ZOH, bool CONV>
 void launch_step(bool pair, unsigned grid, int threads, cudaStream_t stream, int64_t batch, int64_t dim, int N,
                  int sp, const void *x, const void *dt, const void *z, const void *Bm, const void *Cm,
-                 const float *A, const float *Dskip, const float *dt_bias, float *h, void *y) {
+                 const float *A, const float *Dskip, const float *dt_bias, float *h, void *y, const float *conv_w,
+                 const float *conv_b, void *conv_state) {
     if (pair)
-        step_pair_kernel<T, ZOH><<<grid, threads, 0, stream>>>(
+        step_pair_kernel<T, ZOH, CONV><<<grid, threads, 0, stream>>>(
             batch, dim, sp, static_cast<const T *>(x), static_cast<const T *>(dt), static_cast<const T *>(z),
-            static_cast<const T *>(Bm), static_cast<const T *>(Cm), A, Dskip, dt_bias, h, static_cast<T *>(y));
+            static_cast<const T *>(Bm), static_cast<const T *>(Cm), A, Dskip, dt_bias, h, static_cast<T *>(y),
+            conv_w, conv_b, static_cast<T *>(conv_state));
     else
-        step_kernel<T, ZOH><<<grid, threads, 0, stream>>>(
+        step_kernel<T, ZOH, CONV><<<grid, threads, 0, stream>>>(
             batch, dim, N, sp, static_cast<const T *>(x), static_cast<const T *>(dt), static_cast<const T *>(z),
-            static_cast<const T *>(Bm), static_cast<const T *>(Cm), A, Dskip, dt_bias, h, static_cast<T *>(y));
+            static_cast<const T *>(Bm), static_cast<const T *>(Cm), A, Dskip, dt_bias, h, static_cast<T *>(y),
+            conv_w, conv_b, static_cast<T *>(conv_state));
 }
 
+// The exact zero-order hold and the short convolution are separate instantiations.
+template <typename T>
+void dispatch_step(bool zoh, bool conv, bool pair, unsigned grid, int threads, cudaStream_t stream, int64_t batch,
+                   int64_t dim, int N, int sp, const void *x, const void *dt, const void *z, const void *Bm,
+                   const void *Cm, const float *A, const float *Dskip, const float *dt_bias, float *h, void *y,
+                   const float *conv_w, const float *conv_b, void *conv_state) {
+    if (conv) {
+        if (zoh)
+            launch_step<T, true, true>(pair, grid, threads, stream, batch, dim, N, sp, x, dt, z, Bm, Cm, A, Dskip,
+                                       dt_bias, h, y, conv_w, conv_b, conv_state);
+        else
+            launch_step<T, false, true>(pair, grid, threads, stream, batch, dim, N, sp, x, dt, z, Bm, Cm, A, Dskip,
+                                        dt_bias, h, y, conv_w, conv_b, conv_state);
+    } else {
+        if (zoh)
+            launch_step<T, true, false>(pair, grid, threads, stream, batch, dim, N, sp, x, dt, z, Bm, Cm, A, Dskip,
+                                        dt_bias, h, y, nullptr, nullptr, nullptr);
+        else
+            launch_step<T, false, false>(pair, grid, threads, stream, batch, dim, N, sp, x, dt, z, Bm, Cm, A, Dskip,
+                                         dt_bias, h, y, nullptr, nullptr, nullptr);
+    }
+}
+
+// Checks and launch of one decode step; conv_w == NULL: no short convolution.
+ssm_status step_impl(int64_t batch, int64_t dim, int64_t dstate, ssm_dtype dtype, uint32_t flags, const void *x,
+                     const void *dt, const void *z, const void *Bm, const void *Cm, const float *A,
+                     const float *Dskip, const float *dt_bias, const float *conv_w, const float *conv_b,
+                     void *conv_state, float *h, void *y, void *stream_) {
+    ssm_status s = check_common(batch, dim, dstate, dtype, flags);
+    if (s != SSM_OK) return s;
+    if (batch == 0 || dim == 0) return SSM_OK;
+    if (!x || !dt || !Bm || !Cm || !A || !h || !y) return SSM_ERR_INVALID;
+    const bool conv = conv_w != nullptr;
+    if (conv && !conv_state) return SSM_ERR_INVALID;
+    const size_t es = dtype == SSM_BF16 ? 2 : 4;
+    const void *pes[] = {x, dt, z, Bm, Cm, y, conv_state};
+    for (const void *p : pes)
+        if (p && !aligned(p, es)) return SSM_ERR_UNSUPPORTED;
+    const void *p4[] = {A, Dskip, dt_bias, conv_b};
+    for (const void *p : p4)
+        if (p && !aligned(p, 4)) return SSM_ERR_UNSUPPORTED;
+    if (conv && !aligned(conv_w, 16)) return SSM_ERR_UNSUPPORTED;
+    if (!aligned(h, dstate == kMaxN ? 16 : 4)) return SSM_ERR_UNSUPPORTED;  // float4 state rows when N = 16
+    cudaStream_t stream = static_cast<cudaStream_t>(stream_);
+    const int64_t nch = batch * dim;
+    const int sp = (flags & SSM_DELTA_SOFTPLUS) != 0;
+    const bool zoh = (flags & SSM_EXACT_ZOH) != 0;
+    // Two threads per channel when the state rows are whole float4 rows and B, C rows
+    // can be read four elements at a time; one thread per channel otherwise.
+    const bool pair = dstate == kMaxN && aligned(A, 16) && aligned(Bm, 4 * es) && aligned(Cm, 4 * es);
+    const int threads = pair ? 256 : 128;
+    const int64_t blocks = ((pair ? 2 : 1) * nch + threads - 1) / threads;
+    if (blocks > INT32_MAX) return SSM_ERR_UNSUPPORTED;
+    const unsigned grid = unsigned(blocks);
+    if (dtype == SSM_BF16)
+        dispatch_step<__nv_bfloat16>(zoh, conv, pair, grid, threads, stream, batch, dim, int(dstate), sp, x, dt, z,
+                                     Bm, Cm, A, Dskip, dt_bias, h, y, conv_w, conv_b, conv_state);
+    else
+        dispatch_step<float>(zoh, conv, pair, grid, threads, stream, batch, dim, int(dstate), sp, x, dt, z, Bm, Cm,
+                             A, Dskip, dt_bias, h, y, conv_w, conv_b, conv_state);
+    return cudaGetLastError() == cudaSuccess ? SSM_OK : SSM_ERR_CUDA;
+}
+
+
+}  // namespace
 
 extern "C" {
 
@@ -467,46 +582,18 @@ ssm_status ssm_scan_fwd(const ssm_scan_args *a, void *stream_) {
 
 ssm_status ssm_step(int64_t batch, int64_t dim, int64_t dstate, ssm_dtype dtype, uint32_t flags, const void *x,
                     const void *dt, const void *z, const void *Bm, const void *Cm, const float *A,
-                    const float *Dskip, const float *dt_bias, float *h, void *y, void *stream_) {
-    ssm_status s = check_common(batch, dim, dstate, dtype, flags);
-    if (s != SSM_OK) return s;
-    if (batch == 0 || dim == 0) return SSM_OK;
-    if (!x || !dt || !Bm || !Cm || !A || !h || !y) return SSM_ERR_INVALID;
-    const size_t es = dtype == SSM_BF16 ? 2 : 4;
-    const void *pes[] = {x, dt, z, Bm, Cm, y};
-    for (const void *p : pes)
-        if (p && !aligned(p, es)) return SSM_ERR_UNSUPPORTED;
-    const void *p4[] = {A, Dskip, dt_bias};
-    for (const void *p : p4)
-        if (p && !aligned(p, 4)) return SSM_ERR_UNSUPPORTED;
-    if (!aligned(h, dstate == kMaxN ? 16 : 4)) return SSM_ERR_UNSUPPORTED;  // float4 state rows when N = 16
-    cudaStream_t stream = static_cast<cudaStream_t>(stream_);
-    const int64_t nch = batch * dim;
-    const int sp = (flags & SSM_DELTA_SOFTPLUS) != 0;
-    const int zoh = (flags & SSM_EXACT_ZOH) != 0;
-    // Two threads per channel when the state rows are whole float4 rows and B, C rows
-    // can be read four elements at a time; one thread per channel otherwise.
-    const bool pair = dstate == kMaxN && aligned(A, 16) && aligned(Bm, 4 * es) && aligned(Cm, 4 * es);
-    const int threads = pair ? 256 : 128;
-    const int64_t blocks = ((pair ? 2 : 1) * nch + threads - 1) / threads;
-    if (blocks > INT32_MAX) return SSM_ERR_UNSUPPORTED;
-    const unsigned grid = unsigned(blocks);
-    if (dtype == SSM_BF16) {
-        if (zoh)
-            launch_step<__nv_bfloat16, true>(pair, grid, threads, stream, batch, dim, int(dstate), sp, x, dt, z, Bm,
-                                             Cm, A, Dskip, dt_bias, h, y);
-        else
-            launch_step<__nv_bfloat16, false>(pair, grid, threads, stream, batch, dim, int(dstate), sp, x, dt, z,
-                                              Bm, Cm, A, Dskip, dt_bias, h, y);
-    } else {
-        if (zoh)
-            launch_step<float, true>(pair, grid, threads, stream, batch, dim, int(dstate), sp, x, dt, z, Bm, Cm, A,
-                                     Dskip, dt_bias, h, y);
-        else
-            launch_step<float, false>(pair, grid, threads, stream, batch, dim, int(dstate), sp, x, dt, z, Bm, Cm, A,
-                                      Dskip, dt_bias, h, y);
-    }
-    return cudaGetLastError() == cudaSuccess ? SSM_OK : SSM_ERR_CUDA;
+                    const float *Dskip, const float *dt_bias, float *h, void *y, void *stream) {
+    return step_impl(batch, dim, dstate, dtype, flags, x, dt, z, Bm, Cm, A, Dskip, dt_bias, nullptr, nullptr, nullptr,
+                     h, y, stream);
+}
+
+ssm_status ssm_step_conv(int64_t batch, int64_t dim, int64_t dstate, ssm_dtype dtype, uint32_t flags,
+                         const void *x, const void *dt, const void *z, const void *Bm, const void *Cm,
+                         const float *A, const float *Dskip, const float *dt_bias, const float *conv_w,
+                         const float *conv_b, void *conv_state, float *h, void *y, void *stream) {
+    if (!conv_w) return SSM_ERR_INVALID;
+    return step_impl(batch, dim, dstate, dtype, flags, x, dt, z, Bm, Cm, A, Dskip, dt_bias, conv_w, conv_b,
+                     conv_state, h, y, stream);
 }
 
 ssm_status ssm_workspace_status(const void *workspace, void *stream_) {

@@ -42,9 +42,10 @@
 // Short convolution (the CONV instantiations): the block's causal depthwise conv1d of
 // width 4 and SiLU in front of the SSM, u_t = silu(cb + sum_k w_k x_{t-3+k}) (Mamba
 // summary, block-architecture paragraph). The x box of every stage carries the three
-// rows before the tile (TMA fills rows before t = 0 with zeros, or the prologue and
-// epilogue take them from the caller's prefix), and both P and E evaluate u from it:
-// P for Delta u, E for D u. Nothing else changes, and x still crosses HBM once.
+// rows before the tile (TMA fills rows before t = 0 with zeros, or the prologue takes
+// them from the caller's prefix). P evaluates u once per (t, channel), uses it for Delta
+// u and writes it, in the token type, over the dt rows it has just read; E reads u there
+// for D u in place of x. x still crosses HBM once.
 //
 // Exponentials: Abar_n = 2^(Delta log2 e * A[d,n]) on the SFU (ex2.approx). Where
 // every row of A in the block is an arithmetic progression in n (A[d,n] = A[d,0] +
@@ -355,9 +356,9 @@ __device__ __forceinline__ bool conv_prefix(const Params &p, const long long g, 
 // Delta log2 e), with Delta = softplus(dt + bias) (or dt + bias); with `zoh` (exact
 // zero-order hold) u = x, the consumers apply the weight. Rows at or past tlen get
 // (0, 0): Abar = 1, no input. CONV: x is the short convolution's output (cw, cb, and
-// use_x0 / x0 as for conv_silu_rows).
+// use_x0 / x0 as for conv_silu_rows), which is also written over the dt rows read.
 template <typename T, bool CONV>
-__device__ __forceinline__ void prologue_rows(const T *__restrict__ sx, const T *__restrict__ sdt,
+__device__ __forceinline__ void prologue_rows(const T *__restrict__ sx, T *__restrict__ sdt,
                                               float2 *__restrict__ rec, const int t0, const int tlen,
                                               const float bias, const bool softplus, const bool zoh,
                                               const float4 cw, const float cb, const bool use_x0, const float3 x0) {
@@ -390,21 +391,26 @@ __device__ __forceinline__ void prologue_rows(const T *__restrict__ sx, const T 
         rec[t * CH] = t < tlen ? f2(u[q].x, dl[q].x) : f2(0.f, 0.f);
         rec[(t + 1) * CH] = t + 1 < tlen ? f2(u[q].y, dl[q].y) : f2(0.f, 0.f);
     }
+    if (CONV) {  // the epilogue's D u
+#pragma unroll
+        for (int q = 0; q < NPR; ++q) {
+            const int t = t0 + 2 * q;
+            sdt[t * CH] = Tok<T>::from_f(xv[q].x);
+            sdt[(t + 1) * CH] = Tok<T>::from_f(xv[q].y);
+        }
+    }
 }
 
 // ---------------------------------------------------------------- epilogue
 // y for TE steps (rows t0 .. t0+TE-1) of channel c: sum of the four consumer
-// partials, + D x, times silu(z), rounded to T. CONV: x is the short convolution's
-// output, recomputed here from the stage (as in the prologue).
-template <typename T, bool CONV>
+// partials, + D x, times silu(z), rounded to T. (With the short convolution sx points
+// at the u rows the prologue wrote.)
+template <typename T>
 __device__ __forceinline__ void epilogue_rows(const float4 *__restrict__ part, const T *__restrict__ sx,
                                               const T *__restrict__ sz, T *__restrict__ yo, const int t0,
-                                              const float dd, const bool gate, const float4 cw, const float cb,
-                                              const bool use_x0, const float3 x0) {
+                                              const float dd, const bool gate) {
     constexpr int NB = TE / 4;  // blocks of four steps
     float2 y01[NB], y23[NB];
-    float2 xc[CONV ? TE / 2 : 1];
-    if constexpr (CONV) conv_silu_rows<T, TE / 2>(sx, t0, cw, cb, use_x0, x0, xc);
 #pragma unroll
     for (int b = 0; b < NB; ++b) {
         const int blk = t0 / 4 + b;
@@ -418,9 +424,8 @@ __device__ __forceinline__ void epilogue_rows(const float4 *__restrict__ part, c
         lo = __fadd2_rn(lo, lo2);
         hi = __fadd2_rn(hi, hi2);
         const int t = t0 + 4 * b;
-        const float2 x01 = CONV ? xc[2 * b] : f2(Tok<T>::to_f(sx[t * CH]), Tok<T>::to_f(sx[(t + 1) * CH]));
-        const float2 x23 =
-            CONV ? xc[2 * b + 1] : f2(Tok<T>::to_f(sx[(t + 2) * CH]), Tok<T>::to_f(sx[(t + 3) * CH]));
+        const float2 x01 = f2(Tok<T>::to_f(sx[t * CH]), Tok<T>::to_f(sx[(t + 1) * CH]));
+        const float2 x23 = f2(Tok<T>::to_f(sx[(t + 2) * CH]), Tok<T>::to_f(sx[(t + 3) * CH]));
         y01[b] = __ffma2_rn(f2(dd, dd), x01, lo);
         y23[b] = __ffma2_rn(f2(dd, dd), x23, hi);
     }
@@ -556,8 +561,7 @@ __global__ void __launch_bounds__(NTHREADS, C::MINB)
         // ================================================================ E: epilogue
         const int h = warp - WARP_E0;
         const int c = lane;
-        float dd = 0.f, cb = 0.f;
-        float4 cw = make_float4(0.f, 0.f, 0.f, 0.f);
+        float dd = 0.f;
         for (int i = 0;; ++i) {
             const int pr = i % R_PART, st = i % STAGES;
             if (!warp_wait(&bar_part_full[pr], uint32_t(i / R_PART) & 1u)) {
@@ -573,16 +577,14 @@ __global__ void __launch_bounds__(NTHREADS, C::MINB)
             if (m.flags & F_FIRST) {
                 const int64_t d = (m.g % p.Dg) * CH + c;
                 dd = (d < p.D && p.Dskip) ? __ldg(p.Dskip + d) : 0.f;
-                if (CONV) load_conv(p, d, cw, cb);
             }
-            float3 x0 = make_float3(0.f, 0.f, 0.f);
-            const bool use_x0 = CONV && h == 0 && m.t0 == 0 && conv_prefix<T>(p, m.g, c, x0);
             const unsigned char *stage = smem + S::stage_off + size_t(st) * S::stage_bytes;
-            const T *sx = reinterpret_cast<const T *>(stage + S::st_x) + S::HALO * CH + c;
+            // the SSM's input: x, or the short convolution's u that P left in the dt rows
+            const T *sx = reinterpret_cast<const T *>(stage + (CONV ? S::st_dt : S::st_x)) + c;
             const T *sz = reinterpret_cast<const T *>(stage + S::st_z) + c;
             const float4 *part = reinterpret_cast<const float4 *>(smem + S::part_off + pr * S::part_bytes) + c;
             T *yo = reinterpret_cast<T *>(smem + S::yout_off + (i % YBUF) * S::yout_bytes) + c;
-            epilogue_rows<T, CONV>(part, sx, sz, yo, h * TE, dd, p.has_gate != 0, cw, cb, use_x0, x0);
+            epilogue_rows<T>(part, sx, sz, yo, h * TE, dd, p.has_gate != 0);
             warp_arrive(&bar_part_free[pr]);  // the consumers may reuse this partial slot
             warp_arrive(&bar_sfree[st]);      // x and z of this stage are no longer needed
             fence_proxy_async_smem();         // y rows written by this thread -> visible to the TMA store
@@ -644,8 +646,11 @@ __global__ void __launch_bounds__(NTHREADS, C::MINB)
             float3 x0 = make_float3(0.f, 0.f, 0.f);
             const bool use_x0 = CONV && h == 0 && m.t0 == 0 && conv_prefix<T>(p, m.g, c, x0);
             prologue_rows<T, CONV>(reinterpret_cast<const T *>(stage + S::st_x) + S::HALO * CH + c,
-                                   reinterpret_cast<const T *>(stage + S::st_dt) + c, rec, h * TP, m.tlen, bias_c,
-                                   p.softplus != 0, ZOH, cw, cb, use_x0, x0);
+                                   reinterpret_cast<T *>(smem + S::stage_off + size_t(st) * S::stage_bytes +
+                                                         S::st_dt) + c,
+                                   rec, h * TP, m.tlen, bias_c, p.softplus != 0, ZOH, cw, cb, use_x0, x0);
+            // u written over dt: order it before the TMA refill of this stage (async proxy)
+            if (CONV) fence_proxy_async_smem();
             // B and C rows of this half widened to float32: row t = [B_0 .. B_15 | C_0 .. C_15],
             // in 16-byte chunks; chunk id = q * 32 + lane covers row h*TP + id / 8 and chunk
             // id % 8 (0-3: B, 4-7: C), so eight consecutive lanes write one 128-byte row.

@@ -152,6 +152,23 @@ def test_step_rejects_on_host(lib):
     assert call(0, 32, 16, 1, 1, *ptrs, None) == _native.SSM_OK
 
 
+def test_step_conv_rejects_on_host(lib):
+    """ssm_step_conv: the taps and the window are required; alignment as documented."""
+    f = 1 << 20
+    p = [f + (i << 16) for i in range(15)]
+    # x dt z Bm Cm A Dskip dt_bias conv_w conv_b conv_state h y
+    args = lambda **kw: [kw.get(k, v) for k, v in zip(
+        ("x", "dt", "z", "Bm", "Cm", "A", "Dskip", "dt_bias", "conv_w", "conv_b", "conv_state", "h", "y"), p)]
+    call = lambda *a: lib.ssm_step_conv(2, 32, 16, 1, 1, *a, None)
+    assert call(*args(conv_w=None)) == _native.SSM_ERR_INVALID
+    assert call(*args(conv_state=None)) == _native.SSM_ERR_INVALID
+    assert call(*args(conv_w=f + 4)) == _native.SSM_ERR_UNSUPPORTED      # taps on 16 bytes
+    assert call(*args(conv_b=f + 2)) == _native.SSM_ERR_UNSUPPORTED      # bias on 4 bytes
+    assert call(*args(conv_state=f + 1)) == _native.SSM_ERR_UNSUPPORTED  # bf16 window on 2 bytes
+    assert lib.ssm_step_conv(2, 32, 17, 1, 1, *args(), None) == _native.SSM_ERR_UNSUPPORTED
+    assert lib.ssm_step_conv(0, 32, 16, 1, 1, *args(), None) == _native.SSM_OK
+
+
 def test_python_binding_refuses_cpu_tensors():
     import torch
     import selective_state_space_47_b200 as ssm

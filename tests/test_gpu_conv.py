@@ -12,7 +12,7 @@ import torch
 
 from selective_state_space_47_b200 import synth
 from tests.conftest import cuda_available
-from tests.gpu_util import TOL, dtype_name, h_err, oracle_scan, y_err
+from tests.gpu_util import TOL, dtype_name, h_err, oracle_scan, rowwise_rel, y_err
 
 pytestmark = pytest.mark.gpu
 
@@ -100,3 +100,52 @@ def test_host_path_with_conv_equals_device_path(ssm, chunk):
     torch.cuda.synchronize()
     assert torch.equal(y_host, y_dev.cpu())
     assert torch.equal(h_host, h_dev)
+
+
+@pytest.mark.parametrize("N", [16, 5])
+def test_conv_step_matches_oracle(ssm, N):
+    """Decode behind the short convolution: 20 chained steps of ssm_step_conv (two threads
+    per channel for N = 16, one for N = 5) against the oracle's step; the window ends as
+    the last three tokens, bit for bit."""
+    import oracle
+    Bsz, Dm, steps = 4, 96, 20
+    inp = synth.step_inputs(Bsz, Dm, N, steps, torch.bfloat16, seed=58)
+    conv = synth.conv_params(Dm, Bsz, torch.bfloat16, seed=59)
+    dev, cv = _cuda(inp), _cuda(conv)
+    h = dev["h"].clone()
+    hr = inp["h"].double().numpy().copy()
+    win = cv["conv_x0"].clone()
+    st = synth.to_numpy_storage
+    win_r = st(conv["conv_x0"]).copy()
+    worst = 0.0
+    for s in range(steps):
+        y = ssm.step(dev["x"][s], dev["dt"][s], dev["A"], dev["B"][s], dev["C"][s], h, dev["D"], dev["z"][s],
+                     dev["dt_bias"], conv_w=cv["conv_w"], conv_b=cv["conv_b"], conv_state=win)
+        yr = oracle.step(st(inp["x"][s]), st(inp["dt"][s]), inp["A"].numpy(), st(inp["B"][s]), st(inp["C"][s]),
+                         hr, D=inp["D"].numpy(), z=st(inp["z"][s]), dt_bias=inp["dt_bias"].numpy(), dtype="bf16",
+                         conv_w=conv["conv_w"].numpy(), conv_b=conv["conv_b"].numpy(), conv_state=win_r)
+        worst = max(worst, rowwise_rel(y.float().cpu().numpy(), yr, axis=1))
+    torch.cuda.synchronize()
+    print(f"conv step N={N}: y {worst:.2e}")
+    assert worst <= 1e-2
+    assert rowwise_rel(h.cpu().numpy(), hr, axis=2) <= 1e-2
+    assert torch.equal(win.cpu(), inp["x"][steps - 3:].permute(1, 0, 2))
+
+
+def test_prefill_then_conv_step_continues_the_sequence(ssm):
+    """A scan with the convolution over L tokens, then one ssm_step_conv from its final
+    state and last three tokens, gives the oracle's y at t = L of the L + 1 token scan."""
+    Bsz, L, Dm, N = 2, 77, 64, 16
+    inp = synth.scan_inputs(Bsz, L + 1, Dm, N, torch.float32, seed=60, gate=True, h0=True)
+    conv = synth.conv_params(Dm, Bsz, torch.float32, seed=61)
+    y_ref, _ = oracle_scan(inp, conv=conv)
+    dev, cv = _cuda(inp), _cuda(conv)
+    pre = {k: dev[k][:, :L].contiguous() for k in ("x", "dt", "z", "B", "C")}
+    _, hL = ssm.scan_fwd(pre["x"], pre["dt"], dev["A"], pre["B"], pre["C"], dev["D"], pre["z"], dev["dt_bias"],
+                         dev["h0"], return_last_state=True, **cv)
+    win = dev["x"][:, L - 3:L].contiguous()
+    y = ssm.step(dev["x"][:, L].contiguous(), dev["dt"][:, L].contiguous(), dev["A"], dev["B"][:, L].contiguous(),
+                 dev["C"][:, L].contiguous(), hL, dev["D"], dev["z"][:, L].contiguous(), dev["dt_bias"],
+                 conv_w=cv["conv_w"], conv_b=cv["conv_b"], conv_state=win)
+    torch.cuda.synchronize()
+    assert rowwise_rel(y.cpu().numpy(), y_ref[:, L], axis=1) <= 1e-4
