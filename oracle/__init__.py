@@ -30,6 +30,8 @@ def _open(path):
     lib.oracle_step_f64.restype = c_int
     lib.oracle_step_conv_f64.argtypes = [i64, i64, i64, c_int, c_uint] + [vp] * 13 + [c_int]
     lib.oracle_step_conv_f64.restype = c_int
+    lib.oracle_scan_bwd_f64.argtypes = [i64, i64, i64, i64, c_int, c_uint] + [vp] * 20
+    lib.oracle_scan_bwd_f64.restype = c_int
     return lib
 
 
@@ -72,6 +74,10 @@ class Oracle:
         return _scan(self.lib, x, dt, A, B, C, D, z, dt_bias, h0, dtype, delta_softplus,
                      exact_zoh, nthreads, conv_w, conv_b, conv_x0)
 
+    def scan_bwd(self, x, dt, A, B, C, dy, D=None, z=None, dt_bias=None, h0=None, dh_last=None,
+                 dtype="f32", delta_softplus=True):
+        return _scan_bwd(self.lib, x, dt, A, B, C, dy, D, z, dt_bias, h0, dh_last, dtype, delta_softplus)
+
     def step(self, x, dt, A, B, C, h, D=None, z=None, dt_bias=None, dtype="f32",
              delta_softplus=True, exact_zoh=False, nthreads=None, conv_w=None, conv_b=None,
              conv_state=None):
@@ -97,6 +103,11 @@ def scan(*args, **kw):
 def step(*args, **kw):
     """One decode step with the default oracle build; see ``_step``."""
     return default().step(*args, **kw)
+
+
+def scan_bwd(*args, **kw):
+    """Backward of the scan with the default oracle build; see ``_scan_bwd``."""
+    return default().scan_bwd(*args, **kw)
 
 
 def _scan(lib, x, dt, A, B, C, D=None, z=None, dt_bias=None, h0=None, dtype="f32",
@@ -188,3 +199,39 @@ def _step(lib, x, dt, A, B, C, h, D=None, z=None, dt_bias=None, dtype="f32",
     if rc != 0:
         raise ValueError("oracle step rejected its arguments")
     return y
+
+
+def _scan_bwd(lib, x, dt, A, B, C, dy, D=None, z=None, dt_bias=None, h0=None, dh_last=None, dtype="f32",
+              delta_softplus=True):
+    """Gradients of the scan (default discretisation, no convolution) given dy = dL/dy
+    ([Bsz, L, Dm], token storage type) and dh_last = dL/dh_L ([Bsz, Dm, N] float64 or None).
+    Returns a dict of float64 arrays: dx, ddt, dz (None without z) [Bsz, L, Dm]; dB, dC
+    [Bsz, L, N]; dA [Dm, N]; dD, ddt_bias [Dm]; dh0 [Bsz, Dm, N]."""
+    Bsz, L, Dm = np.shape(x)
+    N = np.shape(A)[1]
+    x = _tok(x, dtype, (Bsz, L, Dm), "x")
+    dt = _tok(dt, dtype, (Bsz, L, Dm), "dt")
+    z = None if z is None else _tok(z, dtype, (Bsz, L, Dm), "z")
+    B = _tok(B, dtype, (Bsz, L, N), "B")
+    C = _tok(C, dtype, (Bsz, L, N), "C")
+    dy = _tok(dy, dtype, (Bsz, L, Dm), "dy")
+    A = _f32(A, (Dm, N), "A")
+    D = _f32(D, (Dm,), "D")
+    dt_bias = _f32(dt_bias, (Dm,), "dt_bias")
+    h0 = _f32(h0, (Bsz, Dm, N), "h0")
+    if dh_last is not None:
+        dh_last = np.ascontiguousarray(dh_last, dtype=np.float64)
+        if dh_last.shape != (Bsz, Dm, N):
+            raise ValueError("dh_last must have shape [Bsz, Dm, N]")
+    out = dict(dx=np.empty((Bsz, L, Dm)), ddt=np.empty((Bsz, L, Dm)),
+               dz=None if z is None else np.empty((Bsz, L, Dm)), dB=np.empty((Bsz, L, N)),
+               dC=np.empty((Bsz, L, N)), dA=np.empty((Dm, N)), dD=np.empty(Dm), ddt_bias=np.empty(Dm),
+               dh0=np.empty((Bsz, Dm, N)))
+    rc = lib.oracle_scan_bwd_f64(Bsz, L, Dm, N, 0 if dtype == "f32" else 1, DELTA_SOFTPLUS if delta_softplus else 0,
+                                 _ptr(x), _ptr(dt), _ptr(z), _ptr(B), _ptr(C), _ptr(A), _ptr(D), _ptr(dt_bias),
+                                 _ptr(h0), _ptr(dy), _ptr(dh_last), _ptr(out["dx"]), _ptr(out["ddt"]),
+                                 _ptr(out["dz"]), _ptr(out["dB"]), _ptr(out["dC"]), _ptr(out["dA"]), _ptr(out["dD"]),
+                                 _ptr(out["ddt_bias"]), _ptr(out["dh0"]))
+    if rc != 0:
+        raise ValueError("oracle_scan_bwd_f64 rejected its arguments")
+    return out

@@ -46,6 +46,7 @@
 #include <math.h>
 #include <pthread.h>
 #include <stdint.h>
+#include <stdlib.h>
 #include <string.h>
 
 #define ORACLE_DELTA_SOFTPLUS 1u /* Delta = softplus(dt + dt_bias); else Delta = dt + dt_bias */
@@ -237,5 +238,107 @@ int oracle_step_conv_f64(int64_t Bsz, int64_t Dm, int64_t N, int dtype, unsigned
     scan_job base = {Bsz, 1, Dm, N, dtype, flags, x, dt, z, Bm, Cm, A, Dskip, dt_bias, NULL,
                      y, h, h, 0, Bsz * Dm, conv_w, conv_b, conv_state};
     run_jobs(&base, nthreads);
+    return 0;
+}
+
+/*
+ * Backward of the scan: the gradients of a loss with respect to every input, given
+ * dL/dy (dy, storage type of the tokens) and optionally dL/dh_L (dh_last, double, or
+ * NULL for 0). The pages print no backward formulas; the plain definition is the
+ * derivative of the forward above, and this is reverse-mode differentiation of it,
+ * written step by step. The Mamba summary's hardware-aware paragraph (recomputation)
+ * says the backward recomputes the states instead of storing them; here, on the CPU,
+ * each channel's forward states are simply kept for its reverse sweep.
+ *
+ * Per channel (b, d), with v_t = dt_t + bias, Delta_t = softplus(v_t) (or v_t),
+ * Abar_tn = exp(Delta_t A_n), q_t = C_t . h_t + D x_t and y_t = q_t silu(z_t) (or q_t):
+ *   dq_t = dy_t silu(z_t);  dz_t = dy_t q_t silu'(z_t)
+ *   g_t  = dL/dh_t = dq_t C_t + Abar_{t+1} g_{t+1},  g_L = dq_L C_L + dh_last
+ *   dx_t = dq_t D + sum_n g_tn Delta_t B_tn
+ *   dDelta_t = sum_n g_tn (A_n Abar_tn h_{t-1,n} + B_tn x_t);  ddt_t = dDelta_t sigma(v_t)
+ *   dA_n += g_tn Delta_t Abar_tn h_{t-1,n};  dB_tn += g_tn Delta_t x_t;  dC_tn += dq_t h_tn
+ *   dD += dq_t x_t;  dbias += ddt_t;  dh0 = Abar_1 g_1
+ * dB, dC ([Bsz, L, N]) sum over the channels of a sequence; dA ([Dm, N]), dD and dbias
+ * ([Dm]) over sequences and time. Only the default discretisation (Bbar = Delta B) and
+ * no convolution. Single-threaded. Returns 0, or -1 on invalid arguments.
+ */
+int oracle_scan_bwd_f64(int64_t Bsz, int64_t L, int64_t Dm, int64_t N, int dtype, unsigned flags,
+                        const void *x, const void *dt, const void *z, const void *Bm, const void *Cm,
+                        const float *A, const float *Dskip, const float *dt_bias, const float *h0,
+                        const void *dy, const double *dh_last, double *dx, double *ddt, double *dz,
+                        double *dB, double *dC, double *dA, double *dD, double *dbias, double *dh0) {
+    if (Bsz < 0 || L < 0 || Dm < 0 || N < 1 || N > 256 || (dtype != 0 && dtype != 1)) return -1;
+    if (flags & ~ORACLE_DELTA_SOFTPLUS) return -1;
+    if (!x || !dt || !Bm || !Cm || !A || !dy || !dx || !ddt || !dB || !dC || !dA || !dD || !dbias) return -1;
+    if (z && !dz) return -1;
+    const int softplus_on = (flags & ORACLE_DELTA_SOFTPLUS) != 0;
+    memset(dB, 0, sizeof(double) * (size_t)(Bsz * L * N));
+    memset(dC, 0, sizeof(double) * (size_t)(Bsz * L * N));
+    memset(dA, 0, sizeof(double) * (size_t)(Dm * N));
+    memset(dD, 0, sizeof(double) * (size_t)Dm);
+    memset(dbias, 0, sizeof(double) * (size_t)Dm);
+    /* forward states of one channel: hs[t * N + n] = h_{t-1,n} for t = 0..L (hs[0] = h0) */
+    double *hs = (double *)malloc(sizeof(double) * (size_t)((L + 1) * N));
+    double *delta = (double *)malloc(sizeof(double) * (size_t)(L > 0 ? L : 1));
+    double *g = (double *)malloc(sizeof(double) * (size_t)N);
+    if (!hs || !delta || !g) {
+        free(hs);
+        free(delta);
+        free(g);
+        return -1;
+    }
+    for (int64_t b = 0; b < Bsz; b++) {
+        for (int64_t d = 0; d < Dm; d++) {
+            const double bias = dt_bias ? (double)dt_bias[d] : 0.0;
+            const double dsk = Dskip ? (double)Dskip[d] : 0.0;
+            for (int64_t n = 0; n < N; n++) hs[n] = h0 ? (double)h0[(b * Dm + d) * N + n] : 0.0;
+            /* forward, keeping every state */
+            for (int64_t t = 0; t < L; t++) {
+                const int64_t i = (b * L + t) * Dm + d, bc = (b * L + t) * N;
+                const double v = widen(dt, dtype, i) + bias;
+                delta[t] = softplus_on ? softplus(v) : v;
+                const double xv = widen(x, dtype, i);
+                for (int64_t n = 0; n < N; n++)
+                    hs[(t + 1) * N + n] = exp(delta[t] * (double)A[d * N + n]) * hs[t * N + n] +
+                                          delta[t] * widen(Bm, dtype, bc + n) * xv;
+            }
+            /* reverse */
+            for (int64_t n = 0; n < N; n++) g[n] = dh_last ? dh_last[(b * Dm + d) * N + n] : 0.0;
+            for (int64_t t = L - 1; t >= 0; t--) {
+                const int64_t i = (b * L + t) * Dm + d, bc = (b * L + t) * N;
+                const double xv = widen(x, dtype, i);
+                double q = dsk * xv;
+                for (int64_t n = 0; n < N; n++) q += widen(Cm, dtype, bc + n) * hs[(t + 1) * N + n];
+                double dq = widen(dy, dtype, i);
+                if (z) {
+                    const double zv = widen(z, dtype, i), sg = sigmoid(zv);
+                    dz[i] = dq * q * sg * (1.0 + zv * (1.0 - sg));
+                    dq *= zv * sg;
+                }
+                double dxv = dq * dsk, ddel = 0.0;
+                dD[d] += dq * xv;
+                for (int64_t n = 0; n < N; n++) {
+                    const double a = (double)A[d * N + n], abar = exp(delta[t] * a);
+                    const double bn = widen(Bm, dtype, bc + n), hp = hs[t * N + n];
+                    g[n] += dq * widen(Cm, dtype, bc + n);
+                    dC[bc + n] += dq * hs[(t + 1) * N + n];
+                    dxv += g[n] * delta[t] * bn;
+                    ddel += g[n] * (a * abar * hp + bn * xv);
+                    dA[d * N + n] += g[n] * delta[t] * abar * hp;
+                    dB[bc + n] += g[n] * delta[t] * xv;
+                    g[n] *= abar; /* now dL/dh_{t-1} through h_t */
+                }
+                const double v = widen(dt, dtype, i) + bias;
+                ddt[i] = softplus_on ? ddel * sigmoid(v) : ddel;
+                dbias[d] += ddt[i];
+                dx[i] = dxv;
+            }
+            if (dh0)
+                for (int64_t n = 0; n < N; n++) dh0[(b * Dm + d) * N + n] = g[n];
+        }
+    }
+    free(hs);
+    free(delta);
+    free(g);
     return 0;
 }

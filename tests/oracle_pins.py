@@ -458,3 +458,77 @@ def pin_conv_step_matches_conv_scan(orc, seed=14):
 
 
 ALL_PINS += [pin_conv_front_end, pin_conv_front_end_bf16, pin_conv_step_matches_conv_scan]
+
+
+def _bwd_case(rng, Bsz, L, Dm, N, gate=True):
+    f = lambda *shape: rng.standard_normal(shape).astype(np.float32)
+    return dict(x=f(Bsz, L, Dm), dt=(0.7 * f(Bsz, L, Dm)).astype(np.float32), z=f(Bsz, L, Dm) if gate else None,
+                B=f(Bsz, L, N), C=f(Bsz, L, N), A=(-0.2 - rng.random((Dm, N)) * 2.0).astype(np.float32),
+                D=f(Dm), dt_bias=(0.5 * f(Dm)).astype(np.float32), h0=f(Bsz, Dm, N))
+
+
+def pin_bwd_finite_differences(orc, seed=15, softplus=True, gate=True):
+    """Every gradient of the backward equals the central difference of the forward.
+
+    The loss is L = sum(dy * y) + sum(dh_last * h_L) with random dy, dh_last, so dL/dp is
+    what the backward returns for dy, dh_last. Each input element p (float32) is moved by
+    +-2^-12, exactly representable, and (L(p+) - L(p-)) / (p+ - p-) is compared with the
+    gradient (truncation ~1e-7 relative at this step). A plain derivative check, by a
+    route independent of the reverse sweep."""
+    rng = _rng(seed)
+    Bsz, L, Dm, N = 2, 6, 3, 3
+    inp = _bwd_case(rng, Bsz, L, Dm, N, gate)
+    dy = rng.standard_normal((Bsz, L, Dm)).astype(np.float32)
+    dh_last = rng.standard_normal((Bsz, Dm, N))
+
+    def loss(v):
+        y, h = orc.scan(v["x"], v["dt"], v["A"], v["B"], v["C"], D=v["D"], z=v["z"], dt_bias=v["dt_bias"],
+                        h0=v["h0"], delta_softplus=softplus)
+        return float(np.sum(dy * y) + np.sum(dh_last * h))
+
+    g = orc.scan_bwd(inp["x"], inp["dt"], inp["A"], inp["B"], inp["C"], dy, D=inp["D"], z=inp["z"],
+                     dt_bias=inp["dt_bias"], h0=inp["h0"], dh_last=dh_last, delta_softplus=softplus)
+    names = {"x": "dx", "dt": "ddt", "z": "dz", "B": "dB", "C": "dC", "A": "dA", "D": "dD",
+             "dt_bias": "ddt_bias", "h0": "dh0"}
+    step = np.float32(2.0 ** -12)
+    for key, gname in names.items():
+        if inp[key] is None:
+            assert g[gname] is None
+            continue
+        fd = np.empty(inp[key].shape)
+        for idx in np.ndindex(inp[key].shape):
+            p0 = inp[key][idx]
+            hi, lo = np.float32(p0 + step), np.float32(p0 - step)
+            inp[key][idx] = hi
+            up = loss(inp)
+            inp[key][idx] = lo
+            down = loss(inp)
+            inp[key][idx] = p0
+            fd[idx] = (up - down) / (float(hi) - float(lo))
+        assert _rel(g[gname] - fd, fd) < 2e-5, f"backward {gname} differs from the central difference"
+
+
+def pin_bwd_finite_differences_plain(orc):
+    """The same without softplus and without the gate."""
+    pin_bwd_finite_differences(orc, seed=16, softplus=False, gate=False)
+
+
+def pin_bwd_bf16_storage(orc, seed=17):
+    """bfloat16 storage is read as its exact float32 values, dy included."""
+    rng = _rng(seed)
+    inp = _bwd_case(rng, 2, 9, 4, 3)
+    dy = rng.standard_normal((2, 9, 4)).astype(np.float32)
+    toks = ("x", "dt", "z", "B", "C")
+    bits = {k: _bf16_bits(inp[k]) for k in toks}
+    vals = {k: _bf16_value(bits[k]).astype(np.float32) for k in toks}
+    dyb = _bf16_bits(dy)
+    g16 = orc.scan_bwd(bits["x"], bits["dt"], inp["A"], bits["B"], bits["C"], dyb, D=inp["D"], z=bits["z"],
+                       dt_bias=inp["dt_bias"], h0=inp["h0"], dtype="bf16")
+    g32 = orc.scan_bwd(vals["x"], vals["dt"], inp["A"], vals["B"], vals["C"],
+                       _bf16_value(dyb).astype(np.float32), D=inp["D"], z=vals["z"], dt_bias=inp["dt_bias"],
+                       h0=inp["h0"])
+    for k in g32:
+        assert np.array_equal(g16[k], g32[k]), f"bf16 backward {k} differs"
+
+
+ALL_PINS += [pin_bwd_finite_differences, pin_bwd_finite_differences_plain, pin_bwd_bf16_storage]

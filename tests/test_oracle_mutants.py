@@ -49,6 +49,15 @@ MUTANTS = {
     "conv_reads_next_token": ("t - (ORACLE_CONV_K - 1) + k", "t - (ORACLE_CONV_K - 2) + k"),
     "conv_skip_uses_raw_x": ("y += dskip * xv;", "y += dskip * widen(J->x, J->dtype, i);"),
     "conv_update_uses_raw_x": ("h[n] = abar * h[n] + bbar * xv;", "h[n] = abar * h[n] + bbar * widen(J->x, J->dtype, i);"),
+    "bwd_gate_derivative": ("dz[i] = dq * q * sg * (1.0 + zv * (1.0 - sg));", "dz[i] = dq * q * sg;"),
+    "bwd_adjoint_decay_first": ("                    g[n] += dq * widen(Cm, dtype, bc + n);\n",
+                                "                    g[n] = g[n] * exp(delta[t] * a) + dq * widen(Cm, dtype, bc + n);\n"),
+    "bwd_dA_without_abar": ("dA[d * N + n] += g[n] * delta[t] * abar * hp;", "dA[d * N + n] += g[n] * delta[t] * hp;"),
+    "bwd_dC_previous_state": ("dC[bc + n] += dq * hs[(t + 1) * N + n];", "dC[bc + n] += dq * hs[t * N + n];"),
+    "bwd_ddt_without_sigmoid": ("ddt[i] = softplus_on ? ddel * sigmoid(v) : ddel;", "ddt[i] = ddel;"),
+    "bwd_dD_ungated": ("dD[d] += dq * xv;", "dD[d] += widen(dy, dtype, i) * xv;"),
+    "bwd_dh_last_ignored": ("g[n] = dh_last ? dh_last[(b * Dm + d) * N + n] : 0.0;", "g[n] = 0.0;"),
+    "bwd_ddelta_drops_input_term": ("ddel += g[n] * (a * abar * hp + bn * xv);", "ddel += g[n] * (a * abar * hp);"),
     "conv_step_ignores_window": ("y, h, h, 0, Bsz * Dm, conv_w, conv_b, conv_state};",
                                  "y, h, h, 0, Bsz * Dm, conv_w, conv_b, NULL};"),
 }
