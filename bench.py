@@ -53,6 +53,8 @@ def parse_args(argv=None):
                     help="skip the e2e, decode, general-A and CPU-baseline legs (profiling runs)")
     ap.add_argument("--seqlen", type=int, default=None,
                     help="shorten the workload's sequence (profiling captures of a smaller case)")
+    ap.add_argument("--bwd-only", action="store_true",
+                    help="time only the backward scan on the workload (profiling runs)")
     ap.add_argument("--decode-only", action="store_true",
                     help="run only the recurrent-decode leg (1000 chained steps) and print its line")
     return ap.parse_args(argv)
@@ -304,6 +306,15 @@ def run_ours(args):
         return 0
     inp = synth.scan_inputs(w.batch, w.seqlen, w.dim, w.dstate, w.dtype, seed=rank_seed(w.seed, rank),
                             device=dev, gate=w.gate)
+    if args.bwd_only:
+        line = {"metric": METRIC, "n_gpus": world, "data": "synthetic",
+                "backward": run_backward(ssm, inp, dev, stream, rank, hbm_peak, w, steps=max(1, args.steps))}
+        if world > 1:
+            dist.barrier()
+            dist.destroy_process_group()
+        if rank == 0:
+            print(json.dumps(line), flush=True)
+        return 0
     y = torch.empty_like(inp["x"])
     ws = ssm.ScanWorkspace()
     conv = synth.conv_params(w.dim, w.batch, w.dtype, seed=rank_seed(w.seed + 5, rank), device=dev)
@@ -384,6 +395,10 @@ def run_ours(args):
                                     "separate_pass_ms_at_hbm_peak": sep / (hbm_peak * 1e9) * 1e3,
                                     "kernel": "scan_ws_kernel (short-convolution instantiation)"}
             line["gpu_launches"] += csteps
+        # Backward of the scan (recomputed states) on the same tokens, given a random dL/dy.
+        if not args.conv:
+            line["backward"] = run_backward(ssm, inp, dev, stream, rank, hbm_peak, w, steps=max(2, args.steps // 20))
+            line["gpu_launches"] += line["backward"]["launches"]
         # End to end through the public API: pinned host inputs in, result back each step.
         names = ["x", "dt", "z", "B", "C"] if w.gate else ["x", "dt", "B", "C"]
         host = {k: torch.empty(inp[k].shape, dtype=inp[k].dtype, pin_memory=True) for k in names}
@@ -431,6 +446,32 @@ def run_ours(args):
     if rank == 0:
         print(json.dumps(line), flush=True)
     return 0
+
+
+def run_backward(ssm, inp, dev, stream, rank, hbm_peak, w, steps=3):
+    """ssm_scan_bwd on the benchmark's tokens. Algorithmic bytes: x, dt, z, dy read and
+    dx, ddt, dz written ([B, L, D] each), B, C read and dB, dC (float32) written."""
+    import torch
+    gen = torch.Generator(device=dev).manual_seed(rank_seed(20270, rank))
+    dy = torch.randn(inp["x"].shape, generator=gen, device=dev).to(inp["x"].dtype)
+    ws = ssm.ScanWorkspace()
+
+    def bwd_step():
+        ssm.scan_bwd(inp["x"], inp["dt"], inp["A"], inp["B"], inp["C"], dy, inp["D"], inp["z"], inp["dt_bias"],
+                     workspace=ws)
+
+    bwd_step()
+    torch.cuda.synchronize(dev)
+    ms = time_region(bwd_step, steps, stream) / steps
+    es = 2 if w.dtype == torch.bfloat16 else 4
+    ntok = 7 if w.gate else 5
+    nbytes = ntok * w.batch * w.seqlen * w.dim * es + 2 * w.batch * w.seqlen * w.dstate * (es + 4)
+    gbs = nbytes / (ms / 1e3) / 1e9
+    del dy, ws
+    torch.cuda.empty_cache()
+    return {"workload": f"{w.name} backward (dx, ddt, dz, dB, dC, dA, dD, ddt_bias)", "ms_per_step": ms,
+            "value": w.updates / (ms / 1e3), "unit": UNIT, "algorithmic_bytes": nbytes, "achieved_GBs": gbs,
+            "hbm_frac": gbs / hbm_peak, "kernel": "scan_bwd_kernel", "launches": steps + 1}
 
 
 def run_decode(ssm, synth, dev, stream, rank, hbm_peak, reps=3, conv=False):

@@ -230,6 +230,51 @@ size_t ssm_scan_host_staging_size(const ssm_scan_args *args, int64_t chunk_len);
 ssm_status ssm_scan_fwd_host(const ssm_scan_args *args, int64_t chunk_len, void *staging, size_t staging_bytes,
                              void *stream);
 
+/*
+ * Backward of ssm_scan_fwd: the gradients of a loss with respect to every input, given
+ * dy = dL/dy and optionally dh_last = dL/dh_L. The pages print no backward formulas;
+ * this is the derivative of the forward above, with the states recomputed rather than
+ * stored (Mamba summary, hardware-aware algorithm paragraph: recomputation in the
+ * backward pass). The library runs one forward sweep that keeps only the state at the
+ * start of every 32 steps (in the workspace), then walks the sequence backwards,
+ * recomputing each 16 steps' states from those checkpoints.
+ *
+ * Shapes and types as for ssm_scan_fwd; x, dt, z, Bm, Cm, A, Dskip, dt_bias, h0 are the
+ * forward's inputs. Outputs (all overwritten; device memory the caller owns):
+ *   dx, ddt, dz : [B, L, D], dtype of x (dz is required exactly when z is given);
+ *                 ddt is dL/d(dt), the raw step size before bias and softplus
+ *   dB, dC      : [B, L, N] float32 (B_t and C_t are shared by the channels of a
+ *                 sequence: their gradients sum over the channels)
+ *   dA          : [D, N] float32;  dD, ddt_bias : [D] float32, or NULL to skip
+ *   dh0         : [B, D, N] float32 dL/dh0, or NULL to skip
+ * dB, dC, dA, dD and ddt_bias are sums accumulated with float atomics: their last bits
+ * can vary from run to run with the order of the additions. Only SSM_DELTA_SOFTPLUS
+ * (and SSM_A_GENERAL, which changes nothing here) is honoured; SSM_EXACT_ZOH returns
+ * SSM_ERR_UNSUPPORTED, and the short convolution has no backward here. The workspace
+ * holds the checkpoints: ssm_scan_bwd_workspace_size() bytes = 64 x B x ceil(L/32) x
+ * ceil(D/32) x 32 (as large as one [B, L, D] bfloat16 tensor), 16-byte aligned.
+ * Errors: as ssm_scan_fwd (x, dt, z, dy and workspace on 16 bytes).
+ */
+typedef struct {
+    int64_t batch, seqlen, dim, dstate;
+    ssm_dtype dtype;
+    uint32_t flags;          /* SSM_DELTA_SOFTPLUS as in the forward call */
+    const void *x, *dt, *z, *Bm, *Cm;          /* the forward's tokens (z may be NULL) */
+    const float *A, *Dskip, *dt_bias, *h0;     /* the forward's parameters (NULL as there) */
+    const void *dy;          /* [B, L, D] dL/dy, dtype of x                          */
+    const float *dh_last;    /* [B, D, N] dL/dh_L, or NULL for 0                       */
+    void *dx, *ddt, *dz;     /* [B, L, D] outputs, dtype of x (dz NULL iff z NULL)    */
+    float *dB, *dC;          /* [B, L, N] float32 outputs                            */
+    float *dA;               /* [D, N] float32 output                                */
+    float *dD, *ddt_bias;    /* [D] float32 outputs, or NULL                          */
+    float *dh0;              /* [B, D, N] float32 output, or NULL                     */
+    void *workspace;         /* ssm_scan_bwd_workspace_size() bytes                  */
+    size_t workspace_bytes;
+} ssm_scan_bwd_args;
+
+size_t ssm_scan_bwd_workspace_size(const ssm_scan_bwd_args *args);
+ssm_status ssm_scan_bwd(const ssm_scan_bwd_args *args, void *stream);
+
 /* Human-readable name of a status code (static storage). */
 const char *ssm_status_string(ssm_status status);
 

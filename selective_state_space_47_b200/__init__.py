@@ -229,6 +229,57 @@ def scan_fwd_host(x, dt, A, B, C, D=None, z=None, dt_bias=None, h0=None, *, chun
     return (y, h_last) if return_last_state else y
 
 
+def scan_bwd(x, dt, A, B, C, dy, D=None, z=None, dt_bias=None, h0=None, dh_last=None, *, delta_softplus=True,
+             workspace=None, stream=None):
+    """Backward of scan_fwd (see include/ssm_scan.h, ssm_scan_bwd): gradients given
+    dy = dL/dy [B, L, D] (dtype of x) and optionally dh_last = dL/dh_L [B, D, N] float32.
+
+    Returns a dict: dx, ddt, dz (None without z) in x's dtype [B, L, D]; dB, dC float32
+    [B, L, N]; dA float32 [D, N]; dD, ddt_bias float32 [D]; dh0 float32 [B, D, N].
+    """
+    dev = x.device
+    if x.dtype not in _TOKEN_DTYPES:
+        raise TypeError(f"x: dtype must be float32 or bfloat16, got {x.dtype}")
+    if x.dim() != 3 or A.dim() != 2:
+        raise ValueError("x must be [B, L, D] and A [D, N]")
+    Bsz, L, Dm = x.shape
+    N = A.shape[1]
+    tok = x.dtype
+    for t, name, shape in ((x, "x", (Bsz, L, Dm)), (dt, "dt", (Bsz, L, Dm)), (dy, "dy", (Bsz, L, Dm)),
+                           (B, "B", (Bsz, L, N)), (C, "C", (Bsz, L, N))):
+        _need(t, name, shape, tok, dev)
+    if z is not None:
+        _need(z, "z", (Bsz, L, Dm), tok, dev)
+    _need(A, "A", (Dm, N), torch.float32, dev)
+    for t, name, shape in ((D, "D", (Dm,)), (dt_bias, "dt_bias", (Dm,)), (h0, "h0", (Bsz, Dm, N)),
+                           (dh_last, "dh_last", (Bsz, Dm, N))):
+        if t is not None:
+            _need(t, name, shape, torch.float32, dev)
+    f32 = dict(dtype=torch.float32, device=dev)
+    out = dict(dx=torch.empty_like(x), ddt=torch.empty_like(x), dz=None if z is None else torch.empty_like(x),
+               dB=torch.empty((Bsz, L, N), **f32), dC=torch.empty((Bsz, L, N), **f32),
+               dA=torch.empty((Dm, N), **f32), dD=torch.empty((Dm,), **f32),
+               ddt_bias=torch.empty((Dm,), **f32), dh0=torch.empty((Bsz, Dm, N), **f32))
+    a = _native.ScanBwdArgs()
+    a.batch, a.seqlen, a.dim, a.dstate = Bsz, L, Dm, N
+    a.dtype = _TOKEN_DTYPES[tok]
+    a.flags = _flags(delta_softplus, False)
+    a.x, a.dt, a.z, a.Bm, a.Cm = (_ptr(t) for t in (x, dt, z, B, C))
+    a.A, a.Dskip, a.dt_bias, a.h0 = (_ptr(t) for t in (A, D, dt_bias, h0))
+    a.dy, a.dh_last = _ptr(dy), _ptr(dh_last)
+    a.dx, a.ddt, a.dz = _ptr(out["dx"]), _ptr(out["ddt"]), _ptr(out["dz"])
+    a.dB, a.dC, a.dA, a.dD, a.ddt_bias, a.dh0 = (_ptr(out[k]) for k in ("dB", "dC", "dA", "dD", "ddt_bias", "dh0"))
+    lib = _native.lib()
+    nbytes = int(lib.ssm_scan_bwd_workspace_size(ctypes.byref(a)))
+    if workspace is None:
+        workspace = ScanWorkspace()
+    ws = workspace.get(nbytes, dev) if isinstance(workspace, ScanWorkspace) else workspace
+    a.workspace = ctypes.c_void_p(ws.data_ptr())
+    a.workspace_bytes = ws.numel() * ws.element_size()
+    _native.check(lib.ssm_scan_bwd(ctypes.byref(a), _stream_handle(stream)), "ssm_scan_bwd")
+    return out
+
+
 def workspace_status(workspace, stream=None):
     """Synchronise and return the device status code of the last scan on this workspace."""
     ws = workspace.buf if isinstance(workspace, ScanWorkspace) else workspace

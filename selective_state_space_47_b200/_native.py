@@ -14,7 +14,8 @@ SSM_TEST_DROP_HANDOFF = 0x80000000
 
 # Every symbol the header declares (checked by the CPU test suite).
 EXPORTS = ("ssm_scan_workspace_size", "ssm_scan_fwd", "ssm_step", "ssm_step_conv", "ssm_workspace_status",
-           "ssm_status_string", "ssm_scan_fwd_noalloc", "ssm_scan_host_staging_size", "ssm_scan_fwd_host")
+           "ssm_status_string", "ssm_scan_fwd_noalloc", "ssm_scan_host_staging_size", "ssm_scan_fwd_host",
+           "ssm_scan_bwd_workspace_size", "ssm_scan_bwd")
 
 
 class ScanArgs(ctypes.Structure):
@@ -27,6 +28,20 @@ class ScanArgs(ctypes.Structure):
         ("y", ctypes.c_void_p), ("h_last", ctypes.c_void_p), ("workspace", ctypes.c_void_p),
         ("workspace_bytes", ctypes.c_size_t),
         ("conv_w", ctypes.c_void_p), ("conv_b", ctypes.c_void_p), ("conv_x0", ctypes.c_void_p),
+    ]
+
+
+class ScanBwdArgs(ctypes.Structure):
+    _fields_ = [
+        ("batch", ctypes.c_int64), ("seqlen", ctypes.c_int64), ("dim", ctypes.c_int64),
+        ("dstate", ctypes.c_int64), ("dtype", ctypes.c_int), ("flags", ctypes.c_uint32),
+        ("x", ctypes.c_void_p), ("dt", ctypes.c_void_p), ("z", ctypes.c_void_p),
+        ("Bm", ctypes.c_void_p), ("Cm", ctypes.c_void_p), ("A", ctypes.c_void_p),
+        ("Dskip", ctypes.c_void_p), ("dt_bias", ctypes.c_void_p), ("h0", ctypes.c_void_p),
+        ("dy", ctypes.c_void_p), ("dh_last", ctypes.c_void_p), ("dx", ctypes.c_void_p),
+        ("ddt", ctypes.c_void_p), ("dz", ctypes.c_void_p), ("dB", ctypes.c_void_p), ("dC", ctypes.c_void_p),
+        ("dA", ctypes.c_void_p), ("dD", ctypes.c_void_p), ("ddt_bias", ctypes.c_void_p), ("dh0", ctypes.c_void_p),
+        ("workspace", ctypes.c_void_p), ("workspace_bytes", ctypes.c_size_t),
     ]
 
 
@@ -56,6 +71,10 @@ def lib():
         L.ssm_step.restype = ctypes.c_int
         L.ssm_step_conv.argtypes = [i64, i64, i64, ctypes.c_int, ctypes.c_uint32] + [vp] * 13 + [vp]
         L.ssm_step_conv.restype = ctypes.c_int
+        L.ssm_scan_bwd_workspace_size.argtypes = [ctypes.POINTER(ScanBwdArgs)]
+        L.ssm_scan_bwd_workspace_size.restype = ctypes.c_size_t
+        L.ssm_scan_bwd.argtypes = [ctypes.POINTER(ScanBwdArgs), vp]
+        L.ssm_scan_bwd.restype = ctypes.c_int
         L.ssm_workspace_status.argtypes = [vp, vp]
         L.ssm_workspace_status.restype = ctypes.c_int
         L.ssm_status_string.argtypes = [ctypes.c_int]

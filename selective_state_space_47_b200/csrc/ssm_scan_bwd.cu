@@ -1,0 +1,521 @@
+// ssm_scan_bwd.cu -- backward of the selective scan (S6) on the B200 (sm_100a):
+// the gradients of a loss with respect to every input of ssm_scan_fwd, given dL/dy
+// (and optionally dL/dh_L), with the states recomputed instead of stored (Mamba
+// summary, azimuth.plus, hardware-aware algorithm paragraph: recomputation in the
+// backward pass).
+//
+// One thread block owns one group of CH = 32 channels of one sequence for the whole
+// sequence; lane c is channel c, warp w holds states 4w .. 4w+3 (as in the forward).
+//   1. Forward sweep: the state at the start of every chunk of KC = 32 steps goes to
+//      the workspace (2 KB per chunk and group), nothing else is kept.
+//   2. Reverse sweep over the chunks, each in two halves of TH = 16 steps (second
+//      half first): the half's states are recomputed from the chunk's checkpoint into
+//      shared memory, then walked backwards with the adjoint g = dL/dh:
+//        g += dq_t C_t;  dx_t += g Delta_t B_t;  dDelta_t += g (A Abar_t h_{t-1} + B_t x_t)
+//        dA += g Delta_t Abar_t h_{t-1};  dB_t += g Delta_t x_t;  dC_t += dq_t h_t;  g *= Abar_t
+//      with dq_t = dy_t silu(z_t) (or dy_t) from the recomputed readout.
+// Token tiles move into shared memory with cp.async (double-buffered by chunk). dB and
+// dC (shared by the channels of a sequence) are reduced over the 32 lanes with a
+// shuffle reduce-scatter and added to global memory with one atomic per (t, n) and
+// group; dA, dD and dt_bias's gradient are kept in registers and added once per block.
+// The atomics make dB, dC, dA, dD and dt_bias's gradient independent of any schedule
+// only up to the order of float additions.
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/ssm_scan.h"
+#include "ssm_device.cuh"
+
+namespace ssm {
+namespace bwd {
+
+constexpr int CH = 32;           // channels per block (one per lane)
+constexpr int CW = 4;            // warps (4 states each)
+constexpr int NT = CW * 32;      // threads per block
+constexpr int KC = 32;           // steps per chunk (checkpoint interval)
+constexpr int TH = 16;           // steps per half chunk (the reverse unit)
+constexpr int kMaxN = 16;
+
+struct Params {
+    int64_t Bsz, L, D, N, Dg, nchunks;
+    const void *x, *dt, *z, *Bm, *Cm, *dy;
+    const float *A, *Dskip, *dt_bias, *h0, *dh_last;
+    void *dx, *ddt, *dz;
+    float *dB, *dC, *dA, *dD, *dbias, *dh0;
+    float4 *ckpt;  // [G][nchunks][CW][CH] states at chunk starts
+    int softplus, bc_async;
+};
+
+// Shared memory: two chunk buffers (x | dt | z | dy as [KC][CH] tokens, B | C as
+// [KC][16] tokens), the recomputed states of a half [TH][CW][CH] float4, per-warp
+// partial sums [CW][TH][CH] (readout, then dDelta) and [CW][TH][CH] (dx), and per
+// (t, channel) values dq, Delta, sigma(v) [TH][CH].
+template <typename T>
+struct Smem {
+    static constexpr size_t tok = size_t(KC) * CH * sizeof(T);
+    static constexpr size_t bc = size_t(KC) * kMaxN * sizeof(T);
+    static constexpr size_t o_x = 0, o_dt = tok, o_z = 2 * tok, o_dy = 3 * tok, o_b = 4 * tok, o_c = 4 * tok + bc;
+    static constexpr size_t buf = 4 * tok + 2 * bc;
+    static constexpr size_t off_h = 2 * buf;
+    static constexpr size_t off_pa = off_h + size_t(TH) * CW * CH * 16;
+    static constexpr size_t off_pb = off_pa + size_t(CW) * TH * CH * 4;
+    static constexpr size_t off_dq = off_pb + size_t(CW) * TH * CH * 4;
+    static constexpr size_t off_del = off_dq + size_t(TH) * CH * 4;
+    static constexpr size_t off_sig = off_del + size_t(TH) * CH * 4;
+    static constexpr size_t total = off_sig + size_t(TH) * CH * 4;
+    static_assert(buf % 16 == 0 && off_h % 16 == 0, "16-byte copies and float4 rows");
+};
+
+// 16-byte asynchronous copy global -> shared; valid == false fills zeros (reads nothing).
+__device__ __forceinline__ void cp_async16(void *dst, const void *src, bool valid) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem_u32(dst)), "l"(src),
+                 "r"(valid ? 16 : 0)
+                 : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+    asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+
+// Chunk j of group (b, d0) into `buf`: x, dt (and with `all`, z and dy) by 16-byte
+// copies; rows past L and channels past D read as zeros (D is a multiple of the
+// copy's elements, so a copy is wholly inside or outside). B and C rows by 16-byte
+// copies when a row is a whole number of them (bc_async), else element by element.
+template <typename T>
+__device__ __forceinline__ void load_chunk(unsigned char *buf, const Params &p, int64_t b, int64_t d0, int64_t t0,
+                                           bool all) {
+    using S = Smem<T>;
+    constexpr int VPC = 16 / sizeof(T);  // elements per copy
+    constexpr int CPR = CH / VPC;        // copies per row
+    const T *src[4] = {static_cast<const T *>(p.x), static_cast<const T *>(p.dt), static_cast<const T *>(p.z),
+                       static_cast<const T *>(p.dy)};
+    const size_t dst[4] = {S::o_x, S::o_dt, S::o_z, S::o_dy};
+    for (int k = threadIdx.x; k < KC * CPR; k += NT) {
+        const int r = k / CPR, cc = (k % CPR) * VPC;
+        const int64_t t = t0 + r, d = d0 + cc;
+        const bool ok = t < p.L && d < p.D;
+        const int64_t off = ok ? (b * p.L + t) * p.D + d : 0;
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            if (q >= 2 && !all) break;
+            if (!src[q]) continue;  // no gate
+            cp_async16(buf + dst[q] + size_t(r * CH + cc) * sizeof(T), src[q] + off, ok);
+        }
+    }
+    const T *Bm = static_cast<const T *>(p.Bm), *Cm = static_cast<const T *>(p.Cm);
+    if (p.bc_async) {
+        const int cpr = int(p.N) / VPC;  // copies per B (or C) row
+        for (int k = threadIdx.x; k < KC * cpr; k += NT) {
+            const int r = k / cpr, n0 = (k % cpr) * VPC;
+            const int64_t t = t0 + r;
+            const bool ok = t < p.L;
+            const int64_t off = ok ? (b * p.L + t) * p.N + n0 : 0;
+            cp_async16(buf + S::o_b + size_t(r * kMaxN + n0) * sizeof(T), Bm + off, ok);
+            cp_async16(buf + S::o_c + size_t(r * kMaxN + n0) * sizeof(T), Cm + off, ok);
+        }
+    } else {
+        for (int k = threadIdx.x; k < KC * kMaxN; k += NT) {
+            const int r = k / kMaxN, n = k % kMaxN;
+            const int64_t t = t0 + r;
+            const bool ok = t < p.L && n < p.N;
+            const int64_t off = (b * p.L + t) * p.N + n;
+            reinterpret_cast<T *>(buf + S::o_b)[r * kMaxN + n] = ok ? Bm[off] : Tok<T>::from_f(0.f);
+            reinterpret_cast<T *>(buf + S::o_c)[r * kMaxN + n] = ok ? Cm[off] : Tok<T>::from_f(0.f);
+        }
+    }
+}
+
+__device__ __forceinline__ float delta_of(const float v, const bool softplus) { return softplus ? softplus_f(v) : v; }
+__device__ __forceinline__ float sigmoid_f(const float v) { return rcp_approx(1.0f + ex2_approx(-v * kLog2e)); }
+
+// Four consecutive entries of a [.][16] token row (B or C), widened.
+template <typename T>
+__device__ __forceinline__ float4 row4(const unsigned char *base, const int r, const int n0) {
+    const T *p = reinterpret_cast<const T *>(base) + r * kMaxN + n0;
+    return make_float4(Tok<T>::to_f(p[0]), Tok<T>::to_f(p[1]), Tok<T>::to_f(p[2]), Tok<T>::to_f(p[3]));
+}
+
+// One forward step of a lane's four states.
+__device__ __forceinline__ float4 fwd_step(const float4 h, const float4 a, const float u, const float4 bv) {
+    return make_float4(fmaf(a.x, h.x, u * bv.x), fmaf(a.y, h.y, u * bv.y), fmaf(a.z, h.z, u * bv.z),
+                       fmaf(a.w, h.w, u * bv.w));
+}
+__device__ __forceinline__ float4 abar4(const float dl, const float4 A) {  // dl = Delta log2 e
+    return make_float4(ex2_approx(dl * A.x), ex2_approx(dl * A.y), ex2_approx(dl * A.z), ex2_approx(dl * A.w));
+}
+
+// Sum over the warp's 32 lanes of eight values per lane (a reduce-scatter in 9
+// shuffles): on return, lanes with (lane & 3) == 0 hold the total of value
+// ((lane >> 4) & 1) * 4 + ((lane >> 3) & 1) * 2 + ((lane >> 2) & 1).
+__device__ __forceinline__ float warp_sum8(const float (&v)[8], const int lane) {
+    float u[4], w2[2];
+    const bool h16 = lane & 16, h8 = lane & 8, h4 = lane & 4;
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+        const float send = h16 ? v[k] : v[k + 4], keep = h16 ? v[k + 4] : v[k];
+        u[k] = keep + __shfl_xor_sync(0xffffffffu, send, 16);
+    }
+#pragma unroll
+    for (int k = 0; k < 2; ++k) {
+        const float send = h8 ? u[k] : u[k + 2], keep = h8 ? u[k + 2] : u[k];
+        w2[k] = keep + __shfl_xor_sync(0xffffffffu, send, 8);
+    }
+    float r = (h4 ? w2[1] : w2[0]) + __shfl_xor_sync(0xffffffffu, h4 ? w2[0] : w2[1], 4);
+    r += __shfl_xor_sync(0xffffffffu, r, 2);
+    r += __shfl_xor_sync(0xffffffffu, r, 1);
+    return r;
+}
+
+template <typename T>
+__global__ void __launch_bounds__(NT) scan_bwd_kernel(const Params p) {
+    using S = Smem<T>;
+    extern __shared__ __align__(16) unsigned char smem[];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int64_t g = blockIdx.x;
+    const int64_t b = g / p.Dg, d0 = (g % p.Dg) * CH, d = d0 + lane;
+    const bool dvalid = d < p.D;
+    const bool gate = p.z != nullptr, softplus = p.softplus != 0;
+
+    // zero the B/C rows once: copies never touch the padding past N
+    for (int k = threadIdx.x; k < int(2 * S::buf / 16); k += NT) reinterpret_cast<float4 *>(smem)[k] = make_float4(0, 0, 0, 0);
+    __syncthreads();
+
+    float4 Aq = make_float4(0.f, 0.f, 0.f, 0.f);
+    {
+        float a[4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const int n = 4 * warp + j;
+            a[j] = (dvalid && n < p.N) ? __ldg(p.A + d * p.N + n) : 0.f;
+        }
+        Aq = make_float4(a[0], a[1], a[2], a[3]);
+    }
+    const float bias = (dvalid && p.dt_bias) ? __ldg(p.dt_bias + d) : 0.f;
+    const float dskip = (dvalid && p.Dskip) ? __ldg(p.Dskip + d) : 0.f;
+    float4 *ck = p.ckpt + (g * p.nchunks) * (CW * CH) + warp * CH + lane;
+
+    // ------------------------------------------------------------ 1. forward sweep
+    float4 h = make_float4(0.f, 0.f, 0.f, 0.f);
+    {
+        float hv[4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const int n = 4 * warp + j;
+            hv[j] = (dvalid && n < p.N && p.h0) ? __ldg(p.h0 + (b * p.D + d) * p.N + n) : 0.f;
+        }
+        h = make_float4(hv[0], hv[1], hv[2], hv[3]);
+    }
+    load_chunk<T>(smem, p, b, d0, 0, false);
+    cp_async_commit();
+    for (int64_t j = 0; j < p.nchunks; ++j) {
+        unsigned char *buf = smem + (j & 1) * S::buf;
+        if (j + 1 < p.nchunks) {
+            load_chunk<T>(smem + ((j + 1) & 1) * S::buf, p, b, d0, (j + 1) * KC, false);
+            cp_async_commit();
+            cp_async_wait<1>();
+        } else {
+            cp_async_wait<0>();
+        }
+        __syncthreads();
+        ck[j * CW * CH] = h;
+        const T *sx = reinterpret_cast<const T *>(buf + S::o_x) + lane;
+        const T *sdt = reinterpret_cast<const T *>(buf + S::o_dt) + lane;
+#pragma unroll 4
+        for (int t = 0; t < KC; ++t) {
+            const float delta = delta_of(Tok<T>::to_f(sdt[t * CH]) + bias, softplus);
+            const float4 a = abar4(delta * kLog2e, Aq);
+            h = fwd_step(h, a, delta * Tok<T>::to_f(sx[t * CH]), row4<T>(buf + S::o_b, t, 4 * warp));
+        }
+        __syncthreads();  // the buffer is refilled next
+    }
+
+    // ------------------------------------------------------------ 2. reverse sweep
+    float4 gq = make_float4(0.f, 0.f, 0.f, 0.f);  // dL/dh of the warp's four states
+    if (p.dh_last) {
+        float gv[4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const int n = 4 * warp + j;
+            gv[j] = (dvalid && n < p.N) ? __ldg(p.dh_last + (b * p.D + d) * p.N + n) : 0.f;
+        }
+        gq = make_float4(gv[0], gv[1], gv[2], gv[3]);
+    }
+    float4 dA = make_float4(0.f, 0.f, 0.f, 0.f);
+    float dD = 0.f, dbias = 0.f;  // of channel `lane`, over this thread's (t, channel) pairs
+    float4 *hb = reinterpret_cast<float4 *>(smem + S::off_h);
+    float *pa = reinterpret_cast<float *>(smem + S::off_pa);
+    float *pb = reinterpret_cast<float *>(smem + S::off_pb);
+    float *sdq = reinterpret_cast<float *>(smem + S::off_dq);
+    float *sdel = reinterpret_cast<float *>(smem + S::off_del);
+    float *ssig = reinterpret_cast<float *>(smem + S::off_sig);
+    T *dxo = static_cast<T *>(p.dx);
+    T *ddto = static_cast<T *>(p.ddt);
+    T *dzo = static_cast<T *>(p.dz);
+
+    const int64_t last = p.nchunks - 1;
+    load_chunk<T>(smem + (last & 1) * S::buf, p, b, d0, last * KC, true);
+    cp_async_commit();
+    for (int64_t j = last; j >= 0; --j) {
+        const unsigned char *buf = smem + (j & 1) * S::buf;
+        if (j > 0) {
+            load_chunk<T>(smem + ((j - 1) & 1) * S::buf, p, b, d0, (j - 1) * KC, true);
+            cp_async_commit();
+            cp_async_wait<1>();
+        } else {
+            cp_async_wait<0>();
+        }
+        __syncthreads();
+        const int64_t t0 = j * KC;
+        const T *sx = reinterpret_cast<const T *>(buf + S::o_x);
+        const T *sdt = reinterpret_cast<const T *>(buf + S::o_dt);
+        const T *sz = reinterpret_cast<const T *>(buf + S::o_z);
+        const T *sdy = reinterpret_cast<const T *>(buf + S::o_dy);
+        const float4 hck = ck[j * CW * CH];
+        // the state after the first half, from the checkpoint
+        float4 hmid = hck;
+#pragma unroll 4
+        for (int t = 0; t < TH; ++t) {
+            const float delta = delta_of(Tok<T>::to_f(sdt[t * CH + lane]) + bias, softplus);
+            hmid = fwd_step(hmid, abar4(delta * kLog2e, Aq), delta * Tok<T>::to_f(sx[t * CH + lane]),
+                            row4<T>(buf + S::o_b, t, 4 * warp));
+        }
+        for (int half = 1; half >= 0; --half) {
+            const int tb = half * TH;                   // first step of the half in the chunk
+            const float4 hs = half ? hmid : hck;        // state before the half
+            // (a) recompute the half's states and the warps' partial readouts
+            float4 hh = hs;
+#pragma unroll 4
+            for (int s = 0; s < TH; ++s) {
+                const int t = tb + s;
+                const float delta = delta_of(Tok<T>::to_f(sdt[t * CH + lane]) + bias, softplus);
+                hh = fwd_step(hh, abar4(delta * kLog2e, Aq), delta * Tok<T>::to_f(sx[t * CH + lane]),
+                              row4<T>(buf + S::o_b, t, 4 * warp));
+                hb[(s * CW + warp) * CH + lane] = hh;
+                const float4 c4 = row4<T>(buf + S::o_c, t, 4 * warp);
+                pa[(warp * TH + s) * CH + lane] = fmaf(c4.x, hh.x, fmaf(c4.y, hh.y, fmaf(c4.z, hh.z, c4.w * hh.w)));
+            }
+            __syncthreads();
+            // (b) per (t, channel): readout, gate, dq, dz, Delta, sigma(v)
+#pragma unroll
+            for (int i = 0; i < TH / CW; ++i) {
+                const int s = warp * (TH / CW) + i, t = tb + s;
+                const int64_t tg = t0 + t;
+                const float xv = Tok<T>::to_f(sx[t * CH + lane]);
+                const float q = pa[(0 * TH + s) * CH + lane] + pa[(1 * TH + s) * CH + lane] +
+                                pa[(2 * TH + s) * CH + lane] + pa[(3 * TH + s) * CH + lane] + dskip * xv;
+                const float v = Tok<T>::to_f(sdt[t * CH + lane]) + bias;
+                float dq = Tok<T>::to_f(sdy[t * CH + lane]);
+                if (gate) {
+                    const float zv = Tok<T>::to_f(sz[t * CH + lane]), sg = sigmoid_f(zv);
+                    if (tg < p.L && dvalid)
+                        dzo[(b * p.L + tg) * p.D + d] = Tok<T>::from_f(dq * q * sg * fmaf(zv, 1.f - sg, 1.f));
+                    dq *= zv * sg;
+                }
+                if (tg < p.L) dD = fmaf(dq, xv, dD);
+                sdq[s * CH + lane] = dq;
+                sdel[s * CH + lane] = delta_of(v, softplus);
+                ssig[s * CH + lane] = softplus ? sigmoid_f(v) : 1.f;
+            }
+            __syncthreads();
+            // (c) the adjoint, backwards over the half (steps past L are skipped)
+            for (int s = TH - 1; s >= 0; --s) {
+                const int t = tb + s;
+                const int64_t tg = t0 + t;
+                if (tg >= p.L) continue;  // uniform over the block
+                const float delta = sdel[s * CH + lane], dq = sdq[s * CH + lane];
+                const float xv = Tok<T>::to_f(sx[t * CH + lane]);
+                const float4 bv = row4<T>(buf + S::o_b, t, 4 * warp), cv = row4<T>(buf + S::o_c, t, 4 * warp);
+                const float4 hc = hb[(s * CW + warp) * CH + lane];
+                const float4 hp = s > 0 ? hb[((s - 1) * CW + warp) * CH + lane] : hs;
+                const float4 a = abar4(delta * kLog2e, Aq);
+                gq.x = fmaf(dq, cv.x, gq.x);
+                gq.y = fmaf(dq, cv.y, gq.y);
+                gq.z = fmaf(dq, cv.z, gq.z);
+                gq.w = fmaf(dq, cv.w, gq.w);
+                const float dx_ = delta * xv;
+                // dA_n += g_n Delta Abar_n h_{t-1,n}
+                const float4 ah = make_float4(a.x * hp.x, a.y * hp.y, a.z * hp.z, a.w * hp.w);
+                dA.x = fmaf(gq.x * delta, ah.x, dA.x);
+                dA.y = fmaf(gq.y * delta, ah.y, dA.y);
+                dA.z = fmaf(gq.z * delta, ah.z, dA.z);
+                dA.w = fmaf(gq.w * delta, ah.w, dA.w);
+                // dDelta partial: sum_n g_n (A_n Abar_n h_{t-1,n} + B_n x)
+                float ddel = gq.x * fmaf(Aq.x, ah.x, bv.x * xv);
+                ddel = fmaf(gq.y, fmaf(Aq.y, ah.y, bv.y * xv), ddel);
+                ddel = fmaf(gq.z, fmaf(Aq.z, ah.z, bv.z * xv), ddel);
+                ddel = fmaf(gq.w, fmaf(Aq.w, ah.w, bv.w * xv), ddel);
+                // dx partial: sum_n g_n Delta B_n
+                float dxp = gq.x * bv.x;
+                dxp = fmaf(gq.y, bv.y, dxp);
+                dxp = fmaf(gq.z, bv.z, dxp);
+                dxp = fmaf(gq.w, bv.w, dxp);
+                pa[(warp * TH + s) * CH + lane] = ddel;
+                pb[(warp * TH + s) * CH + lane] = dxp * delta;
+                // dB_tn = sum over channels of g_n Delta x; dC_tn = sum over channels of dq h_tn
+                const float v8[8] = {gq.x * dx_, gq.y * dx_, gq.z * dx_, gq.w * dx_,
+                                     dq * hc.x,  dq * hc.y,  dq * hc.z,  dq * hc.w};
+                const float tot = warp_sum8(v8, lane);
+                if ((lane & 3) == 0) {
+                    const int idx = ((lane >> 4) & 1) * 4 + ((lane >> 3) & 1) * 2 + ((lane >> 2) & 1);
+                    const int n = 4 * warp + (idx & 3);
+                    if (n < p.N) atomicAdd((idx < 4 ? p.dB : p.dC) + (b * p.L + tg) * p.N + n, tot);
+                }
+                gq = make_float4(gq.x * a.x, gq.y * a.y, gq.z * a.z, gq.w * a.w);
+            }
+            __syncthreads();
+            // (d) per (t, channel): dDelta -> ddt, dx
+#pragma unroll
+            for (int i = 0; i < TH / CW; ++i) {
+                const int s = warp * (TH / CW) + i, t = tb + s;
+                const int64_t tg = t0 + t;
+                if (tg >= p.L) continue;
+                const float ddel = pa[(0 * TH + s) * CH + lane] + pa[(1 * TH + s) * CH + lane] +
+                                   pa[(2 * TH + s) * CH + lane] + pa[(3 * TH + s) * CH + lane];
+                const float ddt = ddel * ssig[s * CH + lane];
+                const float dxv = fmaf(sdq[s * CH + lane], dskip,
+                                       pb[(0 * TH + s) * CH + lane] + pb[(1 * TH + s) * CH + lane] +
+                                           pb[(2 * TH + s) * CH + lane] + pb[(3 * TH + s) * CH + lane]);
+                dbias += ddt;
+                if (dvalid) {
+                    ddto[(b * p.L + tg) * p.D + d] = Tok<T>::from_f(ddt);
+                    dxo[(b * p.L + tg) * p.D + d] = Tok<T>::from_f(dxv);
+                }
+            }
+            __syncthreads();
+        }
+    }
+
+    // ------------------------------------------------------------ reductions, dh0
+    if (dvalid) {
+        const float dav[4] = {dA.x, dA.y, dA.z, dA.w};
+        const float gv[4] = {gq.x, gq.y, gq.z, gq.w};
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            const int n = 4 * warp + k;
+            if (n < p.N) {
+                atomicAdd(p.dA + d * p.N + n, dav[k]);
+                if (p.dh0) p.dh0[(b * p.D + d) * p.N + n] = gv[k];
+            }
+        }
+        if (p.dD) atomicAdd(p.dD + d, dD);
+        if (p.dbias) atomicAdd(p.dbias + d, dbias);
+    }
+}
+
+bool aligned(const void *q, size_t a) { return (reinterpret_cast<uintptr_t>(q) & (a - 1)) == 0; }
+
+int64_t groups(const ssm_scan_bwd_args *a) { return a->batch * ((a->dim + CH - 1) / CH); }
+int64_t chunks(const ssm_scan_bwd_args *a) { return (a->seqlen + KC - 1) / KC; }
+
+ssm_status validate(const ssm_scan_bwd_args *a) {
+    if (!a) return SSM_ERR_INVALID;
+    if (a->batch < 0 || a->seqlen < 0 || a->dim < 0 || a->dstate < 1) return SSM_ERR_INVALID;
+    if (a->dtype != SSM_F32 && a->dtype != SSM_BF16) return SSM_ERR_INVALID;
+    if (a->flags & ~uint32_t(SSM_DELTA_SOFTPLUS | SSM_A_GENERAL | SSM_EXACT_ZOH)) return SSM_ERR_INVALID;
+    if (a->flags & SSM_EXACT_ZOH) return SSM_ERR_UNSUPPORTED;
+    if (a->dstate > kMaxN) return SSM_ERR_UNSUPPORTED;
+    if (a->dim % (a->dtype == SSM_BF16 ? 8 : 4) != 0) return SSM_ERR_UNSUPPORTED;
+    if (a->batch > INT32_MAX || a->seqlen > INT32_MAX || a->dim > INT32_MAX) return SSM_ERR_UNSUPPORTED;
+    if ((a->z == nullptr) != (a->dz == nullptr)) return SSM_ERR_INVALID;
+    const bool work = a->batch > 0 && a->dim > 0;
+    if (work && (!a->A || !a->dA)) return SSM_ERR_INVALID;
+    if (work && a->seqlen > 0 &&
+        (!a->x || !a->dt || !a->Bm || !a->Cm || !a->dy || !a->dx || !a->ddt || !a->dB || !a->dC))
+        return SSM_ERR_INVALID;
+    const size_t es = a->dtype == SSM_BF16 ? 2 : 4;
+    const void *p16[] = {a->x, a->dt, a->z, a->dy, a->workspace};
+    for (const void *q : p16)
+        if (q && !aligned(q, 16)) return SSM_ERR_UNSUPPORTED;
+    const void *pes[] = {a->Bm, a->Cm, a->dx, a->ddt, a->dz};
+    for (const void *q : pes)
+        if (q && !aligned(q, es)) return SSM_ERR_UNSUPPORTED;
+    const void *p4[] = {a->A, a->Dskip, a->dt_bias, a->h0, a->dh_last, a->dB, a->dC, a->dA, a->dD, a->ddt_bias, a->dh0};
+    for (const void *q : p4)
+        if (q && !aligned(q, 4)) return SSM_ERR_UNSUPPORTED;
+    if (work && a->seqlen > 0 && (!a->workspace || a->workspace_bytes < ssm_scan_bwd_workspace_size(a)))
+        return SSM_ERR_INVALID;
+    return SSM_OK;
+}
+
+}  // namespace bwd
+}  // namespace ssm
+
+using namespace ssm::bwd;
+
+extern "C" {
+
+size_t ssm_scan_bwd_workspace_size(const ssm_scan_bwd_args *a) {
+    if (!a || a->batch < 0 || a->seqlen < 0 || a->dim < 0) return 0;
+    return size_t(groups(a)) * size_t(chunks(a)) * CW * CH * 16;
+}
+
+ssm_status ssm_scan_bwd(const ssm_scan_bwd_args *a, void *stream_) {
+    const ssm_status s = validate(a);
+    if (s != SSM_OK) return s;
+    cudaStream_t stream = static_cast<cudaStream_t>(stream_);
+    if (a->batch == 0 || a->dim == 0) return SSM_OK;
+    const size_t nd = size_t(a->dim), nbd = size_t(a->batch) * nd * size_t(a->dstate);
+    // every accumulated output starts at zero
+    if (cudaMemsetAsync(a->dA, 0, nd * size_t(a->dstate) * 4, stream) != cudaSuccess) return SSM_ERR_CUDA;
+    if (a->dD && cudaMemsetAsync(a->dD, 0, nd * 4, stream) != cudaSuccess) return SSM_ERR_CUDA;
+    if (a->ddt_bias && cudaMemsetAsync(a->ddt_bias, 0, nd * 4, stream) != cudaSuccess) return SSM_ERR_CUDA;
+    if (a->seqlen == 0) {  // no tokens: dh0 = dh_last (or 0)
+        if (!a->dh0) return SSM_OK;
+        const cudaError_t e = a->dh_last ? cudaMemcpyAsync(a->dh0, a->dh_last, nbd * 4, cudaMemcpyDeviceToDevice, stream)
+                                         : cudaMemsetAsync(a->dh0, 0, nbd * 4, stream);
+        return e == cudaSuccess ? SSM_OK : SSM_ERR_CUDA;
+    }
+    const size_t nbln = size_t(a->batch) * size_t(a->seqlen) * size_t(a->dstate) * 4;
+    if (cudaMemsetAsync(a->dB, 0, nbln, stream) != cudaSuccess || cudaMemsetAsync(a->dC, 0, nbln, stream) != cudaSuccess)
+        return SSM_ERR_CUDA;
+    const size_t es = a->dtype == SSM_BF16 ? 2 : 4;
+    Params p;
+    p.Bsz = a->batch;
+    p.L = a->seqlen;
+    p.D = a->dim;
+    p.N = a->dstate;
+    p.Dg = (a->dim + CH - 1) / CH;
+    p.nchunks = chunks(a);
+    p.x = a->x;
+    p.dt = a->dt;
+    p.z = a->z;
+    p.Bm = a->Bm;
+    p.Cm = a->Cm;
+    p.dy = a->dy;
+    p.A = a->A;
+    p.Dskip = a->Dskip;
+    p.dt_bias = a->dt_bias;
+    p.h0 = a->h0;
+    p.dh_last = a->dh_last;
+    p.dx = a->dx;
+    p.ddt = a->ddt;
+    p.dz = a->dz;
+    p.dB = a->dB;
+    p.dC = a->dC;
+    p.dA = a->dA;
+    p.dD = a->dD;
+    p.dbias = a->ddt_bias;
+    p.dh0 = a->dh0;
+    p.ckpt = static_cast<float4 *>(a->workspace);
+    p.softplus = (a->flags & SSM_DELTA_SOFTPLUS) != 0;
+    p.bc_async = (a->dstate * es) % 16 == 0 && aligned(a->Bm, 16) && aligned(a->Cm, 16);
+    const int64_t G = groups(a);
+    if (G > INT32_MAX) return SSM_ERR_UNSUPPORTED;
+    void *kern;
+    size_t smem;
+    if (a->dtype == SSM_BF16) {
+        kern = reinterpret_cast<void *>(&scan_bwd_kernel<__nv_bfloat16>);
+        smem = Smem<__nv_bfloat16>::total;
+    } else {
+        kern = reinterpret_cast<void *>(&scan_bwd_kernel<float>);
+        smem = Smem<float>::total;
+    }
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem)) != cudaSuccess)
+        return SSM_ERR_CUDA;
+    void *args[] = {&p};
+    const cudaError_t e = cudaLaunchKernel(kern, dim3(unsigned(G)), dim3(NT), args, smem, stream);
+    return e == cudaSuccess ? SSM_OK : SSM_ERR_CUDA;
+}
+
+}  // extern "C"

@@ -36,17 +36,19 @@ def test_header_and_exports_agree(lib):
         assert hasattr(lib, name)
 
 
-def test_args_struct_layout_matches_binding(tmp_path):
-    """The ctypes mirror of ssm_scan_args has the C compiler's field offsets and size."""
-    names = [f[0] for f in _native.ScanArgs._fields_]
+@pytest.mark.parametrize("cname,pyname", [("ssm_scan_args", "ScanArgs"), ("ssm_scan_bwd_args", "ScanBwdArgs")])
+def test_args_struct_layout_matches_binding(tmp_path, cname, pyname):
+    """The ctypes mirrors of the argument structs have the C compiler's field offsets and size."""
+    cls = getattr(_native, pyname)
+    names = [f[0] for f in cls._fields_]
     src = tmp_path / "layout.c"
-    body = "".join(f'printf("%zu\\n", offsetof(ssm_scan_args, {n}));' for n in names)
+    body = "".join(f'printf("%zu\\n", offsetof({cname}, {n}));' for n in names)
     src.write_text('#include <stddef.h>\n#include <stdio.h>\n#include "ssm_scan.h"\n'
-                   f'int main(void){{ {body} printf("%zu\\n", sizeof(ssm_scan_args)); return 0; }}\n')
+                   f'int main(void){{ {body} printf("%zu\\n", sizeof({cname})); return 0; }}\n')
     exe = tmp_path / "layout"
     subprocess.check_call(["gcc", "-std=c99", "-I", os.path.join(ROOT, "include"), "-o", str(exe), str(src)])
     got = [int(v) for v in subprocess.check_output([str(exe)]).decode().split()]
-    want = [getattr(_native.ScanArgs, n).offset for n in names] + [ctypes.sizeof(_native.ScanArgs)]
+    want = [getattr(cls, n).offset for n in names] + [ctypes.sizeof(cls)]
     assert got == want
 
 
@@ -201,3 +203,53 @@ def test_host_scan_staging_size_and_argument_checks(lib):
     a.conv_w = 1 << 30
     assert lib.ssm_scan_host_staging_size(ctypes.byref(a), Lc) == 2 * (4 * tok + 2 * bc + up(3 * 3 * 64 * 2)) + \
         2 * carry
+
+
+def _bwd_args(**kw):
+    a = _native.ScanBwdArgs()
+    a.batch, a.seqlen, a.dim, a.dstate = 2, 100, 64, 16
+    a.dtype = _native.SSM_BF16
+    a.flags = _native.SSM_DELTA_SOFTPLUS
+    fake = 1 << 20  # host-side stand-ins: never dereferenced, the calls must fail first
+    for name in ("x", "dt", "z", "Bm", "Cm", "A", "Dskip", "dt_bias", "h0", "dy", "dh_last", "dx", "ddt", "dz",
+                 "dB", "dC", "dA", "dD", "ddt_bias", "dh0"):
+        setattr(a, name, fake)
+        fake += 1 << 16
+    a.workspace = fake
+    a.workspace_bytes = 1 << 40
+    for k, v in kw.items():
+        setattr(a, k, v)
+    return a
+
+
+def test_bwd_workspace_size(lib):
+    """One float4 per (group, 32-step chunk, warp, lane): 64 B x B x ceil(L/32) x ceil(D/32) x 32."""
+    a = _bwd_args()
+    a.batch, a.seqlen, a.dim = 3, 1000, 100
+    assert lib.ssm_scan_bwd_workspace_size(ctypes.byref(a)) == 3 * 4 * 32 * 4 * 32 * 16
+    a.seqlen = -1
+    assert lib.ssm_scan_bwd_workspace_size(ctypes.byref(a)) == 0
+    assert lib.ssm_scan_bwd_workspace_size(None) == 0
+
+
+@pytest.mark.parametrize("bad,code", [
+    (dict(flags=_native.SSM_DELTA_SOFTPLUS | _native.SSM_EXACT_ZOH), _native.SSM_ERR_UNSUPPORTED),
+    (dict(flags=0x40), _native.SSM_ERR_INVALID),
+    (dict(dstate=17), _native.SSM_ERR_UNSUPPORTED),
+    (dict(dim=12), _native.SSM_ERR_UNSUPPORTED),
+    (dict(dz=None), _native.SSM_ERR_INVALID),              # z given without dz
+    (dict(z=None), _native.SSM_ERR_INVALID),               # dz given without z
+    (dict(dy=None), _native.SSM_ERR_INVALID),
+    (dict(dB=None), _native.SSM_ERR_INVALID),
+    (dict(dA=None), _native.SSM_ERR_INVALID),
+    (dict(dy=(1 << 20) + 8), _native.SSM_ERR_UNSUPPORTED),  # copied 16 bytes at a time
+    (dict(dx=(1 << 20) + 1), _native.SSM_ERR_UNSUPPORTED),
+    (dict(dA=(1 << 20) + 2), _native.SSM_ERR_UNSUPPORTED),
+    (dict(workspace=None), _native.SSM_ERR_INVALID),
+    (dict(workspace_bytes=64), _native.SSM_ERR_INVALID),
+])
+def test_bwd_rejects_on_host(lib, bad, code):
+    a = _bwd_args(**bad)
+    assert lib.ssm_scan_bwd(ctypes.byref(a), None) == code
+    assert lib.ssm_scan_bwd(None, None) == _native.SSM_ERR_INVALID
+    assert lib.ssm_scan_bwd(ctypes.byref(_bwd_args(batch=0)), None) == _native.SSM_OK
