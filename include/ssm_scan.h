@@ -235,9 +235,14 @@ ssm_status ssm_scan_fwd_host(const ssm_scan_args *args, int64_t chunk_len, void 
  * dy = dL/dy and optionally dh_last = dL/dh_L. The pages print no backward formulas;
  * this is the derivative of the forward above, with the states recomputed rather than
  * stored (Mamba summary, hardware-aware algorithm paragraph: recomputation in the
- * backward pass). The library runs one forward sweep that keeps only the state at the
- * start of every 32 steps (in the workspace), then walks the sequence backwards,
- * recomputing each 16 steps' states from those checkpoints.
+ * backward pass). The sequence of every group of 32 channels is cut into segments
+ * (about 1,800 (group, segment) items in all), each a thread block: a first pass gives
+ * each segment's end state from a zero start and its adjoint at the start from a zero
+ * end, a short combine pass chains them into every segment's true start state and end
+ * adjoint (both recurrences are linear), and the main pass runs a forward sweep per
+ * segment that keeps only the state at the start of every 32 steps (in the workspace),
+ * then walks the segment backwards, recomputing each 16 steps' states from those
+ * checkpoints.
  *
  * Shapes and types as for ssm_scan_fwd; x, dt, z, Bm, Cm, A, Dskip, dt_bias, h0 are the
  * forward's inputs. Outputs (all overwritten; device memory the caller owns):
@@ -251,8 +256,8 @@ ssm_status ssm_scan_fwd_host(const ssm_scan_args *args, int64_t chunk_len, void 
  * can vary from run to run with the order of the additions. Only SSM_DELTA_SOFTPLUS
  * (and SSM_A_GENERAL, which changes nothing here) is honoured; SSM_EXACT_ZOH returns
  * SSM_ERR_UNSUPPORTED, and the short convolution has no backward here. The workspace
- * holds the checkpoints: ssm_scan_bwd_workspace_size() bytes = 64 x B x ceil(L/32) x
- * ceil(D/32) x 32 (as large as one [B, L, D] bfloat16 tensor), 16-byte aligned.
+ * holds the checkpoints (64 bytes per channel and 32 steps: about one [B, L, D] bfloat16
+ * tensor) and 8.3 KB per item: ssm_scan_bwd_workspace_size() bytes, 16-byte aligned.
  * Errors: as ssm_scan_fwd (x, dt, z, dy and workspace on 16 bytes).
  */
 typedef struct {

@@ -4,8 +4,18 @@
 // summary, azimuth.plus, hardware-aware algorithm paragraph: recomputation in the
 // backward pass).
 //
-// One thread block owns one group of CH = 32 channels of one sequence for the whole
-// sequence; lane c is channel c, warp w holds states 4w .. 4w+3 (as in the forward).
+// Sequence parallelism: the sequence of every group of CH = 32 channels is cut into K
+// segments, and every (group, segment) item gets its own thread block (lane c is
+// channel c, warp w holds states 4w .. 4w+3, as in the forward). Both recurrences are
+// linear: the state runs forward, h_t = Abar_t h_{t-1} + Delta_t B_t x_t, and the
+// adjoint runs backward, g <- Abar_t (g + dq_t C_t), without reading h. So:
+//   A. scan_bwd_local_kernel, all items at once: the segment's end state from a zero
+//      start, its adjoint at the start from a zero end, and sum_t Delta_t (the product
+//      of the segment's Abar is exp(A sum_t Delta_t)).
+//   B. scan_bwd_combine_kernel, one thread per (group, four states, channel): walks the
+//      K segments forward and backward, giving each segment its true start state and
+//      end adjoint (and dh0).
+//   C. scan_bwd_kernel, all items at once, from those:
 //   1. Forward sweep: the state at the start of every chunk of KC = 32 steps goes to
 //      the workspace (2 KB per chunk and group), nothing else is kept.
 //   2. Reverse sweep over the chunks, each in two halves of TH = 16 steps (second
@@ -38,11 +48,14 @@ constexpr int kMaxN = 16;
 
 struct Params {
     int64_t Bsz, L, D, N, Dg, nchunks;
+    int64_t G, K, segc;  // groups, segments per group, chunks per segment
     const void *x, *dt, *z, *Bm, *Cm, *dy;
     const float *A, *Dskip, *dt_bias, *h0, *dh_last;
     void *dx, *ddt, *dz;
     float *dB, *dC, *dA, *dD, *dbias, *dh0;
     float4 *ckpt;  // [G][nchunks][CW][CH] states at chunk starts
+    float4 *hloc, *gloc, *hs, *ge;  // [G][K][CW][CH]: local end state and start adjoint; true start state, end adjoint
+    float *sdel;                    // [G][K][CH] sum of Delta over the segment
     int softplus, bc_async;
 };
 
@@ -167,12 +180,152 @@ __device__ __forceinline__ float warp_sum8(const float (&v)[8], const int lane) 
     return r;
 }
 
+// The (group, segment) item of this block and its range of chunks [cb, ce).
+struct Item {
+    int64_t g, k, cb, ce;
+};
+__device__ __forceinline__ Item item_of(const Params &p) {
+    Item it;
+    it.g = blockIdx.x % p.G;
+    it.k = blockIdx.x / p.G;
+    it.cb = it.k * p.segc;
+    it.ce = it.cb + p.segc < p.nchunks ? it.cb + p.segc : p.nchunks;
+    return it;
+}
+
+// A quad of four states (4w .. 4w+3) of channel d from a [., D, N] float array, zeros
+// past D or N or for a null array.
+__device__ __forceinline__ float4 quad_of(const float *a, const int64_t row, const int64_t d, const bool dvalid,
+                                          const int warp, const int64_t N) {
+    float v[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+        const int n = 4 * warp + j;
+        v[j] = (a && dvalid && n < N) ? __ldg(a + row * N + n) : 0.f;
+    }
+    return make_float4(v[0], v[1], v[2], v[3]);
+}
+
+// A. Per item: the segment's end state from a zero start (hloc), its adjoint at the start
+// from a zero end (gloc), and sum_t Delta_t (sdel). Steps past L are skipped.
+template <typename T>
+__global__ void __launch_bounds__(NT) scan_bwd_local_kernel(const Params p) {
+    using S = Smem<T>;
+    extern __shared__ __align__(16) unsigned char smem[];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const Item it = item_of(p);
+    const int64_t b = it.g / p.Dg, d0 = (it.g % p.Dg) * CH, d = d0 + lane;
+    const bool dvalid = d < p.D;
+    const bool gate = p.z != nullptr, softplus = p.softplus != 0;
+    for (int k = threadIdx.x; k < int(2 * S::buf / 16); k += NT) reinterpret_cast<float4 *>(smem)[k] = make_float4(0, 0, 0, 0);
+    __syncthreads();
+    const float4 Aq = quad_of(p.A, d, d, dvalid, warp, p.N);
+    const float bias = (dvalid && p.dt_bias) ? __ldg(p.dt_bias + d) : 0.f;
+    const int64_t slot = (it.g * p.K + it.k) * (CW * CH) + warp * CH + lane;
+
+    float4 h = make_float4(0.f, 0.f, 0.f, 0.f);
+    float sd = 0.f;
+    load_chunk<T>(smem + (it.cb & 1) * S::buf, p, b, d0, it.cb * KC, false);
+    cp_async_commit();
+    for (int64_t j = it.cb; j < it.ce; ++j) {
+        const unsigned char *buf = smem + (j & 1) * S::buf;
+        if (j + 1 < it.ce) {
+            load_chunk<T>(smem + ((j + 1) & 1) * S::buf, p, b, d0, (j + 1) * KC, false);
+            cp_async_commit();
+            cp_async_wait<1>();
+        } else {
+            cp_async_wait<0>();
+        }
+        __syncthreads();
+        const T *sx = reinterpret_cast<const T *>(buf + S::o_x) + lane;
+        const T *sdt = reinterpret_cast<const T *>(buf + S::o_dt) + lane;
+        const int tn = p.L - j * KC < KC ? int(p.L - j * KC) : KC;  // valid steps of the chunk
+        for (int t = 0; t < tn; ++t) {
+            const float delta = delta_of(Tok<T>::to_f(sdt[t * CH]) + bias, softplus);
+            h = fwd_step(h, abar4(delta * kLog2e, Aq), delta * Tok<T>::to_f(sx[t * CH]),
+                         row4<T>(buf + S::o_b, t, 4 * warp));
+            sd += delta;
+        }
+        __syncthreads();
+    }
+    p.hloc[slot] = h;
+    if (warp == 0) p.sdel[(it.g * p.K + it.k) * CH + lane] = sd;
+
+    float4 gl = make_float4(0.f, 0.f, 0.f, 0.f);
+    load_chunk<T>(smem + ((it.ce - 1) & 1) * S::buf, p, b, d0, (it.ce - 1) * KC, true);
+    cp_async_commit();
+    for (int64_t j = it.ce - 1; j >= it.cb; --j) {
+        const unsigned char *buf = smem + (j & 1) * S::buf;
+        if (j > it.cb) {
+            load_chunk<T>(smem + ((j - 1) & 1) * S::buf, p, b, d0, (j - 1) * KC, true);
+            cp_async_commit();
+            cp_async_wait<1>();
+        } else {
+            cp_async_wait<0>();
+        }
+        __syncthreads();
+        const T *sdt = reinterpret_cast<const T *>(buf + S::o_dt) + lane;
+        const T *sz = reinterpret_cast<const T *>(buf + S::o_z) + lane;
+        const T *sdy = reinterpret_cast<const T *>(buf + S::o_dy) + lane;
+        const int tn = p.L - j * KC < KC ? int(p.L - j * KC) : KC;
+        for (int t = tn - 1; t >= 0; --t) {
+            const float delta = delta_of(Tok<T>::to_f(sdt[t * CH]) + bias, softplus);
+            float dq = Tok<T>::to_f(sdy[t * CH]);
+            if (gate) dq *= silu_f(Tok<T>::to_f(sz[t * CH]));
+            const float4 cv = row4<T>(buf + S::o_c, t, 4 * warp), a = abar4(delta * kLog2e, Aq);
+            gl = make_float4(a.x * fmaf(dq, cv.x, gl.x), a.y * fmaf(dq, cv.y, gl.y), a.z * fmaf(dq, cv.z, gl.z),
+                             a.w * fmaf(dq, cv.w, gl.w));
+        }
+        __syncthreads();
+    }
+    p.gloc[slot] = gl;
+}
+
+// B. One thread per (group, warp quad, lane): the true start state of every segment
+// (from h0 through the segments before it) and the true adjoint at its end (from dL/dh_L
+// through the segments after it), with P = exp(A sum Delta) per segment; dh0 at the end.
+__global__ void __launch_bounds__(256) scan_bwd_combine_kernel(const Params p) {
+    const int64_t i = int64_t(blockIdx.x) * blockDim.x + threadIdx.x;
+    if (i >= p.G * CW * CH) return;
+    const int64_t g = i / (CW * CH);
+    const int r = int(i % (CW * CH)), warp = r / CH, lane = r % CH;
+    const int64_t b = g / p.Dg, d = (g % p.Dg) * CH + lane;
+    const bool dvalid = d < p.D;
+    const float4 Aq = quad_of(p.A, d, d, dvalid, warp, p.N);
+    float4 H = quad_of(p.h0, b * p.D + d, d, dvalid, warp, p.N);
+    for (int64_t k = 0; k < p.K; ++k) {
+        const int64_t slot = (g * p.K + k) * (CW * CH) + r;
+        p.hs[slot] = H;
+        const float4 P = abar4(p.sdel[(g * p.K + k) * CH + lane] * kLog2e, Aq);
+        const float4 hl = p.hloc[slot];
+        H = make_float4(fmaf(P.x, H.x, hl.x), fmaf(P.y, H.y, hl.y), fmaf(P.z, H.z, hl.z), fmaf(P.w, H.w, hl.w));
+    }
+    float4 Gq = quad_of(p.dh_last, b * p.D + d, d, dvalid, warp, p.N);
+    for (int64_t k = p.K - 1; k >= 0; --k) {
+        const int64_t slot = (g * p.K + k) * (CW * CH) + r;
+        p.ge[slot] = Gq;
+        const float4 P = abar4(p.sdel[(g * p.K + k) * CH + lane] * kLog2e, Aq);
+        const float4 gl = p.gloc[slot];
+        Gq = make_float4(fmaf(P.x, Gq.x, gl.x), fmaf(P.y, Gq.y, gl.y), fmaf(P.z, Gq.z, gl.z), fmaf(P.w, Gq.w, gl.w));
+    }
+    if (p.dh0 && dvalid) {
+        const float gv[4] = {Gq.x, Gq.y, Gq.z, Gq.w};
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const int n = 4 * warp + j;
+            if (n < p.N) p.dh0[(b * p.D + d) * p.N + n] = gv[j];
+        }
+    }
+}
+
+// C. The gradients of one item, from its true start state and end adjoint.
 template <typename T>
 __global__ void __launch_bounds__(NT) scan_bwd_kernel(const Params p) {
     using S = Smem<T>;
     extern __shared__ __align__(16) unsigned char smem[];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int64_t g = blockIdx.x;
+    const Item it = item_of(p);
+    const int64_t g = it.g;
     const int64_t b = g / p.Dg, d0 = (g % p.Dg) * CH, d = d0 + lane;
     const bool dvalid = d < p.D;
     const bool gate = p.z != nullptr, softplus = p.softplus != 0;
@@ -181,36 +334,19 @@ __global__ void __launch_bounds__(NT) scan_bwd_kernel(const Params p) {
     for (int k = threadIdx.x; k < int(2 * S::buf / 16); k += NT) reinterpret_cast<float4 *>(smem)[k] = make_float4(0, 0, 0, 0);
     __syncthreads();
 
-    float4 Aq = make_float4(0.f, 0.f, 0.f, 0.f);
-    {
-        float a[4];
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-            const int n = 4 * warp + j;
-            a[j] = (dvalid && n < p.N) ? __ldg(p.A + d * p.N + n) : 0.f;
-        }
-        Aq = make_float4(a[0], a[1], a[2], a[3]);
-    }
+    const float4 Aq = quad_of(p.A, d, d, dvalid, warp, p.N);
     const float bias = (dvalid && p.dt_bias) ? __ldg(p.dt_bias + d) : 0.f;
     const float dskip = (dvalid && p.Dskip) ? __ldg(p.Dskip + d) : 0.f;
     float4 *ck = p.ckpt + (g * p.nchunks) * (CW * CH) + warp * CH + lane;
+    const int64_t slot = (g * p.K + it.k) * (CW * CH) + warp * CH + lane;
 
     // ------------------------------------------------------------ 1. forward sweep
-    float4 h = make_float4(0.f, 0.f, 0.f, 0.f);
-    {
-        float hv[4];
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-            const int n = 4 * warp + j;
-            hv[j] = (dvalid && n < p.N && p.h0) ? __ldg(p.h0 + (b * p.D + d) * p.N + n) : 0.f;
-        }
-        h = make_float4(hv[0], hv[1], hv[2], hv[3]);
-    }
-    load_chunk<T>(smem, p, b, d0, 0, false);
+    float4 h = p.hs[slot];
+    load_chunk<T>(smem + (it.cb & 1) * S::buf, p, b, d0, it.cb * KC, false);
     cp_async_commit();
-    for (int64_t j = 0; j < p.nchunks; ++j) {
+    for (int64_t j = it.cb; j < it.ce; ++j) {
         unsigned char *buf = smem + (j & 1) * S::buf;
-        if (j + 1 < p.nchunks) {
+        if (j + 1 < it.ce) {
             load_chunk<T>(smem + ((j + 1) & 1) * S::buf, p, b, d0, (j + 1) * KC, false);
             cp_async_commit();
             cp_async_wait<1>();
@@ -231,16 +367,7 @@ __global__ void __launch_bounds__(NT) scan_bwd_kernel(const Params p) {
     }
 
     // ------------------------------------------------------------ 2. reverse sweep
-    float4 gq = make_float4(0.f, 0.f, 0.f, 0.f);  // dL/dh of the warp's four states
-    if (p.dh_last) {
-        float gv[4];
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-            const int n = 4 * warp + j;
-            gv[j] = (dvalid && n < p.N) ? __ldg(p.dh_last + (b * p.D + d) * p.N + n) : 0.f;
-        }
-        gq = make_float4(gv[0], gv[1], gv[2], gv[3]);
-    }
+    float4 gq = p.ge[slot];  // dL/dh of the warp's four states, from the segments after this one
     float4 dA = make_float4(0.f, 0.f, 0.f, 0.f);
     float dD = 0.f, dbias = 0.f;  // of channel `lane`, over this thread's (t, channel) pairs
     float4 *hb = reinterpret_cast<float4 *>(smem + S::off_h);
@@ -253,12 +380,12 @@ __global__ void __launch_bounds__(NT) scan_bwd_kernel(const Params p) {
     T *ddto = static_cast<T *>(p.ddt);
     T *dzo = static_cast<T *>(p.dz);
 
-    const int64_t last = p.nchunks - 1;
+    const int64_t last = it.ce - 1;
     load_chunk<T>(smem + (last & 1) * S::buf, p, b, d0, last * KC, true);
     cp_async_commit();
-    for (int64_t j = last; j >= 0; --j) {
+    for (int64_t j = last; j >= it.cb; --j) {
         const unsigned char *buf = smem + (j & 1) * S::buf;
-        if (j > 0) {
+        if (j > it.cb) {
             load_chunk<T>(smem + ((j - 1) & 1) * S::buf, p, b, d0, (j - 1) * KC, true);
             cp_async_commit();
             cp_async_wait<1>();
@@ -386,17 +513,13 @@ __global__ void __launch_bounds__(NT) scan_bwd_kernel(const Params p) {
         }
     }
 
-    // ------------------------------------------------------------ reductions, dh0
+    // ------------------------------------------------------------ reductions
     if (dvalid) {
         const float dav[4] = {dA.x, dA.y, dA.z, dA.w};
-        const float gv[4] = {gq.x, gq.y, gq.z, gq.w};
 #pragma unroll
         for (int k = 0; k < 4; ++k) {
             const int n = 4 * warp + k;
-            if (n < p.N) {
-                atomicAdd(p.dA + d * p.N + n, dav[k]);
-                if (p.dh0) p.dh0[(b * p.D + d) * p.N + n] = gv[k];
-            }
+            if (n < p.N) atomicAdd(p.dA + d * p.N + n, dav[k]);
         }
         if (p.dD) atomicAdd(p.dD + d, dD);
         if (p.dbias) atomicAdd(p.dbias + d, dbias);
@@ -407,6 +530,24 @@ bool aligned(const void *q, size_t a) { return (reinterpret_cast<uintptr_t>(q) &
 
 int64_t groups(const ssm_scan_bwd_args *a) { return a->batch * ((a->dim + CH - 1) / CH); }
 int64_t chunks(const ssm_scan_bwd_args *a) { return (a->seqlen + KC - 1) / KC; }
+
+// Segments: about kItems (group, segment) items in all (four waves of three blocks on
+// each of 148 SMs), each a whole number of chunks. Depends on the shapes only, so the
+// workspace size does too.
+constexpr int64_t kItems = 1800;
+int64_t seg_chunks(const ssm_scan_bwd_args *a) {
+    const int64_t n = chunks(a), G = groups(a);
+    const int64_t want = (n * G + kItems - 1) / kItems;
+    return want < 1 ? 1 : want;
+}
+int64_t segments(const ssm_scan_bwd_args *a) {
+    const int64_t sc = seg_chunks(a);
+    return (chunks(a) + sc - 1) / sc;
+}
+// Workspace: chunk checkpoints [G][nchunks][CW][CH] float4, then hloc, gloc, hs, ge
+// [G][K][CW][CH] float4 each, then sum of Delta [G][K][CH] float.
+size_t off_items(const ssm_scan_bwd_args *a) { return size_t(groups(a)) * size_t(chunks(a)) * CW * CH * 16; }
+size_t item_bytes(const ssm_scan_bwd_args *a) { return size_t(groups(a)) * size_t(segments(a)) * CW * CH * 16; }
 
 ssm_status validate(const ssm_scan_bwd_args *a) {
     if (!a) return SSM_ERR_INVALID;
@@ -447,7 +588,7 @@ extern "C" {
 
 size_t ssm_scan_bwd_workspace_size(const ssm_scan_bwd_args *a) {
     if (!a || a->batch < 0 || a->seqlen < 0 || a->dim < 0) return 0;
-    return size_t(groups(a)) * size_t(chunks(a)) * CW * CH * 16;
+    return off_items(a) + 4 * item_bytes(a) + size_t(groups(a)) * size_t(segments(a)) * CH * 4;
 }
 
 ssm_status ssm_scan_bwd(const ssm_scan_bwd_args *a, void *stream_) {
@@ -497,24 +638,42 @@ ssm_status ssm_scan_bwd(const ssm_scan_bwd_args *a, void *stream_) {
     p.dD = a->dD;
     p.dbias = a->ddt_bias;
     p.dh0 = a->dh0;
-    p.ckpt = static_cast<float4 *>(a->workspace);
+    p.G = groups(a);
+    p.K = segments(a);
+    p.segc = seg_chunks(a);
+    unsigned char *ws = static_cast<unsigned char *>(a->workspace);
+    p.ckpt = reinterpret_cast<float4 *>(ws);
+    p.hloc = reinterpret_cast<float4 *>(ws + off_items(a));
+    p.gloc = reinterpret_cast<float4 *>(ws + off_items(a) + item_bytes(a));
+    p.hs = reinterpret_cast<float4 *>(ws + off_items(a) + 2 * item_bytes(a));
+    p.ge = reinterpret_cast<float4 *>(ws + off_items(a) + 3 * item_bytes(a));
+    p.sdel = reinterpret_cast<float *>(ws + off_items(a) + 4 * item_bytes(a));
     p.softplus = (a->flags & SSM_DELTA_SOFTPLUS) != 0;
     p.bc_async = (a->dstate * es) % 16 == 0 && aligned(a->Bm, 16) && aligned(a->Cm, 16);
-    const int64_t G = groups(a);
-    if (G > INT32_MAX) return SSM_ERR_UNSUPPORTED;
-    void *kern;
+    const int64_t items = p.G * p.K;
+    if (items > INT32_MAX) return SSM_ERR_UNSUPPORTED;
+    void *local, *kern;
     size_t smem;
     if (a->dtype == SSM_BF16) {
+        local = reinterpret_cast<void *>(&scan_bwd_local_kernel<__nv_bfloat16>);
         kern = reinterpret_cast<void *>(&scan_bwd_kernel<__nv_bfloat16>);
         smem = Smem<__nv_bfloat16>::total;
     } else {
+        local = reinterpret_cast<void *>(&scan_bwd_local_kernel<float>);
         kern = reinterpret_cast<void *>(&scan_bwd_kernel<float>);
         smem = Smem<float>::total;
     }
-    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem)) != cudaSuccess)
+    if (cudaFuncSetAttribute(local, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem)) != cudaSuccess ||
+        cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem)) != cudaSuccess)
         return SSM_ERR_CUDA;
     void *args[] = {&p};
-    const cudaError_t e = cudaLaunchKernel(kern, dim3(unsigned(G)), dim3(NT), args, smem, stream);
+    if (cudaLaunchKernel(local, dim3(unsigned(items)), dim3(NT), args, smem, stream) != cudaSuccess)
+        return SSM_ERR_CUDA;
+    const int64_t threads = p.G * CW * CH;
+    if (cudaLaunchKernel(reinterpret_cast<void *>(&scan_bwd_combine_kernel), dim3(unsigned((threads + 255) / 256)),
+                         dim3(256), args, 0, stream) != cudaSuccess)
+        return SSM_ERR_CUDA;
+    const cudaError_t e = cudaLaunchKernel(kern, dim3(unsigned(items)), dim3(NT), args, smem, stream);
     return e == cudaSuccess ? SSM_OK : SSM_ERR_CUDA;
 }
 
