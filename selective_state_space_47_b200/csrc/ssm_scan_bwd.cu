@@ -142,11 +142,20 @@ __device__ __forceinline__ void load_chunk(unsigned char *buf, const Params &p, 
 __device__ __forceinline__ float delta_of(const float v, const bool softplus) { return softplus ? softplus_f(v) : v; }
 __device__ __forceinline__ float sigmoid_f(const float v) { return rcp_approx(1.0f + ex2_approx(-v * kLog2e)); }
 
-// Four consecutive entries of a [.][16] token row (B or C), widened.
+// Four consecutive entries of a [.][16] token row (B or C), widened: one 8-byte (bf16)
+// or 16-byte (float) load, the warp's four states being 4w .. 4w+3.
 template <typename T>
 __device__ __forceinline__ float4 row4(const unsigned char *base, const int r, const int n0) {
-    const T *p = reinterpret_cast<const T *>(base) + r * kMaxN + n0;
-    return make_float4(Tok<T>::to_f(p[0]), Tok<T>::to_f(p[1]), Tok<T>::to_f(p[2]), Tok<T>::to_f(p[3]));
+    return Tok<T>::quad(reinterpret_cast<const T *>(base) + r * kMaxN + n0);
+}
+
+// Delta of `rows` consecutive rows of a chunk starting at r0, for the thread's channel
+// (lane) and rows spread over the warps: out[(r - r0) * CH + lane]. Computed once per
+// (t, channel) instead of once per warp.
+template <typename T>
+__device__ __forceinline__ void delta_pass(const T *sdt, const int r0, const int rows, const float bias,
+                                           const bool softplus, float *out, const int warp, const int lane) {
+    for (int i = warp; i < rows; i += CW) out[i * CH + lane] = delta_of(Tok<T>::to_f(sdt[(r0 + i) * CH + lane]) + bias, softplus);
 }
 
 // One forward step of a lane's four states.
@@ -222,6 +231,8 @@ __global__ void __launch_bounds__(NT) scan_bwd_local_kernel(const Params p) {
     const float4 Aq = quad_of(p.A, d, d, dvalid, warp, p.N);
     const float bias = (dvalid && p.dt_bias) ? __ldg(p.dt_bias + d) : 0.f;
     const int64_t slot = (it.g * p.K + it.k) * (CW * CH) + warp * CH + lane;
+    float *dc = reinterpret_cast<float *>(smem + S::off_h);            // [KC][CH] Delta of the chunk
+    float *dqc = reinterpret_cast<float *>(smem + S::off_h) + KC * CH;  // [KC][CH] dq of the chunk
 
     float4 h = make_float4(0.f, 0.f, 0.f, 0.f);
     float sd = 0.f;
@@ -238,10 +249,11 @@ __global__ void __launch_bounds__(NT) scan_bwd_local_kernel(const Params p) {
         }
         __syncthreads();
         const T *sx = reinterpret_cast<const T *>(buf + S::o_x) + lane;
-        const T *sdt = reinterpret_cast<const T *>(buf + S::o_dt) + lane;
+        delta_pass<T>(reinterpret_cast<const T *>(buf + S::o_dt), 0, KC, bias, softplus, dc, warp, lane);
+        __syncthreads();
         const int tn = p.L - j * KC < KC ? int(p.L - j * KC) : KC;  // valid steps of the chunk
         for (int t = 0; t < tn; ++t) {
-            const float delta = delta_of(Tok<T>::to_f(sdt[t * CH]) + bias, softplus);
+            const float delta = dc[t * CH + lane];
             h = fwd_step(h, abar4(delta * kLog2e, Aq), delta * Tok<T>::to_f(sx[t * CH]),
                          row4<T>(buf + S::o_b, t, 4 * warp));
             sd += delta;
@@ -264,14 +276,20 @@ __global__ void __launch_bounds__(NT) scan_bwd_local_kernel(const Params p) {
             cp_async_wait<0>();
         }
         __syncthreads();
-        const T *sdt = reinterpret_cast<const T *>(buf + S::o_dt) + lane;
-        const T *sz = reinterpret_cast<const T *>(buf + S::o_z) + lane;
-        const T *sdy = reinterpret_cast<const T *>(buf + S::o_dy) + lane;
+        {
+            const T *sz = reinterpret_cast<const T *>(buf + S::o_z) + lane;
+            const T *sdy = reinterpret_cast<const T *>(buf + S::o_dy) + lane;
+            delta_pass<T>(reinterpret_cast<const T *>(buf + S::o_dt), 0, KC, bias, softplus, dc, warp, lane);
+            for (int t = warp; t < KC; t += CW) {
+                float dq = Tok<T>::to_f(sdy[t * CH]);
+                if (gate) dq *= silu_f(Tok<T>::to_f(sz[t * CH]));
+                dqc[t * CH + lane] = dq;
+            }
+        }
+        __syncthreads();
         const int tn = p.L - j * KC < KC ? int(p.L - j * KC) : KC;
         for (int t = tn - 1; t >= 0; --t) {
-            const float delta = delta_of(Tok<T>::to_f(sdt[t * CH]) + bias, softplus);
-            float dq = Tok<T>::to_f(sdy[t * CH]);
-            if (gate) dq *= silu_f(Tok<T>::to_f(sz[t * CH]));
+            const float delta = dc[t * CH + lane], dq = dqc[t * CH + lane];
             const float4 cv = row4<T>(buf + S::o_c, t, 4 * warp), a = abar4(delta * kLog2e, Aq);
             gl = make_float4(a.x * fmaf(dq, cv.x, gl.x), a.y * fmaf(dq, cv.y, gl.y), a.z * fmaf(dq, cv.z, gl.z),
                              a.w * fmaf(dq, cv.w, gl.w));
@@ -356,10 +374,12 @@ __global__ void __launch_bounds__(NT) scan_bwd_kernel(const Params p) {
         __syncthreads();
         ck[j * CW * CH] = h;
         const T *sx = reinterpret_cast<const T *>(buf + S::o_x) + lane;
-        const T *sdt = reinterpret_cast<const T *>(buf + S::o_dt) + lane;
+        float *dc = reinterpret_cast<float *>(smem + S::off_h);  // [KC][CH] Delta of the chunk (hb is free here)
+        delta_pass<T>(reinterpret_cast<const T *>(buf + S::o_dt), 0, KC, bias, softplus, dc, warp, lane);
+        __syncthreads();
 #pragma unroll 4
         for (int t = 0; t < KC; ++t) {
-            const float delta = delta_of(Tok<T>::to_f(sdt[t * CH]) + bias, softplus);
+            const float delta = dc[t * CH + lane];
             const float4 a = abar4(delta * kLog2e, Aq);
             h = fwd_step(h, a, delta * Tok<T>::to_f(sx[t * CH]), row4<T>(buf + S::o_b, t, 4 * warp));
         }
@@ -400,22 +420,32 @@ __global__ void __launch_bounds__(NT) scan_bwd_kernel(const Params p) {
         const T *sdy = reinterpret_cast<const T *>(buf + S::o_dy);
         const float4 hck = ck[j * CW * CH];
         // the state after the first half, from the checkpoint
+        delta_pass<T>(sdt, 0, TH, bias, softplus, sdel, warp, lane);
+        __syncthreads();
         float4 hmid = hck;
 #pragma unroll 4
         for (int t = 0; t < TH; ++t) {
-            const float delta = delta_of(Tok<T>::to_f(sdt[t * CH + lane]) + bias, softplus);
+            const float delta = sdel[t * CH + lane];
             hmid = fwd_step(hmid, abar4(delta * kLog2e, Aq), delta * Tok<T>::to_f(sx[t * CH + lane]),
                             row4<T>(buf + S::o_b, t, 4 * warp));
         }
+        __syncthreads();  // sdel is rewritten for the second half
         for (int half = 1; half >= 0; --half) {
             const int tb = half * TH;                   // first step of the half in the chunk
             const float4 hs = half ? hmid : hck;        // state before the half
+            // (a0) per (t, channel): Delta and sigma(v) of the half
+            for (int s = warp; s < TH; s += CW) {
+                const float v = Tok<T>::to_f(sdt[(tb + s) * CH + lane]) + bias;
+                sdel[s * CH + lane] = delta_of(v, softplus);
+                ssig[s * CH + lane] = softplus ? sigmoid_f(v) : 1.f;
+            }
+            __syncthreads();
             // (a) recompute the half's states and the warps' partial readouts
             float4 hh = hs;
 #pragma unroll 4
             for (int s = 0; s < TH; ++s) {
                 const int t = tb + s;
-                const float delta = delta_of(Tok<T>::to_f(sdt[t * CH + lane]) + bias, softplus);
+                const float delta = sdel[s * CH + lane];
                 hh = fwd_step(hh, abar4(delta * kLog2e, Aq), delta * Tok<T>::to_f(sx[t * CH + lane]),
                               row4<T>(buf + S::o_b, t, 4 * warp));
                 hb[(s * CW + warp) * CH + lane] = hh;
@@ -423,7 +453,7 @@ __global__ void __launch_bounds__(NT) scan_bwd_kernel(const Params p) {
                 pa[(warp * TH + s) * CH + lane] = fmaf(c4.x, hh.x, fmaf(c4.y, hh.y, fmaf(c4.z, hh.z, c4.w * hh.w)));
             }
             __syncthreads();
-            // (b) per (t, channel): readout, gate, dq, dz, Delta, sigma(v)
+            // (b) per (t, channel): readout, gate, dq, dz
 #pragma unroll
             for (int i = 0; i < TH / CW; ++i) {
                 const int s = warp * (TH / CW) + i, t = tb + s;
@@ -431,7 +461,6 @@ __global__ void __launch_bounds__(NT) scan_bwd_kernel(const Params p) {
                 const float xv = Tok<T>::to_f(sx[t * CH + lane]);
                 const float q = pa[(0 * TH + s) * CH + lane] + pa[(1 * TH + s) * CH + lane] +
                                 pa[(2 * TH + s) * CH + lane] + pa[(3 * TH + s) * CH + lane] + dskip * xv;
-                const float v = Tok<T>::to_f(sdt[t * CH + lane]) + bias;
                 float dq = Tok<T>::to_f(sdy[t * CH + lane]);
                 if (gate) {
                     const float zv = Tok<T>::to_f(sz[t * CH + lane]), sg = sigmoid_f(zv);
@@ -441,8 +470,6 @@ __global__ void __launch_bounds__(NT) scan_bwd_kernel(const Params p) {
                 }
                 if (tg < p.L) dD = fmaf(dq, xv, dD);
                 sdq[s * CH + lane] = dq;
-                sdel[s * CH + lane] = delta_of(v, softplus);
-                ssig[s * CH + lane] = softplus ? sigmoid_f(v) : 1.f;
             }
             __syncthreads();
             // (c) the adjoint, backwards over the half (steps past L are skipped)
