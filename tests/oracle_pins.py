@@ -532,3 +532,39 @@ def pin_bwd_bf16_storage(orc, seed=17):
 
 
 ALL_PINS += [pin_bwd_finite_differences, pin_bwd_finite_differences_plain, pin_bwd_bf16_storage]
+
+
+def pin_ssd_semiseparable_form(orc, seed=18):
+    """With one scalar A per channel (A[d, n] = a_d for every n, the Mamba-2 restriction), the
+    scan equals multiplication by a lower-triangular semiseparable matrix:
+    y_t = sum_{s<=t} (C_t . B_s) exp(a_d (S_t - S_s)) Delta_s x_s + exp(a_d S_t) C_t . h0,
+    S_t = Delta_1 + ... + Delta_t (the structured state space duality of the Mamba-2 article,
+    mugbit.ir, "Mamba-2 and SSD" section: the recurrence as a structured matrix product).
+    The matrix is formed with numpy and applied as one product, independently of the
+    oracle's loop."""
+    rng = _rng(seed)
+    Bsz, L, Dm, N = 2, 23, 3, 4
+    x = rng.standard_normal((Bsz, L, Dm)).astype(np.float32)
+    dt = (0.5 * rng.standard_normal((Bsz, L, Dm))).astype(np.float32)
+    Bm = rng.standard_normal((Bsz, L, N)).astype(np.float32)
+    Cm = rng.standard_normal((Bsz, L, N)).astype(np.float32)
+    a = (-0.3 - rng.random(Dm) * 2.0).astype(np.float32)
+    A = np.repeat(a[:, None], N, axis=1)
+    bias = (0.3 * rng.standard_normal(Dm)).astype(np.float32)
+    h0 = rng.standard_normal((Bsz, Dm, N)).astype(np.float32)
+    y, _ = orc.scan(x, dt, A, Bm, Cm, dt_bias=bias, h0=h0)
+    delta = _softplus(dt.astype(np.float64) + bias.astype(np.float64))       # [Bsz, L, Dm]
+    S = np.cumsum(delta, axis=1)
+    ref = np.empty((Bsz, L, Dm))
+    tri = np.tril(np.ones((L, L), dtype=bool))
+    for b in range(Bsz):
+        CB = Cm[b].astype(np.float64) @ Bm[b].astype(np.float64).T            # [L, L]: C_t . B_s
+        for d in range(Dm):
+            decay = np.where(tri, np.exp(a[d] * (S[b, :, d][:, None] - S[b, :, d][None, :])), 0.0)
+            M = CB * decay                                                     # the semiseparable matrix
+            u = delta[b, :, d] * x[b, :, d]
+            ref[b, :, d] = M @ u + np.exp(a[d] * S[b, :, d]) * (Cm[b].astype(np.float64) @ h0[b, d].astype(np.float64))
+    assert _rel(y - ref, ref) < 1e-11, "scalar-A scan differs from its semiseparable matrix form"
+
+
+ALL_PINS.append(pin_ssd_semiseparable_form)

@@ -73,6 +73,22 @@ def test_scan_random_A_uses_general_path(ssm):
     assert y_err(y, y_ref) <= 1e-2 and h_err(h, h_ref) <= 1e-2
 
 
+@pytest.mark.parametrize("general", [False, True], ids=["auto", "generalA"])
+def test_scalar_A_per_head(ssm, general):
+    """The Mamba-2 restriction: one scalar A per head (A[d, n] = a_h for every n and every
+    channel of the head; rows with zero difference, which the arithmetic-row path takes
+    with ratio 1). The recurrent form of the structured state space duality."""
+    Bsz, L, Dm, N, heads = 2, 3000, 128, 16, 4
+    g = torch.Generator().manual_seed(6)
+    inp = synth.scan_inputs(Bsz, L, Dm, N, torch.bfloat16, seed=78, h0=True)
+    a = -torch.exp(torch.rand(heads, generator=g) * 2.0 - 1.0)
+    inp["A"] = a.repeat_interleave(Dm // heads)[:, None].expand(Dm, N).contiguous()
+    y_ref, h_ref = oracle_scan(inp)
+    y, h = _run(ssm, _to(inp, "cuda"), general_A=general)
+    torch.cuda.synchronize()
+    assert y_err(y, y_ref) <= 1e-2 and h_err(h, h_ref) <= 1e-2
+
+
 def test_scan_without_softplus(ssm):
     inp = synth.scan_inputs(1, 300, 32, 16, torch.float32, seed=78)
     inp["dt"] = inp["dt"].abs() * 0.05
