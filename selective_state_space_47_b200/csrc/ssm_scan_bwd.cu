@@ -62,7 +62,9 @@ struct Params {
 // Shared memory: two chunk buffers (x | dt | z | dy as [KC][CH] tokens, B | C as
 // [KC][16] tokens), the recomputed states of a half [TH][CW][CH] float4, per-warp
 // partial sums [CW][TH][CH] (readout, then dDelta) and [CW][TH][CH] (dx), and per
-// (t, channel) values dq, Delta, sigma(v) [TH][CH].
+// (t, channel) values dq, Delta, sigma(v) [TH][CH]. Where no half's states are live
+// (the forward sweeps and the local pass) their area holds a chunk's Delta (and dq)
+// per (t, channel): each is computed once there, not once per warp.
 template <typename T>
 struct Smem {
     static constexpr size_t tok = size_t(KC) * CH * sizeof(T);
