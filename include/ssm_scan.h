@@ -239,10 +239,10 @@ ssm_status ssm_scan_fwd_host(const ssm_scan_args *args, int64_t chunk_len, void 
  * (about 1,800 (group, segment) items in all), each a thread block: a first pass gives
  * each segment's end state from a zero start and its adjoint at the start from a zero
  * end, a short combine pass chains them into every segment's true start state and end
- * adjoint (both recurrences are linear), and the main pass runs a forward sweep per
- * segment that keeps only the state at the start of every 32 steps (in the workspace),
- * then walks the segment backwards, recomputing each 16 steps' states from those
- * checkpoints.
+ * adjoint (both recurrences are linear). The first pass also keeps, in the workspace,
+ * the zero-start state at every 32 steps and the sum of Delta up to there, from which
+ * the main pass rebuilds the true state at those points; it then walks each segment
+ * backwards, recomputing each 16 steps' states from them.
  *
  * Shapes and types as for ssm_scan_fwd; x, dt, z, Bm, Cm, A, Dskip, dt_bias, h0 are the
  * forward's inputs. Outputs (all overwritten; device memory the caller owns):
@@ -256,7 +256,7 @@ ssm_status ssm_scan_fwd_host(const ssm_scan_args *args, int64_t chunk_len, void 
  * can vary from run to run with the order of the additions. Only SSM_DELTA_SOFTPLUS
  * (and SSM_A_GENERAL, which changes nothing here) is honoured; SSM_EXACT_ZOH returns
  * SSM_ERR_UNSUPPORTED, and the short convolution has no backward here. The workspace
- * holds the checkpoints (64 bytes per channel and 32 steps: about one [B, L, D] bfloat16
+ * holds the checkpoints (68 bytes per channel and 32 steps: about one [B, L, D] bfloat16
  * tensor) and 8.3 KB per item: ssm_scan_bwd_workspace_size() bytes, 16-byte aligned.
  * Errors: as ssm_scan_fwd (x, dt, z, dy and workspace on 16 bytes).
  */

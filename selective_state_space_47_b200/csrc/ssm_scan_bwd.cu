@@ -11,13 +11,14 @@
 // adjoint runs backward, g <- Abar_t (g + dq_t C_t), without reading h. So:
 //   A. scan_bwd_local_kernel, all items at once: the segment's end state from a zero
 //      start, its adjoint at the start from a zero end, and sum_t Delta_t (the product
-//      of the segment's Abar is exp(A sum_t Delta_t)).
+//      of the segment's Abar is exp(A sum_t Delta_t)); on the way, the zero-start state
+//      and the running sum of Delta at the start of every chunk of KC = 32 steps.
 //   B. scan_bwd_combine_kernel, one thread per (group, four states, channel): walks the
 //      K segments forward and backward, giving each segment its true start state and
 //      end adjoint (and dh0).
 //   C. scan_bwd_kernel, all items at once, from those:
-//   1. Forward sweep: the state at the start of every chunk of KC = 32 steps goes to
-//      the workspace (2 KB per chunk and group), nothing else is kept.
+//   1. The true state at the start of chunk j is the zero-start one plus
+//      exp(A sum Delta) times the segment's true start state: no forward sweep.
 //   2. Reverse sweep over the chunks, each in two halves of TH = 16 steps (second
 //      half first): the half's states are recomputed from the chunk's checkpoint into
 //      shared memory, then walked backwards with the adjoint g = dL/dh:
@@ -53,7 +54,8 @@ struct Params {
     const float *A, *Dskip, *dt_bias, *h0, *dh_last;
     void *dx, *ddt, *dz;
     float *dB, *dC, *dA, *dD, *dbias, *dh0;
-    float4 *ckpt;  // [G][nchunks][CW][CH] states at chunk starts
+    float4 *ckpt;  // [G][nchunks][CW][CH] zero-start states at chunk starts (from the segment start)
+    float *cumd;   // [G][nchunks][CH] sum of Delta from the segment start to each chunk start
     float4 *hloc, *gloc, *hs, *ge;  // [G][K][CW][CH]: local end state and start adjoint; true start state, end adjoint
     float *sdel;                    // [G][K][CH] sum of Delta over the segment
     int softplus, bc_async;
@@ -236,6 +238,7 @@ __global__ void __launch_bounds__(NT) scan_bwd_local_kernel(const Params p) {
     float *dc = reinterpret_cast<float *>(smem + S::off_h);            // [KC][CH] Delta of the chunk
     float *dqc = reinterpret_cast<float *>(smem + S::off_h) + KC * CH;  // [KC][CH] dq of the chunk
 
+    float4 *ck = p.ckpt + (it.g * p.nchunks) * (CW * CH) + warp * CH + lane;
     float4 h = make_float4(0.f, 0.f, 0.f, 0.f);
     float sd = 0.f;
     load_chunk<T>(smem + (it.cb & 1) * S::buf, p, b, d0, it.cb * KC, false);
@@ -250,6 +253,8 @@ __global__ void __launch_bounds__(NT) scan_bwd_local_kernel(const Params p) {
             cp_async_wait<0>();
         }
         __syncthreads();
+        ck[j * CW * CH] = h;  // the zero-start state and the sum of Delta at the chunk's start
+        if (warp == 0) p.cumd[(it.g * p.nchunks + j) * CH + lane] = sd;
         const T *sx = reinterpret_cast<const T *>(buf + S::o_x) + lane;
         delta_pass<T>(reinterpret_cast<const T *>(buf + S::o_dt), 0, KC, bias, softplus, dc, warp, lane);
         __syncthreads();
@@ -360,33 +365,11 @@ __global__ void __launch_bounds__(NT) scan_bwd_kernel(const Params p) {
     float4 *ck = p.ckpt + (g * p.nchunks) * (CW * CH) + warp * CH + lane;
     const int64_t slot = (g * p.K + it.k) * (CW * CH) + warp * CH + lane;
 
-    // ------------------------------------------------------------ 1. forward sweep
-    float4 h = p.hs[slot];
-    load_chunk<T>(smem + (it.cb & 1) * S::buf, p, b, d0, it.cb * KC, false);
-    cp_async_commit();
-    for (int64_t j = it.cb; j < it.ce; ++j) {
-        unsigned char *buf = smem + (j & 1) * S::buf;
-        if (j + 1 < it.ce) {
-            load_chunk<T>(smem + ((j + 1) & 1) * S::buf, p, b, d0, (j + 1) * KC, false);
-            cp_async_commit();
-            cp_async_wait<1>();
-        } else {
-            cp_async_wait<0>();
-        }
-        __syncthreads();
-        ck[j * CW * CH] = h;
-        const T *sx = reinterpret_cast<const T *>(buf + S::o_x) + lane;
-        float *dc = reinterpret_cast<float *>(smem + S::off_h);  // [KC][CH] Delta of the chunk (hb is free here)
-        delta_pass<T>(reinterpret_cast<const T *>(buf + S::o_dt), 0, KC, bias, softplus, dc, warp, lane);
-        __syncthreads();
-#pragma unroll 4
-        for (int t = 0; t < KC; ++t) {
-            const float delta = dc[t * CH + lane];
-            const float4 a = abar4(delta * kLog2e, Aq);
-            h = fwd_step(h, a, delta * Tok<T>::to_f(sx[t * CH]), row4<T>(buf + S::o_b, t, 4 * warp));
-        }
-        __syncthreads();  // the buffer is refilled next
-    }
+    // ------------------------------------------------------------ 1. chunk starts
+    // The true state at the start of chunk j: ck[j] (from a zero start at the segment's
+    // start) + exp(A sum of Delta up to the chunk) times the segment's true start state.
+    const float4 hseg = p.hs[slot];
+    const float *cum = p.cumd + (g * p.nchunks) * CH + lane;
 
     // ------------------------------------------------------------ 2. reverse sweep
     float4 gq = p.ge[slot];  // dL/dh of the warp's four states, from the segments after this one
@@ -420,7 +403,9 @@ __global__ void __launch_bounds__(NT) scan_bwd_kernel(const Params p) {
         const T *sdt = reinterpret_cast<const T *>(buf + S::o_dt);
         const T *sz = reinterpret_cast<const T *>(buf + S::o_z);
         const T *sdy = reinterpret_cast<const T *>(buf + S::o_dy);
-        const float4 hck = ck[j * CW * CH];
+        const float4 hz = ck[j * CW * CH], P = abar4(cum[j * CH] * kLog2e, Aq);
+        const float4 hck = make_float4(fmaf(P.x, hseg.x, hz.x), fmaf(P.y, hseg.y, hz.y), fmaf(P.z, hseg.z, hz.z),
+                                       fmaf(P.w, hseg.w, hz.w));
         // the state after the first half, from the checkpoint
         delta_pass<T>(sdt, 0, TH, bias, softplus, sdel, warp, lane);
         __syncthreads();
@@ -574,7 +559,8 @@ int64_t segments(const ssm_scan_bwd_args *a) {
     return (chunks(a) + sc - 1) / sc;
 }
 // Workspace: chunk checkpoints [G][nchunks][CW][CH] float4, then hloc, gloc, hs, ge
-// [G][K][CW][CH] float4 each, then sum of Delta [G][K][CH] float.
+// [G][K][CW][CH] float4 each, sum of Delta per segment [G][K][CH] float, and the sum of
+// Delta up to every chunk start [G][nchunks][CH] float.
 size_t off_items(const ssm_scan_bwd_args *a) { return size_t(groups(a)) * size_t(chunks(a)) * CW * CH * 16; }
 size_t item_bytes(const ssm_scan_bwd_args *a) { return size_t(groups(a)) * size_t(segments(a)) * CW * CH * 16; }
 
@@ -617,7 +603,8 @@ extern "C" {
 
 size_t ssm_scan_bwd_workspace_size(const ssm_scan_bwd_args *a) {
     if (!a || a->batch < 0 || a->seqlen < 0 || a->dim < 0) return 0;
-    return off_items(a) + 4 * item_bytes(a) + size_t(groups(a)) * size_t(segments(a)) * CH * 4;
+    return off_items(a) + 4 * item_bytes(a) + size_t(groups(a)) * size_t(segments(a)) * CH * 4 +
+           size_t(groups(a)) * size_t(chunks(a)) * CH * 4;
 }
 
 ssm_status ssm_scan_bwd(const ssm_scan_bwd_args *a, void *stream_) {
@@ -677,6 +664,7 @@ ssm_status ssm_scan_bwd(const ssm_scan_bwd_args *a, void *stream_) {
     p.hs = reinterpret_cast<float4 *>(ws + off_items(a) + 2 * item_bytes(a));
     p.ge = reinterpret_cast<float4 *>(ws + off_items(a) + 3 * item_bytes(a));
     p.sdel = reinterpret_cast<float *>(ws + off_items(a) + 4 * item_bytes(a));
+    p.cumd = p.sdel + size_t(p.G) * size_t(p.K) * CH;
     p.softplus = (a->flags & SSM_DELTA_SOFTPLUS) != 0;
     p.bc_async = (a->dstate * es) % 16 == 0 && aligned(a->Bm, 16) && aligned(a->Cm, 16);
     const int64_t items = p.G * p.K;

@@ -223,16 +223,18 @@ def _bwd_args(**kw):
 
 
 def test_bwd_workspace_size(lib):
-    """Checkpoints: one float4 per (group, 32-step chunk, warp, lane); per (group, segment)
-    item four float4 per (warp, lane) and one float per lane. Segments: whole chunks, about
-    1800 items in all."""
+    """Checkpoints: one float4 per (group, 32-step chunk, warp, lane) and one float per
+    (group, chunk, lane); per (group, segment) item four float4 per (warp, lane) and one
+    float per lane. Segments: whole chunks, about 1800 items in all."""
     a = _bwd_args()
     a.batch, a.seqlen, a.dim = 3, 1000, 100             # 12 groups, 32 chunks: one chunk per segment
     G, nch, K = 12, 32, 32
-    assert lib.ssm_scan_bwd_workspace_size(ctypes.byref(a)) == G * nch * 2048 + 4 * G * K * 2048 + G * K * 128
+    assert lib.ssm_scan_bwd_workspace_size(ctypes.byref(a)) == \
+        G * nch * 2048 + 4 * G * K * 2048 + G * K * 128 + G * nch * 128
     a.batch, a.seqlen, a.dim = 1, 262144, 5120           # 160 groups, 8192 chunks: 729 per segment
     G, nch, K = 160, 8192, 12
-    assert lib.ssm_scan_bwd_workspace_size(ctypes.byref(a)) == G * nch * 2048 + 4 * G * K * 2048 + G * K * 128
+    assert lib.ssm_scan_bwd_workspace_size(ctypes.byref(a)) == \
+        G * nch * 2048 + 4 * G * K * 2048 + G * K * 128 + G * nch * 128
     a.seqlen = -1
     assert lib.ssm_scan_bwd_workspace_size(ctypes.byref(a)) == 0
     assert lib.ssm_scan_bwd_workspace_size(None) == 0
