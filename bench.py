@@ -16,7 +16,6 @@ over ranks of the device-timed region; value = updates of all ranks / that time.
 import argparse
 import hashlib
 import json
-import math
 import os
 import statistics
 import subprocess

@@ -6,7 +6,6 @@ timed region is the slowest rank's, and the whole-job value sums all ranks' work
 import os
 import socket
 
-import torch
 import torch.distributed as dist
 import torch.multiprocessing as mp
 

@@ -8,7 +8,6 @@ import numpy as np
 import pytest
 import torch
 
-import oracle
 from selective_state_space_47_b200 import synth
 from tests.conftest import cuda_available
 from tests.gpu_util import TOL, dtype_name, h_err, oracle_scan, y_err

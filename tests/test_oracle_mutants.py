@@ -4,7 +4,6 @@ The copy is compiled into a temporary directory; the oracle as built is untouche
 This shows that the pins constrain every term of the oracle: a dropped term, a
 wrong sign, a swapped or shifted index, a transposed operand.
 """
-import os
 import subprocess
 
 import pytest
