@@ -568,3 +568,29 @@ def pin_ssd_semiseparable_form(orc, seed=18):
 
 
 ALL_PINS.append(pin_ssd_semiseparable_form)
+
+
+def pin_segment_affine_maps(orc, seed=19):
+    """Across a segment of the sequence both recurrences are affine with the same slope
+    P = exp(A sum_t Delta_t): the end state is P h_start + (the end state from a zero
+    start), and the adjoint passed out of the segment's start is P g_end + (the one from a
+    zero g_end). This is what lets a segment's work start before its neighbours' is done
+    (Mamba summary, hardware-aware algorithm paragraph: the parallel scan). Checked on the
+    oracle's forward (h_L against h0) and backward (dh0 against dh_last) by superposition."""
+    rng = _rng(seed)
+    inp = _bwd_case(rng, 2, 17, 3, 4)
+    dy = rng.standard_normal((2, 17, 3)).astype(np.float32)
+    g_end = rng.standard_normal((2, 3, 4))
+    P = np.exp(inp["A"].astype(np.float64)[None] *
+               _softplus(inp["dt"].astype(np.float64) + inp["dt_bias"].astype(np.float64)).sum(axis=1)[:, :, None])
+    args = (inp["x"], inp["dt"], inp["A"], inp["B"], inp["C"])
+    kw = dict(D=inp["D"], z=inp["z"], dt_bias=inp["dt_bias"])
+    _, h_full = orc.scan(*args, h0=inp["h0"], **kw)
+    _, h_zero = orc.scan(*args, **kw)
+    assert _rel(h_full - (P * inp["h0"] + h_zero), h_full) < 1e-12, "forward: end state not affine in h0"
+    g_full = orc.scan_bwd(*args, dy, dh_last=g_end, h0=inp["h0"], **kw)["dh0"]
+    g_zero = orc.scan_bwd(*args, dy, h0=inp["h0"], **kw)["dh0"]
+    assert _rel(g_full - (P * g_end + g_zero), g_full) < 1e-12, "backward: start adjoint not affine in dh_last"
+
+
+ALL_PINS.append(pin_segment_affine_maps)
