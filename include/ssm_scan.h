@@ -99,7 +99,8 @@ typedef struct {
 
 /*
  * Bytes of device workspace ssm_scan_fwd needs for these shapes (0 for invalid
- * arguments). The workspace holds the hand-over of the running state between
+ * arguments, for B = 0 or D = 0, which need none, and for more than 2^40 channel slots
+ * B x round_up(D, 32), which ssm_scan_fwd refuses with SSM_ERR_UNSUPPORTED). The workspace holds the hand-over of the running state between
  * consecutive time segments of a channel group, and a status word. It is small:
  * for B=1, L=262144, D=5120, N=16 it is about 330 KB. The library clears what it
  * needs at the start of each call, on the call's stream; one workspace must not
@@ -194,10 +195,23 @@ ssm_status ssm_workspace_status(const void *workspace, void *stream);
  *  - All calls share the one array and the library clears what must start at
  *    zero at each call, so calls that can overlap on the GPU (other streams,
  *    other host threads) race and must be serialised by the caller.
- *  - Its device-side status word also lives in that array; no call reports it.
+ *  - Its device-side status word also lives in that array: ssm_noalloc_status()
+ *    reads it back.
+ * Errors: those of ssm_scan_fwd (shapes, pointers and alignment are checked before
+ * the size bound), SSM_ERR_UNSUPPORTED for shapes beyond the array.
  * The pages have no counterpart: this entry point exists only for such callers.
  */
 ssm_status ssm_scan_fwd_noalloc(const ssm_scan_args *args, void *stream);
+
+/*
+ * Synchronises `stream` and returns the device-side status of the last
+ * ssm_scan_fwd_noalloc on the current device: SSM_OK, or SSM_ERR_TIMEOUT if a bounded
+ * wait for a carried state gave up (the y of that call is then not valid), as
+ * ssm_workspace_status does for a caller's workspace. It copies four bytes to a host
+ * variable and allocates nothing; SSM_ERR_CUDA if the copy or the synchronisation
+ * fails. Like the entry point above, it has no counterpart on the pages.
+ */
+ssm_status ssm_noalloc_status(void *stream);
 
 /*
  * The scan with its token tensors in HOST memory, for callers whose inputs arrive from
@@ -223,7 +237,9 @@ ssm_status ssm_scan_fwd_noalloc(const ssm_scan_args *args, void *stream);
  * first call before any stream capture); calls from several host threads are
  * serialised while they enqueue.
  * Errors: as ssm_scan_fwd; SSM_ERR_INVALID if chunk_len < 1 or staging is NULL or too
- * small; SSM_ERR_UNSUPPORTED if staging is not 256-byte aligned. There is no
+ * small; SSM_ERR_UNSUPPORTED if staging is not 256-byte aligned. When a call fails
+ * after it has queued copies, it waits for the library's copy streams before it
+ * returns, so the host buffers may be reused at once. There is no
  * counterpart on the pages: this is the host side of the layer's input and output.
  */
 size_t ssm_scan_host_staging_size(const ssm_scan_args *args, int64_t chunk_len);

@@ -27,8 +27,18 @@ def _ptr(t):
     return None if t is None else ctypes.c_void_p(t.data_ptr())
 
 
-def _stream_handle(stream):
-    s = torch.cuda.current_stream() if stream is None else stream
+def _resolve_stream(stream, dev):
+    """The stream a call on `dev`'s tensors is launched on: the caller's (which must
+    belong to `dev`), else `dev`'s current stream. The library plans and launches on
+    the current CUDA device, so every call below also runs with `dev` made current."""
+    if stream is None:
+        return torch.cuda.current_stream(dev)
+    if torch.device(stream.device) != torch.device(dev):
+        raise ValueError(f"stream belongs to {stream.device}, the tensors to {dev}")
+    return stream
+
+
+def _handle(s):
     return ctypes.c_void_p(s.cuda_stream)
 
 
@@ -142,16 +152,17 @@ def scan_fwd(x, dt, A, B, C, D=None, z=None, dt_bias=None, h0=None, *, delta_sof
     _need_conv(conv_w, conv_b, conv_x0, Bsz, Dm, tok, dev)
     args = _scan_args(x, dt, A, B, C, D, z, dt_bias, h0, y, h_last, _flags(delta_softplus, general_A, exact_zoh),
                       conv_w, conv_b, conv_x0)
+    s = _resolve_stream(stream, dev)
     nbytes = int(_native.lib().ssm_scan_workspace_size(ctypes.byref(args)))
     if workspace is None:
-        key = (dev, torch.cuda.current_stream(dev).cuda_stream if stream is None else stream.cuda_stream)
-        workspace = _default_ws.setdefault(key, ScanWorkspace())
+        workspace = _default_ws.setdefault((dev, s.cuda_stream), ScanWorkspace())
     ws = workspace.get(nbytes, dev) if isinstance(workspace, ScanWorkspace) else workspace
     if ws.numel() * ws.element_size() < nbytes:
         raise ValueError(f"workspace too small: {ws.numel() * ws.element_size()} < {nbytes} bytes")
     args.workspace = ctypes.c_void_p(ws.data_ptr())
     args.workspace_bytes = ws.numel() * ws.element_size()
-    _native.check(_native.lib().ssm_scan_fwd(ctypes.byref(args), _stream_handle(stream)), "ssm_scan_fwd")
+    with torch.cuda.device(dev):
+        _native.check(_native.lib().ssm_scan_fwd(ctypes.byref(args), _handle(s)), "ssm_scan_fwd")
     return (y, h_last) if return_last_state else y
 
 
@@ -212,7 +223,8 @@ def scan_fwd_host(x, dt, A, B, C, D=None, z=None, dt_bias=None, h0=None, *, chun
     args = _scan_args(x, dt, A, B, C, D, z, dt_bias, h0, y, h_last, _flags(delta_softplus, general_A, exact_zoh),
                       conv_w, conv_b, conv_x0)
     lib = _native.lib()
-    key = (dev, torch.cuda.current_stream(dev).cuda_stream if stream is None else stream.cuda_stream)
+    s = _resolve_stream(stream, dev)
+    key = (dev, s.cuda_stream)
     nbytes = int(lib.ssm_scan_workspace_size(ctypes.byref(args)))
     if workspace is None:
         workspace = _default_ws.setdefault(key, ScanWorkspace())
@@ -223,9 +235,9 @@ def scan_fwd_host(x, dt, A, B, C, D=None, z=None, dt_bias=None, h0=None, *, chun
     if staging is None:
         staging = _default_staging.setdefault(key, ScanWorkspace())
     st = staging.get(sbytes, dev) if isinstance(staging, ScanWorkspace) else staging
-    _native.check(lib.ssm_scan_fwd_host(ctypes.byref(args), int(chunk_len), ctypes.c_void_p(st.data_ptr()),
-                                        st.numel() * st.element_size(), _stream_handle(stream)),
-                  "ssm_scan_fwd_host")
+    with torch.cuda.device(dev):
+        _native.check(lib.ssm_scan_fwd_host(ctypes.byref(args), int(chunk_len), ctypes.c_void_p(st.data_ptr()),
+                                            st.numel() * st.element_size(), _handle(s)), "ssm_scan_fwd_host")
     return (y, h_last) if return_last_state else y
 
 
@@ -276,14 +288,18 @@ def scan_bwd(x, dt, A, B, C, dy, D=None, z=None, dt_bias=None, h0=None, dh_last=
     ws = workspace.get(nbytes, dev) if isinstance(workspace, ScanWorkspace) else workspace
     a.workspace = ctypes.c_void_p(ws.data_ptr())
     a.workspace_bytes = ws.numel() * ws.element_size()
-    _native.check(lib.ssm_scan_bwd(ctypes.byref(a), _stream_handle(stream)), "ssm_scan_bwd")
+    s = _resolve_stream(stream, dev)
+    with torch.cuda.device(dev):
+        _native.check(lib.ssm_scan_bwd(ctypes.byref(a), _handle(s)), "ssm_scan_bwd")
     return out
 
 
 def workspace_status(workspace, stream=None):
     """Synchronise and return the device status code of the last scan on this workspace."""
     ws = workspace.buf if isinstance(workspace, ScanWorkspace) else workspace
-    return int(_native.lib().ssm_workspace_status(ctypes.c_void_p(ws.data_ptr()), _stream_handle(stream)))
+    s = _resolve_stream(stream, ws.device)
+    with torch.cuda.device(ws.device):
+        return int(_native.lib().ssm_workspace_status(ctypes.c_void_p(ws.data_ptr()), _handle(s)))
 
 
 def step(x, dt, A, B, C, h, D=None, z=None, dt_bias=None, *, delta_softplus=True, general_A=False,
@@ -321,7 +337,8 @@ def step(x, dt, A, B, C, h, D=None, z=None, dt_bias=None, *, delta_softplus=True
     if conv_w is None:
         if conv_b is not None or conv_state is not None:
             raise ValueError("conv_b and conv_state need conv_w")
-        rc = _native.lib().ssm_step(*common, _ptr(h), _ptr(y), _stream_handle(stream))
+        with torch.cuda.device(dev):
+            rc = _native.lib().ssm_step(*common, _ptr(h), _ptr(y), _handle(_resolve_stream(stream, dev)))
         _native.check(rc, "ssm_step")
         return y
     _need(conv_w, "conv_w", (Dm, 4), torch.float32, dev)
@@ -330,7 +347,8 @@ def step(x, dt, A, B, C, h, D=None, z=None, dt_bias=None, *, delta_softplus=True
     if conv_state is None:
         raise ValueError("conv_state [B, 3, D] is required with conv_w")
     _need(conv_state, "conv_state", (Bsz, 3, Dm), tok, dev)
-    rc = _native.lib().ssm_step_conv(*common, _ptr(conv_w), _ptr(conv_b), _ptr(conv_state), _ptr(h), _ptr(y),
-                                     _stream_handle(stream))
+    with torch.cuda.device(dev):
+        rc = _native.lib().ssm_step_conv(*common, _ptr(conv_w), _ptr(conv_b), _ptr(conv_state), _ptr(h), _ptr(y),
+                                         _handle(_resolve_stream(stream, dev)))
     _native.check(rc, "ssm_step_conv")
     return y

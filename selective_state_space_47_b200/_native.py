@@ -14,8 +14,8 @@ SSM_TEST_DROP_HANDOFF = 0x80000000
 
 # Every symbol the header declares (checked by the CPU test suite).
 EXPORTS = ("ssm_scan_workspace_size", "ssm_scan_fwd", "ssm_step", "ssm_step_conv", "ssm_workspace_status",
-           "ssm_status_string", "ssm_scan_fwd_noalloc", "ssm_scan_host_staging_size", "ssm_scan_fwd_host",
-           "ssm_scan_bwd_workspace_size", "ssm_scan_bwd")
+           "ssm_status_string", "ssm_scan_fwd_noalloc", "ssm_noalloc_status", "ssm_scan_host_staging_size",
+           "ssm_scan_fwd_host", "ssm_scan_bwd_workspace_size", "ssm_scan_bwd")
 
 
 class ScanArgs(ctypes.Structure):
@@ -63,6 +63,8 @@ def lib():
         L.ssm_scan_fwd.restype = ctypes.c_int
         L.ssm_scan_fwd_noalloc.argtypes = [ctypes.POINTER(ScanArgs), vp]
         L.ssm_scan_fwd_noalloc.restype = ctypes.c_int
+        L.ssm_noalloc_status.argtypes = [vp]
+        L.ssm_noalloc_status.restype = ctypes.c_int
         L.ssm_scan_host_staging_size.argtypes = [ctypes.POINTER(ScanArgs), i64]
         L.ssm_scan_host_staging_size.restype = ctypes.c_size_t
         L.ssm_scan_fwd_host.argtypes = [ctypes.POINTER(ScanArgs), i64, vp, ctypes.c_size_t, vp]

@@ -140,9 +140,16 @@ ssm_status ssm_scan_fwd_host(const ssm_scan_args *a, int64_t chunk_len, void *st
     float *carry[2] = {reinterpret_cast<float *>(base + s.off_carry),
                        reinterpret_cast<float *>(base + s.off_carry + s.carry)};
     const int64_t nc = (a->seqlen + Lc - 1) / Lc;
-#define SSM_CK(call)                                  \
-    do {                                              \
-        if ((call) != cudaSuccess) return SSM_ERR_CUDA; \
+    // On an error after copies were queued, wait for both copy streams before returning,
+    // so that the caller may reuse or free its page-locked buffers at once.
+    auto fail = [&](ssm_status st) {
+        cudaStreamSynchronize(e.in);
+        cudaStreamSynchronize(e.out);
+        return st;
+    };
+#define SSM_CK(call)                                          \
+    do {                                                      \
+        if ((call) != cudaSuccess) return fail(SSM_ERR_CUDA); \
     } while (0)
     // Everything starts after the work already on `stream` (it may still use the staging memory).
     SSM_CK(cudaEventRecord(e.ev_start, stream));
@@ -176,7 +183,7 @@ ssm_status ssm_scan_fwd_host(const ssm_scan_args *a, int64_t chunk_len, void *st
         b.h_last = c == nc - 1 ? a->h_last : carry[c & 1];
         if (a->conv_w) b.conv_x0 = c == 0 ? a->conv_x0 : buf + s.off_x0;
         const ssm_status st = ssm_scan_fwd(&b, stream);
-        if (st != SSM_OK) return st;
+        if (st != SSM_OK) return fail(st);
         SSM_CK(cudaEventRecord(e.ev_scan[k], stream));
         // Copy out the y of chunk c.
         SSM_CK(cudaStreamWaitEvent(e.out, e.ev_scan[k], 0));

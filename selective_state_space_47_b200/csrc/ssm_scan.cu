@@ -271,13 +271,31 @@ size_t pick_smem(ssm_dtype dt, bool deep, bool conv) {
     return conv ? pick_smem_t<true>(dt, deep) : pick_smem_t<false>(dt, deep);
 }
 
-// Largest group count over both block shapes: bounds the flag and state arrays.
-int64_t max_groups(int64_t Bsz, int64_t D) { return Bsz * ((D + 15) / 16); }
+// Channel slots B x round_up(D, 32) beyond which no workspace is planned: far above any
+// shape whose tokens fit in memory, and low enough that no size below overflows 64 bits.
+constexpr uint64_t kMaxChannelSlots = uint64_t(1) << 40;
+
+// B x round_up(D, 32), or 0 when B or D is negative or the count exceeds kMaxChannelSlots
+// (tested by division, so nothing overflows on the way).
+uint64_t channel_slots(int64_t Bsz, int64_t D) {
+    if (Bsz <= 0 || D <= 0 || D > INT64_MAX - 31) return 0;
+    const uint64_t d32 = (uint64_t(D) + 31) / 32 * 32;
+    if (d32 > kMaxChannelSlots / uint64_t(Bsz)) return 0;
+    return uint64_t(Bsz) * d32;
+}
+
+// Largest group count over both block shapes (groups of 16 or 32 channels): bounds the
+// flag and state arrays; at most channel_slots / 16.
+size_t max_groups(int64_t Bsz, int64_t D) { return size_t(Bsz) * size_t((D + 15) / 16); }
 
 size_t ws_flags_off() { return kWsHeader; }
-size_t ws_carry_off(int64_t Bsz, int64_t D) { return round_up(kWsHeader + size_t(max_groups(Bsz, D)) * 4, 256); }
+size_t ws_carry_off(int64_t Bsz, int64_t D) { return round_up(kWsHeader + max_groups(Bsz, D) * 4, 256); }
+// Workspace bytes of a scan over B sequences of D channels; 0 for shapes channel_slots
+// refuses (and for B = 0 or D = 0, which need none).
 size_t ws_total(int64_t Bsz, int64_t D) {
-    return ws_carry_off(Bsz, D) + size_t(Bsz) * size_t(round_up(size_t(D), 32)) * kMaxN * 4;
+    const uint64_t slots = channel_slots(Bsz, D);
+    if (slots == 0) return 0;
+    return ws_carry_off(Bsz, D) + size_t(slots) * kMaxN * 4;
 }
 
 // Blocks per SM of the shallow and deep kernel configurations for a token type, with or
@@ -358,7 +376,8 @@ ssm_status check_common(int64_t Bsz, int64_t D, int64_t N, ssm_dtype dt, uint32_
     return SSM_OK;
 }
 
-ssm_status validate_scan(const ssm_scan_args *a) {
+// Shapes, flags, pointers and alignment of a scan; the workspace is checked separately.
+ssm_status validate_shapes(const ssm_scan_args *a) {
     if (!a) return SSM_ERR_INVALID;
     if (a->seqlen < 0) return SSM_ERR_INVALID;
     ssm_status s = check_common(a->batch, a->dim, a->dstate, a->dtype, a->flags);
@@ -381,6 +400,14 @@ ssm_status validate_scan(const ssm_scan_args *a) {
     if (!a->conv_w && (a->conv_b || a->conv_x0)) return SSM_ERR_INVALID;
     if (a->conv_w && !aligned(a->conv_w, 16)) return SSM_ERR_UNSUPPORTED;
     if (a->conv_x0 && !aligned(a->conv_x0, es)) return SSM_ERR_UNSUPPORTED;
+    if (a->batch > 0 && a->dim > 0 && channel_slots(a->batch, a->dim) == 0) return SSM_ERR_UNSUPPORTED;
+    return SSM_OK;
+}
+
+ssm_status validate_scan(const ssm_scan_args *a) {
+    const ssm_status s = validate_shapes(a);
+    if (s != SSM_OK) return s;
+    const bool work = a->batch > 0 && a->dim > 0 && a->seqlen > 0;
     if (work && (!a->workspace || a->workspace_bytes < ws_total(a->batch, a->dim))) return SSM_ERR_INVALID;
     return SSM_OK;
 }
@@ -608,7 +635,8 @@ ssm_status ssm_workspace_status(const void *workspace, void *stream_) {
 }
 
 ssm_status ssm_scan_fwd_noalloc(const ssm_scan_args *a, void *stream) {
-    if (!a || a->batch < 0 || a->dim < 0) return SSM_ERR_INVALID;
+    const ssm_status v = validate_shapes(a);  // before any size arithmetic on the shape
+    if (v != SSM_OK) return v;
     if (ws_total(a->batch, a->dim) > kStaticScratchBytes) return SSM_ERR_UNSUPPORTED;
     unsigned char *scratch = static_scratch();
     if (!scratch) return SSM_ERR_CUDA;
@@ -616,6 +644,16 @@ ssm_status ssm_scan_fwd_noalloc(const ssm_scan_args *a, void *stream) {
     b.workspace = scratch;
     b.workspace_bytes = kStaticScratchBytes;
     return ssm_scan_fwd(&b, stream);
+}
+
+ssm_status ssm_noalloc_status(void *stream_) {
+    if (!static_scratch()) return SSM_ERR_CUDA;
+    cudaStream_t stream = static_cast<cudaStream_t>(stream_);
+    uint32_t v = 0;  // the status word sits 4 bytes into the array, as in a caller's workspace
+    if (cudaMemcpyFromSymbolAsync(&v, g_scan_scratch, 4, 4, cudaMemcpyDeviceToHost, stream) != cudaSuccess ||
+        cudaStreamSynchronize(stream) != cudaSuccess)
+        return SSM_ERR_CUDA;
+    return v == 0 ? SSM_OK : static_cast<ssm_status>(v);
 }
 
 const char *ssm_status_string(ssm_status s) {

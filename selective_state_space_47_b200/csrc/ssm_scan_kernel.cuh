@@ -102,6 +102,7 @@ enum : int { F_FIRST = 1, F_LAST = 2, F_END = 4, F_STRUCT = 8 };
 
 struct TileMeta {
     long long g, k;  // channel group and time segment of the tile's item
+    int b, d0;       // the group's sequence and first channel (divided out once per item)
     int t0, tlen;    // first step of the tile and its number of valid steps
     int flags;       // F_FIRST | F_LAST | F_END | F_STRUCT
     int j;           // tile index inside the item
@@ -143,7 +144,7 @@ struct Layout {
     static constexpr size_t stage_bytes = x_bytes + 2 * tok_bytes + 2 * bc_bytes;
     static constexpr size_t stage_off = 0;
     static constexpr size_t rec_off = stage_off + STAGES * stage_bytes;
-    static constexpr size_t rec_bytes = size_t(BOX) * 8;            // float2 (u, Delta log2 e) per (t, c)
+    static constexpr size_t rec_bytes = size_t(BOX) * 8;            // float4 (u, Delta log2 e) x 2 per (t pair, c)
     static constexpr size_t bcf_off = rec_off + R_REC * rec_bytes;
     static constexpr size_t bcf_bytes = size_t(TT) * 32 * 4;        // [TT][B 16 | C 16] float
     static constexpr size_t part_off = bcf_off + R_REC * bcf_bytes;
@@ -223,86 +224,189 @@ __device__ __forceinline__ float2 zoh_weight(const float2 z, const float2 a, con
 }
 
 // ---------------------------------------------------------------- consumers
-// TT steps of one tile for one lane (its channel, the warp's four states), in
-// blocks of four steps. rec: this lane's records (stride CH float2 per step); bc: B
-// of the warp's states (stride 32 floats per step; C at +16); part: this lane's
-// partials (stride CH float4 per block of four steps). Aq: A[c][4w .. 4w+3]; del:
-// A[c][1] - A[c][0]; ZOH (exact zero-order hold): zA = A ln 2 and iA = 1/A of the
-// four states, and the records carry x in place of Delta x.
-template <bool STRUCT, bool ZOH>
-__device__ __forceinline__ void consume_tile(const float2 *__restrict__ rec, const float *__restrict__ bc,
+// 2^x on the FMA pipe for two values (x clamped to [-127, 127]): x = j + f with j the
+// nearest integer (x + 1.5 * 2^23 + 127 leaves j + 127 in the float's low mantissa
+// bits) and f in [-1/2, 1/2]; 2^f = 1 + c1 f + ... + c5 f^5, the minimax polynomial of
+// the relative error with the constant term fixed at 1 (Lawson's iteratively
+// reweighted least squares: 9.1e-8 before rounding, 1.7e-7 in float32), times 2^j
+// built from j + 127 in the exponent field, which is exactly 0 for j = -127 (the
+// flush to zero of the special-function unit's result there). 2^0 is exactly 1.
+// Takes part of the exponentials off the special-function unit.
+__device__ __forceinline__ float2 exp2_fma(float2 x) {
+    x.x = fminf(fmaxf(x.x, -127.f), 127.f);
+    x.y = fminf(fmaxf(x.y, -127.f), 127.f);
+    constexpr float kShift = 12583039.f;  // 1.5 * 2^23 + 127
+    const float2 t = __fadd2_rn(x, f2(kShift, kShift));
+    const float2 j = __fadd2_rn(t, f2(-kShift, -kShift));
+    const float2 f = __ffma2_rn(j, f2(-1.f, -1.f), x);
+    float2 q = __ffma2_rn(f, f2(1.326472848e-03f, 1.326472848e-03f), f2(9.671512991e-03f, 9.671512991e-03f));
+    q = __ffma2_rn(f, q, f2(5.550733581e-02f, 5.550733581e-02f));
+    q = __ffma2_rn(f, q, f2(2.402224243e-01f, 2.402224243e-01f));
+    q = __ffma2_rn(f, q, f2(6.931470037e-01f, 6.931470037e-01f));
+    q = __ffma2_rn(f, q, f2(1.f, 1.f));
+    return __fmul2_rn(q, f2(__uint_as_float(__float_as_uint(t.x) << 23), __uint_as_float(__float_as_uint(t.y) << 23)));
+}
+
+#ifndef SSM_FACTORS_AHEAD
+#define SSM_FACTORS_AHEAD 1  // one block per SM: exponentials formed one block ahead of the recurrence
+#endif
+#ifndef SSM_FMA_EXP
+#define SSM_FMA_EXP 0  // general path: exponentials on the FMA pipe per block of 16 (0, 2 or 4)
+#endif
+
+// One block of four steps for one lane: the factors Abar and the inputs u B of the
+// warp's four states (pairs 01 and 23) from the block's records (two steps each) and B
+// rows. The general path takes kPoly exponentials of state 4w+3 on the FMA pipe.
+template <bool STRUCT, bool ZOH, int kPoly>
+__device__ __forceinline__ void block_factors(const float4 r0, const float4 r1, const float4 (&b4)[4], const float4 Aq,
+                                              const float del, const float4 zA, const float4 iA, float2 (&a01)[4],
+                                              float2 (&a23)[4], float2 (&ub01)[4], float2 (&ub23)[4]) {
+    constexpr int S = 4;
+    const float2 p[S] = {f2(r0.x, r0.y), f2(r0.z, r0.w), f2(r1.x, r1.y), f2(r1.z, r1.w)};
+    if (STRUCT) {
+        float2 x[S];
+#pragma unroll
+        for (int s = 0; s < S; ++s) x[s] = __fmul2_rn(f2(p[s].y, p[s].y), f2(Aq.x, del));
+        float a0[S], r[S];
+#pragma unroll
+        for (int s = 0; s < S; ++s) {
+            a0[s] = ex2_approx(x[s].x);
+            r[s] = ex2_approx(x[s].y);
+        }
+#pragma unroll
+        for (int s = 0; s < S; ++s) a01[s] = f2(a0[s], a0[s] * r[s]);
+#pragma unroll
+        for (int s = 0; s < S; ++s) a23[s] = __fmul2_rn(a01[s], f2(r[s] * r[s], r[s] * r[s]));
+    } else {
+        static_assert(kPoly % 2 == 0 && kPoly <= S, "FMA-pipe exponentials go in pairs");
+        float2 x01[S], x23[S];
+#pragma unroll
+        for (int s = 0; s < S; ++s) {
+            x01[s] = __fmul2_rn(f2(p[s].y, p[s].y), f2(Aq.x, Aq.y));
+            x23[s] = __fmul2_rn(f2(p[s].y, p[s].y), f2(Aq.z, Aq.w));
+        }
+#pragma unroll
+        for (int s = 0; s < S; ++s) {
+            a01[s] = f2(ex2_approx(x01[s].x), ex2_approx(x01[s].y));
+            a23[s].x = ex2_approx(x23[s].x);
+            if (s < S - kPoly) a23[s].y = ex2_approx(x23[s].y);
+        }
+#pragma unroll
+        for (int s = S - kPoly; s < S; s += 2) {
+            const float2 e = exp2_fma(f2(x23[s].y, x23[s + 1].y));
+            a23[s].y = e.x;
+            a23[s + 1].y = e.y;
+        }
+    }
+#pragma unroll
+    for (int s = 0; s < S; ++s) {
+        ub01[s] = __fmul2_rn(f2(p[s].x, p[s].x), f2(b4[s].x, b4[s].y));
+        ub23[s] = __fmul2_rn(f2(p[s].x, p[s].x), f2(b4[s].z, b4[s].w));
+    }
+    if (ZOH) {  // the record carries x; Bbar x = B x (Abar - 1) / A
+#pragma unroll
+        for (int s = 0; s < S; ++s) {
+            const float delta = p[s].y * kLn2;
+            const float2 z01 = __fmul2_rn(f2(p[s].y, p[s].y), f2(zA.x, zA.y));
+            const float2 z23 = __fmul2_rn(f2(p[s].y, p[s].y), f2(zA.z, zA.w));
+            ub01[s] = __fmul2_rn(ub01[s], zoh_weight(z01, a01[s], f2(iA.x, iA.y), delta));
+            ub23[s] = __fmul2_rn(ub23[s], zoh_weight(z23, a23[s], f2(iA.z, iA.w), delta));
+        }
+    }
+}
+
+// The recurrence of one block of four steps and the partial readout over the warp's
+// four states, the last additions of two steps paired; returns the four partials.
+__device__ __forceinline__ float4 block_recur(const float2 (&a01)[4], const float2 (&a23)[4], const float2 (&ub01)[4],
+                                              const float2 (&ub23)[4], const float4 (&c4)[4], float2 &h01, float2 &h23) {
+    constexpr int S = 4;
+    float2 q[S];
+#pragma unroll
+    for (int s = 0; s < S; ++s) {
+        h01 = __ffma2_rn(a01[s], h01, ub01[s]);
+        h23 = __ffma2_rn(a23[s], h23, ub23[s]);
+        q[s] = __ffma2_rn(f2(c4[s].z, c4[s].w), h23, __fmul2_rn(f2(c4[s].x, c4[s].y), h01));
+    }
+    const float2 y01 = __fadd2_rn(f2(q[0].x, q[1].x), f2(q[0].y, q[1].y));
+    const float2 y23 = __fadd2_rn(f2(q[2].x, q[3].x), f2(q[2].y, q[3].y));
+    return make_float4(y01.x, y01.y, y23.x, y23.y);
+}
+
+// TT steps of one tile for one lane (its channel, the warp's four states), in blocks of
+// four steps, software-pipelined: the shared-memory operands of a block are loaded
+// LOOK blocks ahead of its recurrence and, with AHEAD, its factors (the exponentials and
+// u B) are formed one block ahead, so that the latency of the loads and of the
+// special-function unit overlaps the recurrence of the block before. rec: this lane's
+// records, one float4 (u, Delta log2 e) x 2 per two steps (stride CH); bc: B of the
+// warp's states (stride 32 floats per step; C at +16); part: this lane's partials
+// (stride CH float4 per block of four steps). Aq: A[c][4w .. 4w+3]; del: A[c][1] -
+// A[c][0]; ZOH (exact zero-order hold): zA = A ln 2 and iA = 1/A of the four states, and
+// the records carry x in place of Delta x.
+template <bool STRUCT, bool ZOH, bool AHEAD>
+__device__ __forceinline__ void consume_tile(const float4 *__restrict__ rec, const float *__restrict__ bc,
                                              float4 *__restrict__ part, const float4 Aq, const float del,
                                              const float4 zA, const float4 iA, float2 &h01, float2 &h23) {
-    constexpr int S = 4;
-#pragma unroll 2
-    for (int t0 = 0; t0 < TT; t0 += S) {
-        float2 p[S];
-        float4 b4[S], c4[S];
-#pragma unroll
-        for (int s = 0; s < S; ++s) p[s] = rec[(t0 + s) * CH];
-#pragma unroll
-        for (int s = 0; s < S; ++s) b4[s] = *reinterpret_cast<const float4 *>(bc + (t0 + s) * 32);  // uniform
-#pragma unroll
-        for (int s = 0; s < S; ++s) c4[s] = *reinterpret_cast<const float4 *>(bc + (t0 + s) * 32 + 16);
-        float2 a01[S], a23[S];
-        if (STRUCT) {
-            float2 x[S];
-#pragma unroll
-            for (int s = 0; s < S; ++s) x[s] = __fmul2_rn(f2(p[s].y, p[s].y), f2(Aq.x, del));
-            float a0[S], r[S];
-#pragma unroll
-            for (int s = 0; s < S; ++s) {
-                a0[s] = ex2_approx(x[s].x);
-                r[s] = ex2_approx(x[s].y);
-            }
-#pragma unroll
-            for (int s = 0; s < S; ++s) a01[s] = f2(a0[s], a0[s] * r[s]);
-#pragma unroll
-            for (int s = 0; s < S; ++s) a23[s] = __fmul2_rn(a01[s], f2(r[s] * r[s], r[s] * r[s]));
-        } else {
-            float2 x01[S], x23[S];
-#pragma unroll
-            for (int s = 0; s < S; ++s) {
-                x01[s] = __fmul2_rn(f2(p[s].y, p[s].y), f2(Aq.x, Aq.y));
-                x23[s] = __fmul2_rn(f2(p[s].y, p[s].y), f2(Aq.z, Aq.w));
-            }
-#pragma unroll
-            for (int s = 0; s < S; ++s) {
-                a01[s] = f2(ex2_approx(x01[s].x), ex2_approx(x01[s].y));
-                a23[s] = f2(ex2_approx(x23[s].x), ex2_approx(x23[s].y));
-            }
-        }
-        float2 ub01[S], ub23[S];
+    constexpr int S = 4, NB = TT / S;
+    constexpr int kPoly = (STRUCT || ZOH) ? 0 : SSM_FMA_EXP;
+    auto load = [&](int blk, float4 &r0, float4 &r1, float4 (&b4)[S], float4 (&c4)[S]) {
+        r0 = rec[(2 * blk) * CH];
+        r1 = rec[(2 * blk + 1) * CH];
 #pragma unroll
         for (int s = 0; s < S; ++s) {
-            ub01[s] = __fmul2_rn(f2(p[s].x, p[s].x), f2(b4[s].x, b4[s].y));
-            ub23[s] = __fmul2_rn(f2(p[s].x, p[s].x), f2(b4[s].z, b4[s].w));
+            b4[s] = *reinterpret_cast<const float4 *>(bc + (blk * S + s) * 32);  // warp-uniform
+            c4[s] = *reinterpret_cast<const float4 *>(bc + (blk * S + s) * 32 + 16);
         }
-        if (ZOH) {  // the record carries x; Bbar x = B x (Abar - 1) / A
+    };
+    if (AHEAD) {
+        float4 r0, r1, b4[S], c4[S], rn0, rn1, bn[S], cn[S];
+        float2 a01[S], a23[S], ub01[S], ub23[S];
+        float4 cc[S];  // C rows of the block whose factors are in a01 .. ub23
+        load(0, r0, r1, b4, c4);
+        block_factors<STRUCT, ZOH, kPoly>(r0, r1, b4, Aq, del, zA, iA, a01, a23, ub01, ub23);
 #pragma unroll
-            for (int s = 0; s < S; ++s) {
-                const float delta = p[s].y * kLn2;
-                const float2 z01 = __fmul2_rn(f2(p[s].y, p[s].y), f2(zA.x, zA.y));
-                const float2 z23 = __fmul2_rn(f2(p[s].y, p[s].y), f2(zA.z, zA.w));
-                ub01[s] = __fmul2_rn(ub01[s], zoh_weight(z01, a01[s], f2(iA.x, iA.y), delta));
-                ub23[s] = __fmul2_rn(ub23[s], zoh_weight(z23, a23[s], f2(iA.z, iA.w), delta));
+        for (int s = 0; s < S; ++s) cc[s] = c4[s];
+        load(1, rn0, rn1, bn, cn);
+#pragma unroll
+        for (int blk = 0; blk < NB; ++blk) {
+            float2 na01[S], na23[S], nub01[S], nub23[S];
+            float4 ncc[S];
+            if (blk + 1 < NB) {  // factors of the next block (its operands were loaded last time)
+                block_factors<STRUCT, ZOH, kPoly>(rn0, rn1, bn, Aq, del, zA, iA, na01, na23, nub01, nub23);
+#pragma unroll
+                for (int s = 0; s < S; ++s) ncc[s] = cn[s];
+            }
+            if (blk + 2 < NB) load(blk + 2, rn0, rn1, bn, cn);
+            part[blk * CH] = block_recur(a01, a23, ub01, ub23, cc, h01, h23);
+            if (blk + 1 < NB) {
+#pragma unroll
+                for (int s = 0; s < S; ++s) {
+                    a01[s] = na01[s];
+                    a23[s] = na23[s];
+                    ub01[s] = nub01[s];
+                    ub23[s] = nub23[s];
+                    cc[s] = ncc[s];
+                }
             }
         }
-        float2 g01[S], g23[S];
+    } else {
+        float4 r0, r1, b4[S], c4[S], rn0, rn1, bn[S], cn[S];
+        load(0, r0, r1, b4, c4);
 #pragma unroll
-        for (int s = 0; s < S; ++s) {
-            h01 = __ffma2_rn(a01[s], h01, ub01[s]);
-            h23 = __ffma2_rn(a23[s], h23, ub23[s]);
-            g01[s] = h01;
-            g23[s] = h23;
-        }
-        float yv[S];
+        for (int blk = 0; blk < NB; ++blk) {
+            if (blk + 1 < NB) load(blk + 1, rn0, rn1, bn, cn);
+            float2 a01[S], a23[S], ub01[S], ub23[S];
+            block_factors<STRUCT, ZOH, kPoly>(r0, r1, b4, Aq, del, zA, iA, a01, a23, ub01, ub23);
+            part[blk * CH] = block_recur(a01, a23, ub01, ub23, c4, h01, h23);
+            if (blk + 1 < NB) {
+                r0 = rn0;
+                r1 = rn1;
 #pragma unroll
-        for (int s = 0; s < S; ++s) {
-            const float2 yy = __ffma2_rn(f2(c4[s].z, c4[s].w), g23[s], __fmul2_rn(f2(c4[s].x, c4[s].y), g01[s]));
-            yv[s] = yy.x + yy.y;
+                for (int s = 0; s < S; ++s) {
+                    b4[s] = bn[s];
+                    c4[s] = cn[s];
+                }
+            }
         }
-        part[(t0 / 4) * CH] = make_float4(yv[0], yv[1], yv[2], yv[3]);
     }
 }
 
@@ -340,11 +444,10 @@ __device__ __forceinline__ void load_conv(const Params &p, const int64_t d, floa
     b = (ok && p.conv_b) ? __ldg(p.conv_b + d) : 0.f;
 }
 
-// The caller's three tokens before t = 0 for lane c of group g, oldest first; false
+// The caller's three tokens before t = 0 for channel d of sequence b, oldest first; false
 // (the halo keeps TMA's zeros) without a prefix or past the last channel.
 template <typename T>
-__device__ __forceinline__ bool conv_prefix(const Params &p, const long long g, const int c, float3 &x0) {
-    const int64_t b = g / p.Dg, d = (g % p.Dg) * CH + c;
+__device__ __forceinline__ bool conv_prefix(const Params &p, const int64_t b, const int64_t d, float3 &x0) {
     if (!p.conv_x0 || d >= p.D) return false;
     const T *src = static_cast<const T *>(p.conv_x0) + b * (KCONV - 1) * p.D + d;
     x0 = make_float3(Tok<T>::ldg(src), Tok<T>::ldg(src + p.D), Tok<T>::ldg(src + 2 * p.D));
@@ -359,7 +462,7 @@ __device__ __forceinline__ bool conv_prefix(const Params &p, const long long g, 
 // use_x0 / x0 as for conv_silu_rows), which is also written over the dt rows read.
 template <typename T, bool CONV>
 __device__ __forceinline__ void prologue_rows(const T *__restrict__ sx, T *__restrict__ sdt,
-                                              float2 *__restrict__ rec, const int t0, const int tlen,
+                                              float4 *__restrict__ rec, const int t0, const int tlen,
                                               const float bias, const bool softplus, const bool zoh,
                                               const float4 cw, const float cb, const bool use_x0, const float3 x0) {
     constexpr int NPR = TP / 2;  // pairs of steps
@@ -388,8 +491,8 @@ __device__ __forceinline__ void prologue_rows(const T *__restrict__ sx, T *__res
 #pragma unroll
     for (int q = 0; q < NPR; ++q) {
         const int t = t0 + 2 * q;
-        rec[t * CH] = t < tlen ? f2(u[q].x, dl[q].x) : f2(0.f, 0.f);
-        rec[(t + 1) * CH] = t + 1 < tlen ? f2(u[q].y, dl[q].y) : f2(0.f, 0.f);
+        const bool v0 = t < tlen, v1 = t + 1 < tlen;
+        rec[(t / 2) * CH] = make_float4(v0 ? u[q].x : 0.f, v0 ? dl[q].x : 0.f, v1 ? u[q].y : 0.f, v1 ? dl[q].y : 0.f);
     }
     if (CONV) {  // the epilogue's D u
 #pragma unroll
@@ -505,7 +608,7 @@ __global__ void __launch_bounds__(NTHREADS, C::MINB)
             }
         }
         long long li_g = 0, li_k = 0, li_beg = 0, li_end = 0;
-        int li_j = 0, li_n = 0;
+        int li_j = 0, li_n = 0, li_b = 0, li_d0 = 0;
         bool li_ok = false;
         auto claim = [&]() {
             unsigned int it = 0;
@@ -515,6 +618,8 @@ __global__ void __launch_bounds__(NTHREADS, C::MINB)
             if (li_ok) {
                 li_k = (long long)it / p.G;
                 li_g = (long long)it % p.G;
+                li_b = int(li_g / p.Dg);
+                li_d0 = int((li_g - (long long)li_b * p.Dg) * CH);
                 li_beg = li_k * p.seg_len;
                 li_end = min((long long)p.L, li_beg + p.seg_len);
                 li_n = int((li_end - li_beg + TT - 1) / TT);
@@ -530,6 +635,8 @@ __global__ void __launch_bounds__(NTHREADS, C::MINB)
             }
             TileMeta m;
             m.g = li_g;
+            m.b = li_b;
+            m.d0 = li_d0;
             m.k = li_k;
             m.j = li_j;
             m.t0 = int(li_beg + (long long)li_j * TT);
@@ -539,7 +646,7 @@ __global__ void __launch_bounds__(NTHREADS, C::MINB)
                 smeta[st] = m;
                 if (li_ok) {
                     unsigned char *stage = smem + S::stage_off + size_t(st) * S::stage_bytes;
-                    const int b = int(m.g / p.Dg), d0 = int((m.g % p.Dg) * CH);
+                    const int b = m.b, d0 = m.d0;
                     mbar_arrive_expect_tx(&bar_full[st], tx_bytes);
                     // CONV: the box starts HALO rows early (before t = 0 TMA reads zeros)
                     tma_load_3d(stage + S::st_x, &tm_x, &bar_full[st], d0, m.t0 - S::HALO, b);
@@ -575,7 +682,7 @@ __global__ void __launch_bounds__(NTHREADS, C::MINB)
                 break;
             }
             if (m.flags & F_FIRST) {
-                const int64_t d = (m.g % p.Dg) * CH + c;
+                const int64_t d = m.d0 + c;
                 dd = (d < p.D && p.Dskip) ? __ldg(p.Dskip + d) : 0.f;
             }
             const unsigned char *stage = smem + S::stage_off + size_t(st) * S::stage_bytes;
@@ -590,7 +697,7 @@ __global__ void __launch_bounds__(NTHREADS, C::MINB)
             fence_proxy_async_smem();         // y rows written by this thread -> visible to the TMA store
             epilogue_sync();
             if (h == 0 && lane == 0) {
-                const int b = int(m.g / p.Dg), d0 = int((m.g % p.Dg) * CH);
+                const int b = m.b, d0 = m.d0;
                 tma_store_3d(&tm_y, smem + S::yout_off + (i % YBUF) * S::yout_bytes, d0, m.t0, b);
                 bulk_commit();
                 bulk_wait_read<1>();  // the store of the previous tile has read its buffer
@@ -625,9 +732,9 @@ __global__ void __launch_bounds__(NTHREADS, C::MINB)
                 warp_arrive(&bar_rec_full[r]);
                 break;
             }
-            const int64_t b = m.g / p.Dg;
+            const int64_t b = m.b;
             if (m.flags & F_FIRST) {  // new item: channel parameters and the structure of A
-                const int64_t d = (m.g % p.Dg) * CH + c;
+                const int64_t d = m.d0 + c;
                 const bool ok = d < p.D;
                 bias_c = (ok && p.dt_bias) ? __ldg(p.dt_bias + d) : 0.f;
                 if (CONV) load_conv(p, d, cw, cb);
@@ -642,9 +749,9 @@ __global__ void __launch_bounds__(NTHREADS, C::MINB)
                 struct_item = p.allow_structured && __all_sync(0xffffffffu, arith);
             }
             const unsigned char *stage = smem + S::stage_off + size_t(st) * S::stage_bytes;
-            float2 *rec = reinterpret_cast<float2 *>(smem + S::rec_off + r * S::rec_bytes) + c;
+            float4 *rec = reinterpret_cast<float4 *>(smem + S::rec_off + r * S::rec_bytes) + c;
             float3 x0 = make_float3(0.f, 0.f, 0.f);
-            const bool use_x0 = CONV && h == 0 && m.t0 == 0 && conv_prefix<T>(p, m.g, c, x0);
+            const bool use_x0 = CONV && h == 0 && m.t0 == 0 && conv_prefix<T>(p, m.b, m.d0 + c, x0);
             prologue_rows<T, CONV>(reinterpret_cast<const T *>(stage + S::st_x) + S::HALO * CH + c,
                                    reinterpret_cast<T *>(smem + S::stage_off + size_t(st) * S::stage_bytes +
                                                          S::st_dt) + c,
@@ -703,8 +810,8 @@ __global__ void __launch_bounds__(NTHREADS, C::MINB)
                     warp_arrive(&bar_part_full[pr]);
                 break;
             }
-            const int64_t b = m.g / p.Dg;
-            const int64_t d = (m.g % p.Dg) * CH + c;
+            const int64_t b = m.b;
+            const int64_t d = m.d0 + c;
             const bool dvalid = d < p.D;
             if (m.flags & F_FIRST) {
                 float a[4];
@@ -753,11 +860,13 @@ __global__ void __launch_bounds__(NTHREADS, C::MINB)
                 set_timeout(p.status, lane);
                 break;
             }
-            const float2 *rec = reinterpret_cast<const float2 *>(smem + S::rec_off + r * S::rec_bytes) + c;
+            const float4 *rec = reinterpret_cast<const float4 *>(smem + S::rec_off + r * S::rec_bytes) + c;
             const float *bc = reinterpret_cast<const float *>(smem + S::bcf_off + r * S::bcf_bytes) + 4 * w;
             float4 *part = reinterpret_cast<float4 *>(smem + S::part_off + pr * S::part_bytes) + w * (TT / 4) * CH + c;
-            if (m.flags & F_STRUCT) consume_tile<true, ZOH>(rec, bc, part, Aq, del, zA, iA, h01, h23);
-            else consume_tile<false, ZOH>(rec, bc, part, Aq, del, zA, iA, h01, h23);
+            // With one block per SM the registers allow the factors to run a block ahead.
+            constexpr bool kAhead = C::MINB == 1 && SSM_FACTORS_AHEAD;
+            if (m.flags & F_STRUCT) consume_tile<true, ZOH, kAhead>(rec, bc, part, Aq, del, zA, iA, h01, h23);
+            else consume_tile<false, ZOH, kAhead>(rec, bc, part, Aq, del, zA, iA, h01, h23);
             warp_arrive(&bar_rec_free[r]);
             warp_arrive(&bar_part_full[pr]);
             if (m.flags & F_LAST) {
