@@ -66,6 +66,9 @@ enum {
                                 the Mamba summary's Theorem 1 (a gated RNN for N = 1) is exact. The
                                 kernels evaluate (exp(z) - 1) / z, z = Delta A, by a series for
                                 |z| < 1/16, where the subtraction would lose relative precision */
+    SSM_TEST_SHORT_SEGMENTS = 0x40000000u, /* test hook: time segments of one 32-step tile each,
+                                so that every tile boundary is a carry between segments (the
+                                result is the same; it runs slower) */
     SSM_TEST_DROP_HANDOFF = 0x80000000u /* fault-injection hook for tests: the first time segment of
                                 channel group 0 does not publish its state, so its successor's
                                 bounded wait runs out; ssm_workspace_status() then reports

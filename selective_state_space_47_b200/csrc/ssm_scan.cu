@@ -28,7 +28,7 @@ namespace {
 
 constexpr int kMaxN = 16;   // states per channel handled by the kernels
 constexpr int kMinSegTiles = 32;  // shortest time segment, in tiles (unless the sequence is shorter)
-constexpr int kMaxSegTiles = 64;  // longest time segment, in tiles
+constexpr int kMaxSegTiles = 256;  // longest time segment, in tiles
 
 // ------------------------------------------------------------- workspace
 // [0, 4) item counter; [4, 8) device status; [256, ...) per-group flags;
@@ -361,6 +361,7 @@ bool plan_scan(const ssm_scan_args *a, ScanPlan *pl) {
     const int64_t lmin = std::min<int64_t>((a->seqlen + TT - 1) / TT * TT, int64_t(kMinSegTiles) * TT);
     pl->seg_len = std::min<int64_t>(int64_t(kMaxSegTiles) * TT,
                                     std::max<int64_t>(std::max<int64_t>(TT, lmin), (per + TT - 1) / TT * TT));
+    if (a->flags & SSM_TEST_SHORT_SEGMENTS) pl->seg_len = TT;
     pl->K = (a->seqlen + pl->seg_len - 1) / pl->seg_len;
     pl->items = pl->G * pl->K;
     return true;
@@ -369,7 +370,8 @@ bool plan_scan(const ssm_scan_args *a, ScanPlan *pl) {
 ssm_status check_common(int64_t Bsz, int64_t D, int64_t N, ssm_dtype dt, uint32_t flags) {
     if (Bsz < 0 || D < 0 || N < 1) return SSM_ERR_INVALID;
     if (dt != SSM_F32 && dt != SSM_BF16) return SSM_ERR_INVALID;
-    if (flags & ~uint32_t(SSM_DELTA_SOFTPLUS | SSM_A_GENERAL | SSM_EXACT_ZOH | SSM_TEST_DROP_HANDOFF))
+    if (flags & ~uint32_t(SSM_DELTA_SOFTPLUS | SSM_A_GENERAL | SSM_EXACT_ZOH | SSM_TEST_SHORT_SEGMENTS |
+                          SSM_TEST_DROP_HANDOFF))
         return SSM_ERR_INVALID;
     if (N > kMaxN) return SSM_ERR_UNSUPPORTED;
     if (D % (dt == SSM_BF16 ? 8 : 4) != 0) return SSM_ERR_UNSUPPORTED;

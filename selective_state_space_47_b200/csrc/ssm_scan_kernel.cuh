@@ -224,40 +224,10 @@ __device__ __forceinline__ float2 zoh_weight(const float2 z, const float2 a, con
 }
 
 // ---------------------------------------------------------------- consumers
-// 2^x on the FMA pipe for two values (x clamped to [-127, 127]): x = j + f with j the
-// nearest integer (x + 1.5 * 2^23 + 127 leaves j + 127 in the float's low mantissa
-// bits) and f in [-1/2, 1/2]; 2^f = 1 + c1 f + ... + c5 f^5, the minimax polynomial of
-// the relative error with the constant term fixed at 1 (Lawson's iteratively
-// reweighted least squares: 9.1e-8 before rounding, 1.7e-7 in float32), times 2^j
-// built from j + 127 in the exponent field, which is exactly 0 for j = -127 (the
-// flush to zero of the special-function unit's result there). 2^0 is exactly 1.
-// Takes part of the exponentials off the special-function unit.
-__device__ __forceinline__ float2 exp2_fma(float2 x) {
-    x.x = fminf(fmaxf(x.x, -127.f), 127.f);
-    x.y = fminf(fmaxf(x.y, -127.f), 127.f);
-    constexpr float kShift = 12583039.f;  // 1.5 * 2^23 + 127
-    const float2 t = __fadd2_rn(x, f2(kShift, kShift));
-    const float2 j = __fadd2_rn(t, f2(-kShift, -kShift));
-    const float2 f = __ffma2_rn(j, f2(-1.f, -1.f), x);
-    float2 q = __ffma2_rn(f, f2(1.326472848e-03f, 1.326472848e-03f), f2(9.671512991e-03f, 9.671512991e-03f));
-    q = __ffma2_rn(f, q, f2(5.550733581e-02f, 5.550733581e-02f));
-    q = __ffma2_rn(f, q, f2(2.402224243e-01f, 2.402224243e-01f));
-    q = __ffma2_rn(f, q, f2(6.931470037e-01f, 6.931470037e-01f));
-    q = __ffma2_rn(f, q, f2(1.f, 1.f));
-    return __fmul2_rn(q, f2(__uint_as_float(__float_as_uint(t.x) << 23), __uint_as_float(__float_as_uint(t.y) << 23)));
-}
-
-#ifndef SSM_FACTORS_AHEAD
-#define SSM_FACTORS_AHEAD 1  // one block per SM: exponentials formed one block ahead of the recurrence
-#endif
-#ifndef SSM_FMA_EXP
-#define SSM_FMA_EXP 0  // general path: exponentials on the FMA pipe per block of 16 (0, 2 or 4)
-#endif
-
 // One block of four steps for one lane: the factors Abar and the inputs u B of the
 // warp's four states (pairs 01 and 23) from the block's records (two steps each) and B
-// rows. The general path takes kPoly exponentials of state 4w+3 on the FMA pipe.
-template <bool STRUCT, bool ZOH, int kPoly>
+// rows.
+template <bool STRUCT, bool ZOH>
 __device__ __forceinline__ void block_factors(const float4 r0, const float4 r1, const float4 (&b4)[4], const float4 Aq,
                                               const float del, const float4 zA, const float4 iA, float2 (&a01)[4],
                                               float2 (&a23)[4], float2 (&ub01)[4], float2 (&ub23)[4]) {
@@ -278,7 +248,6 @@ __device__ __forceinline__ void block_factors(const float4 r0, const float4 r1, 
 #pragma unroll
         for (int s = 0; s < S; ++s) a23[s] = __fmul2_rn(a01[s], f2(r[s] * r[s], r[s] * r[s]));
     } else {
-        static_assert(kPoly % 2 == 0 && kPoly <= S, "FMA-pipe exponentials go in pairs");
         float2 x01[S], x23[S];
 #pragma unroll
         for (int s = 0; s < S; ++s) {
@@ -288,14 +257,7 @@ __device__ __forceinline__ void block_factors(const float4 r0, const float4 r1, 
 #pragma unroll
         for (int s = 0; s < S; ++s) {
             a01[s] = f2(ex2_approx(x01[s].x), ex2_approx(x01[s].y));
-            a23[s].x = ex2_approx(x23[s].x);
-            if (s < S - kPoly) a23[s].y = ex2_approx(x23[s].y);
-        }
-#pragma unroll
-        for (int s = S - kPoly; s < S; s += 2) {
-            const float2 e = exp2_fma(f2(x23[s].y, x23[s + 1].y));
-            a23[s].y = e.x;
-            a23[s + 1].y = e.y;
+            a23[s] = f2(ex2_approx(x23[s].x), ex2_approx(x23[s].y));
         }
     }
 #pragma unroll
@@ -347,7 +309,6 @@ __device__ __forceinline__ void consume_tile(const float4 *__restrict__ rec, con
                                              float4 *__restrict__ part, const float4 Aq, const float del,
                                              const float4 zA, const float4 iA, float2 &h01, float2 &h23) {
     constexpr int S = 4, NB = TT / S;
-    constexpr int kPoly = (STRUCT || ZOH) ? 0 : SSM_FMA_EXP;
     auto load = [&](int blk, float4 &r0, float4 &r1, float4 (&b4)[S], float4 (&c4)[S]) {
         r0 = rec[(2 * blk) * CH];
         r1 = rec[(2 * blk + 1) * CH];
@@ -362,7 +323,7 @@ __device__ __forceinline__ void consume_tile(const float4 *__restrict__ rec, con
         float2 a01[S], a23[S], ub01[S], ub23[S];
         float4 cc[S];  // C rows of the block whose factors are in a01 .. ub23
         load(0, r0, r1, b4, c4);
-        block_factors<STRUCT, ZOH, kPoly>(r0, r1, b4, Aq, del, zA, iA, a01, a23, ub01, ub23);
+        block_factors<STRUCT, ZOH>(r0, r1, b4, Aq, del, zA, iA, a01, a23, ub01, ub23);
 #pragma unroll
         for (int s = 0; s < S; ++s) cc[s] = c4[s];
         load(1, rn0, rn1, bn, cn);
@@ -371,7 +332,7 @@ __device__ __forceinline__ void consume_tile(const float4 *__restrict__ rec, con
             float2 na01[S], na23[S], nub01[S], nub23[S];
             float4 ncc[S];
             if (blk + 1 < NB) {  // factors of the next block (its operands were loaded last time)
-                block_factors<STRUCT, ZOH, kPoly>(rn0, rn1, bn, Aq, del, zA, iA, na01, na23, nub01, nub23);
+                block_factors<STRUCT, ZOH>(rn0, rn1, bn, Aq, del, zA, iA, na01, na23, nub01, nub23);
 #pragma unroll
                 for (int s = 0; s < S; ++s) ncc[s] = cn[s];
             }
@@ -395,7 +356,7 @@ __device__ __forceinline__ void consume_tile(const float4 *__restrict__ rec, con
         for (int blk = 0; blk < NB; ++blk) {
             if (blk + 1 < NB) load(blk + 1, rn0, rn1, bn, cn);
             float2 a01[S], a23[S], ub01[S], ub23[S];
-            block_factors<STRUCT, ZOH, kPoly>(r0, r1, b4, Aq, del, zA, iA, a01, a23, ub01, ub23);
+            block_factors<STRUCT, ZOH>(r0, r1, b4, Aq, del, zA, iA, a01, a23, ub01, ub23);
             part[blk * CH] = block_recur(a01, a23, ub01, ub23, c4, h01, h23);
             if (blk + 1 < NB) {
                 r0 = rn0;
@@ -864,7 +825,7 @@ __global__ void __launch_bounds__(NTHREADS, C::MINB)
             const float *bc = reinterpret_cast<const float *>(smem + S::bcf_off + r * S::bcf_bytes) + 4 * w;
             float4 *part = reinterpret_cast<float4 *>(smem + S::part_off + pr * S::part_bytes) + w * (TT / 4) * CH + c;
             // With one block per SM the registers allow the factors to run a block ahead.
-            constexpr bool kAhead = C::MINB == 1 && SSM_FACTORS_AHEAD;
+            constexpr bool kAhead = C::MINB == 1;
             if (m.flags & F_STRUCT) consume_tile<true, ZOH, kAhead>(rec, bc, part, Aq, del, zA, iA, h01, h23);
             else consume_tile<false, ZOH, kAhead>(rec, bc, part, Aq, del, zA, iA, h01, h23);
             warp_arrive(&bar_rec_free[r]);

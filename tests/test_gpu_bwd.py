@@ -2,9 +2,11 @@
 which is itself pinned to central differences of the forward oracle.
 
 Per-(t, channel) gradients (dx, ddt, dz) are compared row by row over t per (b, d), like
-y; the reduced ones (dB, dC, dA, dD, ddt_bias) and dh0 against the largest reference
-entry of the tensor. Tolerances: float32 1e-4 everywhere; bfloat16 tokens 1e-2 for the
-[B, L, D] gradients (stored in bfloat16) and 1e-4 for the float32 reductions.
+y; the reduced ones row by row too, so that a wrong small row cannot hide under a large
+one: dB and dC per (b, t) over n, dA per channel over n, dh0 per (b, d) over n; dD and
+ddt_bias ([D] vectors) against their largest entry. Tolerances: float32 1e-4 everywhere;
+bfloat16 tokens 1e-2 for the [B, L, D] gradients (stored in bfloat16) and 1e-4 for the
+float32 reductions.
 """
 import numpy as np
 import pytest
@@ -60,9 +62,13 @@ def _check(g, ref, tok_tol, red_tol, sel=None, check_bc=True):
     red = ["dA", "dD", "ddt_bias", "dh0"] + (["dB", "dC"] if check_bc else [])
     for k in red:
         got = g[k]
-        if sel is not None:
+        if sel is not None and k not in ("dB", "dC"):
             got = got.index_select(0 if k in ("dA", "dD", "ddt_bias") else 1, sel.to(got.device))
-        errs[k] = _rel(got.cpu().numpy(), ref[k])
+        got = got.cpu().numpy()
+        if k in ("dD", "ddt_bias"):
+            errs[k] = _rel(got, ref[k])
+        else:  # rows over the state index n: dA [D, N], dB / dC [B, L, N], dh0 [B, D, N]
+            errs[k] = rowwise_rel(got, ref[k], axis=got.ndim - 1)
     print("  ".join(f"{k} {v:.1e}" for k, v in errs.items()))
     for k, v in errs.items():
         assert v <= (tok_tol if k in ("dx", "ddt", "dz") else red_tol), f"{k}: {v:.3e}"
@@ -116,16 +122,37 @@ def test_bwd_empty_sequence(ssm):
 
 
 def test_bwd_long_context_sampled(ssm):
-    """B=1, L=262144, D=5120 at full size; the oracle runs on 8 channels spread over D
-    (all 262,144 steps): dx, ddt, dz, dA, dD, ddt_bias and dh0 of those channels (dB, dC
-    sum over all channels and are checked at the smaller sizes above)."""
+    """B=1, L=262144, D=5120 at full size; the oracle runs on 34 channels spread over D, at
+    a lane that moves with the channel group (all 262,144 steps): dx, ddt, dz, dA, dD,
+    ddt_bias and dh0 of those channels (dB, dC sum over all channels: the next test checks
+    them against an oracle over every channel)."""
     inp = synth.workload_inputs("long_context", device="cuda", h0=True)
     gen = torch.Generator(device="cuda").manual_seed(74)
     dy = torch.randn(inp["x"].shape, generator=gen, device="cuda").to(inp["x"].dtype)
     g = ssm.scan_bwd(inp["x"], inp["dt"], inp["A"], inp["B"], inp["C"], dy, inp["D"], inp["z"], inp["dt_bias"],
                      inp["h0"])
     torch.cuda.synchronize()
-    sel = torch.tensor([0, 1, 777, 2048, 3001, 4095, 5118, 5119])
+    groups = torch.arange(0, 160, 5)
+    sel = torch.unique(torch.cat([groups * 32 + (groups * 11) % 32, torch.tensor([0, 5119])]))
     ref = _oracle_bwd(inp, dy, None, sel=sel)
-    print("\nbwd long_context (8 channels, all steps): ", end="")
+    print(f"\nbwd long_context ({len(sel)} channels, all steps): ", end="")
     _check(g, ref, 1e-2, 1e-4, sel=sel, check_bc=False)
+
+
+def test_bwd_long_context_width_all_channels(ssm):
+    """The long-context width (B=1, D=5120, N=16, bf16, with h0 and dL/dh_L) on a sequence
+    shortened to L=2048, so that the oracle runs over every channel: dB and dC, which sum
+    the contributions of all 5120 channels, compared for every (b, t) row, and every other
+    gradient in full."""
+    w = synth.WORKLOADS["long_context"]
+    inp = synth.scan_inputs(w.batch, 2048, w.dim, w.dstate, w.dtype, seed=75, h0=True)
+    gen = torch.Generator().manual_seed(76)
+    dy = torch.randn(inp["x"].shape, generator=gen).to(w.dtype)
+    dh_last = torch.randn((w.batch, w.dim, w.dstate), generator=gen)
+    ref = _oracle_bwd(inp, dy, dh_last)
+    dev = {k: (v.cuda() if isinstance(v, torch.Tensor) else v) for k, v in inp.items()}
+    g = ssm.scan_bwd(dev["x"], dev["dt"], dev["A"], dev["B"], dev["C"], dy.cuda(), dev["D"], dev["z"],
+                     dev["dt_bias"], dev["h0"], dh_last.cuda())
+    torch.cuda.synchronize()
+    print("\nbwd long_context width, L=2048, all channels: ", end="")
+    _check(g, ref, 1e-2, 1e-4)
