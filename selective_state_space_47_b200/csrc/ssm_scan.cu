@@ -16,6 +16,7 @@
 
 #include <algorithm>
 #include <mutex>
+#include <type_traits>
 
 #include "../../include/ssm_scan.h"
 #include "ssm_device.cuh"
@@ -245,14 +246,24 @@ struct ScanPlan {
     size_t smem = 0;
 };
 
+// The deep configuration of the short-convolution kernels has four prologue warps.
+template <bool CONV>
+using DeepFor = typename std::conditional<CONV, ssm::scan::DeepConv, ssm::scan::Deep>::type;
+
 template <bool ZOH, bool CONV>
 void *pick_kernel_t(ssm_dtype dt, bool deep) {
     using namespace ssm::scan;
     if (dt == SSM_BF16)
-        return deep ? reinterpret_cast<void *>(&scan_ws_kernel<__nv_bfloat16, Deep, ZOH, CONV>)
+        return deep ? reinterpret_cast<void *>(&scan_ws_kernel<__nv_bfloat16, DeepFor<CONV>, ZOH, CONV>)
                     : reinterpret_cast<void *>(&scan_ws_kernel<__nv_bfloat16, Shallow, ZOH, CONV>);
-    return deep ? reinterpret_cast<void *>(&scan_ws_kernel<float, Deep, ZOH, CONV>)
+    return deep ? reinterpret_cast<void *>(&scan_ws_kernel<float, DeepFor<CONV>, ZOH, CONV>)
                 : reinterpret_cast<void *>(&scan_ws_kernel<float, Shallow, ZOH, CONV>);
+}
+// Threads per block of a configuration.
+int pick_threads(bool deep, bool conv) {
+    using namespace ssm::scan;
+    if (!deep) return Shallow::NTHREADS;
+    return conv ? DeepConv::NTHREADS : Deep::NTHREADS;
 }
 // The exact zero-order hold and the short convolution are separate instantiations, so
 // the default kernel carries none of their code.
@@ -264,8 +275,8 @@ template <bool CONV>
 size_t pick_smem_t(ssm_dtype dt, bool deep) {
     using namespace ssm::scan;
     if (dt == SSM_BF16)
-        return deep ? Layout<__nv_bfloat16, Deep, CONV>::total : Layout<__nv_bfloat16, Shallow, CONV>::total;
-    return deep ? Layout<float, Deep, CONV>::total : Layout<float, Shallow, CONV>::total;
+        return deep ? Layout<__nv_bfloat16, DeepFor<CONV>, CONV>::total : Layout<__nv_bfloat16, Shallow, CONV>::total;
+    return deep ? Layout<float, DeepFor<CONV>, CONV>::total : Layout<float, Shallow, CONV>::total;
 }
 size_t pick_smem(ssm_dtype dt, bool deep, bool conv) {
     return conv ? pick_smem_t<true>(dt, deep) : pick_smem_t<false>(dt, deep);
@@ -322,7 +333,8 @@ bool scan_occupancy(ssm_dtype dt, bool conv, int occ[2]) {
                 if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem)) != cudaSuccess ||
                     cudaFuncSetAttribute(kern_zoh, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem)) !=
                         cudaSuccess ||
-                    cudaOccupancyMaxActiveBlocksPerMultiprocessor(&o, kern, ssm::scan::NTHREADS, smem) != cudaSuccess)
+                    cudaOccupancyMaxActiveBlocksPerMultiprocessor(&o, kern, pick_threads(deep != 0, conv), smem) !=
+                        cudaSuccess)
                     return false;
             }
             cache[dev][ti][ci][deep] = o;
@@ -605,7 +617,7 @@ ssm_status ssm_scan_fwd(const ssm_scan_args *a, void *stream_) {
 
     void *kern = pick_kernel(a->dtype, pl.deep, (a->flags & SSM_EXACT_ZOH) != 0, conv);
     void *args[] = {&tx, &tdt, &tz, &tb, &tc, &ty, &p};
-    cudaError_t e = cudaLaunchKernel(kern, dim3(pl.grid), dim3(ssm::scan::NTHREADS), args, pl.smem, stream);
+    cudaError_t e = cudaLaunchKernel(kern, dim3(pl.grid), dim3(pick_threads(pl.deep, conv)), args, pl.smem, stream);
     return e == cudaSuccess ? SSM_OK : SSM_ERR_CUDA;
 }
 

@@ -62,25 +62,29 @@ namespace ssm {
 namespace scan {
 
 constexpr int CW = 4;                             // consumer warps (4 states each)
-constexpr int NP = 2;                             // prologue warps
 constexpr int NE = 2;                             // epilogue warps
 constexpr int CH = 32;                            // channels per block (one per lane)
-constexpr int WARP_P0 = CW, WARP_E0 = CW + NP, WARP_L = CW + NP + NE;
-constexpr int NTHREADS = (CW + NP + NE + 1) * 32;
+constexpr int WARP_P0 = CW;
 constexpr int TT = 32;                            // time steps per tile
-constexpr int TP = TT / NP;                       // steps per prologue warp and tile
 constexpr int TE = TT / NE;                       // steps per epilogue warp and tile
 constexpr int KCONV = 4;                          // width of the short causal convolution
-// Ring depths and blocks per SM. Shallow: 113 KB of shared memory (bf16), two blocks
-// per SM. Deep: rings twice as deep, one block per SM; it decouples the roles further
-// and is the better choice when there are too few channel groups to fill two blocks per
-// SM (the long-context workload has 160 groups for 148 SMs).
-template <int STAGES_, int R_REC_, int R_PART_, int MINB_>
+// Ring depths, blocks per SM and prologue warps. Shallow: 113 KB of shared memory (bf16),
+// two blocks per SM. Deep: rings twice as deep, one block per SM; it decouples the roles
+// further and is the better choice when there are too few channel groups to fill two
+// blocks per SM (the long-context workload has 160 groups for 148 SMs). With the short
+// convolution the prologue does about twice the work (the convolution and its SiLU), so
+// the deep configuration spreads it over four prologue warps, one per SM sub-partition.
+template <int STAGES_, int R_REC_, int R_PART_, int MINB_, int NP_ = 2>
 struct Cfg {
     static constexpr int STAGES = STAGES_;  // TMA ring depth (tiles)
     static constexpr int R_REC = R_REC_;    // record ring depth
     static constexpr int R_PART = R_PART_;  // partial-sum ring depth
     static constexpr int MINB = MINB_;      // blocks per SM the registers are budgeted for
+    static constexpr int NP = NP_;          // prologue warps
+    static constexpr int TP = TT / NP;      // steps per prologue warp and tile
+    static constexpr int WARP_E0 = CW + NP, WARP_L = CW + NP + NE;
+    static constexpr int NTHREADS = (CW + NP + NE + 1) * 32;
+    static_assert(TP % 8 == 0, "a prologue warp takes whole pairs of steps and whole 16-byte B/C chunks");
 };
 #ifndef SSM_DEEP_STAGES
 #define SSM_DEEP_STAGES 8
@@ -93,6 +97,7 @@ struct Cfg {
 #endif
 using Shallow = Cfg<6, 2, 2, 2>;
 using Deep = Cfg<SSM_DEEP_STAGES, SSM_DEEP_REC, SSM_DEEP_PART, 1>;
+using DeepConv = Cfg<SSM_DEEP_STAGES, SSM_DEEP_REC, SSM_DEEP_PART, 1, 4>;
 constexpr int YBUF = 3;                           // y staging buffers for the TMA store
 constexpr int kMaxN = 16;                         // state slots per channel
 constexpr uint64_t kWaitLimitNs = 2000000000ull;  // every device-side wait gives up after 2 s
@@ -421,7 +426,7 @@ __device__ __forceinline__ bool conv_prefix(const Params &p, const int64_t b, co
 // zero-order hold) u = x, the consumers apply the weight. Rows at or past tlen get
 // (0, 0): Abar = 1, no input. CONV: x is the short convolution's output (cw, cb, and
 // use_x0 / x0 as for conv_silu_rows), which is also written over the dt rows read.
-template <typename T, bool CONV>
+template <typename T, bool CONV, int TP>
 __device__ __forceinline__ void prologue_rows(const T *__restrict__ sx, T *__restrict__ sdt,
                                               float4 *__restrict__ rec, const int t0, const int tlen,
                                               const float bias, const bool softplus, const bool zoh,
@@ -520,13 +525,14 @@ __device__ __forceinline__ void epilogue_rows(const float4 *__restrict__ part, c
 
 // ------------------------------------------------------------------- kernel
 template <typename T, typename C, bool ZOH, bool CONV>
-__global__ void __launch_bounds__(NTHREADS, C::MINB)
+__global__ void __launch_bounds__(C::NTHREADS, C::MINB)
     scan_ws_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_dt,
                    const __grid_constant__ CUtensorMap tm_z, const __grid_constant__ CUtensorMap tm_b,
                    const __grid_constant__ CUtensorMap tm_c, const __grid_constant__ CUtensorMap tm_y,
                    const Params p) {
     using S = Layout<T, C, CONV>;
     constexpr int STAGES = C::STAGES, R_REC = C::R_REC, R_PART = C::R_PART;
+    constexpr int NP = C::NP, TP = C::TP, WARP_E0 = C::WARP_E0, WARP_L = C::WARP_L;
     extern __shared__ __align__(1024) unsigned char smem[];
     TileMeta *smeta = reinterpret_cast<TileMeta *>(smem + S::smeta_off);  // per stage
     TileMeta *tmeta = reinterpret_cast<TileMeta *>(smem + S::tmeta_off);  // per record slot
@@ -713,7 +719,7 @@ __global__ void __launch_bounds__(NTHREADS, C::MINB)
             float4 *rec = reinterpret_cast<float4 *>(smem + S::rec_off + r * S::rec_bytes) + c;
             float3 x0 = make_float3(0.f, 0.f, 0.f);
             const bool use_x0 = CONV && h == 0 && m.t0 == 0 && conv_prefix<T>(p, m.b, m.d0 + c, x0);
-            prologue_rows<T, CONV>(reinterpret_cast<const T *>(stage + S::st_x) + S::HALO * CH + c,
+            prologue_rows<T, CONV, TP>(reinterpret_cast<const T *>(stage + S::st_x) + S::HALO * CH + c,
                                    reinterpret_cast<T *>(smem + S::stage_off + size_t(st) * S::stage_bytes +
                                                          S::st_dt) + c,
                                    rec, h * TP, m.tlen, bias_c, p.softplus != 0, ZOH, cw, cb, use_x0, x0);
