@@ -299,6 +299,55 @@ typedef struct {
 size_t ssm_scan_bwd_workspace_size(const ssm_scan_bwd_args *args);
 ssm_status ssm_scan_bwd(const ssm_scan_bwd_args *args, void *stream);
 
+/*
+ * The state space model in its chunked matrix form (structured state space duality;
+ * Mamba-2 article, mugbit.ir, "Mamba-2 / SSD" section: the recurrence is a product with a
+ * lower-triangular semiseparable matrix, computed by matrix multiplications on tensor
+ * cores). It is the same model as ssm_scan_fwd restricted the Mamba-2 way: H heads of P
+ * channels each; the P channels of a head share one step size dt[b, t, h] and one scalar
+ * A[h] (A[d, n] = A[h] for all n), and D[h], dt_bias[h] per head; B_t, C_t [N] shared by
+ * all heads, as in ssm_scan_fwd. Per head h and channel p (d = h P + p):
+ *   Delta_t = softplus(dt[b, t, h] + dt_bias[h])  (or dt + dt_bias without the flag)
+ *   state[p, n] <- exp(Delta_t A[h]) state[p, n] + Delta_t B_t[n] x_t[d]
+ *   y_t[d] = (sum_n C_t[n] state[p, n] + D[h] x_t[d]) * silu(z_t[d])   (no gate if z NULL)
+ * Evaluated per chunk of 128 steps as four tcgen05 matrix products with float32
+ * accumulation: C B^T, the decay-masked matrix times x (the skip D x on its diagonal), C
+ * times the chunk's starting state, and B^T times the decay-weighted x for the next state.
+ * The operands of the products are rounded to bfloat16 (the decay matrix and the state
+ * among them); the state is carried between chunks in float32.
+ * Shapes: x, z, y [B, L, H, P]; dt [B, L, H]; Bm, Cm [B, L, N]; A, Dskip, dt_bias [H];
+ * h0, h_last [B, H, P, N] float32 (state[p, n] of head h), NULL for 0 / not wanted.
+ * Supported: dtype SSM_BF16, headdim P = 64, dstate N = 128 (the Mamba-2 head shape);
+ * anything else returns SSM_ERR_UNSUPPORTED (ssm_scan_fwd computes the same model for
+ * other shapes and float32, one exponential per state). Alignment: x, z, y, Bm, Cm, h0,
+ * h_last and the workspace on 16 bytes, A, Dskip, dt_bias on 4. flags: SSM_DELTA_SOFTPLUS
+ * only. The workspace (ssm_ssd_workspace_size bytes, caller-owned device memory, one
+ * per concurrently running call) holds a counter, a status word (ssm_workspace_status
+ * reads it: SSM_ERR_TIMEOUT if a bounded device wait gave up), a flag per (sequence,
+ * head) and the float32 state handed between the time segments of each (B x H x 32 KB).
+ * L == 0 writes h_last = h0 (or 0). The call enqueues work on `stream` and returns.
+ */
+typedef struct {
+    int64_t batch, seqlen, nheads, headdim, dstate;  /* B, L, H, P, N */
+    ssm_dtype dtype;
+    uint32_t flags;          /* SSM_DELTA_SOFTPLUS                                     */
+    const void *x;           /* [B, L, H, P] input tokens                             */
+    const void *dt;          /* [B, L, H] raw step sizes                              */
+    const void *z;           /* [B, L, H, P] gate, or NULL                            */
+    const void *Bm, *Cm;     /* [B, L, N]                                             */
+    const float *A;          /* [H] one scalar per head                               */
+    const float *Dskip;      /* [H] or NULL                                           */
+    const float *dt_bias;    /* [H] or NULL                                           */
+    const float *h0;         /* [B, H, P, N] or NULL                                  */
+    void *y;                 /* [B, L, H, P] output                                   */
+    float *h_last;           /* [B, H, P, N] output or NULL                           */
+    void *workspace;         /* ssm_ssd_workspace_size() bytes                         */
+    size_t workspace_bytes;
+} ssm_ssd_args;
+
+size_t ssm_ssd_workspace_size(const ssm_ssd_args *args);  /* 0 for invalid shapes */
+ssm_status ssm_ssd_fwd(const ssm_ssd_args *args, void *stream);
+
 /* Human-readable name of a status code (static storage). */
 const char *ssm_status_string(ssm_status status);
 

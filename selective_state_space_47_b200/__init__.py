@@ -18,7 +18,8 @@ import torch
 from . import _native
 from ._native import SSM_A_GENERAL, SSM_DELTA_SOFTPLUS, SSM_EXACT_ZOH
 
-__all__ = ["scan_fwd", "scan_fwd_host", "step", "workspace_size", "workspace_status", "ScanWorkspace"]
+__all__ = ["scan_fwd", "scan_fwd_host", "scan_bwd", "ssd_fwd", "step", "workspace_size", "workspace_status",
+           "ScanWorkspace"]
 
 _TOKEN_DTYPES = {torch.float32: _native.SSM_F32, torch.bfloat16: _native.SSM_BF16}
 
@@ -352,3 +353,58 @@ def step(x, dt, A, B, C, h, D=None, z=None, dt_bias=None, *, delta_softplus=True
                                          _handle(_resolve_stream(stream, dev)))
     _native.check(rc, "ssm_step_conv")
     return y
+
+
+def ssd_fwd(x, dt, A, B, C, D=None, z=None, dt_bias=None, h0=None, *, delta_softplus=True,
+            return_last_state=False, out=None, h_last=None, workspace=None, stream=None):
+    """The chunked (Mamba-2) form on the tensor cores (see include/ssm_scan.h, ssm_ssd_fwd).
+
+    x, z: [B, L, H, P] bfloat16 (P = 64); dt: [B, L, H] bfloat16 (one step size per head);
+    B, C: [B, L, N] bfloat16 (N = 128); A, D, dt_bias: [H] float32 (one scalar A per head);
+    h0: [B, H, P, N] float32. Returns y [B, L, H, P] and, with return_last_state, the final
+    state [B, H, P, N] float32.
+    """
+    dev = x.device
+    if x.dim() != 4:
+        raise ValueError("x must be [B, L, H, P]")
+    Bsz, L, H, Pd = x.shape
+    N = B.shape[-1]
+    tok = x.dtype
+    if tok not in _TOKEN_DTYPES:
+        raise TypeError(f"x: dtype must be float32 or bfloat16, got {tok}")
+    _need(x, "x", (Bsz, L, H, Pd), tok, dev)
+    _need(dt, "dt", (Bsz, L, H), tok, dev)
+    if z is not None:
+        _need(z, "z", (Bsz, L, H, Pd), tok, dev)
+    _need(B, "B", (Bsz, L, N), tok, dev)
+    _need(C, "C", (Bsz, L, N), tok, dev)
+    _need(A, "A", (H,), torch.float32, dev)
+    for t, name in ((D, "D"), (dt_bias, "dt_bias")):
+        if t is not None:
+            _need(t, name, (H,), torch.float32, dev)
+    if h0 is not None:
+        _need(h0, "h0", (Bsz, H, Pd, N), torch.float32, dev)
+    y = torch.empty_like(x) if out is None else out
+    _need(y, "out", (Bsz, L, H, Pd), tok, dev)
+    if return_last_state and h_last is None:
+        h_last = torch.empty((Bsz, H, Pd, N), dtype=torch.float32, device=dev)
+    if h_last is not None:
+        _need(h_last, "h_last", (Bsz, H, Pd, N), torch.float32, dev)
+    a = _native.SsdArgs()
+    a.batch, a.seqlen, a.nheads, a.headdim, a.dstate = Bsz, L, H, Pd, N
+    a.dtype = _TOKEN_DTYPES[tok]
+    a.flags = SSM_DELTA_SOFTPLUS if delta_softplus else 0
+    a.x, a.dt, a.z, a.Bm, a.Cm = (_ptr(t) for t in (x, dt, z, B, C))
+    a.A, a.Dskip, a.dt_bias, a.h0 = (_ptr(t) for t in (A, D, dt_bias, h0))
+    a.y, a.h_last = _ptr(y), _ptr(h_last)
+    lib = _native.lib()
+    s = _resolve_stream(stream, dev)
+    nbytes = int(lib.ssm_ssd_workspace_size(ctypes.byref(a)))
+    if workspace is None:
+        workspace = _default_ws.setdefault((dev, s.cuda_stream, "ssd"), ScanWorkspace())
+    ws = workspace.get(max(nbytes, 256), dev) if isinstance(workspace, ScanWorkspace) else workspace
+    a.workspace = ctypes.c_void_p(ws.data_ptr())
+    a.workspace_bytes = ws.numel() * ws.element_size()
+    with torch.cuda.device(dev):
+        _native.check(lib.ssm_ssd_fwd(ctypes.byref(a), _handle(s)), "ssm_ssd_fwd")
+    return (y, h_last) if return_last_state else y

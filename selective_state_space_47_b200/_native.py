@@ -16,7 +16,8 @@ SSM_TEST_DROP_HANDOFF = 0x80000000
 # Every symbol the header declares (checked by the CPU test suite).
 EXPORTS = ("ssm_scan_workspace_size", "ssm_scan_fwd", "ssm_step", "ssm_step_conv", "ssm_workspace_status",
            "ssm_status_string", "ssm_scan_fwd_noalloc", "ssm_noalloc_status", "ssm_scan_host_staging_size",
-           "ssm_scan_fwd_host", "ssm_scan_bwd_workspace_size", "ssm_scan_bwd")
+           "ssm_scan_fwd_host", "ssm_scan_bwd_workspace_size", "ssm_scan_bwd", "ssm_ssd_workspace_size",
+           "ssm_ssd_fwd")
 
 
 class ScanArgs(ctypes.Structure):
@@ -46,6 +47,17 @@ class ScanBwdArgs(ctypes.Structure):
     ]
 
 
+class SsdArgs(ctypes.Structure):
+    _fields_ = [
+        ("batch", ctypes.c_int64), ("seqlen", ctypes.c_int64), ("nheads", ctypes.c_int64),
+        ("headdim", ctypes.c_int64), ("dstate", ctypes.c_int64), ("dtype", ctypes.c_int),
+        ("flags", ctypes.c_uint32), ("x", ctypes.c_void_p), ("dt", ctypes.c_void_p), ("z", ctypes.c_void_p),
+        ("Bm", ctypes.c_void_p), ("Cm", ctypes.c_void_p), ("A", ctypes.c_void_p), ("Dskip", ctypes.c_void_p),
+        ("dt_bias", ctypes.c_void_p), ("h0", ctypes.c_void_p), ("y", ctypes.c_void_p),
+        ("h_last", ctypes.c_void_p), ("workspace", ctypes.c_void_p), ("workspace_bytes", ctypes.c_size_t),
+    ]
+
+
 _lib = None
 
 
@@ -64,6 +76,10 @@ def lib():
         L.ssm_scan_fwd.restype = ctypes.c_int
         L.ssm_scan_fwd_noalloc.argtypes = [ctypes.POINTER(ScanArgs), vp]
         L.ssm_scan_fwd_noalloc.restype = ctypes.c_int
+        L.ssm_ssd_workspace_size.argtypes = [ctypes.POINTER(SsdArgs)]
+        L.ssm_ssd_workspace_size.restype = ctypes.c_size_t
+        L.ssm_ssd_fwd.argtypes = [ctypes.POINTER(SsdArgs), vp]
+        L.ssm_ssd_fwd.restype = ctypes.c_int
         L.ssm_noalloc_status.argtypes = [vp]
         L.ssm_noalloc_status.restype = ctypes.c_int
         L.ssm_scan_host_staging_size.argtypes = [ctypes.POINTER(ScanArgs), i64]

@@ -9,7 +9,8 @@ import sys
 PKG = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
-SOURCES = [os.path.join(CSRC, "ssm_scan.cu"), os.path.join(CSRC, "ssm_host.cu"), os.path.join(CSRC, "ssm_scan_bwd.cu")]
+SOURCES = [os.path.join(CSRC, "ssm_scan.cu"), os.path.join(CSRC, "ssm_host.cu"), os.path.join(CSRC, "ssm_scan_bwd.cu"),
+           os.path.join(CSRC, "ssm_ssd.cu")]
 DEPS = SOURCES + [os.path.join(CSRC, "ssm_device.cuh"), os.path.join(CSRC, "ssm_scan_kernel.cuh"), os.path.join(ROOT, "include", "ssm_scan.h")]
 LIB = os.path.join(PKG, "libssmscan.so")
 NVCC_FLAGS = ["-O3", "-std=c++17", "-gencode", "arch=compute_100a,code=sm_100a", "-lineinfo",

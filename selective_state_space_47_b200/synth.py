@@ -12,6 +12,12 @@ x, z, B, C ~ N(0, 1); dt_raw ~ N(0, 0.5^2); per channel dt log-uniform in
   mid_layer       B=8  L=4096    D=2048 N=16  bfloat16, gate on, final state out
   long_context    B=1  L=262144  D=5120 N=16  bfloat16 (sequence-parallel case)
   decode          B=256 D=5120 N=16, 1000 chained one-token steps, h ~ N(0, 1)
+
+The chunked (Mamba-2) form with one scalar A per head, H heads of P = 64 channels
+sharing the head's step size, N = 128 states (the Mamba-2 2.7B layer's head shape):
+
+  ssd_layer       B=2  L=16384   H=80 (D=5120) P=64 N=128  bfloat16, gate on
+  A[h] = -U[1, 16] (Mamba-2's initialisation range), dt per head as above, D ~ N(0, 1)
 """
 from dataclasses import dataclass
 import math
@@ -34,6 +40,17 @@ class ScanWorkload:
 
 
 @dataclass(frozen=True)
+class SsdWorkload:
+    name: str
+    batch: int
+    seqlen: int
+    nheads: int
+    headdim: int
+    dstate: int
+    dtype: torch.dtype = torch.bfloat16
+
+
+@dataclass(frozen=True)
 class StepWorkload:
     name: str
     batch: int
@@ -49,9 +66,10 @@ WORKLOADS = {
     "mid_layer": ScanWorkload("mid_layer", 8, 4096, 2048, 16, torch.bfloat16, True, True),
     "long_context": ScanWorkload("long_context", 1, 262144, 5120, 16, torch.bfloat16, True, True),
     "decode": StepWorkload("decode", 256, 5120, 16, 1000),
+    "ssd_layer": SsdWorkload("ssd_layer", 2, 16384, 80, 64, 128),
 }
 SEEDS = {"tiny_f32": SEED_BASE + 0, "small_layer": SEED_BASE + 1, "mid_layer": SEED_BASE + 2,
-         "long_context": SEED_BASE + 3, "decode": SEED_BASE + 4}
+         "long_context": SEED_BASE + 3, "decode": SEED_BASE + 4, "ssd_layer": SEED_BASE + 5}
 
 
 def _gen(seed, device):
@@ -135,3 +153,23 @@ def to_numpy_storage(t):
     if t.dtype == torch.float32:
         return t.numpy()
     raise TypeError(f"unsupported storage dtype {t.dtype}")
+
+
+def ssd_inputs(batch, seqlen, nheads, headdim=64, dstate=128, dtype=torch.bfloat16, seed=SEED_BASE + 5,
+               device="cpu", gate=True, h0=False):
+    """Tokens of the chunked (one A per head) form: x, z [B, L, H, P]; dt [B, L, H]; B, C
+    [B, L, N]; A, D, dt_bias [H] float32; h0 [B, H, P, N] float32 (or None)."""
+    g = _gen(seed, device)
+    x = _normal((batch, seqlen, nheads, headdim), g, device, dtype)
+    dt = _normal((batch, seqlen, nheads), g, device, dtype, std=0.5)
+    z = _normal((batch, seqlen, nheads, headdim), g, device, dtype) if gate else None
+    Bm = _normal((batch, seqlen, dstate), g, device, dtype)
+    Cm = _normal((batch, seqlen, dstate), g, device, dtype)
+    gp = _gen(seed + 7919, "cpu")
+    A = -(1.0 + 15.0 * torch.rand(nheads, generator=gp, dtype=torch.float32))
+    Dskip = torch.randn(nheads, generator=gp, dtype=torch.float32)
+    u = torch.rand(nheads, generator=gp, dtype=torch.float64)
+    dtv = torch.exp(math.log(1e-3) + u * (math.log(0.1) - math.log(1e-3)))
+    dt_bias = torch.log(torch.expm1(dtv)).to(torch.float32)
+    h = _normal((batch, nheads, headdim, dstate), g, device, torch.float32) if h0 else None
+    return dict(x=x, dt=dt, z=z, B=Bm, C=Cm, A=A.to(device), D=Dskip.to(device), dt_bias=dt_bias.to(device), h0=h)

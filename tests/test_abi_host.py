@@ -36,7 +36,8 @@ def test_header_and_exports_agree(lib):
         assert hasattr(lib, name)
 
 
-@pytest.mark.parametrize("cname,pyname", [("ssm_scan_args", "ScanArgs"), ("ssm_scan_bwd_args", "ScanBwdArgs")])
+@pytest.mark.parametrize("cname,pyname", [("ssm_scan_args", "ScanArgs"), ("ssm_scan_bwd_args", "ScanBwdArgs"),
+                                          ("ssm_ssd_args", "SsdArgs")])
 def test_args_struct_layout_matches_binding(tmp_path, cname, pyname):
     """The ctypes mirrors of the argument structs have the C compiler's field offsets and size."""
     cls = getattr(_native, pyname)
