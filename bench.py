@@ -29,6 +29,7 @@ if ROOT not in sys.path:
 METRIC = "selective-scan state-updates/s (B·L·D·N) and % of B200 HBM roofline"
 UNIT = "state-updates/s"
 FALLBACK_HBM_GBS = 6650.0
+FALLBACK_BF16_TFLOPS = 1590.0
 SCAN_SOURCES = ["selective_state_space_47_b200/csrc/ssm_scan.cu",
                 "selective_state_space_47_b200/csrc/ssm_scan_kernel.cuh",
                 "selective_state_space_47_b200/csrc/ssm_device.cuh"]
@@ -57,6 +58,8 @@ def parse_args(argv=None):
                     help="time only the backward scan on the workload (profiling runs)")
     ap.add_argument("--decode-only", action="store_true",
                     help="run only the recurrent-decode leg (1000 chained steps) and print its line")
+    ap.add_argument("--ssd-only", action="store_true",
+                    help="run only the chunked tensor-core (Mamba-2) leg on ssd_layer and print its line")
     return ap.parse_args(argv)
 
 
@@ -294,6 +297,16 @@ def run_ours(args):
     hbm_peak = peaks["hbm_gbs"] if peaks else FALLBACK_HBM_GBS
     peak_src = "measured" if peaks else "fallback"
 
+    tensor_peak = (peaks or {}).get("bf16_tflops") or FALLBACK_BF16_TFLOPS
+    if args.ssd_only:
+        line = {"metric": METRIC, "n_gpus": world, "data": "synthetic",
+                "ssd": run_ssd(ssm, synth, dev, stream, rank, hbm_peak, tensor_peak, reps=max(1, args.steps))}
+        if world > 1:
+            dist.barrier()
+            dist.destroy_process_group()
+        if rank == 0:
+            print(json.dumps(line), flush=True)
+        return 0
     if args.decode_only:
         line = {"metric": "decode state-updates/s (B·D·N per token step)", "n_gpus": world, "data": "synthetic",
                 "decode": run_decode(ssm, synth, dev, stream, rank, hbm_peak, reps=max(1, args.steps),
@@ -436,6 +449,9 @@ def run_ours(args):
                        "api": f"ssm_scan_fwd_host, pinned host tokens, {n_chunks} chunks of {chunk} steps"}
         line["gpu_launches"] += esteps * n_chunks
         del host, y_host, staging
+        # The chunked (Mamba-2) form on the tensor cores, its own workload.
+        line["ssd"] = run_ssd(ssm, synth, dev, stream, rank, hbm_peak, tensor_peak, reps=max(3, args.steps // 4))
+        line["gpu_launches"] += line["ssd"]["launches"]
         # Recurrent decode (one-token step): 1000 chained steps in one CUDA graph.
         line["decode"] = run_decode(ssm, synth, dev, stream, rank, hbm_peak)
         line["gpu_launches"] += line["decode"]["launches"]
@@ -478,6 +494,47 @@ def run_backward(ssm, inp, dev, stream, rank, hbm_peak, w, steps=3):
     return {"workload": f"{w.name} backward (dx, ddt, dz, dB, dC, dA, dD, ddt_bias)", "ms_per_step": ms,
             "value": w.updates / (ms / 1e3), "unit": UNIT, "algorithmic_bytes": nbytes, "achieved_GBs": gbs,
             "hbm_frac": gbs / hbm_peak, "kernel": "scan_bwd_kernel", "launches": steps + 1}
+
+
+def run_ssd(ssm, synth, dev, stream, rank, hbm_peak, tensor_peak, reps=3):
+    """ssm_ssd_fwd on ssd_layer (B=2, L=16384, H=80 heads of P=64 channels, N=128, bf16).
+
+    Algorithmic bytes: x, z read and y written ([B, L, H, P]), dt [B, L, H], B and C [B, L,
+    N]. Tensor FLOPs executed per launch: per chunk of Q=128 steps and head, C B^T (2 Q Q N),
+    C S twice (S in two bfloat16 parts, 2 x 2 Q N P), M x (2 Q Q P) and B^T (w x) (2 N Q P)."""
+    import torch
+    w = synth.WORKLOADS["ssd_layer"]
+    inp = synth.ssd_inputs(w.batch, w.seqlen, w.nheads, w.headdim, w.dstate, seed=rank_seed(synth.SEEDS["ssd_layer"], rank),
+                           device=dev)
+    y = torch.empty_like(inp["x"])
+    ws = ssm.ScanWorkspace()
+
+    def f():
+        ssm.ssd_fwd(inp["x"], inp["dt"], inp["A"], inp["B"], inp["C"], inp["D"], inp["z"], inp["dt_bias"], out=y,
+                    workspace=ws)
+
+    for _ in range(2):
+        f()
+    torch.cuda.synchronize(dev)
+    if ssm.workspace_status(ws) != 0:
+        raise RuntimeError("device-side status of ssm_ssd_fwd is not SSM_OK")
+    ms = time_region(f, reps, stream) / reps
+    B, L, H, P, N, Q = w.batch, w.seqlen, w.nheads, w.headdim, w.dstate, 128
+    nbytes = (3 * B * L * H * P + B * L * H + 2 * B * L * N) * 2
+    nchunk = (L + Q - 1) // Q
+    flops = B * nchunk * H * (2 * Q * Q * N + 2 * 2 * Q * N * P + 2 * Q * Q * P + 2 * N * Q * P)
+    gbs = nbytes / (ms / 1e3) / 1e9
+    tfs = flops / (ms / 1e3) / 1e12
+    upd = B * L * H * P * N
+    del inp, y, ws
+    torch.cuda.empty_cache()
+    return {"workload": f"ssd_layer B={B} L={L} H={H} P={P} N={N} bf16, gate on", "kernel": "ssd_kernel",
+            "ms_per_step": ms, "value": upd / (ms / 1e3), "unit": UNIT,
+            "roofline_hbm": {"achieved": gbs, "peak": hbm_peak, "unit": "GB/s", "frac": gbs / hbm_peak,
+                             "algorithmic_bytes_per_launch": nbytes},
+            "roofline_tensor": {"achieved": tfs, "peak": tensor_peak, "unit": "TFLOP/s", "frac": tfs / tensor_peak,
+                                "tensor_flops_per_launch": flops},
+            "launches": reps + 2}
 
 
 def run_decode(ssm, synth, dev, stream, rank, hbm_peak, reps=3, conv=False):

@@ -40,7 +40,8 @@ namespace ssd {
 constexpr int Q = 128;        // chunk length (rows of every MMA)
 constexpr int NS = 128;       // states per head
 constexpr int P = 64;         // channels per head
-constexpr int NTHREADS = 128; // four warps: warp w owns tensor-memory lanes (rows) 32w .. 32w+31
+constexpr int PH = P / 2;     // channels (columns) per thread: each row is split between two warps
+constexpr int NTHREADS = 256; // eight warps: warps w and w+4 own tensor-memory lanes (rows) 32w .. 32w+31
 constexpr int SEG = 16;       // chunks per segment (2048 steps)
 constexpr uint64_t kWaitLimitNs = 2000000000ull;
 
@@ -57,7 +58,7 @@ constexpr uint32_t OFF_SLO = OFF_S + kTile64;        // S - high part, rounded t
 constexpr uint32_t OFF_MISC = OFF_SLO + kTile64;
 constexpr uint32_t OFF_ALPHA = OFF_MISC;             // a_t log2 e per row [Q] f32
 constexpr uint32_t OFF_DELTA = OFF_ALPHA + Q * 4;    // Delta_t [Q] f32
-constexpr uint32_t OFF_WSUM = OFF_DELTA + Q * 4;     // per-warp sums [4] f32
+constexpr uint32_t OFF_WSUM = OFF_DELTA + Q * 4;     // per-warp sums of the low-half warps [4] f32
 constexpr uint32_t OFF_BAR = OFF_WSUM + 64;          // mbarriers: load[2], mma
 constexpr uint32_t OFF_TMEM = OFF_BAR + 64;          // tensor-memory base address
 constexpr uint32_t OFF_ITEM = OFF_TMEM + 16;         // claimed item
@@ -155,6 +156,32 @@ __device__ __forceinline__ float2 unpack_bf16(uint32_t w) {
     return make_float2(__uint_as_float(w << 16), __uint_as_float(w & 0xffff0000u));
 }
 
+// Global loads issued where they stand (volatile): their results are consumed much later in
+// the chunk, so their latency must not be moved next to the use.
+__device__ __forceinline__ uint16_t ldg_u16_early(const void *p) {
+    uint16_t v;
+    asm volatile("ld.global.nc.u16 %0, [%1];" : "=h"(v) : "l"(p));
+    return v;
+}
+__device__ __forceinline__ uint4 ldg_v4_early(const void *p) {
+    uint4 v;
+    asm volatile("ld.global.nc.v4.u32 {%0, %1, %2, %3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "l"(p));
+    return v;
+}
+
+// silu(z) = z / (1 + e^-z) with one special-function-unit operation: the exponential there,
+// the reciprocal of d = 1 + e^-z by Newton's method from a seed taken from d's bits
+// (0x7EF311C2 minus them: at most 5% relative error, the constant chosen to minimise that
+// over a binade) and three steps r <- r + r (1 - d r) (6e-8). -z log2 e is clamped at 125,
+// which keeps d inside the seed's range; silu(z) is then z 2^-125, zero to float precision.
+__device__ __forceinline__ float silu_1sfu(float z) {
+    const float d = 1.0f + ex2_approx(fminf(-z * kLog2e, 125.f));
+    float r = __int_as_float(0x7EF311C2 - __float_as_int(d));
+#pragma unroll
+    for (int i = 0; i < 3; ++i) r = fmaf(r, fmaf(-d, r, 1.f), r);
+    return z * r;
+}
+
 __device__ __forceinline__ void sts128(uint32_t saddr, uint4 v) {
     asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(saddr), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w)
                  : "memory");
@@ -181,6 +208,9 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + OFF_TMEM);
     int *item_slot = reinterpret_cast<int *>(smem + OFF_ITEM);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    // Row (tensor-memory lane) and column half of this thread: warps w and w+4 share the
+    // lanes 32 (w mod 4) .. +31, the first taking the low half of every row's columns.
+    const int row = tid & (Q - 1), half = tid >> 7, quarter = warp & 3;
 
     if (tid == 0) {
         mbar_init(&bar_load[0], 1);
@@ -199,9 +229,9 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
-    const uint32_t tlane = uint32_t(warp * 32) << 16;  // this warp's lane block in tensor-memory addresses
+    const uint32_t tlane = uint32_t(quarter * 32) << 16;  // this warp's lane block in tensor-memory addresses
     uint32_t ph_load[2] = {0, 0}, ph_mma = 0;
-    bool ok = true;  // every wait of this block so far completed
+    bool ok = true;  // every wait of this thread so far completed
 
     auto mma_wait = [&]() {
         if (!wait_phase(bar_mma, ph_mma)) ok = false;
@@ -221,12 +251,12 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         const float bias = p.dt_bias ? __ldg(p.dt_bias + h) : 0.f;
         const float dskip = p.Dskip ? __ldg(p.Dskip + h) : 0.f;
 
-        // The state at the segment's start, thread n holding row n of S [n][p] in float32.
-        float S[P];
+        // The state at the segment's start: this thread holds S[row][PH half .. +PH) in float32.
+        float S[PH];
         if (k == 0) {
 #pragma unroll
-            for (int q = 0; q < P; ++q)
-                S[q] = p.h0 ? __ldg(p.h0 + ((int64_t(b) * p.H + h) * P + q) * NS + tid) : 0.f;
+            for (int q = 0; q < PH; ++q)
+                S[q] = p.h0 ? __ldg(p.h0 + ((int64_t(b) * p.H + h) * P + PH * half + q) * NS + row) : 0.f;
         } else {
             if (tid == 0 && ld_acquire_gpu(p.flags + bh) < uint32_t(k)) {
                 const uint64_t start = globaltimer_ns();
@@ -241,9 +271,9 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             }
             __syncthreads();
             __threadfence();
-            const float4 *src = reinterpret_cast<const float4 *>(p.carry + (bh * NS + tid) * P);
+            const float4 *src = reinterpret_cast<const float4 *>(p.carry + (bh * NS + row) * P + PH * half);
 #pragma unroll
-            for (int q = 0; q < P / 4; ++q) {
+            for (int q = 0; q < PH / 4; ++q) {
                 const float4 v = __ldcg(src + q);
                 S[4 * q] = v.x;
                 S[4 * q + 1] = v.y;
@@ -255,7 +285,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         // bfloat16 parts, S = hi + lo to about 2^-17, so that C S keeps the float32 state's precision
         auto store_S = [&]() {
 #pragma unroll
-            for (int j = 0; j < 8; ++j) {
+            for (int j = 0; j < 4; ++j) {
                 uint32_t hi[4], lo[4];
 #pragma unroll
                 for (int e = 0; e < 4; ++e) {
@@ -263,8 +293,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                     const float2 r = unpack_bf16(hi[e]);
                     lo[e] = pack_bf16(S[8 * j + 2 * e] - r.x, S[8 * j + 2 * e + 1] - r.y);
                 }
-                sts128(sbase + OFF_S + sw_off(tid, j), make_uint4(hi[0], hi[1], hi[2], hi[3]));
-                sts128(sbase + OFF_SLO + sw_off(tid, j), make_uint4(lo[0], lo[1], lo[2], lo[3]));
+                sts128(sbase + OFF_S + sw_off(row, 4 * half + j), make_uint4(hi[0], hi[1], hi[2], hi[3]));
+                sts128(sbase + OFF_SLO + sw_off(row, 4 * half + j), make_uint4(lo[0], lo[1], lo[2], lo[3]));
             }
         };
         store_S();
@@ -280,68 +310,15 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             tma_load_3d(cc + kTile64, &tm_c, &bar_load[buf], 64, t0, b);
             tma_load_3d(smem + OFF_X + buf * kTile64, &tm_x, &bar_load[buf], h * P, t0, b);
         };
-        if (tid == 0) issue_loads(c0, 0);
-        // make S (written by threads) visible to the tensor cores before the first C S
-        fence_proxy_async_smem();
-        tc_fence_before();
-        __syncthreads();
-        tc_fence_after();
-
-        // dt of this thread's row for the first chunk (prefetched one chunk ahead)
-        const __nv_bfloat16 *dtp = p.dt + (int64_t(b) * p.L) * p.H + h;
-        auto load_dt = [&](int64_t c) -> float {
-            const int64_t t = c * Q + tid;
-            return t < p.L ? __bfloat162float(dtp[t * p.H]) : 0.f;
-        };
-        float dt_next = load_dt(c0);
-
-        for (int64_t c = c0; c < c1; ++c) {
-            const int buf = int((c - c0) & 1);
-            const int64_t t0 = c * Q;
-            const int64_t trow = t0 + tid;
-            const bool rvalid = trow < p.L;
-            // the next chunk's loads go into the other buffer, whose last readers (the
-            // previous chunk's MMAs) have completed
-            if (tid == 0 && c + 1 < c1) issue_loads(c + 1, buf ^ 1);
-            const float dtv = dt_next;
-            if (c + 1 < c1) dt_next = load_dt(c + 1);
-            // z of this row (the gate), read early so its latency overlaps the MMAs
-            uint4 zr[8];
-            if (p.z && rvalid) {
-                const uint4 *zp = reinterpret_cast<const uint4 *>(p.z + (int64_t(b) * p.L + trow) * (p.H * P) + h * P);
-#pragma unroll
-                for (int j = 0; j < 8; ++j) zr[j] = __ldg(zp + j);
-            }
-
-            // Delta and the running sum of A Delta (log2 units) over the chunk's rows
-            float d = 0.f;
-            if (rvalid) {
-                const float v = dtv + bias;
-                d = p.softplus ? softplus_f(v) : v;
-            }
-            float a = d * A2;
-#pragma unroll
-            for (int o = 1; o < 32; o <<= 1) {
-                const float n = __shfl_up_sync(0xffffffffu, a, o);
-                if (lane >= o) a += n;
-            }
-            if (lane == 31) wsum[warp] = a;
-            __syncthreads();
-#pragma unroll
-            for (int w = 0; w < 3; ++w)
-                if (w < warp) a += wsum[w];
-            alpha[tid] = a;
-            dlt[tid] = d;
-
+        // G = C B^T and Y_off = C S of chunk c (buffer buf), once its tiles have landed and S is
+        // in shared memory: issued as soon as possible, ahead of the chunk's own work
+        auto issue_G_Yoff = [&](int buf) {
             if (!wait_phase(&bar_load[buf], ph_load[buf])) ok = false;
             ph_load[buf] ^= 1u;
-            __syncthreads();  // alpha, delta visible; the chunk's tiles landed
-
-            const uint32_t sB = sbase + OFF_B + buf * kTile128, sC = sbase + OFF_C + buf * kTile128;
-            const uint32_t sX = sbase + OFF_X + buf * kTile64, sM = sbase + OFF_M, sS = sbase + OFF_S;
-            // ---- G = C B^T and Y_off = C S
             if (tid == 0) {
                 tc_fence_after();
+                const uint32_t sB = sbase + OFF_B + buf * kTile128, sC = sbase + OFF_C + buf * kTile128;
+                const uint32_t sS = sbase + OFF_S;
                 constexpr uint32_t iG = idesc_bf16(128, 128, 0, 0), iO = idesc_bf16(128, 64, 0, 1);
 #pragma unroll
                 for (int kk = 0; kk < NS / 16; ++kk) {
@@ -358,17 +335,81 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                 }
                 umma_commit(bar_mma);
             }
-            mma_wait();
+        };
+        if (tid == 0) issue_loads(c0, 0);
+        // make S (written by threads) visible to the tensor cores before the first C S
+        fence_proxy_async_smem();
+        tc_fence_before();
+        __syncthreads();
+        tc_fence_after();
+        issue_G_Yoff(0);
 
-            // ---- M = G o exp(a_t - a_s) Delta_s [s <= t], bfloat16, row t per thread
-            {
-                const float at = alpha[tid];
-                const int t = tid;
+        // dt of this thread's row for the first chunk (prefetched one chunk ahead; the low half)
+        const __nv_bfloat16 *dtp = p.dt + (int64_t(b) * p.L) * p.H + h;
+        auto load_dt = [&](int64_t c) -> float {
+            const int64_t t = c * Q + row;
+            return (half == 0 && t < p.L) ? __uint_as_float(uint32_t(ldg_u16_early(dtp + t * p.H)) << 16) : 0.f;
+        };
+        float dt_next = load_dt(c0);
+
+        for (int64_t c = c0; c < c1; ++c) {
+            const int buf = int((c - c0) & 1);
+            const int64_t t0 = c * Q;
+            const int64_t trow = t0 + row;
+            const bool rvalid = trow < p.L;
+            // the next chunk's loads go into the other buffer, whose last readers (the
+            // previous chunk's MMAs) have completed
+            if (tid == 0 && c + 1 < c1) issue_loads(c + 1, buf ^ 1);
+            const float dtv = dt_next;
+            if (c + 1 < c1) dt_next = load_dt(c + 1);
+            // z of this row's column half (the gate), read early so its latency overlaps the MMAs
+            uint4 zr[4];
+            if (p.z && rvalid) {
+                const uint4 *zp = reinterpret_cast<const uint4 *>(p.z + (int64_t(b) * p.L + trow) * (p.H * P) + h * P);
 #pragma unroll
-                for (int q = 0; q < 4; ++q) {  // 32 columns at a time
+                for (int j = 0; j < 4; ++j) zr[j] = ldg_v4_early(zp + 4 * half + j);
+            }
+
+            // Delta and the running sum of A Delta (log2 units) over the chunk's rows (low half)
+            float d = 0.f, a = 0.f;
+            if (half == 0) {
+                if (rvalid) {
+                    const float v = dtv + bias;
+                    d = p.softplus ? softplus_f(v) : v;
+                }
+                a = d * A2;
+#pragma unroll
+                for (int o = 1; o < 32; o <<= 1) {
+                    const float n = __shfl_up_sync(0xffffffffu, a, o);
+                    if (lane >= o) a += n;
+                }
+                if (lane == 31) wsum[quarter] = a;
+            }
+            __syncthreads();
+            if (half == 0) {
+#pragma unroll
+                for (int w = 0; w < 3; ++w)
+                    if (w < quarter) a += wsum[w];
+                alpha[row] = a;
+                dlt[row] = d;
+            }
+
+            __syncthreads();  // alpha, delta visible
+
+            const uint32_t sB = sbase + OFF_B + buf * kTile128;
+            const uint32_t sX = sbase + OFF_X + buf * kTile64, sM = sbase + OFF_M;
+            mma_wait();  // G and Y_off of this chunk, issued when its tiles and the state were ready
+
+            // ---- M = G o exp(a_t - a_s) Delta_s [s <= t], bfloat16: row t, columns of this half
+            {
+                const float at = alpha[row];
+                const int t = row;
+#pragma unroll
+                for (int qq = 0; qq < 2; ++qq) {  // 32 columns at a time
+                    const int q = 2 * half + qq;
                     float g[32];
                     tmem_ld32(tmem + tlane + TM_G + q * 32, g);
-                    const bool any = q * 32 <= warp * 32 + 31;  // some row of this warp reaches these columns
+                    const bool any = q * 32 <= quarter * 32 + 31;  // some row of this warp reaches these columns
 #pragma unroll
                     for (int j4 = 0; j4 < 4; ++j4) {  // 8 columns per 16-byte chunk
                         const int sb = q * 32 + j4 * 8;
@@ -385,8 +426,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                             if (any && s <= t) v = g[j4 * 8 + e] * ex2_approx(at - as[e]) * ds[e];
                             m[e] = v;
                         }
-                        const int s0 = q * 32 + j4 * 8;
-                        sts128(sM + (s0 >> 6) * kTile64 + sw_off(t, (s0 & 63) >> 3),
+                        sts128(sM + (sb >> 6) * kTile64 + sw_off(t, (sb & 63) >> 3),
                                make_uint4(pack_bf16(m[0], m[1]), pack_bf16(m[2], m[3]), pack_bf16(m[4], m[5]),
                                           pack_bf16(m[6], m[7])));
                     }
@@ -415,13 +455,13 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             // skip term rounded to bfloat16 inside M would cost up to 2^-9 |D x| where C h and D x
             // nearly cancel)
             const float alast = alpha[Q - 1];
-            uint4 xr[8];
+            uint4 xr[4];
             {
-                const int s = tid;
+                const int s = row;
                 const float w = ex2_approx(alast - alpha[s]) * dlt[s];
 #pragma unroll
-                for (int j = 0; j < 8; ++j) {
-                    const uint32_t ad = sX + sw_off(s, j);
+                for (int j = 0; j < 4; ++j) {
+                    const uint32_t ad = sX + sw_off(s, 4 * half + j);
                     const uint4 v = lds128(ad);
                     xr[j] = v;
                     const float2 e0 = unpack_bf16(v.x), e1 = unpack_bf16(v.y), e2 = unpack_bf16(v.z), e3 = unpack_bf16(v.w);
@@ -444,48 +484,40 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                 umma_commit(bar_mma);
             }
 
-            // ---- epilogue (overlaps the state MMA): y = Y_diag + exp(a_t) Y_off, gate, store
+            // ---- epilogue (overlaps the state MMA): y = Y_diag + exp(a_t) Y_off + D x, gate, store
             {
-                const float et = ex2_approx(alpha[tid]);
-                __nv_bfloat16 *yp = p.y + (int64_t(b) * p.L + trow) * (p.H * P) + h * P;
+                const float et = ex2_approx(alpha[row]);
+                float yd[32], yo[32];
+                tmem_ld32(tmem + tlane + TM_YDIAG + half * 32, yd);
+                tmem_ld32(tmem + tlane + TM_YOFF + half * 32, yo);
+                uint32_t out[16];
 #pragma unroll
-                for (int q = 0; q < 2; ++q) {
-                    float yd[32], yo[32];
-                    tmem_ld32(tmem + tlane + TM_YDIAG + q * 32, yd);
-                    tmem_ld32(tmem + tlane + TM_YOFF + q * 32, yo);
-                    uint32_t out[16];
-#pragma unroll
-                    for (int e = 0; e < 32; e += 2) {
-                        const float2 xx = unpack_bf16((&xr[q * 4].x)[e >> 1]);
-                        float v0 = fmaf(dskip, xx.x, fmaf(et, yo[e], yd[e]));
-                        float v1 = fmaf(dskip, xx.y, fmaf(et, yo[e + 1], yd[e + 1]));
-                        if (p.z) {
-                            const float2 zz = unpack_bf16(rvalid ? (&zr[q * 4].x)[e >> 1] : 0u);
-                            v0 *= silu_f(zz.x);
-                            v1 *= silu_f(zz.y);
-                        }
-                        out[e >> 1] = pack_bf16(v0, v1);
+                for (int e = 0; e < 32; e += 2) {
+                    const float2 xx = unpack_bf16((&xr[0].x)[e >> 1]);
+                    float v0 = fmaf(dskip, xx.x, fmaf(et, yo[e], yd[e]));
+                    float v1 = fmaf(dskip, xx.y, fmaf(et, yo[e + 1], yd[e + 1]));
+                    if (p.z) {
+                        const float2 zz = unpack_bf16(rvalid ? (&zr[0].x)[e >> 1] : 0u);
+                        v0 *= silu_1sfu(zz.x);
+                        v1 *= silu_1sfu(zz.y);
                     }
-                    if (rvalid) {
-                        uint4 *dst = reinterpret_cast<uint4 *>(yp + q * 32);
+                    out[e >> 1] = pack_bf16(v0, v1);
+                }
+                if (rvalid) {
+                    uint4 *dst = reinterpret_cast<uint4 *>(p.y + (int64_t(b) * p.L + trow) * (p.H * P) + h * P + half * 32);
 #pragma unroll
-                        for (int j = 0; j < 4; ++j)
-                            dst[j] = make_uint4(out[4 * j], out[4 * j + 1], out[4 * j + 2], out[4 * j + 3]);
-                    }
+                    for (int j = 0; j < 4; ++j) dst[j] = make_uint4(out[4 * j], out[4 * j + 1], out[4 * j + 2], out[4 * j + 3]);
                 }
             }
             mma_wait();
 
-            // ---- S <- exp(a_Q) S + S_acc (row n per thread), and its bfloat16 copy for the next chunk
+            // ---- S <- exp(a_Q) S + S_acc (row n, this half's columns), and its bfloat16 parts
             {
                 const float eq = ex2_approx(alast);
+                float sa[32];
+                tmem_ld32(tmem + tlane + TM_S + half * 32, sa);
 #pragma unroll
-                for (int q = 0; q < 2; ++q) {
-                    float sa[32];
-                    tmem_ld32(tmem + tlane + TM_S + q * 32, sa);
-#pragma unroll
-                    for (int e = 0; e < 32; ++e) S[q * 32 + e] = fmaf(eq, S[q * 32 + e], sa[e]);
-                }
+                for (int e = 0; e < 32; ++e) S[e] = fmaf(eq, S[e], sa[e]);
             }
             store_S();
             fence_proxy_async_smem();
@@ -494,6 +526,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             const int all_ok = __syncthreads_and(ok);
             tc_fence_after();
             if (!all_ok) break;
+            if (c + 1 < c1) issue_G_Yoff(buf ^ 1);
         }
         if (!__syncthreads_and(ok)) break;
 
@@ -501,19 +534,19 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         if (k == p.K - 1) {
             if (p.h_last) {
 #pragma unroll
-                for (int q = 0; q < P; ++q) p.h_last[((int64_t(b) * p.H + h) * P + q) * NS + tid] = S[q];
+                for (int q = 0; q < PH; ++q) p.h_last[((int64_t(b) * p.H + h) * P + PH * half + q) * NS + row] = S[q];
             }
         } else {
-            float4 *dst = reinterpret_cast<float4 *>(p.carry + (bh * NS + tid) * P);
+            float4 *dst = reinterpret_cast<float4 *>(p.carry + (bh * NS + row) * P + PH * half);
 #pragma unroll
-            for (int q = 0; q < P / 4; ++q) dst[q] = make_float4(S[4 * q], S[4 * q + 1], S[4 * q + 2], S[4 * q + 3]);
+            for (int q = 0; q < PH / 4; ++q) dst[q] = make_float4(S[4 * q], S[4 * q + 1], S[4 * q + 2], S[4 * q + 3]);
             __threadfence();
             __syncthreads();
             if (tid == 0) st_release_gpu(p.flags + bh, uint32_t(k + 1));
         }
         __syncthreads();
     }
-    if (!ok && tid == 0) atomicExch(p.status, uint32_t(SSM_ERR_TIMEOUT));
+    if (!ok) atomicExch(p.status, uint32_t(SSM_ERR_TIMEOUT));
     tc_fence_before();
     __syncthreads();
     if (warp == 0) tmem_dealloc(tmem, kTmemCols);
