@@ -66,6 +66,15 @@ enum {
                                 the Mamba summary's Theorem 1 (a gated RNN for N = 1) is exact. The
                                 kernels evaluate (exp(z) - 1) / z, z = Delta A, by a series for
                                 |z| < 1/16, where the subtraction would lose relative precision */
+    SSM_SEQ_PARALLEL = 8u,   /* evaluate the sequence in parallel segments: a local pass runs every
+                                segment from a zero state, a combine pass chains the segments'
+                                carries, a main pass runs every segment from its true start; about
+                                twice the work, used automatically when the channel groups (B x
+                                D / 32) fill at most a quarter of the GPU's block slots and L >=
+                                2048, and forced by this flag; needs the workspace
+                                ssm_scan_workspace_size() gives (a smaller one means the hand-off) */
+    SSM_SEQ_HANDOFF = 16u,   /* never the sequence-parallel evaluation (with SSM_SEQ_PARALLEL:
+                                SSM_ERR_INVALID) */
     SSM_TEST_SHORT_SEGMENTS = 0x40000000u, /* test hook: time segments of one 32-step tile each,
                                 so that every tile boundary is a carry between segments (the
                                 result is the same; it runs slower) */
@@ -103,11 +112,15 @@ typedef struct {
 /*
  * Bytes of device workspace ssm_scan_fwd needs for these shapes (0 for invalid
  * arguments, for B = 0 or D = 0, which need none, and for more than 2^40 channel slots
- * B x round_up(D, 32), which ssm_scan_fwd refuses with SSM_ERR_UNSUPPORTED). The workspace holds the hand-over of the running state between
- * consecutive time segments of a channel group, and a status word. It is small:
- * for B=1, L=262144, D=5120, N=16 it is about 330 KB. The library clears what it
- * needs at the start of each call, on the call's stream; one workspace must not
- * be shared by calls that can overlap on the GPU.
+ * B x round_up(D, 32), which ssm_scan_fwd refuses with SSM_ERR_UNSUPPORTED). The workspace
+ * holds a status word, the hand-over of the running state between consecutive time
+ * segments of a channel group (B x round_up(D, 32) x 64 bytes and a little more: about
+ * 330 KB for B=1, D=5120), and after it a fixed 4.5 MiB area for the sequence-parallel
+ * evaluation (SSM_SEQ_PARALLEL: the segments' local end states, start states and sums). A
+ * workspace with the hand-over part only (4.5 MiB less) is accepted and never takes the
+ * sequence-parallel evaluation. The library clears what it needs at the start of each
+ * call, on the call's stream; one workspace must not be shared by calls that can overlap
+ * on the GPU.
  */
 size_t ssm_scan_workspace_size(const ssm_scan_args *args);
 
@@ -119,8 +132,12 @@ size_t ssm_scan_workspace_size(const ssm_scan_args *args);
  * Sequence parallelism: the sequence of every group of channels is cut into
  * time segments; a segment starts from the state its predecessor hands over
  * (a bounded wait on a flag in the workspace), so no exponential is evaluated
- * twice. The chunked form is exact: the recurrence is associative (Mamba
- * summary, hardware-aware algorithm paragraph: parallel scan).
+ * twice. With few groups (B x D / 32 at most half the SMs) and a long sequence, or
+ * with SSM_SEQ_PARALLEL, the segments run concurrently instead: a local pass from zero
+ * states, a combine of the segments' affine maps h -> a h + l, and a main pass from
+ * the combined start states, all on the call's stream. The chunked form is exact: the
+ * recurrence is associative (Mamba summary, hardware-aware algorithm paragraph:
+ * parallel scan).
  *
  * Where every row of A used by a thread block is an exact arithmetic progression
  * in n (A[d,n] = A[d,0] + n * (A[d,1] - A[d,0]) in float32; the S4D-real
@@ -188,8 +205,10 @@ ssm_status ssm_workspace_status(const void *workspace, void *stream);
  * ssm_scan_fwd computes and takes the same arguments, but ignores
  * args->workspace: its scratch is a fixed 2 MiB array in the library's device
  * memory, which every GPU that loads the library keeps until the process
- * exits. Shapes for which ssm_scan_workspace_size() exceeds 2 MiB (a little over
- * 32,000 channels B x D) return SSM_ERR_UNSUPPORTED, with nothing launched. The
+ * exits. It holds the hand-over part of the workspace only, so the evaluation is
+ * always the hand-off (never sequence-parallel); shapes whose hand-over part exceeds
+ * 2 MiB (a little over 32,000 channels B x D) return SSM_ERR_UNSUPPORTED, with
+ * nothing launched. The
  * caller still provides all inputs
  * and outputs. Nothing is allocated: no cudaMalloc, cudaFree or allocating
  * library routine is called.
@@ -228,7 +247,8 @@ ssm_status ssm_noalloc_status(void *stream);
  * on two copy streams of the library, so both transfer directions overlap each other
  * and the kernels. The state passes from chunk to chunk through h0/h_last in the
  * staging memory, so the result equals ssm_scan_fwd over the whole sequence bit for
- * bit. Batch rows are strided in host memory ([B, L, ...]); each chunk moves them with
+ * bit where both take the hand-off evaluation (SSM_SEQ_HANDOFF makes sure of it; the
+ * sequence-parallel one differs from it by float32 rounding only). Batch rows are strided in host memory ([B, L, ...]); each chunk moves them with
  * one two-dimensional copy per tensor. With the short convolution (conv_w, conv_b and
  * conv_x0 device pointers), every chunk after the first also copies in the three host
  * tokens before it as its prefix; the staging size then includes room for them.

@@ -56,9 +56,10 @@ def _need(t, name, shape, dtype, device):
         raise ValueError(f"{name}: must be contiguous")
 
 
-def _flags(delta_softplus, general_A, exact_zoh=False):
+def _flags(delta_softplus, general_A, exact_zoh=False, seq_parallel=None):
     return ((SSM_DELTA_SOFTPLUS if delta_softplus else 0) | (SSM_A_GENERAL if general_A else 0)
-            | (SSM_EXACT_ZOH if exact_zoh else 0))
+            | (SSM_EXACT_ZOH if exact_zoh else 0)
+            | {None: 0, True: _native.SSM_SEQ_PARALLEL, False: _native.SSM_SEQ_HANDOFF}[seq_parallel])
 
 
 def _need_conv(conv_w, conv_b, conv_x0, Bsz, Dm, tok, dev):
@@ -113,7 +114,7 @@ _default_ws = {}
 
 def scan_fwd(x, dt, A, B, C, D=None, z=None, dt_bias=None, h0=None, *, delta_softplus=True,
              general_A=False, exact_zoh=False, return_last_state=False, out=None, h_last=None, workspace=None,
-             stream=None, conv_w=None, conv_b=None, conv_x0=None):
+             stream=None, conv_w=None, conv_b=None, conv_x0=None, seq_parallel=None):
     """Selective scan forward over whole sequences (see include/ssm_scan.h, ssm_scan_fwd).
 
     x, dt, z: [B, L, D] float32 or bfloat16; B, C: [B, L, N] same dtype; A: [D, N]
@@ -121,7 +122,9 @@ def scan_fwd(x, dt, A, B, C, D=None, z=None, dt_bias=None, h0=None, *, delta_sof
     as x) and, with return_last_state, the final state [B, D, N] float32. exact_zoh:
     Bbar = (exp(Delta A) - 1) / A B instead of Delta B. conv_w [D, 4] float32 (with
     conv_b [D] and conv_x0 [B, 3, D], the tokens before t = 0, both optional) runs the
-    block's causal convolution and SiLU on x inside the scan kernel.
+    block's causal convolution and SiLU on x inside the scan kernel. seq_parallel: None
+    lets the library choose between the hand-off and the sequence-parallel evaluation,
+    True forces the latter, False the former.
     """
     dev = x.device
     if x.dtype not in _TOKEN_DTYPES:
@@ -151,8 +154,8 @@ def scan_fwd(x, dt, A, B, C, D=None, z=None, dt_bias=None, h0=None, *, delta_sof
     if h_last is not None:
         _need(h_last, "h_last", (Bsz, Dm, N), torch.float32, dev)
     _need_conv(conv_w, conv_b, conv_x0, Bsz, Dm, tok, dev)
-    args = _scan_args(x, dt, A, B, C, D, z, dt_bias, h0, y, h_last, _flags(delta_softplus, general_A, exact_zoh),
-                      conv_w, conv_b, conv_x0)
+    args = _scan_args(x, dt, A, B, C, D, z, dt_bias, h0, y, h_last,
+                      _flags(delta_softplus, general_A, exact_zoh, seq_parallel), conv_w, conv_b, conv_x0)
     s = _resolve_stream(stream, dev)
     nbytes = int(_native.lib().ssm_scan_workspace_size(ctypes.byref(args)))
     if workspace is None:

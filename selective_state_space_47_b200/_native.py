@@ -10,6 +10,8 @@ SSM_F32, SSM_BF16 = 0, 1
 SSM_DELTA_SOFTPLUS = 1
 SSM_A_GENERAL = 2
 SSM_EXACT_ZOH = 4
+SSM_SEQ_PARALLEL = 8
+SSM_SEQ_HANDOFF = 16
 SSM_TEST_SHORT_SEGMENTS = 0x40000000
 SSM_TEST_DROP_HANDOFF = 0x80000000
 

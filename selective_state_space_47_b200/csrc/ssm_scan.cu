@@ -241,6 +241,7 @@ int sm_count() {
 struct ScanPlan {
     int ch = ssm::scan::CH;
     bool deep = false;
+    bool seqpar = false;  // local pass + combine + main pass instead of the hand-off
     int64_t G = 0, Dg = 0, K = 0, seg_len = 0, items = 0;
     int grid = 0;
     size_t smem = 0;
@@ -281,6 +282,68 @@ size_t pick_smem_t(ssm_dtype dt, bool deep) {
 size_t pick_smem(ssm_dtype dt, bool deep, bool conv) {
     return conv ? pick_smem_t<true>(dt, deep) : pick_smem_t<false>(dt, deep);
 }
+// Prologue warps of a configuration (each writes its own slot of the segment sums).
+int pick_np(bool deep, bool conv) {
+    using namespace ssm::scan;
+    if (!deep) return Shallow::NP;
+    return conv ? DeepConv::NP : Deep::NP;
+}
+
+// ------------------------------------------------- sequence-parallel combine
+// Between the local pass and the main pass of the sequence-parallel evaluation. Over one
+// segment k the recurrence is an affine map of the state, h_end = a_k h_start + l_k, with
+// a_k = prod_t Abar_t = 2^(A[d,n] sum_t Delta_t log2 e) (the segment's sum from the
+// prologue warps' slots) and l_k the end state the local pass reached from zero. Segment
+// 0's local pass started from h0, so a_0 = 0 and its l_0 is already exact; the start state
+// of segment k is the composition of maps 0 .. k-1 applied to 0. One warp per state
+// h[b, d, n]: lane j composes a run of consecutive segments, the lanes' runs are composed
+// by a shuffle scan ((a1, b1) then (a2, b2) is (a2 a1, a2 b1 + b2)), and each lane walks
+// its run again writing every segment's start state (segment 0's is h0 and not written).
+__global__ void __launch_bounds__(256)
+    seqpar_combine_kernel(int64_t G, int64_t K, int64_t Dg, int64_t D, int N, int np, const float *__restrict__ A,
+                          const float *__restrict__ seg_local, const float *__restrict__ seg_dsum,
+                          float *__restrict__ seg_state) {
+    constexpr int CH = ssm::scan::CH, CW = ssm::scan::CW;
+    const int64_t wid = (int64_t(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+    const int lane = threadIdx.x & 31;
+    if (wid >= G * CH * 16) return;
+    const int n = int(wid & 15), c = int((wid >> 4) % CH);
+    const int64_t g = wid / (16 * CH);
+    const int64_t d = (g % Dg) * CH + c;
+    const bool valid = d < D && n < N;
+    const float An = valid ? A[d * N + n] : 0.f;
+    const int w = n >> 2, j = n & 3;
+    auto at = [&](int64_t k) { return (((g * K + k) * CW + w) * CH + c) * 4 + j; };
+    auto factor = [&](int64_t k) {
+        if (k == 0) return 0.f;
+        float ds = 0.f;
+        for (int h = 0; h < np; ++h) ds += seg_dsum[((g * K + k) * 4 + h) * CH + c];
+        return exp2f(An * ds);
+    };
+    const int64_t per = (K + 31) / 32;
+    const int64_t k0 = lane * per < K ? lane * per : K, k1 = k0 + per < K ? k0 + per : K;
+    float ar = 1.f, br = 0.f;  // the run's map: h -> ar h + br
+    for (int64_t k = k0; k < k1; ++k) {
+        const float ak = factor(k), lk = valid ? seg_local[at(k)] : 0.f;
+        ar *= ak;
+        br = fmaf(ak, br, lk);
+    }
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const float ap = __shfl_up_sync(0xffffffffu, ar, o), bp = __shfl_up_sync(0xffffffffu, br, o);
+        if (lane >= o) {
+            br = fmaf(ar, bp, br);
+            ar *= ap;
+        }
+    }
+    float h = __shfl_up_sync(0xffffffffu, br, 1);  // the state entering this lane's run
+    if (lane == 0) h = 0.f;
+    for (int64_t k = k0; k < k1; ++k) {
+        if (k > 0) seg_state[at(k)] = valid ? h : 0.f;
+        const float ak = factor(k), lk = valid ? seg_local[at(k)] : 0.f;
+        h = fmaf(ak, h, lk);
+    }
+}
 
 // Channel slots B x round_up(D, 32) beyond which no workspace is planned: far above any
 // shape whose tokens fit in memory, and low enough that no size below overflows 64 bits.
@@ -301,12 +364,25 @@ size_t max_groups(int64_t Bsz, int64_t D) { return size_t(Bsz) * size_t((D + 15)
 
 size_t ws_flags_off() { return kWsHeader; }
 size_t ws_carry_off(int64_t Bsz, int64_t D) { return round_up(kWsHeader + max_groups(Bsz, D) * 4, 256); }
-// Workspace bytes of a scan over B sequences of D channels; 0 for shapes channel_slots
-// refuses (and for B = 0 or D = 0, which need none).
+// Workspace bytes of the hand-off evaluation over B sequences of D channels; 0 for shapes
+// channel_slots refuses (and for B = 0 or D = 0, which need none).
 size_t ws_total(int64_t Bsz, int64_t D) {
     const uint64_t slots = channel_slots(Bsz, D);
     if (slots == 0) return 0;
     return ws_carry_off(Bsz, D) + size_t(slots) * kMaxN * 4;
+}
+
+// The sequence-parallel evaluation's area after it, for at most kSeqParMaxItems (group,
+// segment) items: each item's local end state and true start state ([CW][CH] float4 each)
+// and its prologue warps' sums of Delta log2 e ([4][CH] float).
+constexpr int64_t kSeqParMaxItems = 1024;
+constexpr size_t kSeqParItemState = size_t(ssm::scan::CW) * ssm::scan::CH * 16;
+constexpr size_t kSeqParItemDsum = size_t(4) * ssm::scan::CH * 4;
+size_t ws_seqpar_off(int64_t Bsz, int64_t D) { return round_up(ws_total(Bsz, D), 256); }
+size_t ws_full(int64_t Bsz, int64_t D) {
+    const size_t base = ws_total(Bsz, D);
+    if (base == 0) return 0;
+    return ws_seqpar_off(Bsz, D) + size_t(kSeqParMaxItems) * (2 * kSeqParItemState + kSeqParItemDsum);
 }
 
 // Blocks per SM of the shallow and deep kernel configurations for a token type, with or
@@ -376,15 +452,40 @@ bool plan_scan(const ssm_scan_args *a, ScanPlan *pl) {
     if (a->flags & SSM_TEST_SHORT_SEGMENTS) pl->seg_len = TT;
     pl->K = (a->seqlen + pl->seg_len - 1) / pl->seg_len;
     pl->items = pl->G * pl->K;
+
+    // Sequence-parallel evaluation: when the groups fill at most a quarter of the block
+    // slots (it does about twice the work of the hand-off) and the sequence is long, or when
+    // the caller asks; only if the workspace has its area and the sequence gives at least
+    // two segments.
+    const int64_t slots = int64_t(occ[pl->deep ? 1 : 0]) * sms;
+    const bool want = !(a->flags & SSM_SEQ_HANDOFF) &&
+                      ((a->flags & SSM_SEQ_PARALLEL) || (4 * pl->G <= slots && a->seqlen >= 64 * TT));
+    if (want && a->workspace_bytes >= ws_full(a->batch, a->dim)) {
+        // about two items per block and pass, segments of at least 16 tiles
+        int64_t K = std::max<int64_t>(2, (2 * slots + pl->G - 1) / pl->G);
+        K = std::min<int64_t>(K, (a->seqlen + 16 * TT - 1) / (16 * TT));
+        int64_t seg = (a->seqlen + K - 1) / std::max<int64_t>(K, 1);
+        seg = (seg + TT - 1) / TT * TT;
+        if (a->flags & SSM_TEST_SHORT_SEGMENTS) seg = TT;
+        K = (a->seqlen + seg - 1) / seg;
+        if (K >= 2 && pl->G * K <= kSeqParMaxItems) {
+            pl->seqpar = true;
+            pl->seg_len = seg;
+            pl->K = K;
+            pl->items = pl->G * K;
+            pl->grid = int(std::min<int64_t>(pl->items, slots));
+        }
+    }
     return true;
 }
 
 ssm_status check_common(int64_t Bsz, int64_t D, int64_t N, ssm_dtype dt, uint32_t flags) {
     if (Bsz < 0 || D < 0 || N < 1) return SSM_ERR_INVALID;
     if (dt != SSM_F32 && dt != SSM_BF16) return SSM_ERR_INVALID;
-    if (flags & ~uint32_t(SSM_DELTA_SOFTPLUS | SSM_A_GENERAL | SSM_EXACT_ZOH | SSM_TEST_SHORT_SEGMENTS |
-                          SSM_TEST_DROP_HANDOFF))
+    if (flags & ~uint32_t(SSM_DELTA_SOFTPLUS | SSM_A_GENERAL | SSM_EXACT_ZOH | SSM_SEQ_PARALLEL |
+                          SSM_SEQ_HANDOFF | SSM_TEST_SHORT_SEGMENTS | SSM_TEST_DROP_HANDOFF))
         return SSM_ERR_INVALID;
+    if ((flags & SSM_SEQ_PARALLEL) && (flags & SSM_SEQ_HANDOFF)) return SSM_ERR_INVALID;
     if (N > kMaxN) return SSM_ERR_UNSUPPORTED;
     if (D % (dt == SSM_BF16 ? 8 : 4) != 0) return SSM_ERR_UNSUPPORTED;
     return SSM_OK;
@@ -544,7 +645,7 @@ extern "C" {
 
 size_t ssm_scan_workspace_size(const ssm_scan_args *a) {
     if (!a || a->batch < 0 || a->dim < 0) return 0;
-    return ws_total(a->batch, a->dim);
+    return ws_full(a->batch, a->dim);
 }
 
 ssm_status ssm_scan_fwd(const ssm_scan_args *a, void *stream_) {
@@ -614,10 +715,36 @@ ssm_status ssm_scan_fwd(const ssm_scan_args *a, void *stream_) {
     p.allow_structured = (a->flags & SSM_A_GENERAL) == 0;
     p.drop_handoff = (a->flags & SSM_TEST_DROP_HANDOFF) != 0;
     p.bc_tma = bc_tma;
+    p.mode = ssm::scan::kModeHandoff;
+    p.item_base = 0;
+    p.seg_local = p.seg_state = p.seg_dsum = nullptr;
 
     void *kern = pick_kernel(a->dtype, pl.deep, (a->flags & SSM_EXACT_ZOH) != 0, conv);
     void *args[] = {&tx, &tdt, &tz, &tb, &tc, &ty, &p};
-    cudaError_t e = cudaLaunchKernel(kern, dim3(pl.grid), dim3(pick_threads(pl.deep, conv)), args, pl.smem, stream);
+    const int threads = pick_threads(pl.deep, conv);
+    if (!pl.seqpar) {
+        cudaError_t e = cudaLaunchKernel(kern, dim3(pl.grid), dim3(threads), args, pl.smem, stream);
+        return e == cudaSuccess ? SSM_OK : SSM_ERR_CUDA;
+    }
+    // Sequence-parallel: local pass, combine, main pass over segments 1 .. K-1 (segment 0's
+    // outputs come from the local pass, which started it from h0).
+    unsigned char *sp = ws + ws_seqpar_off(a->batch, a->dim);
+    p.seg_local = reinterpret_cast<float *>(sp);
+    p.seg_state = reinterpret_cast<float *>(sp + size_t(kSeqParMaxItems) * kSeqParItemState);
+    p.seg_dsum = reinterpret_cast<float *>(sp + size_t(kSeqParMaxItems) * 2 * kSeqParItemState);
+    p.mode = ssm::scan::kModeLocal;
+    if (cudaLaunchKernel(kern, dim3(pl.grid), dim3(threads), args, pl.smem, stream) != cudaSuccess)
+        return SSM_ERR_CUDA;
+    if (cudaMemsetAsync(ws, 0, 4, stream) != cudaSuccess) return SSM_ERR_CUDA;  // the item counter
+    const int64_t warps = pl.G * ssm::scan::CH * 16;
+    seqpar_combine_kernel<<<unsigned((warps + 7) / 8), 256, 0, stream>>>(
+        pl.G, pl.K, pl.Dg, a->dim, int(a->dstate), pick_np(pl.deep, conv), a->A, p.seg_local, p.seg_dsum,
+        p.seg_state);
+    if (cudaGetLastError() != cudaSuccess) return SSM_ERR_CUDA;
+    p.mode = ssm::scan::kModeFromCarry;
+    p.item_base = pl.G;
+    const int grid2 = int(std::min<int64_t>(pl.items - pl.G, int64_t(pl.grid)));
+    cudaError_t e = cudaLaunchKernel(kern, dim3(grid2), dim3(threads), args, pl.smem, stream);
     return e == cudaSuccess ? SSM_OK : SSM_ERR_CUDA;
 }
 

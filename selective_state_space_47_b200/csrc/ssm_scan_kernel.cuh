@@ -131,7 +131,18 @@ struct Params {
     const float *conv_b;  // [D] or null
     const void *conv_x0;  // [B, 3, D] tokens before t = 0, or null for zeros
     int has_gate, softplus, allow_structured, drop_handoff, bc_tma;
+    // Sequence-parallel evaluation (kModeHandoff: segment k waits for k-1's state):
+    // kModeLocal: every segment runs from a zero state (segment 0 from h0, so its outputs
+    // are final and only its y is stored), writes its end state to seg_local and its sum of
+    // Delta log2 e per channel to seg_dsum; kModeFromCarry: segments 1 .. K-1 (the items
+    // from item_base = G on) start from seg_state (the combine kernel's result).
+    int mode;
+    int64_t item_base;  // the first item this launch claims
+    float *seg_local;  // [G K][CW][CH] float4
+    float *seg_state;  // [G K][CW][CH] float4
+    float *seg_dsum;   // [G K][4 prologue slots][CH]
 };
+enum : int { kModeHandoff = 0, kModeLocal = 1, kModeFromCarry = 2 };
 
 template <typename T, typename C, bool CONV = false>
 struct Layout {
@@ -426,8 +437,9 @@ __device__ __forceinline__ bool conv_prefix(const Params &p, const int64_t b, co
 // zero-order hold) u = x, the consumers apply the weight. Rows at or past tlen get
 // (0, 0): Abar = 1, no input. CONV: x is the short convolution's output (cw, cb, and
 // use_x0 / x0 as for conv_silu_rows), which is also written over the dt rows read.
+// Returns the sum of the valid rows' Delta log2 e.
 template <typename T, bool CONV, int TP>
-__device__ __forceinline__ void prologue_rows(const T *__restrict__ sx, T *__restrict__ sdt,
+__device__ __forceinline__ float prologue_rows(const T *__restrict__ sx, T *__restrict__ sdt,
                                               float4 *__restrict__ rec, const int t0, const int tlen,
                                               const float bias, const bool softplus, const bool zoh,
                                               const float4 cw, const float cb, const bool use_x0, const float3 x0) {
@@ -449,6 +461,7 @@ __device__ __forceinline__ void prologue_rows(const T *__restrict__ sx, T *__res
     for (int q = 0; q < NPR; ++q)
         delta[q] = softplus ? f2(softplus_f(v[q].x), softplus_f(v[q].y)) : v[q];
     float2 u[NPR], dl[NPR];
+    float dsum = 0.f;  // sum of the valid rows' Delta log2 e (the sequence-parallel local pass)
 #pragma unroll
     for (int q = 0; q < NPR; ++q) {
         u[q] = zoh ? xv[q] : __fmul2_rn(delta[q], xv[q]);
@@ -459,6 +472,7 @@ __device__ __forceinline__ void prologue_rows(const T *__restrict__ sx, T *__res
         const int t = t0 + 2 * q;
         const bool v0 = t < tlen, v1 = t + 1 < tlen;
         rec[(t / 2) * CH] = make_float4(v0 ? u[q].x : 0.f, v0 ? dl[q].x : 0.f, v1 ? u[q].y : 0.f, v1 ? dl[q].y : 0.f);
+        dsum += (v0 ? dl[q].x : 0.f) + (v1 ? dl[q].y : 0.f);
     }
     if (CONV) {  // the epilogue's D u
 #pragma unroll
@@ -468,6 +482,7 @@ __device__ __forceinline__ void prologue_rows(const T *__restrict__ sx, T *__res
             sdt[(t + 1) * CH] = Tok<T>::from_f(xv[q].y);
         }
     }
+    return dsum;
 }
 
 // ---------------------------------------------------------------- epilogue
@@ -581,6 +596,7 @@ __global__ void __launch_bounds__(C::NTHREADS, C::MINB)
             unsigned int it = 0;
             if (lane == 0) it = atomicAdd(p.counter, 1u);
             it = __shfl_sync(0xffffffffu, it, 0);
+            it += (unsigned int)p.item_base;
             li_ok = (long long)it < p.items;
             if (li_ok) {
                 li_k = (long long)it / p.G;
@@ -663,7 +679,7 @@ __global__ void __launch_bounds__(C::NTHREADS, C::MINB)
             warp_arrive(&bar_sfree[st]);      // x and z of this stage are no longer needed
             fence_proxy_async_smem();         // y rows written by this thread -> visible to the TMA store
             epilogue_sync();
-            if (h == 0 && lane == 0) {
+            if (h == 0 && lane == 0 && (p.mode != kModeLocal || m.k == 0)) {  // the local pass: segment 0
                 const int b = m.b, d0 = m.d0;
                 tma_store_3d(&tm_y, smem + S::yout_off + (i % YBUF) * S::yout_bytes, d0, m.t0, b);
                 bulk_commit();
@@ -681,6 +697,7 @@ __global__ void __launch_bounds__(C::NTHREADS, C::MINB)
         float bias_c = 0.f, cb = 0.f;
         float4 cw = make_float4(0.f, 0.f, 0.f, 0.f);
         bool struct_item = false;
+        float seg_dsum = 0.f;  // this warp's rows' sum of Delta log2 e over the item
         for (int i = 0;; ++i) {
             const int r = i % R_REC, st = i % STAGES;
             TileMeta *tm = &tmeta[r];
@@ -719,10 +736,13 @@ __global__ void __launch_bounds__(C::NTHREADS, C::MINB)
             float4 *rec = reinterpret_cast<float4 *>(smem + S::rec_off + r * S::rec_bytes) + c;
             float3 x0 = make_float3(0.f, 0.f, 0.f);
             const bool use_x0 = CONV && h == 0 && m.t0 == 0 && conv_prefix<T>(p, m.b, m.d0 + c, x0);
-            prologue_rows<T, CONV, TP>(reinterpret_cast<const T *>(stage + S::st_x) + S::HALO * CH + c,
-                                   reinterpret_cast<T *>(smem + S::stage_off + size_t(st) * S::stage_bytes +
-                                                         S::st_dt) + c,
-                                   rec, h * TP, m.tlen, bias_c, p.softplus != 0, ZOH, cw, cb, use_x0, x0);
+            if (m.flags & F_FIRST) seg_dsum = 0.f;
+            seg_dsum += prologue_rows<T, CONV, TP>(
+                reinterpret_cast<const T *>(stage + S::st_x) + S::HALO * CH + c,
+                reinterpret_cast<T *>(smem + S::stage_off + size_t(st) * S::stage_bytes + S::st_dt) + c, rec, h * TP,
+                m.tlen, bias_c, p.softplus != 0, ZOH, cw, cb, use_x0, x0);
+            if (p.mode == kModeLocal && (m.flags & F_LAST))
+                p.seg_dsum[((m.g * p.K + m.k) * 4 + h) * CH + c] = seg_dsum;
             // u written over dt: order it before the TMA refill of this stage (async proxy)
             if (CONV) fence_proxy_async_smem();
             // B and C rows of this half widened to float32: row t = [B_0 .. B_15 | C_0 .. C_15],
@@ -794,7 +814,15 @@ __global__ void __launch_bounds__(C::NTHREADS, C::MINB)
                                      a[2] != 0.f ? 1.f / a[2] : 0.f, a[3] != 0.f ? 1.f / a[3] : 0.f);
                 }
                 del = (dvalid && p.N >= 2) ? __ldg(p.A + d * p.N + 1) - __ldg(p.A + d * p.N) : 0.f;
-                if (m.k == 0) {
+                if (m.k > 0 && p.mode == kModeLocal) {  // the local pass: every later segment from zero
+                    h01 = f2(0.f, 0.f);
+                    h23 = f2(0.f, 0.f);
+                } else if (m.k > 0 && p.mode == kModeFromCarry) {  // the combine kernel's start state
+                    const float4 hv =
+                        __ldcg(reinterpret_cast<const float4 *>(p.seg_state) + ((m.g * p.K + m.k) * CW + w) * CH + c);
+                    h01 = f2(hv.x, hv.y);
+                    h23 = f2(hv.z, hv.w);
+                } else if (m.k == 0) {
                     float hv[4];
 #pragma unroll
                     for (int j = 0; j < 4; ++j) {
@@ -836,7 +864,19 @@ __global__ void __launch_bounds__(C::NTHREADS, C::MINB)
             else consume_tile<false, ZOH, kAhead>(rec, bc, part, Aq, del, zA, iA, h01, h23);
             warp_arrive(&bar_rec_free[r]);
             warp_arrive(&bar_part_full[pr]);
-            if (m.flags & F_LAST) {
+            if ((m.flags & F_LAST) && p.mode == kModeLocal) {
+                reinterpret_cast<float4 *>(p.seg_local)[((m.g * p.K + m.k) * CW + w) * CH + c] =
+                    make_float4(h01.x, h01.y, h23.x, h23.y);
+            } else if ((m.flags & F_LAST) && p.mode == kModeFromCarry) {
+                if (m.k == p.K - 1 && p.h_last && dvalid) {
+                    const float hv[4] = {h01.x, h01.y, h23.x, h23.y};
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) {
+                        const int n = 4 * w + j;
+                        if (n < p.N) p.h_last[(b * p.D + d) * p.N + n] = hv[j];
+                    }
+                }
+            } else if (m.flags & F_LAST) {
                 if (m.k == p.K - 1) {
                     if (p.h_last && dvalid) {
                         const float hv[4] = {h01.x, h01.y, h23.x, h23.y};

@@ -91,9 +91,12 @@ def test_workspace_size(lib):
     a = _args()
     a.batch, a.seqlen, a.dim = 1, 262144, 5120
     n = lib_ws(a)
-    # per-group flags (rounded) plus one float32 state of 16 per channel
-    assert n == 256 * ((256 + 4 * (5120 // 16) + 255) // 256) + 5120 * 16 * 4
-    assert n < 400_000
+    # per-group flags (rounded) plus one float32 state of 16 per channel: the hand-over part
+    handover = 256 * ((256 + 4 * (5120 // 16) + 255) // 256) + 5120 * 16 * 4
+    assert handover < 400_000
+    # then, 256-aligned, the sequence-parallel area: 1024 items x (two [4][32] float4 states
+    # + [4][32] float sums)
+    assert n == 256 * ((handover + 255) // 256) + 1024 * (2 * 4 * 32 * 16 + 4 * 32 * 4)
     a.batch = -1
     assert lib_ws(a) == 0
     assert lib.ssm_scan_workspace_size(None) == 0
@@ -105,6 +108,7 @@ def test_workspace_size(lib):
     (dict(dim=12), _native.SSM_ERR_UNSUPPORTED),          # bf16 needs dim % 8 == 0
     (dict(dtype=7), _native.SSM_ERR_INVALID),
     (dict(flags=0x40), _native.SSM_ERR_INVALID),
+    (dict(flags=_native.SSM_SEQ_PARALLEL | _native.SSM_SEQ_HANDOFF), _native.SSM_ERR_INVALID),
     (dict(seqlen=-1), _native.SSM_ERR_INVALID),
     (dict(x=None), _native.SSM_ERR_INVALID),
     (dict(Bm=None), _native.SSM_ERR_INVALID),
@@ -244,6 +248,7 @@ def test_bwd_workspace_size(lib):
 @pytest.mark.parametrize("bad,code", [
     (dict(flags=_native.SSM_DELTA_SOFTPLUS | _native.SSM_EXACT_ZOH), _native.SSM_ERR_UNSUPPORTED),
     (dict(flags=0x40), _native.SSM_ERR_INVALID),
+    (dict(flags=_native.SSM_SEQ_PARALLEL | _native.SSM_SEQ_HANDOFF), _native.SSM_ERR_INVALID),
     (dict(dstate=17), _native.SSM_ERR_UNSUPPORTED),
     (dict(dim=12), _native.SSM_ERR_UNSUPPORTED),
     (dict(dz=None), _native.SSM_ERR_INVALID),              # z given without dz

@@ -70,16 +70,17 @@ def test_split_sequence_equals_one_call(ssm, dtype, L, split):
     conv = _cuda(synth.conv_params(Dm, Bsz, dtype, seed=55))
     args = lambda s: [inp[k][:, s].contiguous() for k in ("x", "dt", "B", "C")]
     y, h = ssm.scan_fwd(inp["x"], inp["dt"], inp["A"], inp["B"], inp["C"], inp["D"], inp["z"], inp["dt_bias"],
-                        inp["h0"], return_last_state=True, **conv)
+                        inp["h0"], return_last_state=True, seq_parallel=False, **conv)
     a, b = slice(0, split), slice(split, L)
     xa, dta, Ba, Ca = args(a)
     xb, dtb, Bb, Cb = args(b)
     ya, ha = ssm.scan_fwd(xa, dta, inp["A"], Ba, Ca, inp["D"], inp["z"][:, a].contiguous(), inp["dt_bias"],
-                          inp["h0"], return_last_state=True, **conv)
+                          inp["h0"], return_last_state=True, seq_parallel=False, **conv)
     # the second call's prefix: the three tokens before `split` (from the first prefix if split < 3)
     x0 = torch.cat([conv["conv_x0"], xa], dim=1)[:, -3:].contiguous()
     yb, hb = ssm.scan_fwd(xb, dtb, inp["A"], Bb, Cb, inp["D"], inp["z"][:, b].contiguous(), inp["dt_bias"], ha,
-                          return_last_state=True, conv_w=conv["conv_w"], conv_b=conv["conv_b"], conv_x0=x0)
+                          return_last_state=True, conv_w=conv["conv_w"], conv_b=conv["conv_b"], conv_x0=x0,
+                          seq_parallel=False)
     torch.cuda.synchronize()
     assert torch.equal(torch.cat([ya, yb], dim=1), y)
     assert torch.equal(hb, h)
@@ -93,7 +94,7 @@ def test_host_path_with_conv_equals_device_path(ssm, chunk):
     conv = _cuda(synth.conv_params(Dm, Bsz, dtype, seed=57))
     dev = _cuda(host)
     y_dev, h_dev = ssm.scan_fwd(dev["x"], dev["dt"], dev["A"], dev["B"], dev["C"], dev["D"], dev["z"],
-                                dev["dt_bias"], dev["h0"], return_last_state=True, **conv)
+                                dev["dt_bias"], dev["h0"], return_last_state=True, seq_parallel=False, **conv)
     pin = {k: (v.pin_memory() if k in ("x", "dt", "z", "B", "C") else v) for k, v in host.items()}
     y_host, h_host = ssm.scan_fwd_host(pin["x"], pin["dt"], dev["A"], pin["B"], pin["C"], dev["D"], pin["z"],
                                        dev["dt_bias"], dev["h0"], chunk_len=chunk, return_last_state=True, **conv)

@@ -169,7 +169,7 @@ def test_handoff_timeout_is_reported(ssm):
     ws = ssm.ScanWorkspace()
     a = ssm._scan_args(inp["x"], inp["dt"], inp["A"], inp["B"], inp["C"], inp["D"], inp["z"],
                        inp["dt_bias"], None, torch.empty_like(inp["x"]), None,
-                       _native.SSM_DELTA_SOFTPLUS | _native.SSM_TEST_DROP_HANDOFF)
+                       _native.SSM_DELTA_SOFTPLUS | _native.SSM_TEST_DROP_HANDOFF | _native.SSM_SEQ_HANDOFF)
     import ctypes
     nbytes = _native.lib().ssm_scan_workspace_size(ctypes.byref(a))
     buf = ws.get(nbytes, inp["x"].device)
@@ -237,7 +237,8 @@ def test_many_short_segments(ssm, dtype):
     for general in (False, True):
         y = torch.empty_like(inp["x"])
         h = torch.empty((2, 96, 16), dtype=torch.float32, device="cuda")
-        flags = _native.SSM_DELTA_SOFTPLUS | _native.SSM_TEST_SHORT_SEGMENTS | (_native.SSM_A_GENERAL if general else 0)
+        flags = (_native.SSM_DELTA_SOFTPLUS | _native.SSM_TEST_SHORT_SEGMENTS | _native.SSM_SEQ_HANDOFF
+                 | (_native.SSM_A_GENERAL if general else 0))
         a = ssm._scan_args(inp["x"], inp["dt"], inp["A"], inp["B"], inp["C"], inp["D"], inp["z"],
                            inp["dt_bias"], inp["h0"], y, h, flags)
         ws = ssm.ScanWorkspace()
@@ -252,6 +253,6 @@ def test_many_short_segments(ssm, dtype):
         print(f"\nshort segments {dtype} general={general}: y {e_y:.3e}, h_L {e_h:.3e}")
         assert e_y <= tol and e_h <= tol
         # the same call with the planner's own segments gives the same result bit for bit
-        y2, h2 = _run(ssm, inp, general_A=general)
+        y2, h2 = _run(ssm, inp, general_A=general, seq_parallel=False)
         torch.cuda.synchronize()
         assert torch.equal(y, y2) and torch.equal(h, h2)

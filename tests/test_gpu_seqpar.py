@@ -1,0 +1,131 @@
+"""GPU parity of the sequence-parallel evaluation of ssm_scan_fwd (SSM_SEQ_PARALLEL):
+a local pass runs every time segment of a channel group from a zero state, a combine
+kernel composes the segments' affine maps h -> a h + l along the sequence, and a main
+pass runs every segment from its combined start state.
+
+Against the float64 oracle on the same bytes (tolerances as for the scan), with one-tile
+segments (test hook SSM_TEST_SHORT_SEGMENTS: every 32-step boundary is a combined carry)
+and with the planner's segments; the general and the structured exponential paths, the
+exact zero-order hold and the fused short convolution (whose three-token window reaches
+across every segment boundary). The hand-off evaluation of the same call is compared
+too: both are float32 evaluations of one recurrence and must agree within tolerance.
+"""
+import ctypes
+
+import pytest
+import torch
+
+from selective_state_space_47_b200 import synth
+from tests.conftest import cuda_available
+from tests.gpu_util import TOL, dtype_name, h_err, oracle_scan, y_err
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def ssm():
+    if not cuda_available():
+        pytest.skip("needs a CUDA device")
+    import selective_state_space_47_b200 as m
+    return m
+
+
+def _cuda(d):
+    return {k: (v.cuda() if isinstance(v, torch.Tensor) else v) for k, v in d.items()}
+
+
+def _call(ssm, inp, flags, conv=None):
+    """ssm_scan_fwd through the C ABI with explicit flags; returns y, h_last, status."""
+    from selective_state_space_47_b200 import _native
+    conv = conv or {}
+    Bsz, L, Dm = inp["x"].shape
+    N = inp["A"].shape[1]
+    y = torch.full_like(inp["x"], float("nan"))
+    h = torch.full((Bsz, Dm, N), float("nan"), dtype=torch.float32, device="cuda")
+    a = ssm._scan_args(inp["x"], inp["dt"], inp["A"], inp["B"], inp["C"], inp["D"], inp["z"], inp["dt_bias"],
+                       inp.get("h0"), y, h, flags, conv.get("conv_w"), conv.get("conv_b"), conv.get("conv_x0"))
+    ws = ssm.ScanWorkspace()
+    buf = ws.get(_native.lib().ssm_scan_workspace_size(ctypes.byref(a)), y.device)
+    a.workspace, a.workspace_bytes = ctypes.c_void_p(buf.data_ptr()), buf.numel()
+    stream = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+    assert _native.lib().ssm_scan_fwd(ctypes.byref(a), stream) == _native.SSM_OK
+    return y, h, ssm.workspace_status(ws)
+
+
+CASES = [
+    # (batch, seqlen, dim, dstate, dtype, one-tile segments, h0)
+    (1, 4097, 64, 16, torch.float32, True, True),     # 129 segments per group, ragged last tile
+    (1, 4097, 64, 16, torch.bfloat16, True, False),
+    (2, 5000, 96, 16, torch.bfloat16, False, True),   # the planner's segments, six groups
+    (1, 20000, 40, 7, torch.float32, False, True),    # lanes past D, odd dstate, long segments
+    (3, 2100, 32, 1, torch.float32, True, False),     # dstate 1, 66 segments x 3 groups
+]
+
+
+@pytest.mark.parametrize("case", CASES, ids=lambda c: f"B{c[0]}L{c[1]}D{c[2]}N{c[3]}{str(c[4])[6:]}"
+                         f"{'short' if c[5] else ''}")
+@pytest.mark.parametrize("general", [False, True], ids=["auto", "generalA"])
+def test_seq_parallel_matches_oracle(ssm, case, general):
+    from selective_state_space_47_b200 import _native
+    Bsz, L, Dm, N, dtype, short, h0 = case
+    cpu = synth.scan_inputs(Bsz, L, Dm, N, dtype, seed=2000 + L + Dm, h0=h0)
+    inp = _cuda(cpu)
+    base = _native.SSM_DELTA_SOFTPLUS | (_native.SSM_A_GENERAL if general else 0)
+    hook = _native.SSM_TEST_SHORT_SEGMENTS if short else 0
+    y, h, st = _call(ssm, inp, base | _native.SSM_SEQ_PARALLEL | hook)
+    assert st == _native.SSM_OK
+    y_ref, h_ref = oracle_scan(cpu)
+    tol = TOL[dtype_name(cpu["x"])]
+    ey, eh = y_err(y, y_ref), h_err(h, h_ref)
+    y_ho, h_ho, st_ho = _call(ssm, inp, base | _native.SSM_SEQ_HANDOFF | hook)
+    assert st_ho == _native.SSM_OK
+    d = h_err(h, h_ho.cpu().double().numpy())
+    print(f"\nseq-parallel {case} general={general}: y {ey:.3e}, h_L {eh:.3e}; h_L vs hand-off {d:.3e}")
+    assert ey <= tol and eh <= tol
+    assert eh <= 1e-4  # the float32 state regression bound of the scan tests
+    assert d <= 1e-4
+    assert y_err(y, y_ho.float().cpu().double().numpy()) <= tol
+
+
+@pytest.mark.parametrize("zoh,conv", [(True, False), (False, True), (True, True)], ids=["zoh", "conv", "zoh+conv"])
+def test_seq_parallel_zoh_and_conv(ssm, zoh, conv):
+    from selective_state_space_47_b200 import _native
+    Bsz, L, Dm, N, dtype = 2, 3001, 64, 16, torch.bfloat16
+    cpu = synth.scan_inputs(Bsz, L, Dm, N, dtype, seed=2101, h0=True)
+    g = torch.Generator().manual_seed(2102)
+    cpu["A"] = -torch.rand((Dm, N), generator=g) * 4.0 - 0.05  # general A
+    cv = synth.conv_params(Dm, Bsz, dtype, seed=2103) if conv else None
+    flags = (_native.SSM_DELTA_SOFTPLUS | _native.SSM_SEQ_PARALLEL | _native.SSM_TEST_SHORT_SEGMENTS
+             | (_native.SSM_EXACT_ZOH if zoh else 0))
+    y, h, st = _call(ssm, _cuda(cpu), flags, _cuda(cv) if cv else None)
+    assert st == _native.SSM_OK
+    y_ref, h_ref = oracle_scan(cpu, exact_zoh=zoh, conv=cv)
+    ey, eh = y_err(y, y_ref), h_err(h, h_ref)
+    print(f"\nseq-parallel zoh={zoh} conv={conv}: y {ey:.3e}, h_L {eh:.3e}")
+    assert ey <= TOL["bf16"] and eh <= TOL["bf16"]
+    assert eh <= 1e-4
+
+
+def test_seq_parallel_chosen_for_few_groups(ssm):
+    """One channel group over a long sequence: the library's own choice (no flag) is the
+    sequence-parallel evaluation, which is correct and gives the same bits as the forced one."""
+    from selective_state_space_47_b200 import _native
+    cpu = synth.scan_inputs(1, 40000, 32, 16, torch.bfloat16, seed=2104, h0=True)
+    inp = _cuda(cpu)
+    y_auto, h_auto, _ = _call(ssm, inp, _native.SSM_DELTA_SOFTPLUS)
+    y_sp, h_sp, _ = _call(ssm, inp, _native.SSM_DELTA_SOFTPLUS | _native.SSM_SEQ_PARALLEL)
+    torch.cuda.synchronize()
+    assert torch.equal(y_auto, y_sp) and torch.equal(h_auto, h_sp)
+    y_ref, h_ref = oracle_scan(cpu)
+    assert y_err(y_auto, y_ref) <= TOL["bf16"] and h_err(h_auto, h_ref) <= 1e-4
+
+
+def test_seq_parallel_flags_conflict(ssm):
+    from selective_state_space_47_b200 import _native
+    inp = _cuda(synth.scan_inputs(1, 64, 32, 16, torch.bfloat16, seed=2105))
+    a = ssm._scan_args(inp["x"], inp["dt"], inp["A"], inp["B"], inp["C"], inp["D"], inp["z"], inp["dt_bias"],
+                       None, torch.empty_like(inp["x"]), None,
+                       _native.SSM_SEQ_PARALLEL | _native.SSM_SEQ_HANDOFF)
+    buf = torch.empty(_native.lib().ssm_scan_workspace_size(ctypes.byref(a)), dtype=torch.uint8, device="cuda")
+    a.workspace, a.workspace_bytes = ctypes.c_void_p(buf.data_ptr()), buf.numel()
+    assert _native.lib().ssm_scan_fwd(ctypes.byref(a), None) == _native.SSM_ERR_INVALID
