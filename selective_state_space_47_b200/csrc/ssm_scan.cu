@@ -252,8 +252,11 @@ template <bool CONV>
 using DeepFor = typename std::conditional<CONV, ssm::scan::DeepConv, ssm::scan::Deep>::type;
 
 template <bool ZOH, bool CONV>
-void *pick_kernel_t(ssm_dtype dt, bool deep) {
+void *pick_kernel_t(ssm_dtype dt, bool deep, bool seq) {
     using namespace ssm::scan;
+    if (seq)  // the sequence-parallel passes: deep rings only
+        return dt == SSM_BF16 ? reinterpret_cast<void *>(&scan_ws_kernel<__nv_bfloat16, DeepFor<CONV>, ZOH, CONV, true>)
+                              : reinterpret_cast<void *>(&scan_ws_kernel<float, DeepFor<CONV>, ZOH, CONV, true>);
     if (dt == SSM_BF16)
         return deep ? reinterpret_cast<void *>(&scan_ws_kernel<__nv_bfloat16, DeepFor<CONV>, ZOH, CONV>)
                     : reinterpret_cast<void *>(&scan_ws_kernel<__nv_bfloat16, Shallow, ZOH, CONV>);
@@ -268,9 +271,9 @@ int pick_threads(bool deep, bool conv) {
 }
 // The exact zero-order hold and the short convolution are separate instantiations, so
 // the default kernel carries none of their code.
-void *pick_kernel(ssm_dtype dt, bool deep, bool zoh, bool conv) {
-    if (conv) return zoh ? pick_kernel_t<true, true>(dt, deep) : pick_kernel_t<false, true>(dt, deep);
-    return zoh ? pick_kernel_t<true, false>(dt, deep) : pick_kernel_t<false, false>(dt, deep);
+void *pick_kernel(ssm_dtype dt, bool deep, bool zoh, bool conv, bool seq = false) {
+    if (conv) return zoh ? pick_kernel_t<true, true>(dt, deep, seq) : pick_kernel_t<false, true>(dt, deep, seq);
+    return zoh ? pick_kernel_t<true, false>(dt, deep, seq) : pick_kernel_t<false, false>(dt, deep, seq);
 }
 template <bool CONV>
 size_t pick_smem_t(ssm_dtype dt, bool deep) {
@@ -406,6 +409,11 @@ bool scan_occupancy(ssm_dtype dt, bool conv, int occ[2]) {
             const size_t smem = pick_smem(dt, deep != 0, conv);
             int o = 0;
             if (smem <= size_t(optin)) {
+                if (deep)  // the sequence-parallel kernels share the deep shape
+                    for (int zoh = 0; zoh < 2; ++zoh)
+                        if (cudaFuncSetAttribute(pick_kernel(dt, true, zoh != 0, conv, true),
+                                                 cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem)) != cudaSuccess)
+                            return false;
                 if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem)) != cudaSuccess ||
                     cudaFuncSetAttribute(kern_zoh, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem)) !=
                         cudaSuccess ||
@@ -457,8 +465,8 @@ bool plan_scan(const ssm_scan_args *a, ScanPlan *pl) {
     // slots (it does about twice the work of the hand-off) and the sequence is long, or when
     // the caller asks; only if the workspace has its area and the sequence gives at least
     // two segments.
-    const int64_t slots = int64_t(occ[pl->deep ? 1 : 0]) * sms;
-    const bool want = !(a->flags & SSM_SEQ_HANDOFF) &&
+    const int64_t slots = int64_t(occ[1]) * sms;  // the sequence-parallel passes use the deep rings
+    const bool want = occ[1] > 0 && !(a->flags & SSM_SEQ_HANDOFF) &&
                       ((a->flags & SSM_SEQ_PARALLEL) || (4 * pl->G <= slots && a->seqlen >= 64 * TT));
     if (want && a->workspace_bytes >= ws_full(a->batch, a->dim)) {
         // about two items per block and pass, segments of at least 16 tiles
@@ -470,6 +478,8 @@ bool plan_scan(const ssm_scan_args *a, ScanPlan *pl) {
         K = (a->seqlen + seg - 1) / seg;
         if (K >= 2 && pl->G * K <= kSeqParMaxItems) {
             pl->seqpar = true;
+            pl->deep = true;
+            pl->smem = pick_smem(a->dtype, true, conv);
             pl->seg_len = seg;
             pl->K = K;
             pl->items = pl->G * K;
@@ -719,7 +729,7 @@ ssm_status ssm_scan_fwd(const ssm_scan_args *a, void *stream_) {
     p.item_base = 0;
     p.seg_local = p.seg_state = p.seg_dsum = nullptr;
 
-    void *kern = pick_kernel(a->dtype, pl.deep, (a->flags & SSM_EXACT_ZOH) != 0, conv);
+    void *kern = pick_kernel(a->dtype, pl.deep, (a->flags & SSM_EXACT_ZOH) != 0, conv, pl.seqpar);
     void *args[] = {&tx, &tdt, &tz, &tb, &tc, &ty, &p};
     const int threads = pick_threads(pl.deep, conv);
     if (!pl.seqpar) {

@@ -437,8 +437,8 @@ __device__ __forceinline__ bool conv_prefix(const Params &p, const int64_t b, co
 // zero-order hold) u = x, the consumers apply the weight. Rows at or past tlen get
 // (0, 0): Abar = 1, no input. CONV: x is the short convolution's output (cw, cb, and
 // use_x0 / x0 as for conv_silu_rows), which is also written over the dt rows read.
-// Returns the sum of the valid rows' Delta log2 e.
-template <typename T, bool CONV, int TP>
+// DSUM: returns the sum of the valid rows' Delta log2 e (else 0).
+template <typename T, bool CONV, int TP, bool DSUM>
 __device__ __forceinline__ float prologue_rows(const T *__restrict__ sx, T *__restrict__ sdt,
                                               float4 *__restrict__ rec, const int t0, const int tlen,
                                               const float bias, const bool softplus, const bool zoh,
@@ -472,7 +472,7 @@ __device__ __forceinline__ float prologue_rows(const T *__restrict__ sx, T *__re
         const int t = t0 + 2 * q;
         const bool v0 = t < tlen, v1 = t + 1 < tlen;
         rec[(t / 2) * CH] = make_float4(v0 ? u[q].x : 0.f, v0 ? dl[q].x : 0.f, v1 ? u[q].y : 0.f, v1 ? dl[q].y : 0.f);
-        dsum += (v0 ? dl[q].x : 0.f) + (v1 ? dl[q].y : 0.f);
+        if (DSUM) dsum += (v0 ? dl[q].x : 0.f) + (v1 ? dl[q].y : 0.f);
     }
     if (CONV) {  // the epilogue's D u
 #pragma unroll
@@ -539,7 +539,9 @@ __device__ __forceinline__ void epilogue_rows(const float4 *__restrict__ part, c
 }
 
 // ------------------------------------------------------------------- kernel
-template <typename T, typename C, bool ZOH, bool CONV>
+// SEQ: the sequence-parallel passes (p.mode kModeLocal or kModeFromCarry); the hand-off
+// kernel (SEQ false) carries none of their code.
+template <typename T, typename C, bool ZOH, bool CONV, bool SEQ = false>
 __global__ void __launch_bounds__(C::NTHREADS, C::MINB)
     scan_ws_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_dt,
                    const __grid_constant__ CUtensorMap tm_z, const __grid_constant__ CUtensorMap tm_b,
@@ -596,7 +598,7 @@ __global__ void __launch_bounds__(C::NTHREADS, C::MINB)
             unsigned int it = 0;
             if (lane == 0) it = atomicAdd(p.counter, 1u);
             it = __shfl_sync(0xffffffffu, it, 0);
-            it += (unsigned int)p.item_base;
+            if (SEQ) it += (unsigned int)p.item_base;
             li_ok = (long long)it < p.items;
             if (li_ok) {
                 li_k = (long long)it / p.G;
@@ -679,7 +681,7 @@ __global__ void __launch_bounds__(C::NTHREADS, C::MINB)
             warp_arrive(&bar_sfree[st]);      // x and z of this stage are no longer needed
             fence_proxy_async_smem();         // y rows written by this thread -> visible to the TMA store
             epilogue_sync();
-            if (h == 0 && lane == 0 && (p.mode != kModeLocal || m.k == 0)) {  // the local pass: segment 0
+            if (h == 0 && lane == 0 && (!SEQ || p.mode != kModeLocal || m.k == 0)) {  // local pass: segment 0
                 const int b = m.b, d0 = m.d0;
                 tma_store_3d(&tm_y, smem + S::yout_off + (i % YBUF) * S::yout_bytes, d0, m.t0, b);
                 bulk_commit();
@@ -736,13 +738,16 @@ __global__ void __launch_bounds__(C::NTHREADS, C::MINB)
             float4 *rec = reinterpret_cast<float4 *>(smem + S::rec_off + r * S::rec_bytes) + c;
             float3 x0 = make_float3(0.f, 0.f, 0.f);
             const bool use_x0 = CONV && h == 0 && m.t0 == 0 && conv_prefix<T>(p, m.b, m.d0 + c, x0);
-            if (m.flags & F_FIRST) seg_dsum = 0.f;
-            seg_dsum += prologue_rows<T, CONV, TP>(
-                reinterpret_cast<const T *>(stage + S::st_x) + S::HALO * CH + c,
-                reinterpret_cast<T *>(smem + S::stage_off + size_t(st) * S::stage_bytes + S::st_dt) + c, rec, h * TP,
-                m.tlen, bias_c, p.softplus != 0, ZOH, cw, cb, use_x0, x0);
-            if (p.mode == kModeLocal && (m.flags & F_LAST))
-                p.seg_dsum[((m.g * p.K + m.k) * 4 + h) * CH + c] = seg_dsum;
+            {
+                const T *sx = reinterpret_cast<const T *>(stage + S::st_x) + S::HALO * CH + c;
+                T *sdt = reinterpret_cast<T *>(smem + S::stage_off + size_t(st) * S::stage_bytes + S::st_dt) + c;
+                // SEQ: the segment's sum of Delta, which the local pass stores
+                if (SEQ && (m.flags & F_FIRST)) seg_dsum = 0.f;
+                seg_dsum += prologue_rows<T, CONV, TP, SEQ>(sx, sdt, rec, h * TP, m.tlen, bias_c, p.softplus != 0,
+                                                            ZOH, cw, cb, use_x0, x0);
+                if (SEQ && p.mode == kModeLocal && (m.flags & F_LAST))
+                    p.seg_dsum[((m.g * p.K + m.k) * 4 + h) * CH + c] = seg_dsum;
+            }
             // u written over dt: order it before the TMA refill of this stage (async proxy)
             if (CONV) fence_proxy_async_smem();
             // B and C rows of this half widened to float32: row t = [B_0 .. B_15 | C_0 .. C_15],
@@ -814,10 +819,10 @@ __global__ void __launch_bounds__(C::NTHREADS, C::MINB)
                                      a[2] != 0.f ? 1.f / a[2] : 0.f, a[3] != 0.f ? 1.f / a[3] : 0.f);
                 }
                 del = (dvalid && p.N >= 2) ? __ldg(p.A + d * p.N + 1) - __ldg(p.A + d * p.N) : 0.f;
-                if (m.k > 0 && p.mode == kModeLocal) {  // the local pass: every later segment from zero
+                if (SEQ && m.k > 0 && p.mode == kModeLocal) {  // the local pass: every later segment from zero
                     h01 = f2(0.f, 0.f);
                     h23 = f2(0.f, 0.f);
-                } else if (m.k > 0 && p.mode == kModeFromCarry) {  // the combine kernel's start state
+                } else if (SEQ && m.k > 0 && p.mode == kModeFromCarry) {  // the combine kernel's start state
                     const float4 hv =
                         __ldcg(reinterpret_cast<const float4 *>(p.seg_state) + ((m.g * p.K + m.k) * CW + w) * CH + c);
                     h01 = f2(hv.x, hv.y);
@@ -864,10 +869,10 @@ __global__ void __launch_bounds__(C::NTHREADS, C::MINB)
             else consume_tile<false, ZOH, kAhead>(rec, bc, part, Aq, del, zA, iA, h01, h23);
             warp_arrive(&bar_rec_free[r]);
             warp_arrive(&bar_part_full[pr]);
-            if ((m.flags & F_LAST) && p.mode == kModeLocal) {
+            if (SEQ && (m.flags & F_LAST) && p.mode == kModeLocal) {
                 reinterpret_cast<float4 *>(p.seg_local)[((m.g * p.K + m.k) * CW + w) * CH + c] =
                     make_float4(h01.x, h01.y, h23.x, h23.y);
-            } else if ((m.flags & F_LAST) && p.mode == kModeFromCarry) {
+            } else if (SEQ && (m.flags & F_LAST) && p.mode == kModeFromCarry) {
                 if (m.k == p.K - 1 && p.h_last && dvalid) {
                     const float hv[4] = {h01.x, h01.y, h23.x, h23.y};
 #pragma unroll

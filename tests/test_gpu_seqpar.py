@@ -12,6 +12,7 @@ too: both are float32 evaluations of one recurrence and must agree within tolera
 """
 import ctypes
 
+import numpy as np
 import pytest
 import torch
 
@@ -76,14 +77,20 @@ def test_seq_parallel_matches_oracle(ssm, case, general):
     assert st == _native.SSM_OK
     y_ref, h_ref = oracle_scan(cpu)
     tol = TOL[dtype_name(cpu["x"])]
-    ey, eh = y_err(y, y_ref), h_err(h, h_ref)
+    # The state's error per (b, d) row over n; with N = 1 a row is a single state, which can
+    # be a near-cancelled sum, so there it is taken relative to the largest state instead.
+    herr = h_err if N > 1 else (lambda g, r: float(np.abs(g.cpu().double().numpy() - r).max() / np.abs(r).max()))
+    ey, eh = y_err(y, y_ref), herr(h, h_ref)
     y_ho, h_ho, st_ho = _call(ssm, inp, base | _native.SSM_SEQ_HANDOFF | hook)
     assert st_ho == _native.SSM_OK
-    d = h_err(h, h_ho.cpu().double().numpy())
-    print(f"\nseq-parallel {case} general={general}: y {ey:.3e}, h_L {eh:.3e}; h_L vs hand-off {d:.3e}")
+    eh_ho = herr(h_ho, h_ref)
+    # the two evaluations against each other, relative to the largest state
+    d = float((h - h_ho).abs().max() / h_ho.abs().max())
+    print(f"\nseq-parallel {case} general={general}: y {ey:.3e}, h_L {eh:.3e} (hand-off {eh_ho:.3e}); "
+          f"max |h_L - hand-off| / max |h_L| {d:.3e}")
     assert ey <= tol and eh <= tol
     assert eh <= 1e-4  # the float32 state regression bound of the scan tests
-    assert d <= 1e-4
+    assert d <= 1e-5
     assert y_err(y, y_ho.float().cpu().double().numpy()) <= tol
 
 
