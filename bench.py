@@ -449,6 +449,10 @@ def run_ours(args):
                        "api": f"ssm_scan_fwd_host, pinned host tokens, {n_chunks} chunks of {chunk} steps"}
         line["gpu_launches"] += esteps * n_chunks
         del host, y_host, staging
+        # Few channel groups over a long sequence: the hand-off against the sequence-parallel
+        # evaluation (the library's own choice there).
+        line["seq_parallel"] = run_seq_parallel(ssm, synth, dev, stream, rank, hbm_peak, reps=max(3, args.steps // 4))
+        line["gpu_launches"] += line["seq_parallel"]["launches"]
         # The chunked (Mamba-2) form on the tensor cores, its own workload.
         line["ssd"] = run_ssd(ssm, synth, dev, stream, rank, hbm_peak, tensor_peak, reps=max(3, args.steps // 4))
         line["gpu_launches"] += line["ssd"]["launches"]
@@ -494,6 +498,42 @@ def run_backward(ssm, inp, dev, stream, rank, hbm_peak, w, steps=3):
     return {"workload": f"{w.name} backward (dx, ddt, dz, dB, dC, dA, dD, ddt_bias)", "ms_per_step": ms,
             "value": w.updates / (ms / 1e3), "unit": UNIT, "algorithmic_bytes": nbytes, "achieved_GBs": gbs,
             "hbm_frac": gbs / hbm_peak, "kernel": "scan_bwd_kernel", "launches": steps + 1}
+
+
+def run_seq_parallel(ssm, synth, dev, stream, rank, hbm_peak, reps=3):
+    """long_narrow (B=1, L=262144, D=1024, N=16, bf16, general exponential path): 32 channel
+    groups, one chain of time segments each under the hand-off; the sequence-parallel
+    evaluation runs a local pass, a combine and a main pass over all segments at once.
+    Algorithmic bytes as for the scan (x, dt, z read, y written, B and C read once)."""
+    import torch
+    w = synth.WORKLOADS["long_narrow"]
+    inp = synth.scan_inputs(w.batch, w.seqlen, w.dim, w.dstate, w.dtype, seed=rank_seed(synth.SEEDS["long_narrow"], rank),
+                            device=dev, gate=w.gate)
+    y = torch.empty_like(inp["x"])
+    ws = ssm.ScanWorkspace()
+    res = {}
+    for name, sp in (("handoff", False), ("seq_parallel", True)):
+        def f(sp=sp):
+            ssm.scan_fwd(inp["x"], inp["dt"], inp["A"], inp["B"], inp["C"], inp["D"], inp["z"], inp["dt_bias"],
+                         out=y, workspace=ws, general_A=True, seq_parallel=sp)
+        f()
+        torch.cuda.synchronize(dev)
+        if ssm.workspace_status(ws) != 0:
+            raise RuntimeError(f"device-side status of the {name} scan is not SSM_OK")
+        res[name] = time_region(f, reps, stream) / reps
+    es = 2
+    nbytes = (4 * w.batch * w.seqlen * w.dim + 2 * w.batch * w.seqlen * w.dstate) * es
+    upd = w.batch * w.seqlen * w.dim * w.dstate
+    ms = res["seq_parallel"]
+    gbs = nbytes / (ms / 1e3) / 1e9
+    del inp, y, ws
+    torch.cuda.empty_cache()
+    return {"workload": f"long_narrow B={w.batch} L={w.seqlen} D={w.dim} N={w.dstate} bf16, gate on, general A",
+            "value": upd / (ms / 1e3), "unit": UNIT, "ms_per_step": ms, "handoff_ms_per_step": res["handoff"],
+            "speedup_over_handoff": res["handoff"] / ms,
+            "roofline": {"bound": "hbm", "achieved": gbs, "peak": hbm_peak, "unit": "GB/s", "frac": gbs / hbm_peak,
+                         "algorithmic_bytes_per_launch": nbytes},
+            "launches": (reps + 1) * 1 + (reps + 1) * 3}  # hand-off: one kernel; sequence-parallel: three
 
 
 def run_ssd(ssm, synth, dev, stream, rank, hbm_peak, tensor_peak, reps=3):

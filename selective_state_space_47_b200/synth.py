@@ -65,11 +65,15 @@ WORKLOADS = {
     "small_layer": ScanWorkload("small_layer", 4, 2048, 1536, 16, torch.bfloat16, True, True),
     "mid_layer": ScanWorkload("mid_layer", 8, 4096, 2048, 16, torch.bfloat16, True, True),
     "long_context": ScanWorkload("long_context", 1, 262144, 5120, 16, torch.bfloat16, True, True),
+    # one sequence of long_context's length over a fifth of its channels: 32 channel groups,
+    # too few to fill the GPU with one chain of segments each
+    "long_narrow": ScanWorkload("long_narrow", 1, 262144, 1024, 16, torch.bfloat16, True, True),
     "decode": StepWorkload("decode", 256, 5120, 16, 1000),
     "ssd_layer": SsdWorkload("ssd_layer", 2, 16384, 80, 64, 128),
 }
 SEEDS = {"tiny_f32": SEED_BASE + 0, "small_layer": SEED_BASE + 1, "mid_layer": SEED_BASE + 2,
-         "long_context": SEED_BASE + 3, "decode": SEED_BASE + 4, "ssd_layer": SEED_BASE + 5}
+         "long_context": SEED_BASE + 3, "decode": SEED_BASE + 4, "ssd_layer": SEED_BASE + 5,
+         "long_narrow": SEED_BASE + 6}
 
 
 def _gen(seed, device):
