@@ -1,4 +1,4 @@
-"""float64 CPU oracle for the selective scan (S6) forward and the recurrent step.
+"""float64 CPU oracle for the selective scan (S6) forward, its backward and the recurrent step.
 
 TEST INFRASTRUCTURE. Only tests/, the package smoke check and the benchmark's
 CPU-baseline leg may import this package. It shares no code with the CUDA path.
@@ -32,6 +32,8 @@ def _open(path):
     lib.oracle_step_conv_f64.restype = c_int
     lib.oracle_scan_bwd_f64.argtypes = [i64, i64, i64, i64, c_int, c_uint] + [vp] * 20
     lib.oracle_scan_bwd_f64.restype = c_int
+    lib.oracle_scan_bwd_conv_f64.argtypes = [i64, i64, i64, i64, c_int, c_uint] + [vp] * 26
+    lib.oracle_scan_bwd_conv_f64.restype = c_int
     return lib
 
 
@@ -75,8 +77,9 @@ class Oracle:
                      exact_zoh, nthreads, conv_w, conv_b, conv_x0)
 
     def scan_bwd(self, x, dt, A, B, C, dy, D=None, z=None, dt_bias=None, h0=None, dh_last=None,
-                 dtype="f32", delta_softplus=True):
-        return _scan_bwd(self.lib, x, dt, A, B, C, dy, D, z, dt_bias, h0, dh_last, dtype, delta_softplus)
+                 dtype="f32", delta_softplus=True, exact_zoh=False, conv_w=None, conv_b=None, conv_x0=None):
+        return _scan_bwd(self.lib, x, dt, A, B, C, dy, D, z, dt_bias, h0, dh_last, dtype, delta_softplus,
+                         exact_zoh, conv_w, conv_b, conv_x0)
 
     def step(self, x, dt, A, B, C, h, D=None, z=None, dt_bias=None, dtype="f32",
              delta_softplus=True, exact_zoh=False, nthreads=None, conv_w=None, conv_b=None,
@@ -202,11 +205,13 @@ def _step(lib, x, dt, A, B, C, h, D=None, z=None, dt_bias=None, dtype="f32",
 
 
 def _scan_bwd(lib, x, dt, A, B, C, dy, D=None, z=None, dt_bias=None, h0=None, dh_last=None, dtype="f32",
-              delta_softplus=True):
-    """Gradients of the scan (default discretisation, no convolution) given dy = dL/dy
-    ([Bsz, L, Dm], token storage type) and dh_last = dL/dh_L ([Bsz, Dm, N] float64 or None).
-    Returns a dict of float64 arrays: dx, ddt, dz (None without z) [Bsz, L, Dm]; dB, dC
-    [Bsz, L, N]; dA [Dm, N]; dD, ddt_bias [Dm]; dh0 [Bsz, Dm, N]."""
+              delta_softplus=True, exact_zoh=False, conv_w=None, conv_b=None, conv_x0=None):
+    """Gradients of the scan given dy = dL/dy ([Bsz, L, Dm], token storage type) and
+    dh_last = dL/dh_L ([Bsz, Dm, N] float64 or None); exact_zoh and the short convolution
+    (conv_w, conv_b, conv_x0) as for ``_scan``. Returns a dict of float64 arrays: dx, ddt,
+    dz (None without z) [Bsz, L, Dm]; dB, dC [Bsz, L, N]; dA [Dm, N]; dD, ddt_bias [Dm];
+    dh0 [Bsz, Dm, N]; with the convolution also dconv_w [Dm, 4], dconv_b [Dm] and
+    dconv_x0 [Bsz, 3, Dm] (dx is then the gradient of the raw tokens before it)."""
     Bsz, L, Dm = np.shape(x)
     N = np.shape(A)[1]
     x = _tok(x, dtype, (Bsz, L, Dm), "x")
@@ -227,11 +232,22 @@ def _scan_bwd(lib, x, dt, A, B, C, dy, D=None, z=None, dt_bias=None, h0=None, dh
                dz=None if z is None else np.empty((Bsz, L, Dm)), dB=np.empty((Bsz, L, N)),
                dC=np.empty((Bsz, L, N)), dA=np.empty((Dm, N)), dD=np.empty(Dm), ddt_bias=np.empty(Dm),
                dh0=np.empty((Bsz, Dm, N)))
-    rc = lib.oracle_scan_bwd_f64(Bsz, L, Dm, N, 0 if dtype == "f32" else 1, DELTA_SOFTPLUS if delta_softplus else 0,
-                                 _ptr(x), _ptr(dt), _ptr(z), _ptr(B), _ptr(C), _ptr(A), _ptr(D), _ptr(dt_bias),
-                                 _ptr(h0), _ptr(dy), _ptr(dh_last), _ptr(out["dx"]), _ptr(out["ddt"]),
-                                 _ptr(out["dz"]), _ptr(out["dB"]), _ptr(out["dC"]), _ptr(out["dA"]), _ptr(out["dD"]),
-                                 _ptr(out["ddt_bias"]), _ptr(out["dh0"]))
+    if conv_w is None:
+        if conv_b is not None or conv_x0 is not None:
+            raise ValueError("conv_b and conv_x0 need conv_w")
+    else:
+        conv_w = _f32(conv_w, (Dm, 4), "conv_w")
+        conv_b = _f32(conv_b, (Dm,), "conv_b")
+        conv_x0 = None if conv_x0 is None else _tok(conv_x0, dtype, (Bsz, 3, Dm), "conv_x0")
+        out.update(dconv_w=np.empty((Dm, 4)), dconv_b=np.empty(Dm), dconv_x0=np.empty((Bsz, 3, Dm)))
+    flags = (DELTA_SOFTPLUS if delta_softplus else 0) | (EXACT_ZOH if exact_zoh else 0)
+    rc = lib.oracle_scan_bwd_conv_f64(Bsz, L, Dm, N, 0 if dtype == "f32" else 1, flags,
+                                      _ptr(x), _ptr(dt), _ptr(z), _ptr(B), _ptr(C), _ptr(A), _ptr(D), _ptr(dt_bias),
+                                      _ptr(h0), _ptr(conv_w), _ptr(conv_b), _ptr(conv_x0), _ptr(dy), _ptr(dh_last),
+                                      _ptr(out["dx"]), _ptr(out["ddt"]), _ptr(out["dz"]), _ptr(out["dB"]),
+                                      _ptr(out["dC"]), _ptr(out["dA"]), _ptr(out["dD"]), _ptr(out["ddt_bias"]),
+                                      _ptr(out["dh0"]), _ptr(out.get("dconv_w")), _ptr(out.get("dconv_b")),
+                                      _ptr(out.get("dconv_x0")))
     if rc != 0:
-        raise ValueError("oracle_scan_bwd_f64 rejected its arguments")
+        raise ValueError("oracle_scan_bwd_conv_f64 rejected its arguments")
     return out

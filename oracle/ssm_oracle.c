@@ -242,6 +242,31 @@ int oracle_step_conv_f64(int64_t Bsz, int64_t Dm, int64_t N, int dtype, unsigned
 }
 
 /*
+ * Weight of the input under the exact zero-order hold and its two derivatives, for one
+ * state: w = (exp(Delta a) - 1) / a (w = Delta for a = 0), dw/dDelta = exp(Delta a), and
+ * dw/da = Delta^2 f(Delta a) with f(s) = (s e^s - e^s + 1) / s^2. Near s = 0 the closed
+ * form of f cancels, so there f is its Taylor series, the sum over k >= 0 of
+ * (k + 1) s^k / (k + 2)! (differentiate w = Delta sum_k s^k / (k + 1)! term by term).
+ */
+static void zoh_weight(double delta, double a, double *w, double *dw_ddelta, double *dw_da) {
+    const double s = delta * a;
+    *dw_ddelta = exp(s);
+    *w = a != 0.0 ? expm1(s) / a : delta;
+    double f;
+    if (fabs(s) < 0.25) {
+        double term = 0.5, sum = 0.0; /* term_k = (k + 1) s^k / (k + 2)! */
+        for (int k = 0; k < 24; k++) {
+            sum += term;
+            term *= s * (double)(k + 2) / ((double)(k + 1) * (double)(k + 3));
+        }
+        f = sum;
+    } else {
+        f = (s * exp(s) - expm1(s)) / (s * s);
+    }
+    *dw_da = delta * delta * f;
+}
+
+/*
  * Backward of the scan: the gradients of a loss with respect to every input, given
  * dL/dy (dy, storage type of the tokens) and optionally dL/dh_L (dh_last, double, or
  * NULL for 0). The pages print no backward formulas; the plain definition is the
@@ -251,39 +276,60 @@ int oracle_step_conv_f64(int64_t Bsz, int64_t Dm, int64_t N, int dtype, unsigned
  * each channel's forward states are simply kept for its reverse sweep.
  *
  * Per channel (b, d), with v_t = dt_t + bias, Delta_t = softplus(v_t) (or v_t),
- * Abar_tn = exp(Delta_t A_n), q_t = C_t . h_t + D x_t and y_t = q_t silu(z_t) (or q_t):
+ * Abar_tn = exp(Delta_t A_n), the SSM input u_t (x_t, or the short convolution's output),
+ * the input weight w_tn = Delta_t (or, with ORACLE_EXACT_ZOH, (Abar_tn - 1) / A_n),
+ * q_t = C_t . h_t + D u_t and y_t = q_t silu(z_t) (or q_t):
  *   dq_t = dy_t silu(z_t);  dz_t = dy_t q_t silu'(z_t)
  *   g_t  = dL/dh_t = dq_t C_t + Abar_{t+1} g_{t+1},  g_L = dq_L C_L + dh_last
- *   dx_t = dq_t D + sum_n g_tn Delta_t B_tn
- *   dDelta_t = sum_n g_tn (A_n Abar_tn h_{t-1,n} + B_tn x_t);  ddt_t = dDelta_t sigma(v_t)
- *   dA_n += g_tn Delta_t Abar_tn h_{t-1,n};  dB_tn += g_tn Delta_t x_t;  dC_tn += dq_t h_tn
- *   dD += dq_t x_t;  dbias += ddt_t;  dh0 = Abar_1 g_1
- * dB, dC ([Bsz, L, N]) sum over the channels of a sequence; dA ([Dm, N]), dD and dbias
- * ([Dm]) over sequences and time. Only the default discretisation (Bbar = Delta B) and
- * no convolution. Single-threaded. Returns 0, or -1 on invalid arguments.
+ *   du_t = dq_t D + sum_n g_tn w_tn B_tn
+ *   dDelta_t = sum_n g_tn (A_n Abar_tn h_{t-1,n} + dw_tn/dDelta B_tn u_t);  ddt_t = dDelta_t sigma(v_t)
+ *   dA_n += g_tn (Delta_t Abar_tn h_{t-1,n} + dw_tn/dA_n B_tn u_t)
+ *   dB_tn += g_tn w_tn u_t;  dC_tn += dq_t h_tn;  dD += dq_t u_t;  dbias += ddt_t;  dh0 = Abar_1 g_1
+ * (dw/dDelta = 1 and dw/dA = 0 for w = Delta.) Without the convolution dx_t = du_t. With it,
+ * u_t = silu(p_t), p_t = conv_b + sum_k conv_w[k] x_{t-3+k}, and dp_t = du_t silu'(p_t):
+ *   dx_tau += conv_w[k] dp_t (tau = t-3+k; tau < 0 goes to dconv_x0[tau + 3])
+ *   dconv_w[k] += dp_t x_{t-3+k};  dconv_b += dp_t
+ * dB, dC ([Bsz, L, N]) sum over the channels of a sequence; dA ([Dm, N]), dD, dbias, dconv_w
+ * and dconv_b over sequences and time. Single-threaded. Returns 0, or -1 on invalid arguments.
  */
-int oracle_scan_bwd_f64(int64_t Bsz, int64_t L, int64_t Dm, int64_t N, int dtype, unsigned flags,
-                        const void *x, const void *dt, const void *z, const void *Bm, const void *Cm,
-                        const float *A, const float *Dskip, const float *dt_bias, const float *h0,
-                        const void *dy, const double *dh_last, double *dx, double *ddt, double *dz,
-                        double *dB, double *dC, double *dA, double *dD, double *dbias, double *dh0) {
+int oracle_scan_bwd_conv_f64(int64_t Bsz, int64_t L, int64_t Dm, int64_t N, int dtype, unsigned flags,
+                             const void *x, const void *dt, const void *z, const void *Bm, const void *Cm,
+                             const float *A, const float *Dskip, const float *dt_bias, const float *h0,
+                             const float *conv_w, const float *conv_b, const void *conv_x0,
+                             const void *dy, const double *dh_last, double *dx, double *ddt, double *dz,
+                             double *dB, double *dC, double *dA, double *dD, double *dbias, double *dh0,
+                             double *dconv_w, double *dconv_b, double *dconv_x0) {
     if (Bsz < 0 || L < 0 || Dm < 0 || N < 1 || N > 256 || (dtype != 0 && dtype != 1)) return -1;
-    if (flags & ~ORACLE_DELTA_SOFTPLUS) return -1;
+    if (flags & ~(ORACLE_DELTA_SOFTPLUS | ORACLE_EXACT_ZOH)) return -1;
     if (!x || !dt || !Bm || !Cm || !A || !dy || !dx || !ddt || !dB || !dC || !dA || !dD || !dbias) return -1;
     if (z && !dz) return -1;
+    if (!conv_w && (conv_b || conv_x0)) return -1;
+    if (conv_w && (!dconv_w || !dconv_b || !dconv_x0)) return -1;
     const int softplus_on = (flags & ORACLE_DELTA_SOFTPLUS) != 0;
+    const int zoh = (flags & ORACLE_EXACT_ZOH) != 0;
+    memset(dx, 0, sizeof(double) * (size_t)(Bsz * L * Dm));
     memset(dB, 0, sizeof(double) * (size_t)(Bsz * L * N));
     memset(dC, 0, sizeof(double) * (size_t)(Bsz * L * N));
     memset(dA, 0, sizeof(double) * (size_t)(Dm * N));
     memset(dD, 0, sizeof(double) * (size_t)Dm);
     memset(dbias, 0, sizeof(double) * (size_t)Dm);
+    if (conv_w) {
+        memset(dconv_w, 0, sizeof(double) * (size_t)(Dm * ORACLE_CONV_K));
+        memset(dconv_b, 0, sizeof(double) * (size_t)Dm);
+        memset(dconv_x0, 0, sizeof(double) * (size_t)(Bsz * (ORACLE_CONV_K - 1) * Dm));
+    }
+    /* the convolution's inputs, read through the forward's own helpers */
+    scan_job cj = {Bsz, L, Dm, N, dtype, flags, x, dt, z, Bm, Cm, A, Dskip, dt_bias, h0,
+                   NULL, NULL, NULL, 0, 0, conv_w, conv_b, conv_x0};
     /* forward states of one channel: hs[t * N + n] = h_{t-1,n} for t = 0..L (hs[0] = h0) */
     double *hs = (double *)malloc(sizeof(double) * (size_t)((L + 1) * N));
     double *delta = (double *)malloc(sizeof(double) * (size_t)(L > 0 ? L : 1));
+    double *u = (double *)malloc(sizeof(double) * (size_t)(L > 0 ? L : 1));
     double *g = (double *)malloc(sizeof(double) * (size_t)N);
-    if (!hs || !delta || !g) {
+    if (!hs || !delta || !u || !g) {
         free(hs);
         free(delta);
+        free(u);
         free(g);
         return -1;
     }
@@ -297,16 +343,19 @@ int oracle_scan_bwd_f64(int64_t Bsz, int64_t L, int64_t Dm, int64_t N, int dtype
                 const int64_t i = (b * L + t) * Dm + d, bc = (b * L + t) * N;
                 const double v = widen(dt, dtype, i) + bias;
                 delta[t] = softplus_on ? softplus(v) : v;
-                const double xv = widen(x, dtype, i);
-                for (int64_t n = 0; n < N; n++)
-                    hs[(t + 1) * N + n] = exp(delta[t] * (double)A[d * N + n]) * hs[t * N + n] +
-                                          delta[t] * widen(Bm, dtype, bc + n) * xv;
+                u[t] = conv_w ? conv_silu(&cj, b, t, d) : widen(x, dtype, i);
+                for (int64_t n = 0; n < N; n++) {
+                    const double a = (double)A[d * N + n];
+                    double w = delta[t], wd, wa;
+                    if (zoh) zoh_weight(delta[t], a, &w, &wd, &wa);
+                    hs[(t + 1) * N + n] = exp(delta[t] * a) * hs[t * N + n] + w * widen(Bm, dtype, bc + n) * u[t];
+                }
             }
             /* reverse */
             for (int64_t n = 0; n < N; n++) g[n] = dh_last ? dh_last[(b * Dm + d) * N + n] : 0.0;
             for (int64_t t = L - 1; t >= 0; t--) {
                 const int64_t i = (b * L + t) * Dm + d, bc = (b * L + t) * N;
-                const double xv = widen(x, dtype, i);
+                const double xv = u[t];
                 double q = dsk * xv;
                 for (int64_t n = 0; n < N; n++) q += widen(Cm, dtype, bc + n) * hs[(t + 1) * N + n];
                 double dq = widen(dy, dtype, i);
@@ -320,18 +369,38 @@ int oracle_scan_bwd_f64(int64_t Bsz, int64_t L, int64_t Dm, int64_t N, int dtype
                 for (int64_t n = 0; n < N; n++) {
                     const double a = (double)A[d * N + n], abar = exp(delta[t] * a);
                     const double bn = widen(Bm, dtype, bc + n), hp = hs[t * N + n];
+                    double w = delta[t], w_dd = 1.0, w_da = 0.0;
+                    if (zoh) zoh_weight(delta[t], a, &w, &w_dd, &w_da);
                     g[n] += dq * widen(Cm, dtype, bc + n);
                     dC[bc + n] += dq * hs[(t + 1) * N + n];
-                    dxv += g[n] * delta[t] * bn;
-                    ddel += g[n] * (a * abar * hp + bn * xv);
-                    dA[d * N + n] += g[n] * delta[t] * abar * hp;
-                    dB[bc + n] += g[n] * delta[t] * xv;
+                    dxv += g[n] * w * bn;
+                    ddel += g[n] * (a * abar * hp + w_dd * bn * xv);
+                    dA[d * N + n] += g[n] * (delta[t] * abar * hp + w_da * bn * xv);
+                    dB[bc + n] += g[n] * w * xv;
                     g[n] *= abar; /* now dL/dh_{t-1} through h_t */
                 }
                 const double v = widen(dt, dtype, i) + bias;
                 ddt[i] = softplus_on ? ddel * sigmoid(v) : ddel;
                 dbias[d] += ddt[i];
-                dx[i] = dxv;
+                if (conv_w) {
+                    /* dx through the convolution: p_t from the taps, u = silu(p) */
+                    double p = conv_b ? (double)conv_b[d] : 0.0;
+                    for (int k = 0; k < ORACLE_CONV_K; k++)
+                        p += (double)conv_w[d * ORACLE_CONV_K + k] * raw_token(&cj, b, t - (ORACLE_CONV_K - 1) + k, d);
+                    const double sp = sigmoid(p), dp = dxv * sp * (1.0 + p * (1.0 - sp));
+                    dconv_b[d] += dp;
+                    for (int k = 0; k < ORACLE_CONV_K; k++) {
+                        const int64_t tau = t - (ORACLE_CONV_K - 1) + k;
+                        dconv_w[d * ORACLE_CONV_K + k] += dp * raw_token(&cj, b, tau, d);
+                        const double dtok = dp * (double)conv_w[d * ORACLE_CONV_K + k];
+                        if (tau >= 0)
+                            dx[(b * L + tau) * Dm + d] += dtok;
+                        else
+                            dconv_x0[(b * (ORACLE_CONV_K - 1) + (tau + ORACLE_CONV_K - 1)) * Dm + d] += dtok;
+                    }
+                } else {
+                    dx[i] = dxv;
+                }
             }
             if (dh0)
                 for (int64_t n = 0; n < N; n++) dh0[(b * Dm + d) * N + n] = g[n];
@@ -339,6 +408,18 @@ int oracle_scan_bwd_f64(int64_t Bsz, int64_t L, int64_t Dm, int64_t N, int dtype
     }
     free(hs);
     free(delta);
+    free(u);
     free(g);
     return 0;
+}
+
+/* The backward without the short convolution (see oracle_scan_bwd_conv_f64). */
+int oracle_scan_bwd_f64(int64_t Bsz, int64_t L, int64_t Dm, int64_t N, int dtype, unsigned flags,
+                        const void *x, const void *dt, const void *z, const void *Bm, const void *Cm,
+                        const float *A, const float *Dskip, const float *dt_bias, const float *h0,
+                        const void *dy, const double *dh_last, double *dx, double *ddt, double *dz,
+                        double *dB, double *dC, double *dA, double *dD, double *dbias, double *dh0) {
+    return oracle_scan_bwd_conv_f64(Bsz, L, Dm, N, dtype, flags, x, dt, z, Bm, Cm, A, Dskip, dt_bias, h0, NULL,
+                                    NULL, NULL, dy, dh_last, dx, ddt, dz, dB, dC, dA, dD, dbias, dh0, NULL, NULL,
+                                    NULL);
 }

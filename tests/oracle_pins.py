@@ -467,29 +467,45 @@ def _bwd_case(rng, Bsz, L, Dm, N, gate=True):
                 D=f(Dm), dt_bias=(0.5 * f(Dm)).astype(np.float32), h0=f(Bsz, Dm, N))
 
 
-def pin_bwd_finite_differences(orc, seed=15, softplus=True, gate=True):
+def pin_bwd_finite_differences(orc, seed=15, softplus=True, gate=True, exact_zoh=False, conv=False):
     """Every gradient of the backward equals the central difference of the forward.
 
     The loss is L = sum(dy * y) + sum(dh_last * h_L) with random dy, dh_last, so dL/dp is
     what the backward returns for dy, dh_last. Each input element p (float32) is moved by
     +-2^-12, exactly representable, and (L(p+) - L(p-)) / (p+ - p-) is compared with the
     gradient (truncation ~1e-7 relative at this step). A plain derivative check, by a
-    route independent of the reverse sweep."""
+    route independent of the reverse sweep. exact_zoh and conv (the short convolution,
+    with bias and the three tokens before the sequence) select those forward variants; the
+    convolution's taps, bias and prefix tokens are then differentiated too."""
     rng = _rng(seed)
     Bsz, L, Dm, N = 2, 6, 3, 3
     inp = _bwd_case(rng, Bsz, L, Dm, N, gate)
+    if exact_zoh:
+        # A spanning the exact hold's regimes: tiny |Delta A| (the series branch of dw/dA),
+        # exactly zero (w = Delta), and ordinary values
+        inp["A"][0, 0], inp["A"][1, 1], inp["A"][2, 2] = np.float32(-1e-3), np.float32(0.0), np.float32(3e-4)
+    cv = {}
+    if conv:
+        cv = dict(conv_w=(rng.random((Dm, 4)) - 0.5).astype(np.float32),
+                  conv_b=(rng.random(Dm) - 0.5).astype(np.float32),
+                  conv_x0=rng.standard_normal((Bsz, 3, Dm)).astype(np.float32))
+        inp.update(cv)
     dy = rng.standard_normal((Bsz, L, Dm)).astype(np.float32)
     dh_last = rng.standard_normal((Bsz, Dm, N))
 
     def loss(v):
+        kw = {k: v[k] for k in cv}
         y, h = orc.scan(v["x"], v["dt"], v["A"], v["B"], v["C"], D=v["D"], z=v["z"], dt_bias=v["dt_bias"],
-                        h0=v["h0"], delta_softplus=softplus)
+                        h0=v["h0"], delta_softplus=softplus, exact_zoh=exact_zoh, **kw)
         return float(np.sum(dy * y) + np.sum(dh_last * h))
 
     g = orc.scan_bwd(inp["x"], inp["dt"], inp["A"], inp["B"], inp["C"], dy, D=inp["D"], z=inp["z"],
-                     dt_bias=inp["dt_bias"], h0=inp["h0"], dh_last=dh_last, delta_softplus=softplus)
+                     dt_bias=inp["dt_bias"], h0=inp["h0"], dh_last=dh_last, delta_softplus=softplus,
+                     exact_zoh=exact_zoh, **cv)
     names = {"x": "dx", "dt": "ddt", "z": "dz", "B": "dB", "C": "dC", "A": "dA", "D": "dD",
              "dt_bias": "ddt_bias", "h0": "dh0"}
+    if conv:
+        names.update(conv_w="dconv_w", conv_b="dconv_b", conv_x0="dconv_x0")
     step = np.float32(2.0 ** -12)
     for key, gname in names.items():
         if inp[key] is None:
@@ -531,7 +547,52 @@ def pin_bwd_bf16_storage(orc, seed=17):
         assert np.array_equal(g16[k], g32[k]), f"bf16 backward {k} differs"
 
 
-ALL_PINS += [pin_bwd_finite_differences, pin_bwd_finite_differences_plain, pin_bwd_bf16_storage]
+def pin_bwd_finite_differences_zoh(orc):
+    """The backward of the exact zero-order hold, against the central difference."""
+    pin_bwd_finite_differences(orc, seed=20, exact_zoh=True)
+
+
+def pin_bwd_finite_differences_conv(orc):
+    """The backward through the short convolution (taps, bias, prefix tokens and the raw
+    tokens), against the central difference."""
+    pin_bwd_finite_differences(orc, seed=21, conv=True)
+
+
+def pin_bwd_finite_differences_zoh_conv(orc):
+    """Both variants at once, without softplus."""
+    pin_bwd_finite_differences(orc, seed=22, softplus=False, exact_zoh=True, conv=True)
+
+
+def pin_zoh_weight_series_matches_closed_form(orc, seed=23):
+    """dL/dA of the exact hold on both sides of |Delta A| = 0.25, where the oracle switches
+    between the closed form of dw/dA and its series: for A in {-0.05, -0.2, -0.3, -1.5}
+    (with Delta about 0.3 to 1.5) it equals the central difference of the loss in A, with
+    a step of 2^-14 and a tolerance of 1e-6."""
+    rng = _rng(seed)
+    Bsz, L, Dm, N = 1, 5, 1, 2
+    inp = _bwd_case(rng, Bsz, L, Dm, N, gate=False)
+    dy = rng.standard_normal((Bsz, L, Dm)).astype(np.float32)
+    for a in (-0.05, -0.2, -0.3, -1.5):  # Delta ~ 0.5..1.5 puts Delta A on both sides of 0.25
+        inp["A"][0, :] = np.float32(a)
+        g = orc.scan_bwd(inp["x"], inp["dt"], inp["A"], inp["B"], inp["C"], dy, D=inp["D"],
+                         dt_bias=inp["dt_bias"], h0=inp["h0"], exact_zoh=True)["dA"]
+
+        def loss(A):
+            y, _ = orc.scan(inp["x"], inp["dt"], A, inp["B"], inp["C"], D=inp["D"], dt_bias=inp["dt_bias"],
+                            h0=inp["h0"], exact_zoh=True)
+            return float(np.sum(dy * y))
+        for n in range(N):
+            A1, A2 = inp["A"].copy(), inp["A"].copy()
+            st = np.float32(2.0 ** -14)
+            A1[0, n] += st
+            A2[0, n] -= st
+            fd = (loss(A1) - loss(A2)) / (float(A1[0, n]) - float(A2[0, n]))
+            assert abs(g[0, n] - fd) <= 1e-6 * max(1.0, abs(fd)), f"dA at A = {a} differs from the central difference"
+
+
+ALL_PINS += [pin_bwd_finite_differences, pin_bwd_finite_differences_plain, pin_bwd_bf16_storage,
+             pin_bwd_finite_differences_zoh, pin_bwd_finite_differences_conv, pin_bwd_finite_differences_zoh_conv,
+             pin_zoh_weight_series_matches_closed_form]
 
 
 def pin_ssd_semiseparable_form(orc, seed=18):

@@ -45,18 +45,32 @@ MUTANTS = {
     "conv_without_silu": ("return v * sigmoid(v);", "return v;"),
     "conv_x0_ignored": ("if (J->conv_x0) return", "if (0) return"),
     "conv_x0_rows_reversed": ("(tau + ORACLE_CONV_K - 1)", "(-1 - tau)"),
-    "conv_reads_next_token": ("t - (ORACLE_CONV_K - 1) + k", "t - (ORACLE_CONV_K - 2) + k"),
+    # (the shifted window stays inside x: it moves one token ahead except at the last step)
+    "conv_reads_next_token": ("raw_token(J, b, t - (ORACLE_CONV_K - 1) + k, d)",
+                              "raw_token(J, b, t - (ORACLE_CONV_K - 1) + k + (t + 1 < J->L), d)"),
     "conv_skip_uses_raw_x": ("y += dskip * xv;", "y += dskip * widen(J->x, J->dtype, i);"),
     "conv_update_uses_raw_x": ("h[n] = abar * h[n] + bbar * xv;", "h[n] = abar * h[n] + bbar * widen(J->x, J->dtype, i);"),
     "bwd_gate_derivative": ("dz[i] = dq * q * sg * (1.0 + zv * (1.0 - sg));", "dz[i] = dq * q * sg;"),
     "bwd_adjoint_decay_first": ("                    g[n] += dq * widen(Cm, dtype, bc + n);\n",
                                 "                    g[n] = g[n] * exp(delta[t] * a) + dq * widen(Cm, dtype, bc + n);\n"),
-    "bwd_dA_without_abar": ("dA[d * N + n] += g[n] * delta[t] * abar * hp;", "dA[d * N + n] += g[n] * delta[t] * hp;"),
+    "bwd_dA_without_abar": ("g[n] * (delta[t] * abar * hp + w_da", "g[n] * (delta[t] * hp + w_da"),
     "bwd_dC_previous_state": ("dC[bc + n] += dq * hs[(t + 1) * N + n];", "dC[bc + n] += dq * hs[t * N + n];"),
     "bwd_ddt_without_sigmoid": ("ddt[i] = softplus_on ? ddel * sigmoid(v) : ddel;", "ddt[i] = ddel;"),
     "bwd_dD_ungated": ("dD[d] += dq * xv;", "dD[d] += widen(dy, dtype, i) * xv;"),
     "bwd_dh_last_ignored": ("g[n] = dh_last ? dh_last[(b * Dm + d) * N + n] : 0.0;", "g[n] = 0.0;"),
-    "bwd_ddelta_drops_input_term": ("ddel += g[n] * (a * abar * hp + bn * xv);", "ddel += g[n] * (a * abar * hp);"),
+    "bwd_ddelta_drops_input_term": ("ddel += g[n] * (a * abar * hp + w_dd * bn * xv);", "ddel += g[n] * (a * abar * hp);"),
+    "bwd_zoh_series_coefficient": ("double term = 0.5, sum = 0.0;", "double term = 1.0 / 3.0, sum = 0.0;"),
+    "bwd_zoh_closed_form_sign": ("f = (s * exp(s) - expm1(s)) / (s * s);", "f = (s * exp(s) + expm1(s)) / (s * s);"),
+    "bwd_zoh_dw_ddelta_one": ("*dw_ddelta = exp(s);", "*dw_ddelta = 1.0;"),
+    "bwd_zoh_dB_uses_delta": ("dB[bc + n] += g[n] * w * xv;", "dB[bc + n] += g[n] * delta[t] * xv;"),
+    "bwd_zoh_dx_uses_delta": ("dxv += g[n] * w * bn;", "dxv += g[n] * delta[t] * bn;"),
+    "bwd_conv_without_silu_derivative": ("dp = dxv * sp * (1.0 + p * (1.0 - sp));", "dp = dxv * sp;"),
+    "bwd_conv_taps_reversed": ("const double dtok = dp * (double)conv_w[d * ORACLE_CONV_K + k];",
+                               "const double dtok = dp * (double)conv_w[d * ORACLE_CONV_K + (ORACLE_CONV_K - 1 - k)];"),
+    "bwd_conv_x0_gradient_dropped": ("(tau + ORACLE_CONV_K - 1)) * Dm + d] += dtok;", "(tau + ORACLE_CONV_K - 1)) * Dm + d] += 0.0 * dtok;"),
+    "bwd_conv_bias_gradient_ungated": ("dconv_b[d] += dp;", "dconv_b[d] += dxv;"),
+    "bwd_conv_tap_gradient_shifted": ("dconv_w[d * ORACLE_CONV_K + k] += dp * raw_token(&cj, b, tau, d);",
+                                      "dconv_w[d * ORACLE_CONV_K + k] += dp * raw_token(&cj, b, tau + (t + 1 < L), d);"),
     "conv_step_ignores_window": ("y, h, h, 0, Bsz * Dm, conv_w, conv_b, conv_state};",
                                  "y, h, h, 0, Bsz * Dm, conv_w, conv_b, NULL};"),
 }
