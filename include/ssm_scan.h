@@ -292,11 +292,16 @@ ssm_status ssm_scan_fwd_host(const ssm_scan_args *args, int64_t chunk_len, void 
  *   dA          : [D, N] float32;  dD, ddt_bias : [D] float32, or NULL to skip
  *   dh0         : [B, D, N] float32 dL/dh0, or NULL to skip
  * dB, dC, dA, dD and ddt_bias are sums accumulated with float atomics: their last bits
- * can vary from run to run with the order of the additions. Only SSM_DELTA_SOFTPLUS
- * (and SSM_A_GENERAL, which changes nothing here) is honoured; SSM_EXACT_ZOH returns
- * SSM_ERR_UNSUPPORTED, and the short convolution has no backward here. The workspace
- * holds the checkpoints (68 bytes per channel and 32 steps: about one [B, L, D] bfloat16
- * tensor) and 8.3 KB per item: ssm_scan_bwd_workspace_size() bytes, 16-byte aligned.
+ * can vary from run to run with the order of the additions. SSM_DELTA_SOFTPLUS and
+ * SSM_EXACT_ZOH as in the forward call (SSM_A_GENERAL changes nothing here). With the
+ * short convolution (conv_w, conv_b, conv_x0 as in the forward) dx is the gradient of
+ * the raw tokens before it, and dconv_w, dconv_b, dconv_x0 those of its taps, bias and
+ * prefix tokens (dconv_w and dconv_b also accumulate with atomics): a first kernel writes
+ * the convolution's output u into the workspace, the passes run on it and write dL/du in
+ * float32 there, and a last kernel takes dL/du back through SiLU and the taps. The
+ * workspace holds the checkpoints (68 bytes per channel and 32 steps: about one [B, L, D]
+ * bfloat16 tensor), 8.3 KB per item and, with the convolution, u and dL/du:
+ * ssm_scan_bwd_workspace_size() bytes, 16-byte aligned.
  * Errors: as ssm_scan_fwd (x, dt, z, dy and workspace on 16 bytes).
  */
 typedef struct {
@@ -314,6 +319,13 @@ typedef struct {
     float *dh0;              /* [B, D, N] float32 output, or NULL                     */
     void *workspace;         /* ssm_scan_bwd_workspace_size() bytes                  */
     size_t workspace_bytes;
+    /* The short convolution of the forward call (conv_w NULL: none), and its gradients:
+       dconv_w [D, 4] and dconv_b [D] float32 (required with conv_w; dconv_b also when
+       conv_b is NULL), dconv_x0 [B, 3, D] dtype of x (exactly when conv_x0 is given). */
+    const float *conv_w, *conv_b;
+    const void *conv_x0;
+    float *dconv_w, *dconv_b;
+    void *dconv_x0;
 } ssm_scan_bwd_args;
 
 size_t ssm_scan_bwd_workspace_size(const ssm_scan_bwd_args *args);

@@ -246,12 +246,15 @@ def scan_fwd_host(x, dt, A, B, C, D=None, z=None, dt_bias=None, h0=None, *, chun
 
 
 def scan_bwd(x, dt, A, B, C, dy, D=None, z=None, dt_bias=None, h0=None, dh_last=None, *, delta_softplus=True,
-             workspace=None, stream=None):
+             exact_zoh=False, conv_w=None, conv_b=None, conv_x0=None, workspace=None, stream=None):
     """Backward of scan_fwd (see include/ssm_scan.h, ssm_scan_bwd): gradients given
     dy = dL/dy [B, L, D] (dtype of x) and optionally dh_last = dL/dh_L [B, D, N] float32.
+    exact_zoh and the short convolution (conv_w, conv_b, conv_x0) as in the forward call.
 
     Returns a dict: dx, ddt, dz (None without z) in x's dtype [B, L, D]; dB, dC float32
-    [B, L, N]; dA float32 [D, N]; dD, ddt_bias float32 [D]; dh0 float32 [B, D, N].
+    [B, L, N]; dA float32 [D, N]; dD, ddt_bias float32 [D]; dh0 float32 [B, D, N]; with
+    the convolution also dconv_w float32 [D, 4], dconv_b float32 [D] and dconv_x0 [B, 3, D]
+    in x's dtype (None without conv_x0), dx then being the gradient of the raw tokens.
     """
     dev = x.device
     if x.dtype not in _TOKEN_DTYPES:
@@ -271,6 +274,7 @@ def scan_bwd(x, dt, A, B, C, dy, D=None, z=None, dt_bias=None, h0=None, dh_last=
                            (dh_last, "dh_last", (Bsz, Dm, N))):
         if t is not None:
             _need(t, name, shape, torch.float32, dev)
+    _need_conv(conv_w, conv_b, conv_x0, Bsz, Dm, tok, dev)
     f32 = dict(dtype=torch.float32, device=dev)
     out = dict(dx=torch.empty_like(x), ddt=torch.empty_like(x), dz=None if z is None else torch.empty_like(x),
                dB=torch.empty((Bsz, L, N), **f32), dC=torch.empty((Bsz, L, N), **f32),
@@ -279,7 +283,12 @@ def scan_bwd(x, dt, A, B, C, dy, D=None, z=None, dt_bias=None, h0=None, dh_last=
     a = _native.ScanBwdArgs()
     a.batch, a.seqlen, a.dim, a.dstate = Bsz, L, Dm, N
     a.dtype = _TOKEN_DTYPES[tok]
-    a.flags = _flags(delta_softplus, False)
+    a.flags = _flags(delta_softplus, False, exact_zoh)
+    if conv_w is not None:
+        out.update(dconv_w=torch.empty((Dm, 4), **f32), dconv_b=torch.empty((Dm,), **f32),
+                   dconv_x0=None if conv_x0 is None else torch.empty((Bsz, 3, Dm), dtype=tok, device=dev))
+        a.conv_w, a.conv_b, a.conv_x0 = _ptr(conv_w), _ptr(conv_b), _ptr(conv_x0)
+        a.dconv_w, a.dconv_b, a.dconv_x0 = _ptr(out["dconv_w"]), _ptr(out["dconv_b"]), _ptr(out["dconv_x0"])
     a.x, a.dt, a.z, a.Bm, a.Cm = (_ptr(t) for t in (x, dt, z, B, C))
     a.A, a.Dskip, a.dt_bias, a.h0 = (_ptr(t) for t in (A, D, dt_bias, h0))
     a.dy, a.dh_last = _ptr(dy), _ptr(dh_last)

@@ -46,6 +46,8 @@ class ScanBwdArgs(ctypes.Structure):
         ("ddt", ctypes.c_void_p), ("dz", ctypes.c_void_p), ("dB", ctypes.c_void_p), ("dC", ctypes.c_void_p),
         ("dA", ctypes.c_void_p), ("dD", ctypes.c_void_p), ("ddt_bias", ctypes.c_void_p), ("dh0", ctypes.c_void_p),
         ("workspace", ctypes.c_void_p), ("workspace_bytes", ctypes.c_size_t),
+        ("conv_w", ctypes.c_void_p), ("conv_b", ctypes.c_void_p), ("conv_x0", ctypes.c_void_p),
+        ("dconv_w", ctypes.c_void_p), ("dconv_b", ctypes.c_void_p), ("dconv_x0", ctypes.c_void_p),
     ]
 
 

@@ -58,6 +58,7 @@ struct Params {
     float *cumd;   // [G][nchunks][CH] sum of Delta from the segment start to each chunk start
     float4 *hloc, *gloc, *hs, *ge;  // [G][K][CW][CH]: local end state and start adjoint; true start state, end adjoint
     float *sdel;                    // [G][K][CH] sum of Delta over the segment
+    float *du32;  // with the short convolution: dL/du [B, L, D] float32 instead of dx
     int softplus, bc_async;
 };
 
@@ -171,6 +172,55 @@ __device__ __forceinline__ float4 abar4(const float dl, const float4 A) {  // dl
     return make_float4(ex2_approx(dl * A.x), ex2_approx(dl * A.y), ex2_approx(dl * A.z), ex2_approx(dl * A.w));
 }
 
+// Exact zero-order hold, one state: the input weight w = (Abar - 1) / A (below |Delta A| =
+// 1/16 by its series Delta (1 + s/2 + s^2/6 + s^3/24 + s^4/120), s = Delta A; Delta for
+// A = 0), and dw/dA = Delta^2 f(s), f(s) = (s e^s - e^s + 1) / s^2, below |s| = 1/2 by its
+// Taylor series sum_k (k + 1) s^k / (k + 2)! (the closed form cancels near 0). dw/dDelta
+// is Abar itself.
+__device__ __forceinline__ float zoh_w1(const float delta, const float A, const float abar) {
+    const float s = delta * A;
+    if (fabsf(s) < 0.0625f)
+        return delta * fmaf(s, fmaf(s, fmaf(s, fmaf(s, 1.f / 120.f, 1.f / 24.f), 1.f / 6.f), 0.5f), 1.f);
+    return __fdividef(abar - 1.f, A);
+}
+__device__ __forceinline__ float zoh_dwdA1(const float delta, const float A, const float abar) {
+    const float s = delta * A;
+    float f;
+    if (fabsf(s) < 0.5f) {
+        f = fmaf(s, 1.f / 403200.f, 1.f / 45360.f);
+        f = fmaf(s, f, 1.f / 5760.f);
+        f = fmaf(s, f, 1.f / 840.f);
+        f = fmaf(s, f, 1.f / 144.f);
+        f = fmaf(s, f, 1.f / 30.f);
+        f = fmaf(s, f, 0.125f);
+        f = fmaf(s, f, 1.f / 3.f);
+        f = fmaf(s, f, 0.5f);
+    } else {
+        f = __fdividef(fmaf(s, abar, 1.f - abar), s * s);
+    }
+    return delta * delta * f;
+}
+__device__ __forceinline__ float4 zoh_w4(const float delta, const float4 A, const float4 a) {
+    return make_float4(zoh_w1(delta, A.x, a.x), zoh_w1(delta, A.y, a.y), zoh_w1(delta, A.z, a.z),
+                       zoh_w1(delta, A.w, a.w));
+}
+__device__ __forceinline__ float4 zoh_dwdA4(const float delta, const float4 A, const float4 a) {
+    return make_float4(zoh_dwdA1(delta, A.x, a.x), zoh_dwdA1(delta, A.y, a.y), zoh_dwdA1(delta, A.z, a.z),
+                       zoh_dwdA1(delta, A.w, a.w));
+}
+
+// One forward step of a lane's four states under either discretisation: the input
+// weight is Delta (ZOH false) or the exact hold's per-state weight.
+template <bool ZOH>
+__device__ __forceinline__ float4 step4(const float4 h, const float delta, const float4 A, const float xv,
+                                        const float4 bv) {
+    const float4 a = abar4(delta * kLog2e, A);
+    if (!ZOH) return fwd_step(h, a, delta * xv, bv);
+    const float4 w = zoh_w4(delta, A, a);
+    return make_float4(fmaf(a.x, h.x, w.x * xv * bv.x), fmaf(a.y, h.y, w.y * xv * bv.y),
+                       fmaf(a.z, h.z, w.z * xv * bv.z), fmaf(a.w, h.w, w.w * xv * bv.w));
+}
+
 // Sum over the warp's 32 lanes of eight values per lane (a reduce-scatter in 9
 // shuffles): on return, lanes with (lane & 3) == 0 hold the total of value
 // ((lane >> 4) & 1) * 4 + ((lane >> 3) & 1) * 2 + ((lane >> 2) & 1).
@@ -221,7 +271,7 @@ __device__ __forceinline__ float4 quad_of(const float *a, const int64_t row, con
 
 // A. Per item: the segment's end state from a zero start (hloc), its adjoint at the start
 // from a zero end (gloc), and sum_t Delta_t (sdel). Steps past L are skipped.
-template <typename T>
+template <typename T, bool ZOH>
 __global__ void __launch_bounds__(NT) scan_bwd_local_kernel(const Params p) {
     using S = Smem<T>;
     extern __shared__ __align__(16) unsigned char smem[];
@@ -261,8 +311,7 @@ __global__ void __launch_bounds__(NT) scan_bwd_local_kernel(const Params p) {
         const int tn = p.L - j * KC < KC ? int(p.L - j * KC) : KC;  // valid steps of the chunk
         for (int t = 0; t < tn; ++t) {
             const float delta = dc[t * CH + lane];
-            h = fwd_step(h, abar4(delta * kLog2e, Aq), delta * Tok<T>::to_f(sx[t * CH]),
-                         row4<T>(buf + S::o_b, t, 4 * warp));
+            h = step4<ZOH>(h, delta, Aq, Tok<T>::to_f(sx[t * CH]), row4<T>(buf + S::o_b, t, 4 * warp));
             sd += delta;
         }
         __syncthreads();
@@ -344,7 +393,7 @@ __global__ void __launch_bounds__(256) scan_bwd_combine_kernel(const Params p) {
 }
 
 // C. The gradients of one item, from its true start state and end adjoint.
-template <typename T>
+template <typename T, bool ZOH>
 __global__ void __launch_bounds__(NT) scan_bwd_kernel(const Params p) {
     using S = Smem<T>;
     extern __shared__ __align__(16) unsigned char smem[];
@@ -413,8 +462,7 @@ __global__ void __launch_bounds__(NT) scan_bwd_kernel(const Params p) {
 #pragma unroll 4
         for (int t = 0; t < TH; ++t) {
             const float delta = sdel[t * CH + lane];
-            hmid = fwd_step(hmid, abar4(delta * kLog2e, Aq), delta * Tok<T>::to_f(sx[t * CH + lane]),
-                            row4<T>(buf + S::o_b, t, 4 * warp));
+            hmid = step4<ZOH>(hmid, delta, Aq, Tok<T>::to_f(sx[t * CH + lane]), row4<T>(buf + S::o_b, t, 4 * warp));
         }
         __syncthreads();  // sdel is rewritten for the second half
         for (int half = 1; half >= 0; --half) {
@@ -433,8 +481,7 @@ __global__ void __launch_bounds__(NT) scan_bwd_kernel(const Params p) {
             for (int s = 0; s < TH; ++s) {
                 const int t = tb + s;
                 const float delta = sdel[s * CH + lane];
-                hh = fwd_step(hh, abar4(delta * kLog2e, Aq), delta * Tok<T>::to_f(sx[t * CH + lane]),
-                              row4<T>(buf + S::o_b, t, 4 * warp));
+                hh = step4<ZOH>(hh, delta, Aq, Tok<T>::to_f(sx[t * CH + lane]), row4<T>(buf + S::o_b, t, 4 * warp));
                 hb[(s * CW + warp) * CH + lane] = hh;
                 const float4 c4 = row4<T>(buf + S::o_c, t, 4 * warp);
                 pa[(warp * TH + s) * CH + lane] = fmaf(c4.x, hh.x, fmaf(c4.y, hh.y, fmaf(c4.z, hh.z, c4.w * hh.w)));
@@ -474,27 +521,39 @@ __global__ void __launch_bounds__(NT) scan_bwd_kernel(const Params p) {
                 gq.y = fmaf(dq, cv.y, gq.y);
                 gq.z = fmaf(dq, cv.z, gq.z);
                 gq.w = fmaf(dq, cv.w, gq.w);
-                const float dx_ = delta * xv;
-                // dA_n += g_n Delta Abar_n h_{t-1,n}
+                // dA_n += g_n Delta Abar_n h_{t-1,n} (+ g_n dw_n/dA_n B_n x, exact hold)
                 const float4 ah = make_float4(a.x * hp.x, a.y * hp.y, a.z * hp.z, a.w * hp.w);
                 dA.x = fmaf(gq.x * delta, ah.x, dA.x);
                 dA.y = fmaf(gq.y * delta, ah.y, dA.y);
                 dA.z = fmaf(gq.z * delta, ah.z, dA.z);
                 dA.w = fmaf(gq.w * delta, ah.w, dA.w);
-                // dDelta partial: sum_n g_n (A_n Abar_n h_{t-1,n} + B_n x)
-                float ddel = gq.x * fmaf(Aq.x, ah.x, bv.x * xv);
-                ddel = fmaf(gq.y, fmaf(Aq.y, ah.y, bv.y * xv), ddel);
-                ddel = fmaf(gq.z, fmaf(Aq.z, ah.z, bv.z * xv), ddel);
-                ddel = fmaf(gq.w, fmaf(Aq.w, ah.w, bv.w * xv), ddel);
-                // dx partial: sum_n g_n Delta B_n
-                float dxp = gq.x * bv.x;
-                dxp = fmaf(gq.y, bv.y, dxp);
-                dxp = fmaf(gq.z, bv.z, dxp);
-                dxp = fmaf(gq.w, bv.w, dxp);
+                // the input weight per state (Delta, or the exact hold's) and dw/dDelta
+                float4 w = make_float4(0.f, 0.f, 0.f, 0.f), wd = make_float4(1.f, 1.f, 1.f, 1.f);
+                if (ZOH) {
+                    w = zoh_w4(delta, Aq, a);
+                    wd = a;
+                    const float4 wa = zoh_dwdA4(delta, Aq, a);
+                    dA.x = fmaf(gq.x * wa.x, bv.x * xv, dA.x);
+                    dA.y = fmaf(gq.y * wa.y, bv.y * xv, dA.y);
+                    dA.z = fmaf(gq.z * wa.z, bv.z * xv, dA.z);
+                    dA.w = fmaf(gq.w * wa.w, bv.w * xv, dA.w);
+                }
+                // dDelta partial: sum_n g_n (A_n Abar_n h_{t-1,n} + dw_n/dDelta B_n x)
+                float ddel = gq.x * fmaf(Aq.x, ah.x, wd.x * bv.x * xv);
+                ddel = fmaf(gq.y, fmaf(Aq.y, ah.y, wd.y * bv.y * xv), ddel);
+                ddel = fmaf(gq.z, fmaf(Aq.z, ah.z, wd.z * bv.z * xv), ddel);
+                ddel = fmaf(gq.w, fmaf(Aq.w, ah.w, wd.w * bv.w * xv), ddel);
+                // dx partial: sum_n g_n w_n B_n; g w (Delta factored out of the sum when w = Delta)
+                const float4 gw = ZOH ? make_float4(gq.x * w.x, gq.y * w.y, gq.z * w.z, gq.w * w.w) : gq;
+                float dxp = gw.x * bv.x;
+                dxp = fmaf(gw.y, bv.y, dxp);
+                dxp = fmaf(gw.z, bv.z, dxp);
+                dxp = fmaf(gw.w, bv.w, dxp);
                 pa[(warp * TH + s) * CH + lane] = ddel;
-                pb[(warp * TH + s) * CH + lane] = dxp * delta;
-                // dB_tn = sum over channels of g_n Delta x; dC_tn = sum over channels of dq h_tn
-                const float v8[8] = {gq.x * dx_, gq.y * dx_, gq.z * dx_, gq.w * dx_,
+                pb[(warp * TH + s) * CH + lane] = ZOH ? dxp : dxp * delta;
+                // dB_tn = sum over channels of g_n w_n x; dC_tn = sum over channels of dq h_tn
+                const float xw = ZOH ? xv : delta * xv;
+                const float v8[8] = {gw.x * xw, gw.y * xw, gw.z * xw, gw.w * xw,
                                      dq * hc.x,  dq * hc.y,  dq * hc.z,  dq * hc.w};
                 const float tot = warp_sum8(v8, lane);
                 if ((lane & 3) == 0) {
@@ -520,7 +579,8 @@ __global__ void __launch_bounds__(NT) scan_bwd_kernel(const Params p) {
                 dbias += ddt;
                 if (dvalid) {
                     ddto[(b * p.L + tg) * p.D + d] = Tok<T>::from_f(ddt);
-                    dxo[(b * p.L + tg) * p.D + d] = Tok<T>::from_f(dxv);
+                    if (p.du32) p.du32[(b * p.L + tg) * p.D + d] = dxv;  // on through the convolution
+                    else dxo[(b * p.L + tg) * p.D + d] = Tok<T>::from_f(dxv);
                 }
             }
             __syncthreads();
@@ -537,6 +597,124 @@ __global__ void __launch_bounds__(NT) scan_bwd_kernel(const Params p) {
         }
         if (p.dD) atomicAdd(p.dD + d, dD);
         if (p.dbias) atomicAdd(p.dbias + d, dbias);
+    }
+}
+
+// ------------------------------------------------------------ short convolution
+// The block's causal convolution and SiLU in front of the SSM: u_t = silu(p_t), p_t =
+// cb + w0 x_{t-3} + w1 x_{t-2} + w2 x_{t-1} + w3 x_t per channel (Mamba summary,
+// block-architecture paragraph), tokens before t = 0 from conv_x0 ([B, 3, D], oldest
+// first) or zero. With it the backward runs on u: conv_u_kernel writes u (dtype of x)
+// into the workspace, the main passes read it where they read x and write dL/du in
+// float32, and conv_bwd_kernel takes dL/du back through SiLU and the taps.
+constexpr int CONV_TCH = 256;  // steps per thread in the convolution kernels
+
+template <typename T>
+__device__ __forceinline__ float raw_x(const T *x, const T *x0, const int64_t b, const int64_t t, const int64_t L,
+                                       const int64_t D, const int64_t d) {
+    if (t >= 0) return Tok<T>::to_f(x[(b * L + t) * D + d]);
+    return x0 ? Tok<T>::to_f(x0[(b * 3 + (t + 3)) * D + d]) : 0.f;
+}
+
+// One thread per (b, d, run of CONV_TCH steps): u_t for the run (the same fused
+// multiply-adds in the same order as the forward's front end).
+template <typename T>
+__global__ void __launch_bounds__(256) conv_u_kernel(int64_t Bsz, int64_t L, int64_t D, const T *__restrict__ x,
+                                                     const T *__restrict__ x0, const float *__restrict__ cw,
+                                                     const float *__restrict__ cb, T *__restrict__ u) {
+    const int64_t runs = (L + CONV_TCH - 1) / CONV_TCH;
+    const int64_t i = int64_t(blockIdx.x) * blockDim.x + threadIdx.x;
+    if (i >= Bsz * runs * D) return;
+    const int64_t d = i % D, r = (i / D) % runs, b = i / (D * runs);
+    const int64_t t0 = r * CONV_TCH, t1 = t0 + CONV_TCH < L ? t0 + CONV_TCH : L;
+    const float4 w = *reinterpret_cast<const float4 *>(cw + d * 4);
+    const float bias = cb ? cb[d] : 0.f;
+    float s0 = raw_x(x, x0, b, t0 - 3, L, D, d), s1 = raw_x(x, x0, b, t0 - 2, L, D, d),
+          s2 = raw_x(x, x0, b, t0 - 1, L, D, d);
+    for (int64_t t = t0; t < t1; ++t) {
+        const float xv = Tok<T>::to_f(x[(b * L + t) * D + d]);
+        float v = fmaf(w.x, s0, bias);
+        v = fmaf(w.y, s1, v);
+        v = fmaf(w.z, s2, v);
+        v = fmaf(w.w, xv, v);
+        u[(b * L + t) * D + d] = Tok<T>::from_f(silu_f(v));
+        s0 = s1;
+        s1 = s2;
+        s2 = xv;
+    }
+}
+
+// The convolution's backward, one thread per (b, d, run [t0, t1) of CONV_TCH steps), four
+// runs of 32 channels per block: dp_t = du_t silu'(p_t) for t in [t0, t1 + 3) (the last
+// three for the run's dx only), dx_tau = sum_k w_k dp_{tau+3-k} for tau in the run (tau < 0:
+// dconv_x0, written by the first run of each sequence), dconv_w[k] = sum_t dp_t x_{t-3+k}
+// and dconv_b = sum_t dp_t over the run, summed over the block's runs and added with one
+// atomic per channel and block.
+template <typename T>
+__global__ void __launch_bounds__(128) conv_bwd_kernel(int64_t Bsz, int64_t L, int64_t D, const T *__restrict__ x,
+                                                       const T *__restrict__ x0, const float *__restrict__ cw,
+                                                       const float *__restrict__ cb, const float *__restrict__ du,
+                                                       T *__restrict__ dx, T *__restrict__ dx0, float *__restrict__ dcw,
+                                                       float *__restrict__ dcb) {
+    __shared__ float red[4][5][32];
+    const int lane = threadIdx.x & 31, wr = threadIdx.x >> 5;
+    const int64_t runs = (L + CONV_TCH - 1) / CONV_TCH, rg = (runs + 3) / 4, Dg = (D + 31) / 32;
+    const int64_t blk = blockIdx.x;
+    const int64_t g = blk % Dg, rr = (blk / Dg) % rg, b = blk / (Dg * rg);
+    const int64_t d = g * 32 + lane, r = rr * 4 + wr;
+    float acc[5] = {0.f, 0.f, 0.f, 0.f, 0.f};  // dconv_w[0..3], dconv_b
+    if (d < D && r < runs && b < Bsz) {
+        const int64_t t0 = r * CONV_TCH, t1 = t0 + CONV_TCH < L ? t0 + CONV_TCH : L;
+        const int64_t tend = t1 + 3 < L ? t1 + 3 : L;
+        const float4 w = *reinterpret_cast<const float4 *>(cw + d * 4);
+        const float bias = cb ? cb[d] : 0.f;
+        float s0 = raw_x(x, x0, b, t0 - 3, L, D, d), s1 = raw_x(x, x0, b, t0 - 2, L, D, d),
+              s2 = raw_x(x, x0, b, t0 - 1, L, D, d);
+        float q0 = 0.f, q1 = 0.f, q2 = 0.f;  // partial dx of tau = t-3, t-2, t-1 before step t
+        auto emit = [&](const int64_t tau, const float v) {
+            if (tau >= t0 && tau < t1) dx[(b * L + tau) * D + d] = Tok<T>::from_f(v);
+            else if (tau < 0 && t0 == 0 && dx0) dx0[(b * 3 + (tau + 3)) * D + d] = Tok<T>::from_f(v);
+        };
+        for (int64_t t = t0; t < tend; ++t) {
+            const float xv = Tok<T>::to_f(x[(b * L + t) * D + d]);
+            float v = fmaf(w.x, s0, bias);
+            v = fmaf(w.y, s1, v);
+            v = fmaf(w.z, s2, v);
+            v = fmaf(w.w, xv, v);
+            const float sg = rcp_approx(1.0f + ex2_approx(-v * kLog2e));
+            const float dp = du[(b * L + t) * D + d] * sg * fmaf(v, 1.f - sg, 1.f);
+            if (t < t1) {
+                acc[0] = fmaf(dp, s0, acc[0]);
+                acc[1] = fmaf(dp, s1, acc[1]);
+                acc[2] = fmaf(dp, s2, acc[2]);
+                acc[3] = fmaf(dp, xv, acc[3]);
+                acc[4] += dp;
+            }
+            // tau = t-3 is complete after this step
+            emit(t - 3, fmaf(w.x, dp, q0));
+            q0 = fmaf(w.y, dp, q1);
+            q1 = fmaf(w.z, dp, q2);
+            q2 = w.w * dp;
+            s0 = s1;
+            s1 = s2;
+            s2 = xv;
+        }
+        if (tend == L) {  // the sequence ends: the last three are complete too
+            emit(L - 3, q0);
+            emit(L - 2, q1);
+            emit(L - 1, q2);
+        }
+    }
+#pragma unroll
+    for (int k = 0; k < 5; ++k) red[wr][k][lane] = acc[k];
+    __syncthreads();
+    if (wr == 0 && d < D && b < Bsz) {
+#pragma unroll
+        for (int k = 0; k < 5; ++k) {
+            const float v = red[0][k][lane] + red[1][k][lane] + red[2][k][lane] + red[3][k][lane];
+            if (k < 4) atomicAdd(dcw + d * 4 + k, v);
+            else atomicAdd(dcb + d, v);
+        }
     }
 }
 
@@ -569,7 +747,6 @@ ssm_status validate(const ssm_scan_bwd_args *a) {
     if (a->batch < 0 || a->seqlen < 0 || a->dim < 0 || a->dstate < 1) return SSM_ERR_INVALID;
     if (a->dtype != SSM_F32 && a->dtype != SSM_BF16) return SSM_ERR_INVALID;
     if (a->flags & ~uint32_t(SSM_DELTA_SOFTPLUS | SSM_A_GENERAL | SSM_EXACT_ZOH)) return SSM_ERR_INVALID;
-    if (a->flags & SSM_EXACT_ZOH) return SSM_ERR_UNSUPPORTED;
     if (a->dstate > kMaxN) return SSM_ERR_UNSUPPORTED;
     if (a->dim % (a->dtype == SSM_BF16 ? 8 : 4) != 0) return SSM_ERR_UNSUPPORTED;
     if (a->batch > INT32_MAX || a->seqlen > INT32_MAX || a->dim > INT32_MAX) return SSM_ERR_UNSUPPORTED;
@@ -589,9 +766,33 @@ ssm_status validate(const ssm_scan_bwd_args *a) {
     const void *p4[] = {a->A, a->Dskip, a->dt_bias, a->h0, a->dh_last, a->dB, a->dC, a->dA, a->dD, a->ddt_bias, a->dh0};
     for (const void *q : p4)
         if (q && !aligned(q, 4)) return SSM_ERR_UNSUPPORTED;
+    // the short convolution: taps required with bias or prefix; its gradients exactly with it
+    if (!a->conv_w && (a->conv_b || a->conv_x0 || a->dconv_w || a->dconv_b || a->dconv_x0)) return SSM_ERR_INVALID;
+    if (a->conv_w && (!a->dconv_w || !a->dconv_b)) return SSM_ERR_INVALID;
+    if ((a->conv_x0 == nullptr) != (a->dconv_x0 == nullptr)) return SSM_ERR_INVALID;
+    if (a->conv_w && !aligned(a->conv_w, 16)) return SSM_ERR_UNSUPPORTED;
+    const void *pc4[] = {a->conv_b, a->dconv_w, a->dconv_b};
+    for (const void *q : pc4)
+        if (q && !aligned(q, 4)) return SSM_ERR_UNSUPPORTED;
+    const void *pces[] = {a->conv_x0, a->dconv_x0};
+    for (const void *q : pces)
+        if (q && !aligned(q, es)) return SSM_ERR_UNSUPPORTED;
     if (work && a->seqlen > 0 && (!a->workspace || a->workspace_bytes < ssm_scan_bwd_workspace_size(a)))
         return SSM_ERR_INVALID;
     return SSM_OK;
+}
+
+// With the short convolution the workspace also holds u ([B, L, D], dtype of x) and dL/du
+// ([B, L, D] float32) after the items' area, each 256-byte aligned.
+size_t base_bytes(const ssm_scan_bwd_args *a) {
+    return off_items(a) + 4 * item_bytes(a) + size_t(groups(a)) * size_t(segments(a)) * CH * 4 +
+           size_t(groups(a)) * size_t(chunks(a)) * CH * 4;
+}
+size_t rup256(size_t v) { return (v + 255) / 256 * 256; }
+size_t tok_count(const ssm_scan_bwd_args *a) { return size_t(a->batch) * size_t(a->seqlen) * size_t(a->dim); }
+size_t off_u(const ssm_scan_bwd_args *a) { return rup256(base_bytes(a)); }
+size_t off_du(const ssm_scan_bwd_args *a) {
+    return rup256(off_u(a) + tok_count(a) * (a->dtype == SSM_BF16 ? 2 : 4));
 }
 
 }  // namespace bwd
@@ -603,8 +804,8 @@ extern "C" {
 
 size_t ssm_scan_bwd_workspace_size(const ssm_scan_bwd_args *a) {
     if (!a || a->batch < 0 || a->seqlen < 0 || a->dim < 0) return 0;
-    return off_items(a) + 4 * item_bytes(a) + size_t(groups(a)) * size_t(segments(a)) * CH * 4 +
-           size_t(groups(a)) * size_t(chunks(a)) * CH * 4;
+    if (!a->conv_w) return base_bytes(a);
+    return off_du(a) + tok_count(a) * 4;
 }
 
 ssm_status ssm_scan_bwd(const ssm_scan_bwd_args *a, void *stream_) {
@@ -617,6 +818,15 @@ ssm_status ssm_scan_bwd(const ssm_scan_bwd_args *a, void *stream_) {
     if (cudaMemsetAsync(a->dA, 0, nd * size_t(a->dstate) * 4, stream) != cudaSuccess) return SSM_ERR_CUDA;
     if (a->dD && cudaMemsetAsync(a->dD, 0, nd * 4, stream) != cudaSuccess) return SSM_ERR_CUDA;
     if (a->ddt_bias && cudaMemsetAsync(a->ddt_bias, 0, nd * 4, stream) != cudaSuccess) return SSM_ERR_CUDA;
+    const bool conv = a->conv_w != nullptr;
+    if (conv) {  // the convolution's gradients accumulate too (dconv_x0 is written whole)
+        if (cudaMemsetAsync(a->dconv_w, 0, nd * 16, stream) != cudaSuccess ||
+            cudaMemsetAsync(a->dconv_b, 0, nd * 4, stream) != cudaSuccess)
+            return SSM_ERR_CUDA;
+        if (a->dconv_x0 && cudaMemsetAsync(a->dconv_x0, 0, size_t(a->batch) * 3 * nd * (a->dtype == SSM_BF16 ? 2 : 4),
+                                           stream) != cudaSuccess)
+            return SSM_ERR_CUDA;
+    }
     if (a->seqlen == 0) {  // no tokens: dh0 = dh_last (or 0)
         if (!a->dh0) return SSM_OK;
         const cudaError_t e = a->dh_last ? cudaMemcpyAsync(a->dh0, a->dh_last, nbd * 4, cudaMemcpyDeviceToDevice, stream)
@@ -667,18 +877,41 @@ ssm_status ssm_scan_bwd(const ssm_scan_bwd_args *a, void *stream_) {
     p.cumd = p.sdel + size_t(p.G) * size_t(p.K) * CH;
     p.softplus = (a->flags & SSM_DELTA_SOFTPLUS) != 0;
     p.bc_async = (a->dstate * es) % 16 == 0 && aligned(a->Bm, 16) && aligned(a->Cm, 16);
+    p.du32 = nullptr;
     const int64_t items = p.G * p.K;
     if (items > INT32_MAX) return SSM_ERR_UNSUPPORTED;
+    const bool zoh = (a->flags & SSM_EXACT_ZOH) != 0;
     void *local, *kern;
     size_t smem;
     if (a->dtype == SSM_BF16) {
-        local = reinterpret_cast<void *>(&scan_bwd_local_kernel<__nv_bfloat16>);
-        kern = reinterpret_cast<void *>(&scan_bwd_kernel<__nv_bfloat16>);
+        local = zoh ? reinterpret_cast<void *>(&scan_bwd_local_kernel<__nv_bfloat16, true>)
+                    : reinterpret_cast<void *>(&scan_bwd_local_kernel<__nv_bfloat16, false>);
+        kern = zoh ? reinterpret_cast<void *>(&scan_bwd_kernel<__nv_bfloat16, true>)
+                   : reinterpret_cast<void *>(&scan_bwd_kernel<__nv_bfloat16, false>);
         smem = Smem<__nv_bfloat16>::total;
     } else {
-        local = reinterpret_cast<void *>(&scan_bwd_local_kernel<float>);
-        kern = reinterpret_cast<void *>(&scan_bwd_kernel<float>);
+        local = zoh ? reinterpret_cast<void *>(&scan_bwd_local_kernel<float, true>)
+                    : reinterpret_cast<void *>(&scan_bwd_local_kernel<float, false>);
+        kern = zoh ? reinterpret_cast<void *>(&scan_bwd_kernel<float, true>)
+                   : reinterpret_cast<void *>(&scan_bwd_kernel<float, false>);
         smem = Smem<float>::total;
+    }
+    // The short convolution: u into the workspace first; the passes read it as x.
+    const int64_t runs = (a->seqlen + CONV_TCH - 1) / CONV_TCH;
+    if (conv) {
+        void *u = ws + off_u(a);
+        p.x = u;
+        p.du32 = reinterpret_cast<float *>(ws + off_du(a));
+        const int64_t n = a->batch * runs * a->dim;
+        if (a->dtype == SSM_BF16)
+            conv_u_kernel<__nv_bfloat16><<<unsigned((n + 255) / 256), 256, 0, stream>>>(
+                a->batch, a->seqlen, a->dim, static_cast<const __nv_bfloat16 *>(a->x),
+                static_cast<const __nv_bfloat16 *>(a->conv_x0), a->conv_w, a->conv_b, static_cast<__nv_bfloat16 *>(u));
+        else
+            conv_u_kernel<float><<<unsigned((n + 255) / 256), 256, 0, stream>>>(
+                a->batch, a->seqlen, a->dim, static_cast<const float *>(a->x), static_cast<const float *>(a->conv_x0),
+                a->conv_w, a->conv_b, static_cast<float *>(u));
+        if (cudaGetLastError() != cudaSuccess) return SSM_ERR_CUDA;
     }
     if (cudaFuncSetAttribute(local, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem)) != cudaSuccess ||
         cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem)) != cudaSuccess)
@@ -690,8 +923,24 @@ ssm_status ssm_scan_bwd(const ssm_scan_bwd_args *a, void *stream_) {
     if (cudaLaunchKernel(reinterpret_cast<void *>(&scan_bwd_combine_kernel), dim3(unsigned((threads + 255) / 256)),
                          dim3(256), args, 0, stream) != cudaSuccess)
         return SSM_ERR_CUDA;
-    const cudaError_t e = cudaLaunchKernel(kern, dim3(unsigned(items)), dim3(NT), args, smem, stream);
-    return e == cudaSuccess ? SSM_OK : SSM_ERR_CUDA;
+    if (cudaLaunchKernel(kern, dim3(unsigned(items)), dim3(NT), args, smem, stream) != cudaSuccess)
+        return SSM_ERR_CUDA;
+    if (conv) {  // dL/du back through SiLU and the taps
+        const int64_t blocks = a->batch * ((runs + 3) / 4) * ((a->dim + 31) / 32);
+        if (blocks > INT32_MAX) return SSM_ERR_UNSUPPORTED;
+        if (a->dtype == SSM_BF16)
+            conv_bwd_kernel<__nv_bfloat16><<<unsigned(blocks), 128, 0, stream>>>(
+                a->batch, a->seqlen, a->dim, static_cast<const __nv_bfloat16 *>(a->x),
+                static_cast<const __nv_bfloat16 *>(a->conv_x0), a->conv_w, a->conv_b, p.du32,
+                static_cast<__nv_bfloat16 *>(a->dx), static_cast<__nv_bfloat16 *>(a->dconv_x0), a->dconv_w, a->dconv_b);
+        else
+            conv_bwd_kernel<float><<<unsigned(blocks), 128, 0, stream>>>(
+                a->batch, a->seqlen, a->dim, static_cast<const float *>(a->x), static_cast<const float *>(a->conv_x0),
+                a->conv_w, a->conv_b, p.du32, static_cast<float *>(a->dx), static_cast<float *>(a->dconv_x0), a->dconv_w,
+                a->dconv_b);
+        if (cudaGetLastError() != cudaSuccess) return SSM_ERR_CUDA;
+    }
+    return SSM_OK;
 }
 
 }  // extern "C"

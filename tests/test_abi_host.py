@@ -240,14 +240,29 @@ def test_bwd_workspace_size(lib):
     G, nch, K = 160, 8192, 12
     assert lib.ssm_scan_bwd_workspace_size(ctypes.byref(a)) == \
         G * nch * 2048 + 4 * G * K * 2048 + G * K * 128 + G * nch * 128
+    # with the short convolution: u (bf16) and dL/du (float32) after it, each on 256 bytes
+    base = G * nch * 2048 + 4 * G * K * 2048 + G * K * 128 + G * nch * 128
+    a.conv_w = 1 << 32
+    r256 = lambda v: (v + 255) // 256 * 256
+    n_tok = 262144 * 5120
+    assert lib.ssm_scan_bwd_workspace_size(ctypes.byref(a)) == r256(r256(base) + 2 * n_tok) + 4 * n_tok
+    a.conv_w = None
     a.seqlen = -1
     assert lib.ssm_scan_bwd_workspace_size(ctypes.byref(a)) == 0
     assert lib.ssm_scan_bwd_workspace_size(None) == 0
 
 
 @pytest.mark.parametrize("bad,code", [
-    (dict(flags=_native.SSM_DELTA_SOFTPLUS | _native.SSM_EXACT_ZOH), _native.SSM_ERR_UNSUPPORTED),
     (dict(flags=0x40), _native.SSM_ERR_INVALID),
+    (dict(conv_b=4294967296), _native.SSM_ERR_INVALID),                            # convolution bias without taps
+    (dict(dconv_w=4294967296), _native.SSM_ERR_INVALID),                           # its gradient without taps
+    (dict(conv_w=4294967296, dconv_b=4294967552), _native.SSM_ERR_INVALID),          # taps without dconv_w
+    (dict(conv_w=4294967296, dconv_w=4294967552), _native.SSM_ERR_INVALID),          # taps without dconv_b
+    (dict(conv_w=4294967296, dconv_w=4294967552, dconv_b=4294967808, conv_x0=4294968064),
+     _native.SSM_ERR_INVALID),                                              # prefix without its gradient
+    (dict(conv_w=4294967300, dconv_w=4294967552, dconv_b=4294967808), _native.SSM_ERR_UNSUPPORTED),  # taps: float4
+    (dict(conv_w=4294967296, dconv_w=4294967552, dconv_b=4294967808, conv_x0=4294968065, dconv_x0=4294968320),
+     _native.SSM_ERR_UNSUPPORTED),                                          # bf16 prefix on 2 bytes
     (dict(flags=_native.SSM_SEQ_PARALLEL | _native.SSM_SEQ_HANDOFF), _native.SSM_ERR_INVALID),
     (dict(dstate=17), _native.SSM_ERR_UNSUPPORTED),
     (dict(dim=12), _native.SSM_ERR_UNSUPPORTED),
