@@ -26,9 +26,11 @@
 //        dA += g Delta_t Abar_t h_{t-1};  dB_t += g Delta_t x_t;  dC_t += dq_t h_t;  g *= Abar_t
 //      with dq_t = dy_t silu(z_t) (or dy_t) from the recomputed readout.
 // Token tiles move into shared memory with cp.async (double-buffered by chunk). dB and
-// dC (shared by the channels of a sequence) are reduced over the 32 lanes with a
-// shuffle reduce-scatter and added to global memory with one atomic per (t, n) and
-// group; dA, dD and dt_bias's gradient are kept in registers and added once per block.
+// dC (shared by the channels of a sequence) are summed over the block's 32 channels in
+// shared memory, from the half's stored states (dC, before the reverse walk) and from
+// the g w x terms the reverse walk leaves in those slots (dB, after it), and added to
+// global memory with one atomic per (t, n) and group; dA, dD and dt_bias's gradient are
+// kept in registers and added once per block.
 // The atomics make dB, dC, dA, dD and dt_bias's gradient independent of any schedule
 // only up to the order of float additions.
 #include <cuda_runtime.h>
@@ -163,13 +165,38 @@ __device__ __forceinline__ void delta_pass(const T *sdt, const int r0, const int
     for (int i = warp; i < rows; i += CW) out[i * CH + lane] = delta_of(Tok<T>::to_f(sdt[(r0 + i) * CH + lane]) + bias, softplus);
 }
 
+// A lane's four states as two pairs: the arithmetic on them uses the packed float32
+// pair instructions (fma.rn.f32x2 and mul.rn.f32x2: one issue slot per pair, each
+// result rounded as the scalar instruction would round it).
+__device__ __forceinline__ float2 lo2(const float4 v) { return make_float2(v.x, v.y); }
+__device__ __forceinline__ float2 hi2(const float4 v) { return make_float2(v.z, v.w); }
+__device__ __forceinline__ float4 cat4(const float2 l, const float2 h) { return make_float4(l.x, l.y, h.x, h.y); }
+__device__ __forceinline__ float2 bc2(const float v) { return make_float2(v, v); }
+__device__ __forceinline__ float4 mul4(const float4 a, const float4 b) {
+    return cat4(__fmul2_rn(lo2(a), lo2(b)), __fmul2_rn(hi2(a), hi2(b)));
+}
+__device__ __forceinline__ float4 mul4s(const float4 a, const float s) {
+    return cat4(__fmul2_rn(lo2(a), bc2(s)), __fmul2_rn(hi2(a), bc2(s)));
+}
+__device__ __forceinline__ float4 fma4(const float4 a, const float4 b, const float4 c) {  // a b + c
+    return cat4(__ffma2_rn(lo2(a), lo2(b), lo2(c)), __ffma2_rn(hi2(a), hi2(b), hi2(c)));
+}
+__device__ __forceinline__ float4 fma4s(const float s, const float4 b, const float4 c) {  // s b + c
+    return cat4(__ffma2_rn(bc2(s), lo2(b), lo2(c)), __ffma2_rn(bc2(s), hi2(b), hi2(c)));
+}
+// a . b as a chain of fused multiply-adds (as many issue slots as a packed product and a
+// sum, with one rounding per term instead of two)
+__device__ __forceinline__ float dot4(const float4 a, const float4 b) {
+    return fmaf(a.w, b.w, fmaf(a.z, b.z, fmaf(a.y, b.y, a.x * b.x)));
+}
+
 // One forward step of a lane's four states.
 __device__ __forceinline__ float4 fwd_step(const float4 h, const float4 a, const float u, const float4 bv) {
-    return make_float4(fmaf(a.x, h.x, u * bv.x), fmaf(a.y, h.y, u * bv.y), fmaf(a.z, h.z, u * bv.z),
-                       fmaf(a.w, h.w, u * bv.w));
+    return fma4(a, h, mul4s(bv, u));
 }
 __device__ __forceinline__ float4 abar4(const float dl, const float4 A) {  // dl = Delta log2 e
-    return make_float4(ex2_approx(dl * A.x), ex2_approx(dl * A.y), ex2_approx(dl * A.z), ex2_approx(dl * A.w));
+    const float4 e = mul4s(A, dl);
+    return make_float4(ex2_approx(e.x), ex2_approx(e.y), ex2_approx(e.z), ex2_approx(e.w));
 }
 
 // Exact zero-order hold, one state: the input weight w = (Abar - 1) / A (below |Delta A| =
@@ -216,31 +243,38 @@ __device__ __forceinline__ float4 step4(const float4 h, const float delta, const
                                         const float4 bv) {
     const float4 a = abar4(delta * kLog2e, A);
     if (!ZOH) return fwd_step(h, a, delta * xv, bv);
-    const float4 w = zoh_w4(delta, A, a);
-    return make_float4(fmaf(a.x, h.x, w.x * xv * bv.x), fmaf(a.y, h.y, w.y * xv * bv.y),
-                       fmaf(a.z, h.z, w.z * xv * bv.z), fmaf(a.w, h.w, w.w * xv * bv.w));
+    return fma4(a, h, mul4(mul4s(zoh_w4(delta, A, a), xv), bv));
 }
 
-// Sum over the warp's 32 lanes of eight values per lane (a reduce-scatter in 9
-// shuffles): on return, lanes with (lane & 3) == 0 hold the total of value
-// ((lane >> 4) & 1) * 4 + ((lane >> 3) & 1) * 2 + ((lane >> 2) & 1).
-__device__ __forceinline__ float warp_sum8(const float (&v)[8], const int lane) {
-    float u[4], w2[2];
-    const bool h16 = lane & 16, h8 = lane & 8, h4 = lane & 4;
-#pragma unroll
-    for (int k = 0; k < 4; ++k) {
-        const float send = h16 ? v[k] : v[k + 4], keep = h16 ? v[k + 4] : v[k];
-        u[k] = keep + __shfl_xor_sync(0xffffffffu, send, 16);
+// dB or dC of a half chunk: for each of its TH steps s and states n, the sum over the 32
+// channels of v[s][warp][channel].n (times w[s][channel] when w is given), taken from
+// shared memory with the channels across a thread's loop rather than across lanes (no
+// shuffle reduction in the reverse step). Thread tid takes step s = tid / 8, the four
+// states of warp slot q = (tid / 2) % 4 and half the channels (tid % 2); the channel
+// order is rotated per thread pair so that a warp's 16-byte loads touch 32 different
+// channels (four wavefronts, the minimum). Pairs combine by one shuffle round; the first
+// of each pair adds the four sums to out[(b L + t) N + n] for steps t < L.
+__device__ __forceinline__ void reduce_channels(const float4 *v, const float *w, float *out, const int64_t row0,
+                                                const int64_t tvalid, const int64_t N) {
+    const int tid = threadIdx.x;
+    const int s = tid >> 3, q = (tid >> 1) & 3, hf = tid & 1, rot = tid >> 1;
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll 4
+    for (int j = 0; j < 16; ++j) {
+        const int c = hf * 16 + ((j + rot) & 15);
+        const float4 x = v[(s * CW + q) * CH + c];
+        acc = w ? fma4s(w[s * CH + c], x, acc) : cat4(__fadd2_rn(lo2(acc), lo2(x)), __fadd2_rn(hi2(acc), hi2(x)));
     }
+    acc.x += __shfl_xor_sync(0xffffffffu, acc.x, 1);
+    acc.y += __shfl_xor_sync(0xffffffffu, acc.y, 1);
+    acc.z += __shfl_xor_sync(0xffffffffu, acc.z, 1);
+    acc.w += __shfl_xor_sync(0xffffffffu, acc.w, 1);
+    if (hf == 0 && s < tvalid) {
+        const float av[4] = {acc.x, acc.y, acc.z, acc.w};
 #pragma unroll
-    for (int k = 0; k < 2; ++k) {
-        const float send = h8 ? u[k] : u[k + 2], keep = h8 ? u[k + 2] : u[k];
-        w2[k] = keep + __shfl_xor_sync(0xffffffffu, send, 8);
+        for (int k = 0; k < 4; ++k)
+            if (4 * q + k < N) atomicAdd(out + (row0 + s) * N + 4 * q + k, av[k]);
     }
-    float r = (h4 ? w2[1] : w2[0]) + __shfl_xor_sync(0xffffffffu, h4 ? w2[0] : w2[1], 4);
-    r += __shfl_xor_sync(0xffffffffu, r, 2);
-    r += __shfl_xor_sync(0xffffffffu, r, 1);
-    return r;
 }
 
 // The (group, segment) item of this block and its range of chunks [cb, ce).
@@ -347,8 +381,7 @@ __global__ void __launch_bounds__(NT) scan_bwd_local_kernel(const Params p) {
         for (int t = tn - 1; t >= 0; --t) {
             const float delta = dc[t * CH + lane], dq = dqc[t * CH + lane];
             const float4 cv = row4<T>(buf + S::o_c, t, 4 * warp), a = abar4(delta * kLog2e, Aq);
-            gl = make_float4(a.x * fmaf(dq, cv.x, gl.x), a.y * fmaf(dq, cv.y, gl.y), a.z * fmaf(dq, cv.z, gl.z),
-                             a.w * fmaf(dq, cv.w, gl.w));
+            gl = mul4(a, fma4s(dq, cv, gl));
         }
         __syncthreads();
     }
@@ -484,7 +517,7 @@ __global__ void __launch_bounds__(NT) scan_bwd_kernel(const Params p) {
                 hh = step4<ZOH>(hh, delta, Aq, Tok<T>::to_f(sx[t * CH + lane]), row4<T>(buf + S::o_b, t, 4 * warp));
                 hb[(s * CW + warp) * CH + lane] = hh;
                 const float4 c4 = row4<T>(buf + S::o_c, t, 4 * warp);
-                pa[(warp * TH + s) * CH + lane] = fmaf(c4.x, hh.x, fmaf(c4.y, hh.y, fmaf(c4.z, hh.z, c4.w * hh.w)));
+                pa[(warp * TH + s) * CH + lane] = dot4(c4, hh);
             }
             __syncthreads();
             // (b) per (t, channel): readout, gate, dq, dz
@@ -506,6 +539,10 @@ __global__ void __launch_bounds__(NT) scan_bwd_kernel(const Params p) {
                 sdq[s * CH + lane] = dq;
             }
             __syncthreads();
+            // (b2) dC_tn = sum over channels of dq_t h_tn, from the half's stored states
+            const int64_t tvalid = p.L - (t0 + tb);  // steps of the half before L
+            reduce_channels(hb, sdq, p.dC, b * p.L + t0 + tb, tvalid, p.N);
+            __syncthreads();  // the reverse step reuses the states' slots
             // (c) the adjoint, backwards over the half (steps past L are skipped)
             for (int s = TH - 1; s >= 0; --s) {
                 const int t = tb + s;
@@ -514,56 +551,38 @@ __global__ void __launch_bounds__(NT) scan_bwd_kernel(const Params p) {
                 const float delta = sdel[s * CH + lane], dq = sdq[s * CH + lane];
                 const float xv = Tok<T>::to_f(sx[t * CH + lane]);
                 const float4 bv = row4<T>(buf + S::o_b, t, 4 * warp), cv = row4<T>(buf + S::o_c, t, 4 * warp);
-                const float4 hc = hb[(s * CW + warp) * CH + lane];
                 const float4 hp = s > 0 ? hb[((s - 1) * CW + warp) * CH + lane] : hs;
                 const float4 a = abar4(delta * kLog2e, Aq);
-                gq.x = fmaf(dq, cv.x, gq.x);
-                gq.y = fmaf(dq, cv.y, gq.y);
-                gq.z = fmaf(dq, cv.z, gq.z);
-                gq.w = fmaf(dq, cv.w, gq.w);
+                gq = fma4s(dq, cv, gq);
                 // dA_n += g_n Delta Abar_n h_{t-1,n} (+ g_n dw_n/dA_n B_n x, exact hold)
-                const float4 ah = make_float4(a.x * hp.x, a.y * hp.y, a.z * hp.z, a.w * hp.w);
-                dA.x = fmaf(gq.x * delta, ah.x, dA.x);
-                dA.y = fmaf(gq.y * delta, ah.y, dA.y);
-                dA.z = fmaf(gq.z * delta, ah.z, dA.z);
-                dA.w = fmaf(gq.w * delta, ah.w, dA.w);
+                const float4 ah = mul4(a, hp);
+                dA = fma4(mul4s(gq, delta), ah, dA);
+                const float4 bx = mul4s(bv, xv);
                 // the input weight per state (Delta, or the exact hold's) and dw/dDelta
-                float4 w = make_float4(0.f, 0.f, 0.f, 0.f), wd = make_float4(1.f, 1.f, 1.f, 1.f);
+                float4 w = make_float4(0.f, 0.f, 0.f, 0.f);
+                float4 ddq;  // dDelta terms: A_n Abar_n h_{t-1,n} + dw_n/dDelta B_n x
                 if (ZOH) {
                     w = zoh_w4(delta, Aq, a);
-                    wd = a;
-                    const float4 wa = zoh_dwdA4(delta, Aq, a);
-                    dA.x = fmaf(gq.x * wa.x, bv.x * xv, dA.x);
-                    dA.y = fmaf(gq.y * wa.y, bv.y * xv, dA.y);
-                    dA.z = fmaf(gq.z * wa.z, bv.z * xv, dA.z);
-                    dA.w = fmaf(gq.w * wa.w, bv.w * xv, dA.w);
+                    dA = fma4(mul4(gq, zoh_dwdA4(delta, Aq, a)), bx, dA);
+                    ddq = fma4(Aq, ah, mul4(a, bx));
+                } else {
+                    ddq = fma4(Aq, ah, bx);
                 }
-                // dDelta partial: sum_n g_n (A_n Abar_n h_{t-1,n} + dw_n/dDelta B_n x)
-                float ddel = gq.x * fmaf(Aq.x, ah.x, wd.x * bv.x * xv);
-                ddel = fmaf(gq.y, fmaf(Aq.y, ah.y, wd.y * bv.y * xv), ddel);
-                ddel = fmaf(gq.z, fmaf(Aq.z, ah.z, wd.z * bv.z * xv), ddel);
-                ddel = fmaf(gq.w, fmaf(Aq.w, ah.w, wd.w * bv.w * xv), ddel);
+                const float ddel = dot4(gq, ddq);
                 // dx partial: sum_n g_n w_n B_n; g w (Delta factored out of the sum when w = Delta)
-                const float4 gw = ZOH ? make_float4(gq.x * w.x, gq.y * w.y, gq.z * w.z, gq.w * w.w) : gq;
-                float dxp = gw.x * bv.x;
-                dxp = fmaf(gw.y, bv.y, dxp);
-                dxp = fmaf(gw.z, bv.z, dxp);
-                dxp = fmaf(gw.w, bv.w, dxp);
+                const float4 gw = ZOH ? mul4(gq, w) : gq;
+                const float dxp = dot4(gw, bv);
                 pa[(warp * TH + s) * CH + lane] = ddel;
                 pb[(warp * TH + s) * CH + lane] = ZOH ? dxp : dxp * delta;
                 // dB_tn = sum over channels of g_n w_n x; dC_tn = sum over channels of dq h_tn
-                const float xw = ZOH ? xv : delta * xv;
-                const float v8[8] = {gw.x * xw, gw.y * xw, gw.z * xw, gw.w * xw,
-                                     dq * hc.x,  dq * hc.y,  dq * hc.z,  dq * hc.w};
-                const float tot = warp_sum8(v8, lane);
-                if ((lane & 3) == 0) {
-                    const int idx = ((lane >> 4) & 1) * 4 + ((lane >> 3) & 1) * 2 + ((lane >> 2) & 1);
-                    const int n = 4 * warp + (idx & 3);
-                    if (n < p.N) atomicAdd((idx < 4 ? p.dB : p.dC) + (b * p.L + tg) * p.N + n, tot);
-                }
-                gq = make_float4(gq.x * a.x, gq.y * a.y, gq.z * a.z, gq.w * a.w);
+                // this step's dB terms g_n w_n x go into its state slot, read for the last time
+                // above (the step before reads its own slot and the one before that)
+                hb[(s * CW + warp) * CH + lane] = mul4s(gw, ZOH ? xv : delta * xv);
+                gq = mul4(gq, a);
             }
             __syncthreads();
+            // (c2) dB_tn = sum over channels of g_n w_n x
+            reduce_channels(hb, nullptr, p.dB, b * p.L + t0 + tb, tvalid, p.N);
             // (d) per (t, channel): dDelta -> ddt, dx
 #pragma unroll
             for (int i = 0; i < TH / CW; ++i) {
