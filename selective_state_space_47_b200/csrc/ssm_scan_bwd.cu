@@ -83,6 +83,8 @@ struct Smem {
     static constexpr size_t off_del = off_dq + size_t(TH) * CH * 4;
     static constexpr size_t off_sig = off_del + size_t(TH) * CH * 4;
     static constexpr size_t total = off_sig + size_t(TH) * CH * 4;
+    // the local pass needs only the chunk buffers and a chunk's Delta and dq
+    static constexpr size_t local_total = off_h + size_t(2) * KC * CH * 4;
     static_assert(buf % 16 == 0 && off_h % 16 == 0, "16-byte copies and float4 rows");
 };
 
@@ -901,19 +903,21 @@ ssm_status ssm_scan_bwd(const ssm_scan_bwd_args *a, void *stream_) {
     if (items > INT32_MAX) return SSM_ERR_UNSUPPORTED;
     const bool zoh = (a->flags & SSM_EXACT_ZOH) != 0;
     void *local, *kern;
-    size_t smem;
+    size_t smem, smem_local;
     if (a->dtype == SSM_BF16) {
         local = zoh ? reinterpret_cast<void *>(&scan_bwd_local_kernel<__nv_bfloat16, true>)
                     : reinterpret_cast<void *>(&scan_bwd_local_kernel<__nv_bfloat16, false>);
         kern = zoh ? reinterpret_cast<void *>(&scan_bwd_kernel<__nv_bfloat16, true>)
                    : reinterpret_cast<void *>(&scan_bwd_kernel<__nv_bfloat16, false>);
         smem = Smem<__nv_bfloat16>::total;
+        smem_local = Smem<__nv_bfloat16>::local_total;
     } else {
         local = zoh ? reinterpret_cast<void *>(&scan_bwd_local_kernel<float, true>)
                     : reinterpret_cast<void *>(&scan_bwd_local_kernel<float, false>);
         kern = zoh ? reinterpret_cast<void *>(&scan_bwd_kernel<float, true>)
                    : reinterpret_cast<void *>(&scan_bwd_kernel<float, false>);
         smem = Smem<float>::total;
+        smem_local = Smem<float>::local_total;
     }
     // The short convolution: u into the workspace first; the passes read it as x.
     const int64_t runs = (a->seqlen + CONV_TCH - 1) / CONV_TCH;
@@ -932,11 +936,11 @@ ssm_status ssm_scan_bwd(const ssm_scan_bwd_args *a, void *stream_) {
                 a->conv_w, a->conv_b, static_cast<float *>(u));
         if (cudaGetLastError() != cudaSuccess) return SSM_ERR_CUDA;
     }
-    if (cudaFuncSetAttribute(local, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem)) != cudaSuccess ||
+    if (cudaFuncSetAttribute(local, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem_local)) != cudaSuccess ||
         cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem)) != cudaSuccess)
         return SSM_ERR_CUDA;
     void *args[] = {&p};
-    if (cudaLaunchKernel(local, dim3(unsigned(items)), dim3(NT), args, smem, stream) != cudaSuccess)
+    if (cudaLaunchKernel(local, dim3(unsigned(items)), dim3(NT), args, smem_local, stream) != cudaSuccess)
         return SSM_ERR_CUDA;
     const int64_t threads = p.G * CW * CH;
     if (cudaLaunchKernel(reinterpret_cast<void *>(&scan_bwd_combine_kernel), dim3(unsigned((threads + 255) / 256)),
