@@ -306,7 +306,11 @@ __device__ __forceinline__ float4 quad_of(const float *a, const int64_t row, con
 }
 
 // A. Per item: the segment's end state from a zero start (hloc), its adjoint at the start
-// from a zero end (gloc), and sum_t Delta_t (sdel). Steps past L are skipped.
+// from a zero end (gloc), and sum_t Delta_t (sdel), in one forward walk. The adjoint
+// recurrence g <- Abar_t (g + dq_t C_t), run backwards from g = 0, gives at the start
+// g = sum_t P_t dq_t C_t with P_t = Abar_start ... Abar_t, and dq_t = dy_t silu(z_t) needs
+// no state: so the walk carries P with h and adds P dq C as it goes. Steps past L are
+// skipped.
 template <typename T, bool ZOH>
 __global__ void __launch_bounds__(NT) scan_bwd_local_kernel(const Params p) {
     using S = Smem<T>;
@@ -326,13 +330,14 @@ __global__ void __launch_bounds__(NT) scan_bwd_local_kernel(const Params p) {
 
     float4 *ck = p.ckpt + (it.g * p.nchunks) * (CW * CH) + warp * CH + lane;
     float4 h = make_float4(0.f, 0.f, 0.f, 0.f);
+    float4 P = make_float4(1.f, 1.f, 1.f, 1.f), gl = make_float4(0.f, 0.f, 0.f, 0.f);
     float sd = 0.f;
-    load_chunk<T>(smem + (it.cb & 1) * S::buf, p, b, d0, it.cb * KC, false);
+    load_chunk<T>(smem + (it.cb & 1) * S::buf, p, b, d0, it.cb * KC, true);
     cp_async_commit();
     for (int64_t j = it.cb; j < it.ce; ++j) {
         const unsigned char *buf = smem + (j & 1) * S::buf;
         if (j + 1 < it.ce) {
-            load_chunk<T>(smem + ((j + 1) & 1) * S::buf, p, b, d0, (j + 1) * KC, false);
+            load_chunk<T>(smem + ((j + 1) & 1) * S::buf, p, b, d0, (j + 1) * KC, true);
             cp_async_commit();
             cp_async_wait<1>();
         } else {
@@ -342,32 +347,6 @@ __global__ void __launch_bounds__(NT) scan_bwd_local_kernel(const Params p) {
         ck[j * CW * CH] = h;  // the zero-start state and the sum of Delta at the chunk's start
         if (warp == 0) p.cumd[(it.g * p.nchunks + j) * CH + lane] = sd;
         const T *sx = reinterpret_cast<const T *>(buf + S::o_x) + lane;
-        delta_pass<T>(reinterpret_cast<const T *>(buf + S::o_dt), 0, KC, bias, softplus, dc, warp, lane);
-        __syncthreads();
-        const int tn = p.L - j * KC < KC ? int(p.L - j * KC) : KC;  // valid steps of the chunk
-        for (int t = 0; t < tn; ++t) {
-            const float delta = dc[t * CH + lane];
-            h = step4<ZOH>(h, delta, Aq, Tok<T>::to_f(sx[t * CH]), row4<T>(buf + S::o_b, t, 4 * warp));
-            sd += delta;
-        }
-        __syncthreads();
-    }
-    p.hloc[slot] = h;
-    if (warp == 0) p.sdel[(it.g * p.K + it.k) * CH + lane] = sd;
-
-    float4 gl = make_float4(0.f, 0.f, 0.f, 0.f);
-    load_chunk<T>(smem + ((it.ce - 1) & 1) * S::buf, p, b, d0, (it.ce - 1) * KC, true);
-    cp_async_commit();
-    for (int64_t j = it.ce - 1; j >= it.cb; --j) {
-        const unsigned char *buf = smem + (j & 1) * S::buf;
-        if (j > it.cb) {
-            load_chunk<T>(smem + ((j - 1) & 1) * S::buf, p, b, d0, (j - 1) * KC, true);
-            cp_async_commit();
-            cp_async_wait<1>();
-        } else {
-            cp_async_wait<0>();
-        }
-        __syncthreads();
         {
             const T *sz = reinterpret_cast<const T *>(buf + S::o_z) + lane;
             const T *sdy = reinterpret_cast<const T *>(buf + S::o_dy) + lane;
@@ -379,15 +358,22 @@ __global__ void __launch_bounds__(NT) scan_bwd_local_kernel(const Params p) {
             }
         }
         __syncthreads();
-        const int tn = p.L - j * KC < KC ? int(p.L - j * KC) : KC;
-        for (int t = tn - 1; t >= 0; --t) {
+        const int tn = p.L - j * KC < KC ? int(p.L - j * KC) : KC;  // valid steps of the chunk
+        for (int t = 0; t < tn; ++t) {
             const float delta = dc[t * CH + lane], dq = dqc[t * CH + lane];
-            const float4 cv = row4<T>(buf + S::o_c, t, 4 * warp), a = abar4(delta * kLog2e, Aq);
-            gl = mul4(a, fma4s(dq, cv, gl));
+            const float4 a = abar4(delta * kLog2e, Aq);
+            const float4 bv = row4<T>(buf + S::o_b, t, 4 * warp), cv = row4<T>(buf + S::o_c, t, 4 * warp);
+            const float xv = Tok<T>::to_f(sx[t * CH]);
+            h = fma4(a, h, ZOH ? mul4(mul4s(zoh_w4(delta, Aq, a), xv), bv) : mul4s(bv, delta * xv));
+            P = mul4(P, a);
+            gl = fma4(P, mul4s(cv, dq), gl);
+            sd += delta;
         }
         __syncthreads();
     }
+    p.hloc[slot] = h;
     p.gloc[slot] = gl;
+    if (warp == 0) p.sdel[(it.g * p.K + it.k) * CH + lane] = sd;
 }
 
 // B. One thread per (group, warp quad, lane): the true start state of every segment
