@@ -253,9 +253,10 @@ __device__ __forceinline__ float4 step4(const float4 h, const float delta, const
 // shared memory with the channels across a thread's loop rather than across lanes (no
 // shuffle reduction in the reverse step). Thread tid takes step s = tid / 8, the four
 // states of warp slot q = (tid / 2) % 4 and half the channels (tid % 2); the channel
-// order is rotated per thread pair so that a warp's 16-byte loads touch 32 different
-// channels (four wavefronts, the minimum). Pairs combine by one shuffle round; the first
-// of each pair adds the four sums to out[(b L + t) N + n] for steps t < L.
+// order is rotated per thread so that each eight threads served together by a 16-byte
+// load read eight different bank groups (channel mod 8: four wavefronts per warp, the
+// minimum) and a warp's 4-byte loads 32 different banks. Pairs combine by one shuffle
+// round; the first of each pair adds the four sums to out[(b L + t) N + n] for t < L.
 __device__ __forceinline__ void reduce_channels(const float4 *v, const float *w, float *out, const int64_t row0,
                                                 const int64_t tvalid, const int64_t N) {
     const int tid = threadIdx.x;
@@ -263,7 +264,7 @@ __device__ __forceinline__ void reduce_channels(const float4 *v, const float *w,
     float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll 4
     for (int j = 0; j < 16; ++j) {
-        const int c = hf * 16 + ((j + rot) & 15);
+        const int c = hf * 16 + ((j + rot + 4 * hf) & 15);
         const float4 x = v[(s * CW + q) * CH + c];
         acc = w ? fma4s(w[s * CH + c], x, acc) : cat4(__fadd2_rn(lo2(acc), lo2(x)), __fadd2_rn(hi2(acc), hi2(x)));
     }
