@@ -477,15 +477,21 @@ __global__ void __launch_bounds__(NT) scan_bwd_kernel(const Params p) {
         const float4 hz = ck[j * CW * CH], P = abar4(cum[j * CH] * kLog2e, Aq);
         const float4 hck = make_float4(fmaf(P.x, hseg.x, hz.x), fmaf(P.y, hseg.y, hz.y), fmaf(P.z, hseg.z, hz.z),
                                        fmaf(P.w, hseg.w, hz.w));
-        // the state after the first half, from the checkpoint
+        // the first half's states from the checkpoint, kept in registers until the first
+        // half's turn (the second half's go to shared memory first)
         delta_pass<T>(sdt, 0, TH, bias, softplus, sdel, warp, lane);
         __syncthreads();
-        float4 hmid = hck;
-#pragma unroll 4
-        for (int t = 0; t < TH; ++t) {
-            const float delta = sdel[t * CH + lane];
-            hmid = step4<ZOH>(hmid, delta, Aq, Tok<T>::to_f(sx[t * CH + lane]), row4<T>(buf + S::o_b, t, 4 * warp));
+        float4 hreg[TH];
+        {
+            float4 hh = hck;
+#pragma unroll
+            for (int t = 0; t < TH; ++t) {
+                const float delta = sdel[t * CH + lane];
+                hh = step4<ZOH>(hh, delta, Aq, Tok<T>::to_f(sx[t * CH + lane]), row4<T>(buf + S::o_b, t, 4 * warp));
+                hreg[t] = hh;
+            }
         }
+        const float4 hmid = hreg[TH - 1];
         __syncthreads();  // sdel is rewritten for the second half
         for (int half = 1; half >= 0; --half) {
             const int tb = half * TH;                   // first step of the half in the chunk
@@ -497,16 +503,24 @@ __global__ void __launch_bounds__(NT) scan_bwd_kernel(const Params p) {
                 ssig[s * CH + lane] = softplus ? sigmoid_f(v) : 1.f;
             }
             __syncthreads();
-            // (a) recompute the half's states and the warps' partial readouts
-            float4 hh = hs;
+            // (a) the half's states into shared memory (the second half recomputed, the first
+            // from registers) and the warps' partial readouts
+            if (half) {
+                float4 hh = hs;
 #pragma unroll 4
-            for (int s = 0; s < TH; ++s) {
-                const int t = tb + s;
-                const float delta = sdel[s * CH + lane];
-                hh = step4<ZOH>(hh, delta, Aq, Tok<T>::to_f(sx[t * CH + lane]), row4<T>(buf + S::o_b, t, 4 * warp));
-                hb[(s * CW + warp) * CH + lane] = hh;
-                const float4 c4 = row4<T>(buf + S::o_c, t, 4 * warp);
-                pa[(warp * TH + s) * CH + lane] = dot4(c4, hh);
+                for (int s = 0; s < TH; ++s) {
+                    const int t = tb + s;
+                    const float delta = sdel[s * CH + lane];
+                    hh = step4<ZOH>(hh, delta, Aq, Tok<T>::to_f(sx[t * CH + lane]), row4<T>(buf + S::o_b, t, 4 * warp));
+                    hb[(s * CW + warp) * CH + lane] = hh;
+                    pa[(warp * TH + s) * CH + lane] = dot4(row4<T>(buf + S::o_c, t, 4 * warp), hh);
+                }
+            } else {
+#pragma unroll
+                for (int s = 0; s < TH; ++s) {
+                    hb[(s * CW + warp) * CH + lane] = hreg[s];
+                    pa[(warp * TH + s) * CH + lane] = dot4(row4<T>(buf + S::o_c, s, 4 * warp), hreg[s]);
+                }
             }
             __syncthreads();
             // (b) per (t, channel): readout, gate, dq, dz
