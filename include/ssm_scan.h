@@ -71,8 +71,10 @@ enum {
                                 carries, a main pass runs every segment from its true start; about
                                 twice the work, used automatically when the channel groups (B x
                                 D / 32) fill at most a quarter of the GPU's block slots and L >=
-                                2048, and forced by this flag; needs the workspace
-                                ssm_scan_workspace_size() gives (a smaller one means the hand-off) */
+                                2048, and asked for by this flag; taken when the workspace is the
+                                one ssm_scan_workspace_size() gives, the sequence spans at least
+                                two segments of 16 tiles (or, under SSM_TEST_SHORT_SEGMENTS, of
+                                one) and groups x segments <= 1024; otherwise the hand-off */
     SSM_SEQ_HANDOFF = 16u,   /* never the sequence-parallel evaluation (with SSM_SEQ_PARALLEL:
                                 SSM_ERR_INVALID) */
     SSM_TEST_SHORT_SEGMENTS = 0x40000000u, /* test hook: time segments of one 32-step tile each,
