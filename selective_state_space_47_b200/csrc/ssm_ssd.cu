@@ -40,8 +40,10 @@ namespace ssd {
 constexpr int Q = 128;        // chunk length (rows of every MMA)
 constexpr int NS = 128;       // states per head
 constexpr int P = 64;         // channels per head
-constexpr int PH = P / 2;     // channels (columns) per thread: each row is split between two warps
-constexpr int NTHREADS = 256; // eight warps: warps w and w+4 own tensor-memory lanes (rows) 32w .. 32w+31
+constexpr int NQ = 4;         // column quarters: each row is split between four warps
+constexpr int PH = P / NQ;    // channels (columns) per thread
+constexpr int PC = PH / 8;    // 16-byte chunks (8 bfloat16) of them
+constexpr int NTHREADS = 128 * NQ;  // 16 warps; warp w owns tensor-memory lanes (rows) 32 (w mod 4) .. +31
 constexpr int SEG = 16;       // chunks per segment (2048 steps)
 constexpr uint64_t kWaitLimitNs = 2000000000ull;
 
@@ -58,7 +60,7 @@ constexpr uint32_t OFF_SLO = OFF_S + kTile64;        // S - high part, rounded t
 constexpr uint32_t OFF_MISC = OFF_SLO + kTile64;
 constexpr uint32_t OFF_ALPHA = OFF_MISC;             // a_t log2 e per row [Q] f32
 constexpr uint32_t OFF_DELTA = OFF_ALPHA + Q * 4;    // Delta_t [Q] f32
-constexpr uint32_t OFF_WSUM = OFF_DELTA + Q * 4;     // per-warp sums of the low-half warps [4] f32
+constexpr uint32_t OFF_WSUM = OFF_DELTA + Q * 4;     // per-warp sums of the first-quarter warps [4] f32
 constexpr uint32_t OFF_BAR = OFF_WSUM + 64;          // mbarriers: load[2], mma
 constexpr uint32_t OFF_TMEM = OFF_BAR + 64;          // tensor-memory base address
 constexpr uint32_t OFF_ITEM = OFF_TMEM + 16;         // claimed item
@@ -135,6 +137,21 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32]) {
     for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
 }
 
+// 16 consecutive float32 columns of this thread's lane (32x32b shape).
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, float (&v)[16]) {
+    uint32_t r[16];
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, "
+        "%15}, [%16];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+        : "r"(taddr)
+        : "memory");
+    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+    for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
+}
+
 // Bounded wait on phase `parity` of an mbarrier (every thread); false if it gave up.
 __device__ __forceinline__ bool wait_phase(uint64_t *bar, uint32_t parity) {
     if (mbar_try_wait(bar, parity)) return true;
@@ -208,9 +225,9 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + OFF_TMEM);
     int *item_slot = reinterpret_cast<int *>(smem + OFF_ITEM);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    // Row (tensor-memory lane) and column half of this thread: warps w and w+4 share the
-    // lanes 32 (w mod 4) .. +31, the first taking the low half of every row's columns.
-    const int row = tid & (Q - 1), half = tid >> 7, quarter = warp & 3;
+    // Row (tensor-memory lane) and column quarter qt of this thread: warps w, w+4, w+8, w+12
+    // share the lanes 32 (w mod 4) .. +31, warp w + 4 qt taking quarter qt of every row.
+    const int row = tid & (Q - 1), qt = tid >> 7, quarter = warp & 3;
 
     if (tid == 0) {
         mbar_init(&bar_load[0], 1);
@@ -251,12 +268,12 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         const float bias = p.dt_bias ? __ldg(p.dt_bias + h) : 0.f;
         const float dskip = p.Dskip ? __ldg(p.Dskip + h) : 0.f;
 
-        // The state at the segment's start: this thread holds S[row][PH half .. +PH) in float32.
+        // The state at the segment's start: this thread holds S[row][PH qt .. +PH) in float32.
         float S[PH];
         if (k == 0) {
 #pragma unroll
             for (int q = 0; q < PH; ++q)
-                S[q] = p.h0 ? __ldg(p.h0 + ((int64_t(b) * p.H + h) * P + PH * half + q) * NS + row) : 0.f;
+                S[q] = p.h0 ? __ldg(p.h0 + ((int64_t(b) * p.H + h) * P + PH * qt + q) * NS + row) : 0.f;
         } else {
             if (tid == 0 && ld_acquire_gpu(p.flags + bh) < uint32_t(k)) {
                 const uint64_t start = globaltimer_ns();
@@ -271,7 +288,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             }
             __syncthreads();
             __threadfence();
-            const float4 *src = reinterpret_cast<const float4 *>(p.carry + (bh * NS + row) * P + PH * half);
+            const float4 *src = reinterpret_cast<const float4 *>(p.carry + (bh * NS + row) * P + PH * qt);
 #pragma unroll
             for (int q = 0; q < PH / 4; ++q) {
                 const float4 v = __ldcg(src + q);
@@ -285,7 +302,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         // bfloat16 parts, S = hi + lo to about 2^-17, so that C S keeps the float32 state's precision
         auto store_S = [&]() {
 #pragma unroll
-            for (int j = 0; j < 4; ++j) {
+            for (int j = 0; j < PC; ++j) {
                 uint32_t hi[4], lo[4];
 #pragma unroll
                 for (int e = 0; e < 4; ++e) {
@@ -293,8 +310,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                     const float2 r = unpack_bf16(hi[e]);
                     lo[e] = pack_bf16(S[8 * j + 2 * e] - r.x, S[8 * j + 2 * e + 1] - r.y);
                 }
-                sts128(sbase + OFF_S + sw_off(row, 4 * half + j), make_uint4(hi[0], hi[1], hi[2], hi[3]));
-                sts128(sbase + OFF_SLO + sw_off(row, 4 * half + j), make_uint4(lo[0], lo[1], lo[2], lo[3]));
+                sts128(sbase + OFF_S + sw_off(row, PC * qt + j), make_uint4(hi[0], hi[1], hi[2], hi[3]));
+                sts128(sbase + OFF_SLO + sw_off(row, PC * qt + j), make_uint4(lo[0], lo[1], lo[2], lo[3]));
             }
         };
         store_S();
@@ -344,11 +361,11 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         tc_fence_after();
         issue_G_Yoff(0);
 
-        // dt of this thread's row for the first chunk (prefetched one chunk ahead; the low half)
+        // dt of this thread's row for the first chunk (prefetched one chunk ahead; first quarter)
         const __nv_bfloat16 *dtp = p.dt + (int64_t(b) * p.L) * p.H + h;
         auto load_dt = [&](int64_t c) -> float {
             const int64_t t = c * Q + row;
-            return (half == 0 && t < p.L) ? __uint_as_float(uint32_t(ldg_u16_early(dtp + t * p.H)) << 16) : 0.f;
+            return (qt == 0 && t < p.L) ? __uint_as_float(uint32_t(ldg_u16_early(dtp + t * p.H)) << 16) : 0.f;
         };
         float dt_next = load_dt(c0);
 
@@ -362,17 +379,17 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             if (tid == 0 && c + 1 < c1) issue_loads(c + 1, buf ^ 1);
             const float dtv = dt_next;
             if (c + 1 < c1) dt_next = load_dt(c + 1);
-            // z of this row's column half (the gate), read early so its latency overlaps the MMAs
-            uint4 zr[4];
+            // z of this row's column quarter (the gate), read early so its latency overlaps the MMAs
+            uint4 zr[PC];
             if (p.z && rvalid) {
                 const uint4 *zp = reinterpret_cast<const uint4 *>(p.z + (int64_t(b) * p.L + trow) * (p.H * P) + h * P);
 #pragma unroll
-                for (int j = 0; j < 4; ++j) zr[j] = ldg_v4_early(zp + 4 * half + j);
+                for (int j = 0; j < PC; ++j) zr[j] = ldg_v4_early(zp + PC * qt + j);
             }
 
-            // Delta and the running sum of A Delta (log2 units) over the chunk's rows (low half)
+            // Delta and the running sum of A Delta (log2 units) over the chunk's rows (first quarter)
             float d = 0.f, a = 0.f;
-            if (half == 0) {
+            if (qt == 0) {
                 if (rvalid) {
                     const float v = dtv + bias;
                     d = p.softplus ? softplus_f(v) : v;
@@ -386,7 +403,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                 if (lane == 31) wsum[quarter] = a;
             }
             __syncthreads();
-            if (half == 0) {
+            if (qt == 0) {
 #pragma unroll
                 for (int w = 0; w < 3; ++w)
                     if (w < quarter) a += wsum[w];
@@ -400,13 +417,13 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             const uint32_t sX = sbase + OFF_X + buf * kTile64, sM = sbase + OFF_M;
             mma_wait();  // G and Y_off of this chunk, issued when its tiles and the state were ready
 
-            // ---- M = G o exp(a_t - a_s) Delta_s [s <= t], bfloat16: row t, columns of this half
+            // ---- M = G o exp(a_t - a_s) Delta_s [s <= t], bfloat16: row t, columns of this quarter
             {
                 const float at = alpha[row];
                 const int t = row;
 #pragma unroll
-                for (int qq = 0; qq < 2; ++qq) {  // 32 columns at a time
-                    const int q = 2 * half + qq;
+                for (int qq = 0; qq < Q / NQ / 32; ++qq) {  // 32 columns at a time
+                    const int q = (Q / NQ / 32) * qt + qq;
                     float g[32];
                     tmem_ld32(tmem + tlane + TM_G + q * 32, g);
                     const bool any = q * 32 <= quarter * 32 + 31;  // some row of this warp reaches these columns
@@ -455,13 +472,13 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             // skip term rounded to bfloat16 inside M would cost up to 2^-9 |D x| where C h and D x
             // nearly cancel)
             const float alast = alpha[Q - 1];
-            uint4 xr[4];
+            uint4 xr[PC];
             {
                 const int s = row;
                 const float w = ex2_approx(alast - alpha[s]) * dlt[s];
 #pragma unroll
-                for (int j = 0; j < 4; ++j) {
-                    const uint32_t ad = sX + sw_off(s, 4 * half + j);
+                for (int j = 0; j < PC; ++j) {
+                    const uint32_t ad = sX + sw_off(s, PC * qt + j);
                     const uint4 v = lds128(ad);
                     xr[j] = v;
                     const float2 e0 = unpack_bf16(v.x), e1 = unpack_bf16(v.y), e2 = unpack_bf16(v.z), e3 = unpack_bf16(v.w);
@@ -487,12 +504,12 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             // ---- epilogue (overlaps the state MMA): y = Y_diag + exp(a_t) Y_off + D x, gate, store
             {
                 const float et = ex2_approx(alpha[row]);
-                float yd[32], yo[32];
-                tmem_ld32(tmem + tlane + TM_YDIAG + half * 32, yd);
-                tmem_ld32(tmem + tlane + TM_YOFF + half * 32, yo);
-                uint32_t out[16];
+                float yd[PH], yo[PH];
+                tmem_ld16(tmem + tlane + TM_YDIAG + qt * PH, yd);
+                tmem_ld16(tmem + tlane + TM_YOFF + qt * PH, yo);
+                uint32_t out[PH / 2];
 #pragma unroll
-                for (int e = 0; e < 32; e += 2) {
+                for (int e = 0; e < PH; e += 2) {
                     const float2 xx = unpack_bf16((&xr[0].x)[e >> 1]);
                     float v0 = fmaf(dskip, xx.x, fmaf(et, yo[e], yd[e]));
                     float v1 = fmaf(dskip, xx.y, fmaf(et, yo[e + 1], yd[e + 1]));
@@ -504,20 +521,20 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                     out[e >> 1] = pack_bf16(v0, v1);
                 }
                 if (rvalid) {
-                    uint4 *dst = reinterpret_cast<uint4 *>(p.y + (int64_t(b) * p.L + trow) * (p.H * P) + h * P + half * 32);
+                    uint4 *dst = reinterpret_cast<uint4 *>(p.y + (int64_t(b) * p.L + trow) * (p.H * P) + h * P + qt * PH);
 #pragma unroll
-                    for (int j = 0; j < 4; ++j) dst[j] = make_uint4(out[4 * j], out[4 * j + 1], out[4 * j + 2], out[4 * j + 3]);
+                    for (int j = 0; j < PC; ++j) dst[j] = make_uint4(out[4 * j], out[4 * j + 1], out[4 * j + 2], out[4 * j + 3]);
                 }
             }
             mma_wait();
 
-            // ---- S <- exp(a_Q) S + S_acc (row n, this half's columns), and its bfloat16 parts
+            // ---- S <- exp(a_Q) S + S_acc (row n, this quarter's columns), and its bfloat16 parts
             {
                 const float eq = ex2_approx(alast);
-                float sa[32];
-                tmem_ld32(tmem + tlane + TM_S + half * 32, sa);
+                float sa[PH];
+                tmem_ld16(tmem + tlane + TM_S + qt * PH, sa);
 #pragma unroll
-                for (int e = 0; e < 32; ++e) S[e] = fmaf(eq, S[e], sa[e]);
+                for (int e = 0; e < PH; ++e) S[e] = fmaf(eq, S[e], sa[e]);
             }
             store_S();
             fence_proxy_async_smem();
@@ -534,10 +551,10 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         if (k == p.K - 1) {
             if (p.h_last) {
 #pragma unroll
-                for (int q = 0; q < PH; ++q) p.h_last[((int64_t(b) * p.H + h) * P + PH * half + q) * NS + row] = S[q];
+                for (int q = 0; q < PH; ++q) p.h_last[((int64_t(b) * p.H + h) * P + PH * qt + q) * NS + row] = S[q];
             }
         } else {
-            float4 *dst = reinterpret_cast<float4 *>(p.carry + (bh * NS + row) * P + PH * half);
+            float4 *dst = reinterpret_cast<float4 *>(p.carry + (bh * NS + row) * P + PH * qt);
 #pragma unroll
             for (int q = 0; q < PH / 4; ++q) dst[q] = make_float4(S[4 * q], S[4 * q + 1], S[4 * q + 2], S[4 * q + 3]);
             __threadfence();
