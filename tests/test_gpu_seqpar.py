@@ -94,10 +94,11 @@ def test_seq_parallel_matches_oracle(ssm, case, general):
     assert y_err(y, y_ho.float().cpu().double().numpy()) <= tol
 
 
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32], ids=["bf16", "f32"])
 @pytest.mark.parametrize("zoh,conv", [(True, False), (False, True), (True, True)], ids=["zoh", "conv", "zoh+conv"])
-def test_seq_parallel_zoh_and_conv(ssm, zoh, conv):
+def test_seq_parallel_zoh_and_conv(ssm, zoh, conv, dtype):
     from selective_state_space_47_b200 import _native
-    Bsz, L, Dm, N, dtype = 2, 3001, 64, 16, torch.bfloat16
+    Bsz, L, Dm, N = 2, 3001, 64, 16
     cpu = synth.scan_inputs(Bsz, L, Dm, N, dtype, seed=2101, h0=True)
     g = torch.Generator().manual_seed(2102)
     cpu["A"] = -torch.rand((Dm, N), generator=g) * 4.0 - 0.05  # general A
@@ -108,8 +109,9 @@ def test_seq_parallel_zoh_and_conv(ssm, zoh, conv):
     assert st == _native.SSM_OK
     y_ref, h_ref = oracle_scan(cpu, exact_zoh=zoh, conv=cv)
     ey, eh = y_err(y, y_ref), h_err(h, h_ref)
-    print(f"\nseq-parallel zoh={zoh} conv={conv}: y {ey:.3e}, h_L {eh:.3e}")
-    assert ey <= TOL["bf16"] and eh <= TOL["bf16"]
+    print(f"\nseq-parallel zoh={zoh} conv={conv} {dtype}: y {ey:.3e}, h_L {eh:.3e}")
+    tol = TOL[dtype_name(cpu["x"])]
+    assert ey <= tol and eh <= tol
     assert eh <= 1e-4
 
 
