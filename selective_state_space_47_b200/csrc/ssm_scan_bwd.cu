@@ -201,51 +201,55 @@ __device__ __forceinline__ float4 abar4(const float dl, const float4 A) {  // dl
     return make_float4(ex2_approx(e.x), ex2_approx(e.y), ex2_approx(e.z), ex2_approx(e.w));
 }
 
-// Exact zero-order hold, one state: the input weight w = (Abar - 1) / A (below |Delta A| =
-// 1/16 by its series Delta (1 + s/2 + s^2/6 + s^3/24 + s^4/120), s = Delta A; Delta for
-// A = 0), and dw/dA = Delta^2 f(s), f(s) = (s e^s - e^s + 1) / s^2, below |s| = 1/2 by its
-// Taylor series sum_k (k + 1) s^k / (k + 2)! (the closed form cancels near 0). dw/dDelta
-// is Abar itself.
-__device__ __forceinline__ float zoh_w1(const float delta, const float A, const float abar) {
-    const float s = delta * A;
-    if (fabsf(s) < 0.0625f)
-        return delta * fmaf(s, fmaf(s, fmaf(s, fmaf(s, 1.f / 120.f, 1.f / 24.f), 1.f / 6.f), 0.5f), 1.f);
-    return __fdividef(abar - 1.f, A);
+// Exact zero-order hold for a lane's four states: the input weight w = (Abar - 1) / A (below
+// |Delta A| = 1/16 by its series Delta (1 + s/2 + s^2/6 + s^3/24 + s^4/120), s = Delta A),
+// and dw/dA = Delta^2 f(s), f(s) = (s e^s - e^s + 1) / s^2 = (s Abar - Abar + 1) / (Delta A)^2,
+// below |s| = 1/2 by its Taylor series sum_k (k + 1) s^k / (k + 2)! (the closed form cancels
+// near 0). dw/dDelta is Abar itself. Both forms are evaluated on packed pairs and the series
+// selected per state (no divergent branch); iA = 1/A (0 for A = 0, where s = 0 always takes
+// the series).
+__device__ __forceinline__ float4 bc4(const float v) { return make_float4(v, v, v, v); }
+__device__ __forceinline__ float4 add4(const float4 a, const float4 b) {
+    return cat4(__fadd2_rn(lo2(a), lo2(b)), __fadd2_rn(hi2(a), hi2(b)));
 }
-__device__ __forceinline__ float zoh_dwdA1(const float delta, const float A, const float abar) {
-    const float s = delta * A;
-    float f;
-    if (fabsf(s) < 0.5f) {
-        f = fmaf(s, 1.f / 403200.f, 1.f / 45360.f);
-        f = fmaf(s, f, 1.f / 5760.f);
-        f = fmaf(s, f, 1.f / 840.f);
-        f = fmaf(s, f, 1.f / 144.f);
-        f = fmaf(s, f, 1.f / 30.f);
-        f = fmaf(s, f, 0.125f);
-        f = fmaf(s, f, 1.f / 3.f);
-        f = fmaf(s, f, 0.5f);
-    } else {
-        f = __fdividef(fmaf(s, abar, 1.f - abar), s * s);
-    }
-    return delta * delta * f;
+__device__ __forceinline__ float4 sel4(const float4 s, const float lim, const float4 ser, const float4 dir) {
+    return make_float4(fabsf(s.x) < lim ? ser.x : dir.x, fabsf(s.y) < lim ? ser.y : dir.y,
+                       fabsf(s.z) < lim ? ser.z : dir.z, fabsf(s.w) < lim ? ser.w : dir.w);
 }
-__device__ __forceinline__ float4 zoh_w4(const float delta, const float4 A, const float4 a) {
-    return make_float4(zoh_w1(delta, A.x, a.x), zoh_w1(delta, A.y, a.y), zoh_w1(delta, A.z, a.z),
-                       zoh_w1(delta, A.w, a.w));
+__device__ __forceinline__ float4 inv4(const float4 A) {  // 1 / A, 0 for A = 0
+    return make_float4(A.x != 0.f ? 1.f / A.x : 0.f, A.y != 0.f ? 1.f / A.y : 0.f, A.z != 0.f ? 1.f / A.z : 0.f,
+                       A.w != 0.f ? 1.f / A.w : 0.f);
 }
-__device__ __forceinline__ float4 zoh_dwdA4(const float delta, const float4 A, const float4 a) {
-    return make_float4(zoh_dwdA1(delta, A.x, a.x), zoh_dwdA1(delta, A.y, a.y), zoh_dwdA1(delta, A.z, a.z),
-                       zoh_dwdA1(delta, A.w, a.w));
+__device__ __forceinline__ float4 zoh_w4(const float delta, const float4 A, const float4 iA, const float4 a) {
+    const float4 s = mul4s(A, delta);
+    float4 q = fma4(s, bc4(1.f / 120.f), bc4(1.f / 24.f));
+    q = fma4(s, q, bc4(1.f / 6.f));
+    q = fma4(s, q, bc4(0.5f));
+    q = fma4(s, q, bc4(1.f));
+    return sel4(s, 0.0625f, mul4s(q, delta), mul4(add4(a, bc4(-1.f)), iA));
+}
+__device__ __forceinline__ float4 zoh_dwdA4(const float delta, const float4 A, const float4 iA, const float4 a) {
+    const float4 s = mul4s(A, delta);
+    float4 f = fma4(s, bc4(1.f / 403200.f), bc4(1.f / 45360.f));
+    f = fma4(s, f, bc4(1.f / 5760.f));
+    f = fma4(s, f, bc4(1.f / 840.f));
+    f = fma4(s, f, bc4(1.f / 144.f));
+    f = fma4(s, f, bc4(1.f / 30.f));
+    f = fma4(s, f, bc4(0.125f));
+    f = fma4(s, f, bc4(1.f / 3.f));
+    f = fma4(s, f, bc4(0.5f));
+    const float4 num = fma4(s, a, add4(bc4(1.f), mul4s(a, -1.f)));
+    return sel4(s, 0.5f, mul4s(f, delta * delta), mul4(num, mul4(iA, iA)));
 }
 
 // One forward step of a lane's four states under either discretisation: the input
 // weight is Delta (ZOH false) or the exact hold's per-state weight.
 template <bool ZOH>
-__device__ __forceinline__ float4 step4(const float4 h, const float delta, const float4 A, const float xv,
-                                        const float4 bv) {
+__device__ __forceinline__ float4 step4(const float4 h, const float delta, const float4 A, const float4 iA,
+                                        const float xv, const float4 bv) {
     const float4 a = abar4(delta * kLog2e, A);
     if (!ZOH) return fwd_step(h, a, delta * xv, bv);
-    return fma4(a, h, mul4(mul4s(zoh_w4(delta, A, a), xv), bv));
+    return fma4(a, h, mul4(mul4s(zoh_w4(delta, A, iA, a), xv), bv));
 }
 
 // dB or dC of a half chunk: for each of its TH steps s and states n, the sum over the 32
@@ -324,6 +328,7 @@ __global__ void __launch_bounds__(NT) scan_bwd_local_kernel(const Params p) {
     for (int k = threadIdx.x; k < int(2 * S::buf / 16); k += NT) reinterpret_cast<float4 *>(smem)[k] = make_float4(0, 0, 0, 0);
     __syncthreads();
     const float4 Aq = quad_of(p.A, d, d, dvalid, warp, p.N);
+    const float4 iAq = ZOH ? inv4(Aq) : make_float4(0.f, 0.f, 0.f, 0.f);
     const float bias = (dvalid && p.dt_bias) ? __ldg(p.dt_bias + d) : 0.f;
     const int64_t slot = (it.g * p.K + it.k) * (CW * CH) + warp * CH + lane;
     float *dc = reinterpret_cast<float *>(smem + S::off_h);            // [KC][CH] Delta of the chunk
@@ -365,7 +370,7 @@ __global__ void __launch_bounds__(NT) scan_bwd_local_kernel(const Params p) {
             const float4 a = abar4(delta * kLog2e, Aq);
             const float4 bv = row4<T>(buf + S::o_b, t, 4 * warp), cv = row4<T>(buf + S::o_c, t, 4 * warp);
             const float xv = Tok<T>::to_f(sx[t * CH]);
-            h = fma4(a, h, ZOH ? mul4(mul4s(zoh_w4(delta, Aq, a), xv), bv) : mul4s(bv, delta * xv));
+            h = fma4(a, h, ZOH ? mul4(mul4s(zoh_w4(delta, Aq, iAq, a), xv), bv) : mul4s(bv, delta * xv));
             P = mul4(P, a);
             gl = fma4(P, mul4s(cv, dq), gl);
             sd += delta;
@@ -431,6 +436,7 @@ __global__ void __launch_bounds__(NT) scan_bwd_kernel(const Params p) {
     __syncthreads();
 
     const float4 Aq = quad_of(p.A, d, d, dvalid, warp, p.N);
+    const float4 iAq = ZOH ? inv4(Aq) : make_float4(0.f, 0.f, 0.f, 0.f);
     const float bias = (dvalid && p.dt_bias) ? __ldg(p.dt_bias + d) : 0.f;
     const float dskip = (dvalid && p.Dskip) ? __ldg(p.Dskip + d) : 0.f;
     float4 *ck = p.ckpt + (g * p.nchunks) * (CW * CH) + warp * CH + lane;
@@ -487,7 +493,7 @@ __global__ void __launch_bounds__(NT) scan_bwd_kernel(const Params p) {
 #pragma unroll
             for (int t = 0; t < TH; ++t) {
                 const float delta = sdel[t * CH + lane];
-                hh = step4<ZOH>(hh, delta, Aq, Tok<T>::to_f(sx[t * CH + lane]), row4<T>(buf + S::o_b, t, 4 * warp));
+                hh = step4<ZOH>(hh, delta, Aq, iAq, Tok<T>::to_f(sx[t * CH + lane]), row4<T>(buf + S::o_b, t, 4 * warp));
                 hreg[t] = hh;
             }
         }
@@ -511,7 +517,7 @@ __global__ void __launch_bounds__(NT) scan_bwd_kernel(const Params p) {
                 for (int s = 0; s < TH; ++s) {
                     const int t = tb + s;
                     const float delta = sdel[s * CH + lane];
-                    hh = step4<ZOH>(hh, delta, Aq, Tok<T>::to_f(sx[t * CH + lane]), row4<T>(buf + S::o_b, t, 4 * warp));
+                    hh = step4<ZOH>(hh, delta, Aq, iAq, Tok<T>::to_f(sx[t * CH + lane]), row4<T>(buf + S::o_b, t, 4 * warp));
                     hb[(s * CW + warp) * CH + lane] = hh;
                     pa[(warp * TH + s) * CH + lane] = dot4(row4<T>(buf + S::o_c, t, 4 * warp), hh);
                 }
@@ -566,8 +572,8 @@ __global__ void __launch_bounds__(NT) scan_bwd_kernel(const Params p) {
                 float4 w = make_float4(0.f, 0.f, 0.f, 0.f);
                 float4 ddq;  // dDelta terms: A_n Abar_n h_{t-1,n} + dw_n/dDelta B_n x
                 if (ZOH) {
-                    w = zoh_w4(delta, Aq, a);
-                    dA = fma4(mul4(gq, zoh_dwdA4(delta, Aq, a)), bx, dA);
+                    w = zoh_w4(delta, Aq, iAq, a);
+                    dA = fma4(mul4(gq, zoh_dwdA4(delta, Aq, iAq, a)), bx, dA);
                     ddq = fma4(Aq, ah, mul4(a, bx));
                 } else {
                     ddq = fma4(Aq, ah, bx);
