@@ -221,7 +221,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     float *dlt = reinterpret_cast<float *>(smem + OFF_DELTA);
     float *wsum = reinterpret_cast<float *>(smem + OFF_WSUM);
     uint64_t *bar_load = reinterpret_cast<uint64_t *>(smem + OFF_BAR);
-    uint64_t *bar_mma = bar_load + 2;
+    uint64_t *bar_mma = bar_load + 2;   // the MMAs thread 0 issues
+    uint64_t *bar_yoff = bar_load + 3;  // Y_off, issued by thread 128 beside thread 0's G
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + OFF_TMEM);
     int *item_slot = reinterpret_cast<int *>(smem + OFF_ITEM);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -233,6 +234,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         mbar_init(&bar_load[0], 1);
         mbar_init(&bar_load[1], 1);
         mbar_init(bar_mma, 1);
+        mbar_init(bar_yoff, 1);
         fence_mbar_init();
         prefetch_tensormap(&tm_b);
         prefetch_tensormap(&tm_c);
@@ -247,7 +249,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
     const uint32_t tlane = uint32_t(quarter * 32) << 16;  // this warp's lane block in tensor-memory addresses
-    uint32_t ph_load[2] = {0, 0}, ph_mma = 0;
+    uint32_t ph_load[2] = {0, 0}, ph_mma = 0, ph_yoff = 0;
     bool ok = true;  // every wait of this thread so far completed
 
     auto mma_wait = [&]() {
@@ -335,13 +337,18 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             if (tid == 0) {
                 tc_fence_after();
                 const uint32_t sB = sbase + OFF_B + buf * kTile128, sC = sbase + OFF_C + buf * kTile128;
-                const uint32_t sS = sbase + OFF_S;
-                constexpr uint32_t iG = idesc_bf16(128, 128, 0, 0), iO = idesc_bf16(128, 64, 0, 1);
+                constexpr uint32_t iG = idesc_bf16(128, 128, 0, 0);
 #pragma unroll
                 for (int kk = 0; kk < NS / 16; ++kk) {
                     const uint32_t koff = (kk >> 2) * kTile64 + (kk & 3) * 32;  // K block, 32 bytes per 16 columns
                     umma(tmem + TM_G, sw128_desc(sC + koff, 16, 1024), sw128_desc(sB + koff, 16, 1024), iG, kk > 0);
                 }
+                umma_commit(bar_mma);
+            } else if (tid == 128) {  // another warp issues C S at the same time (a thread's MMA issue waits)
+                tc_fence_after();
+                const uint32_t sC = sbase + OFF_C + buf * kTile128;
+                const uint32_t sS = sbase + OFF_S;
+                constexpr uint32_t iO = idesc_bf16(128, 64, 0, 1);
 #pragma unroll
                 for (int kk = 0; kk < 2 * (NS / 16); ++kk) {  // C S_hi, then C S_lo into the same accumulator
                     const int k8 = kk & 7;
@@ -350,7 +357,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                     umma(tmem + TM_YOFF, sw128_desc(sC + koff, 16, 1024), sw128_desc(sPart + k8 * 2048, kTile64, 1024),
                          iO, kk > 0);
                 }
-                umma_commit(bar_mma);
+                umma_commit(bar_yoff);
             }
         };
         if (tid == 0) issue_loads(c0, 0);
@@ -416,6 +423,9 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             const uint32_t sB = sbase + OFF_B + buf * kTile128;
             const uint32_t sX = sbase + OFF_X + buf * kTile64, sM = sbase + OFF_M;
             mma_wait();  // G and Y_off of this chunk, issued when its tiles and the state were ready
+            if (!wait_phase(bar_yoff, ph_yoff)) ok = false;
+            ph_yoff ^= 1u;
+            tc_fence_after();
 
             // ---- M = G o exp(a_t - a_s) Delta_s [s <= t], bfloat16: row t, columns of this quarter
             {
