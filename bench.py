@@ -58,6 +58,8 @@ def parse_args(argv=None):
                     help="time only the backward scan on the workload (profiling runs)")
     ap.add_argument("--decode-only", action="store_true",
                     help="run only the recurrent-decode leg (1000 chained steps) and print its line")
+    ap.add_argument("--seqpar-only", action="store_true",
+                    help="run only the long_narrow leg (hand-off against the sequence-parallel evaluation)")
     ap.add_argument("--ssd-only", action="store_true",
                     help="run only the chunked tensor-core (Mamba-2) leg on ssd_layer and print its line")
     return ap.parse_args(argv)
@@ -301,6 +303,15 @@ def run_ours(args):
     if args.ssd_only:
         line = {"metric": METRIC, "n_gpus": world, "data": "synthetic",
                 "ssd": run_ssd(ssm, synth, dev, stream, rank, hbm_peak, tensor_peak, reps=max(1, args.steps))}
+        if world > 1:
+            dist.barrier()
+            dist.destroy_process_group()
+        if rank == 0:
+            print(json.dumps(line), flush=True)
+        return 0
+    if args.seqpar_only:
+        line = {"metric": METRIC, "n_gpus": world, "data": "synthetic",
+                "seq_parallel": run_seq_parallel(ssm, synth, dev, stream, rank, hbm_peak, reps=max(1, args.steps))}
         if world > 1:
             dist.barrier()
             dist.destroy_process_group()

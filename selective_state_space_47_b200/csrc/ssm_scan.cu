@@ -469,13 +469,30 @@ bool plan_scan(const ssm_scan_args *a, ScanPlan *pl) {
     const bool want = occ[1] > 0 && !(a->flags & SSM_SEQ_HANDOFF) &&
                       ((a->flags & SSM_SEQ_PARALLEL) || (4 * pl->G <= slots && a->seqlen >= 64 * TT));
     if (want && a->workspace_bytes >= ws_full(a->batch, a->dim)) {
-        // about two items per block and pass, segments of at least 16 tiles
-        int64_t K = std::max<int64_t>(2, (2 * slots + pl->G - 1) / pl->G);
-        K = std::min<int64_t>(K, (a->seqlen + 16 * TT - 1) / (16 * TT));
-        int64_t seg = (a->seqlen + K - 1) / std::max<int64_t>(K, 1);
-        seg = (seg + TT - 1) / TT * TT;
-        if (a->flags & SSM_TEST_SHORT_SEGMENTS) seg = TT;
-        K = (a->seqlen + seg - 1) / seg;
+        // Segments of at least 16 tiles. The number K of segments minimises the two passes'
+        // length in waves of equal items, (ceil(G K / slots) + ceil(G (K - 1) / slots)) x the
+        // segment length (the smallest such K on ties): e.g. 32 groups on 148 slots take 9
+        // segments (288 + 256 items, two waves each) rather than 10 (320 items need three).
+        const int64_t kmax = std::min<int64_t>(kSeqParMaxItems / std::max<int64_t>(pl->G, 1),
+                                               (a->seqlen + 16 * TT - 1) / (16 * TT));
+        int64_t K = 0, seg = 0;
+        double best = 0.0;
+        for (int64_t k = 2; k <= kmax; ++k) {
+            const int64_t sl = ((a->seqlen + k - 1) / k + TT - 1) / TT * TT;
+            const int64_t kr = (a->seqlen + sl - 1) / sl;
+            if (kr < 2) continue;
+            const double cost = double((pl->G * kr + slots - 1) / slots + (pl->G * (kr - 1) + slots - 1) / slots) *
+                                double(sl);
+            if (K == 0 || cost < best) {
+                best = cost;
+                K = kr;
+                seg = sl;
+            }
+        }
+        if (a->flags & SSM_TEST_SHORT_SEGMENTS) {
+            seg = TT;
+            K = (a->seqlen + seg - 1) / seg;
+        }
         if (K >= 2 && pl->G * K <= kSeqParMaxItems) {
             pl->seqpar = true;
             pl->deep = true;
