@@ -154,3 +154,24 @@ def test_host_path_chunks_take_the_sequence_parallel_evaluation(ssm):
     ey, eh = y_err(y, y_ref), h_err(h, h_ref)
     print(f"\nhost path, 4096-step chunks, one group: y {ey:.3e}, h_L {eh:.3e}")
     assert ey <= TOL["bf16"] and eh <= 1e-4
+
+
+def test_long_narrow_sampled(ssm):
+    """long_narrow (B=1, L=262144, D=1024: the benchmark's sequence-parallel leg) at full size
+    in that leg's launch configuration (general exponentials, the planner's segments); the
+    oracle follows one channel in every one of the 32 groups (at a lane that moves with the
+    group) plus the last channel, over all 262144 steps, so every group's chain of combined
+    carries is compared at full length."""
+    w = synth.WORKLOADS["long_narrow"]
+    inp = synth.scan_inputs(w.batch, w.seqlen, w.dim, w.dstate, w.dtype, seed=synth.SEEDS["long_narrow"],
+                            device="cuda", gate=w.gate)
+    y, h = ssm.scan_fwd(inp["x"], inp["dt"], inp["A"], inp["B"], inp["C"], inp["D"], inp["z"], inp["dt_bias"],
+                        return_last_state=True, general_A=True, seq_parallel=True)
+    torch.cuda.synchronize()
+    groups = torch.arange(w.dim // 32)
+    sel = torch.unique(torch.cat([groups * 32 + (groups * 7) % 32, torch.tensor([w.dim - 1])]))
+    cpu = {k: (v.cpu() if isinstance(v, torch.Tensor) else v) for k, v in inp.items()}
+    y_ref, h_ref = oracle_scan(cpu, sel=sel)
+    e_y, e_h = y_err(y[:, :, sel.cuda()], y_ref), h_err(h[:, sel.cuda()], h_ref)
+    print(f"\nlong_narrow ({len(sel)} channels, all steps, sequence-parallel): y {e_y:.3e}, h_L {e_h:.3e}")
+    assert e_y <= TOL["bf16"] and e_h <= 1e-4
