@@ -18,8 +18,8 @@ import torch
 from . import _native
 from ._native import SSM_A_GENERAL, SSM_DELTA_SOFTPLUS, SSM_EXACT_ZOH
 
-__all__ = ["scan_fwd", "scan_fwd_host", "scan_bwd", "ssd_fwd", "step", "workspace_size", "workspace_status",
-           "ScanWorkspace"]
+__all__ = ["scan_fwd", "scan_fwd_host", "scan_bwd", "selective_scan", "ssd_fwd", "step", "workspace_size",
+           "workspace_status", "ScanWorkspace"]
 
 _TOKEN_DTYPES = {torch.float32: _native.SSM_F32, torch.bfloat16: _native.SSM_BF16}
 
@@ -419,4 +419,43 @@ def ssd_fwd(x, dt, A, B, C, D=None, z=None, dt_bias=None, h0=None, *, delta_soft
     a.workspace_bytes = ws.numel() * ws.element_size()
     with torch.cuda.device(dev):
         _native.check(lib.ssm_ssd_fwd(ctypes.byref(a), _handle(s)), "ssm_ssd_fwd")
+    return (y, h_last) if return_last_state else y
+
+
+class _SelectiveScan(torch.autograd.Function):
+    """scan_fwd as an autograd function: the forward keeps its inputs (the states are not
+    kept: scan_bwd recomputes them) and the backward is scan_bwd."""
+
+    @staticmethod
+    def forward(ctx, x, dt, A, B, C, D, z, dt_bias, h0, conv_w, conv_b, conv_x0, delta_softplus, exact_zoh):
+        conv = {} if conv_w is None else dict(conv_w=conv_w, conv_b=conv_b, conv_x0=conv_x0)
+        y, h_last = scan_fwd(x, dt, A, B, C, D, z, dt_bias, h0, delta_softplus=delta_softplus, exact_zoh=exact_zoh,
+                             return_last_state=True, **conv)
+        ctx.save_for_backward(x, dt, A, B, C, D, z, dt_bias, h0, conv_w, conv_b, conv_x0)
+        ctx.flags = (delta_softplus, exact_zoh)
+        return y, h_last
+
+    @staticmethod
+    def backward(ctx, dy, dh_last):
+        x, dt, A, B, C, D, z, dt_bias, h0, conv_w, conv_b, conv_x0 = ctx.saved_tensors
+        delta_softplus, exact_zoh = ctx.flags
+        conv = {} if conv_w is None else dict(conv_w=conv_w, conv_b=conv_b, conv_x0=conv_x0)
+        dy = torch.zeros_like(x) if dy is None else dy.to(x.dtype).contiguous()
+        dh_last = None if dh_last is None else dh_last.float().contiguous()
+        g = scan_bwd(x, dt, A, B, C, dy, D, z, dt_bias, h0, dh_last, delta_softplus=delta_softplus,
+                     exact_zoh=exact_zoh, **conv)
+        cg = (g.get("dconv_w"), g.get("dconv_b") if conv_b is not None else None, g.get("dconv_x0")) if conv_w is not None \
+            else (None, None, None)
+        return (g["dx"], g["ddt"], g["dA"], g["dB"].to(B.dtype), g["dC"].to(C.dtype),
+                g["dD"] if D is not None else None, g["dz"], g["ddt_bias"] if dt_bias is not None else None,
+                g["dh0"] if h0 is not None else None, *cg, None, None)
+
+
+def selective_scan(x, dt, A, B, C, D=None, z=None, dt_bias=None, h0=None, *, delta_softplus=True, exact_zoh=False,
+                   conv_w=None, conv_b=None, conv_x0=None, return_last_state=False):
+    """The scan with its backward attached for torch.autograd: y (and the final state) from
+    scan_fwd; gradients for every tensor input from scan_bwd (dB and dC in B's and C's
+    dtype). Device tensors as for scan_fwd."""
+    y, h_last = _SelectiveScan.apply(x, dt, A, B, C, D, z, dt_bias, h0, conv_w, conv_b, conv_x0, delta_softplus,
+                                     exact_zoh)
     return (y, h_last) if return_last_state else y
