@@ -676,7 +676,9 @@ __global__ void __launch_bounds__(C::NTHREADS, C::MINB)
             const T *sz = reinterpret_cast<const T *>(stage + S::st_z) + c;
             const float4 *part = reinterpret_cast<const float4 *>(smem + S::part_off + pr * S::part_bytes) + c;
             T *yo = reinterpret_cast<T *>(smem + S::yout_off + (i % YBUF) * S::yout_bytes) + c;
-            epilogue_rows<T>(part, sx, sz, yo, h * TE, dd, p.has_gate != 0);
+            // (the local pass keeps the y of segment 0 only: the other segments' tiles pass through)
+            if (!SEQ || p.mode != kModeLocal || m.k == 0)
+                epilogue_rows<T>(part, sx, sz, yo, h * TE, dd, p.has_gate != 0);
             warp_arrive(&bar_part_free[pr]);  // the consumers may reuse this partial slot
             warp_arrive(&bar_sfree[st]);      // x and z of this stage are no longer needed
             fence_proxy_async_smem();         // y rows written by this thread -> visible to the TMA store
