@@ -23,8 +23,16 @@
 // Work decomposition: one persistent block per SM claims (sequence, head, segment) items in
 // order; a segment of SEG chunks starts from the state its predecessor segment published
 // (bounded release/acquire wait, as in the scan kernel), so the blocks stay balanced for
-// any number of heads. Within an item, the B, C and x tiles of the next chunk are loaded
-// by TMA while the current chunk is computed.
+// any number of heads.
+//
+// Within an item the chunks are software-pipelined. Of a chunk's products only C S needs
+// the state left by the chunk before; G, M X and B^T (w x) do not. So the products of
+// chunk c+1 that do not need the state are issued while chunk c is finished: the sixteen
+// compute warps turn chunk c's accumulators into its rows of y and the new state, then
+// build chunk c+1's M from its G, while a seventeenth warp issues the TMA loads (two
+// chunks ahead) and every MMA as soon as its operands are ready. The weights w of the
+// state update scale B's rows in place (after G has read them), so that M X and
+// B^T (w x) read the same unscaled x and are issued together.
 #include <cudaTypedefs.h>
 #include <stdint.h>
 
@@ -43,7 +51,9 @@ constexpr int P = 64;         // channels per head
 constexpr int NQ = 4;         // column quarters: each row is split between four warps
 constexpr int PH = P / NQ;    // channels (columns) per thread
 constexpr int PC = PH / 8;    // 16-byte chunks (8 bfloat16) of them
-constexpr int NTHREADS = 128 * NQ;  // 16 warps; warp w owns tensor-memory lanes (rows) 32 (w mod 4) .. +31
+constexpr int NCW = 4 * NQ;          // compute warps; warp w owns tensor-memory lanes (rows) 32 (w mod 4) .. +31
+constexpr int NCOMP = 32 * NCW;      // compute threads
+constexpr int NTHREADS = NCOMP + 32; // + the load / MMA warp
 constexpr int SEG = 16;       // chunks per segment (2048 steps)
 constexpr uint64_t kWaitLimitNs = 2000000000ull;
 
@@ -54,22 +64,24 @@ constexpr uint32_t kTile64 = Q * 64 * 2;    // 16 KB: [128][64] bf16
 constexpr uint32_t OFF_B = 0;                        // B chunk [t][n], two buffers
 constexpr uint32_t OFF_C = OFF_B + 2 * kTile128;     // C chunk [t][n], two buffers
 constexpr uint32_t OFF_X = OFF_C + 2 * kTile128;     // x chunk [t][p], two buffers
-constexpr uint32_t OFF_M = OFF_X + 2 * kTile64;      // M [t][s]
-constexpr uint32_t OFF_S = OFF_M + kTile128;         // S [n][p] bfloat16, high part (operand of C S)
+constexpr uint32_t OFF_Z = OFF_X + 2 * kTile64;      // z chunk [t][p] (the gate), one buffer
+constexpr uint32_t OFF_S = OFF_Z + kTile64;          // S [n][p] bfloat16, high part (operand of C S)
 constexpr uint32_t OFF_SLO = OFF_S + kTile64;        // S - high part, rounded to bfloat16 again
 constexpr uint32_t OFF_MISC = OFF_SLO + kTile64;
-constexpr uint32_t OFF_ALPHA = OFF_MISC;             // a_t log2 e per row [Q] f32
-constexpr uint32_t OFF_DELTA = OFF_ALPHA + Q * 4;    // Delta_t [Q] f32
-constexpr uint32_t OFF_WSUM = OFF_DELTA + Q * 4;     // per-warp sums of the first-quarter warps [4] f32
-constexpr uint32_t OFF_BAR = OFF_WSUM + 64;          // mbarriers: load[2], mma
-constexpr uint32_t OFF_TMEM = OFF_BAR + 64;          // tensor-memory base address
-constexpr uint32_t OFF_ITEM = OFF_TMEM + 16;         // claimed item
+constexpr uint32_t OFF_ALPHA = OFF_MISC;             // a_t log2 e per row [2][Q] f32, by the chunk's parity
+constexpr uint32_t OFF_DELTA = OFF_ALPHA + 2 * Q * 4;  // Delta_t per row [2][Q] f32, by the chunk's parity
+constexpr uint32_t OFF_BAR = OFF_DELTA + 2 * Q * 4;  // mbarriers (10)
+constexpr uint32_t OFF_TMEM = OFF_BAR + 128;         // tensor-memory base address
+constexpr uint32_t OFF_ITEM = OFF_TMEM + 16;         // claimed item, abort flag
 constexpr uint32_t SMEM_BYTES = OFF_ITEM + 16 + 1024;  // + slack to align the base to 1024
+static_assert(SMEM_BYTES <= 232448, "227 KB of shared memory per block");
 constexpr uint32_t kLoadBytes = 2 * kTile128 + kTile64;  // one chunk: B, C, x
 
-// Tensor memory: 256 columns x 128 lanes of float32.
-constexpr uint32_t kTmemCols = 256;
-constexpr uint32_t TM_G = 0, TM_S = 0, TM_YOFF = 128, TM_YDIAG = 192;
+// Tensor memory: 512 columns x 128 lanes of 32 bits: G [128 cols], M X [64], B^T (w x) [64],
+// C S as [C S_hi | C S_lo] [128], and M itself [64: two bfloat16 per column], the A operand of
+// M X read by the tensor cores from tensor memory.
+constexpr uint32_t kTmemCols = 512;
+constexpr uint32_t TM_G = 0, TM_YDIAG = 128, TM_S = 192, TM_YOFF = 256, TM_M = 384;
 
 struct Params {
     int64_t Bsz, L, H, nchunks, K, items;  // K: segments per sequence
@@ -116,27 +128,25 @@ __device__ __forceinline__ void umma(uint32_t d_tmem, uint64_t adesc, uint64_t b
         "l"(adesc), "l"(bdesc), "r"(idesc), "r"(acc), "r"(0), "r"(0), "r"(0), "r"(0)
         : "memory");
 }
+// The same with A read from tensor memory (a_tmem: its first column; K = 16 bfloat16 in 8 columns).
+__device__ __forceinline__ void umma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t bdesc, uint32_t idesc, uint32_t acc) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "r"(a_tmem), "l"(bdesc), "r"(idesc), "r"(acc)
+        : "memory");
+}
+// 8 consecutive 32-bit columns of this thread's lane written (32x32b shape); then the wait.
+__device__ __forceinline__ void tmem_st8(uint32_t taddr, const uint32_t (&r)[8]) {
+    asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"r"(taddr), "r"(r[0]),
+                 "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7])
+                 : "memory");
+}
+__device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 __device__ __forceinline__ void umma_commit(uint64_t *bar) {
     asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_u32(bar))
                  : "memory");
 }
-// 32 consecutive float32 columns of this thread's lane (its warp's 32 lanes, 32x32b shape).
-__device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32]) {
-    uint32_t r[32];
-    asm volatile(
-        "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, "
-        "%15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];"
-        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
-          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
-          "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
-          "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
-        : "r"(taddr)
-        : "memory");
-    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
-#pragma unroll
-    for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
-}
-
 // 16 consecutive float32 columns of this thread's lane (32x32b shape).
 __device__ __forceinline__ void tmem_ld16(uint32_t taddr, float (&v)[16]) {
     uint32_t r[16];
@@ -152,13 +162,56 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, float (&v)[16]) {
     for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
 }
 
-// Bounded wait on phase `parity` of an mbarrier (every thread); false if it gave up.
-__device__ __forceinline__ bool wait_phase(uint64_t *bar, uint32_t parity) {
+// Bounded wait on phase `parity` of an mbarrier. A wait that gives up sets the block's abort
+// flag, and every wait returns false at once while it is set, so that a block whose
+// hand-offs broke runs through its remaining steps without waiting and stops at the next item.
+__device__ __forceinline__ bool wait_phase(uint64_t *bar, uint32_t parity, volatile int *abort) {
     if (mbar_try_wait(bar, parity)) return true;
     const uint64_t start = globaltimer_ns();
-    while (!mbar_try_wait(bar, parity))
-        if (globaltimer_ns() - start > kWaitLimitNs) return false;
+    while (!mbar_try_wait(bar, parity)) {
+        if (*abort) return false;
+        if (globaltimer_ns() - start > kWaitLimitNs) {
+            *abort = 1;
+            return false;
+        }
+    }
     return true;
+}
+__device__ __forceinline__ void mbar_arrive1(uint64_t *bar) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+// Barrier of the compute warps alone (named barrier 1).
+__device__ __forceinline__ void comp_sync() { asm volatile("bar.sync 1, %0;" ::"n"(NCOMP) : "memory"); }
+
+// 16 float32 columns of this thread's lane without waiting, and the wait that makes them
+// valid (the registers pass through it, so no use can move above it).
+__device__ __forceinline__ void tmem_ld16_nw(uint32_t taddr, uint32_t (&r)[16]) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, "
+        "%15}, [%16];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+        : "r"(taddr)
+        : "memory");
+}
+__device__ __forceinline__ void tmem_ld8_nw(uint32_t taddr, uint32_t (&r)[8]) {
+    asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7])
+                 : "r"(taddr)
+                 : "memory");
+}
+__device__ __forceinline__ void tmem_wait8(uint32_t (&r)[8]) {
+    asm volatile("tcgen05.wait::ld.sync.aligned;"
+                 : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]), "+r"(r[6]), "+r"(r[7])
+                 :
+                 : "memory");
+}
+__device__ __forceinline__ void tmem_wait16(uint32_t (&r)[16]) {
+    asm volatile("tcgen05.wait::ld.sync.aligned;"
+                 : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]), "+r"(r[6]), "+r"(r[7]),
+                   "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]), "+r"(r[12]), "+r"(r[13]), "+r"(r[14]), "+r"(r[15])
+                 :
+                 : "memory");
 }
 
 // Byte offset of 16-byte chunk j (8 bfloat16) of row r in a [rows][64] block with the
@@ -213,32 +266,47 @@ __device__ __forceinline__ uint4 lds128(uint32_t saddr) {
 // ----------------------------------------------------------------- kernel
 __global__ void __launch_bounds__(NTHREADS, 1)
     ssd_kernel(const __grid_constant__ CUtensorMap tm_b, const __grid_constant__ CUtensorMap tm_c,
-               const __grid_constant__ CUtensorMap tm_x, const Params p) {
+               const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_z, const Params p) {
     extern __shared__ unsigned char smem_raw[];
     unsigned char *smem = reinterpret_cast<unsigned char *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const uint32_t sbase = smem_u32(smem);
     float *alpha = reinterpret_cast<float *>(smem + OFF_ALPHA);
     float *dlt = reinterpret_cast<float *>(smem + OFF_DELTA);
-    float *wsum = reinterpret_cast<float *>(smem + OFF_WSUM);
-    uint64_t *bar_load = reinterpret_cast<uint64_t *>(smem + OFF_BAR);
-    uint64_t *bar_mma = bar_load + 2;   // the MMAs thread 0 issues
-    uint64_t *bar_yoff = bar_load + 3;  // Y_off, issued by thread 128 beside thread 0's G
+    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + OFF_BAR);
+    uint64_t *bar_full = bars;    // [2] a chunk's B, C and x tiles have landed (TMA)
+    uint64_t *bar_g = bars + 2;   // G done
+    uint64_t *bar_ys = bars + 3;  // M X and B^T (w x) done
+    uint64_t *bar_yo = bars + 4;  // C S done
+    uint64_t *bar_sr = bars + 5;  // the compute threads: state stored, the chunk's accumulators, x and z read
+    uint64_t *bar_mr = bars + 6;  // the compute threads: M written, B scaled, G read
+    uint64_t *bar_pf = bars + 7;  // [2] the load warp: a chunk's Delta and prefix stored (by the chunk's parity)
+    uint64_t *bar_z = bars + 9;   // z of the next chunk to finish has landed (TMA)
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + OFF_TMEM);
     int *item_slot = reinterpret_cast<int *>(smem + OFF_ITEM);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + OFF_ITEM + 4);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    // Row (tensor-memory lane) and column quarter qt of this thread: warps w, w+4, w+8, w+12
+    // Compute threads: row (tensor-memory lane) and column quarter qt; warps w, w+4, w+8, w+12
     // share the lanes 32 (w mod 4) .. +31, warp w + 4 qt taking quarter qt of every row.
     const int row = tid & (Q - 1), qt = tid >> 7, quarter = warp & 3;
+    const bool gate = p.z != nullptr;
 
     if (tid == 0) {
-        mbar_init(&bar_load[0], 1);
-        mbar_init(&bar_load[1], 1);
-        mbar_init(bar_mma, 1);
-        mbar_init(bar_yoff, 1);
+        mbar_init(&bar_full[0], 1);
+        mbar_init(&bar_full[1], 1);
+        mbar_init(bar_g, 1);
+        mbar_init(bar_ys, 1);
+        mbar_init(bar_yo, 1);
+        mbar_init(bar_sr, NCOMP);
+        mbar_init(bar_mr, NCOMP);
+        mbar_init(&bar_pf[0], 32);
+        mbar_init(&bar_pf[1], 32);
+        mbar_init(bar_z, 1);
+        *abort_flag = 0;
         fence_mbar_init();
         prefetch_tensormap(&tm_b);
         prefetch_tensormap(&tm_c);
         prefetch_tensormap(&tm_x);
+        if (gate) prefetch_tensormap(&tm_z);
     }
     if (warp == 0) {
         tmem_alloc(tmem_slot, kTmemCols);
@@ -249,12 +317,12 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
     const uint32_t tlane = uint32_t(quarter * 32) << 16;  // this warp's lane block in tensor-memory addresses
-    uint32_t ph_load[2] = {0, 0}, ph_mma = 0, ph_yoff = 0;
-    bool ok = true;  // every wait of this thread so far completed
-
-    auto mma_wait = [&]() {
-        if (!wait_phase(bar_mma, ph_mma)) ok = false;
-        ph_mma ^= 1u;
+    // mbarrier phases, carried across items (each role uses its own)
+    uint32_t ph_full0 = 0, ph_full1 = 0, ph_g = 0, ph_ys = 0, ph_yo = 0, ph_sr = 0, ph_mr = 0, ph_pf0 = 0, ph_pf1 = 0,
+             ph_z = 0;
+    auto wait_bar = [&](uint64_t *bar, uint32_t &ph) {
+        wait_phase(bar, ph, abort_flag);
+        ph ^= 1u;
         tc_fence_after();
     };
 
@@ -262,80 +330,40 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         if (tid == 0) *item_slot = int(atomicAdd(p.counter, 1u));
         __syncthreads();
         const int64_t it = *item_slot;
-        if (it >= p.items) break;
+        if (it >= p.items || *abort_flag) break;
         const int64_t bh = it % (p.Bsz * p.H), k = it / (p.Bsz * p.H);
         const int b = int(bh / p.H), h = int(bh % p.H);
         const int64_t c0 = k * SEG, c1 = c0 + SEG < p.nchunks ? c0 + SEG : p.nchunks;
+        const int nch = int(c1 - c0);
         const float A2 = __ldg(p.A + h) * kLog2e;  // A log2 e
-        const float bias = p.dt_bias ? __ldg(p.dt_bias + h) : 0.f;
-        const float dskip = p.Dskip ? __ldg(p.Dskip + h) : 0.f;
 
-        // The state at the segment's start: this thread holds S[row][PH qt .. +PH) in float32.
-        float S[PH];
-        if (k == 0) {
-#pragma unroll
-            for (int q = 0; q < PH; ++q)
-                S[q] = p.h0 ? __ldg(p.h0 + ((int64_t(b) * p.H + h) * P + PH * qt + q) * NS + row) : 0.f;
-        } else {
-            if (tid == 0 && ld_acquire_gpu(p.flags + bh) < uint32_t(k)) {
-                const uint64_t start = globaltimer_ns();
-                for (uint32_t n = 1;; ++n) {
-                    if (ld_acquire_gpu(p.flags + bh) >= uint32_t(k)) break;
-                    __nanosleep(256);
-                    if ((n & 63u) == 0 && globaltimer_ns() - start > kWaitLimitNs) {
-                        atomicExch(p.status, uint32_t(SSM_ERR_TIMEOUT));
-                        break;
-                    }
-                }
-            }
-            __syncthreads();
-            __threadfence();
-            const float4 *src = reinterpret_cast<const float4 *>(p.carry + (bh * NS + row) * P + PH * qt);
-#pragma unroll
-            for (int q = 0; q < PH / 4; ++q) {
-                const float4 v = __ldcg(src + q);
-                S[4 * q] = v.x;
-                S[4 * q + 1] = v.y;
-                S[4 * q + 2] = v.z;
-                S[4 * q + 3] = v.w;
-            }
-        }
-        // S as the operand of C S: row n, 64 p contiguous (N-major, 128-byte swizzle), in two
-        // bfloat16 parts, S = hi + lo to about 2^-17, so that C S keeps the float32 state's precision
-        auto store_S = [&]() {
-#pragma unroll
-            for (int j = 0; j < PC; ++j) {
-                uint32_t hi[4], lo[4];
-#pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    hi[e] = pack_bf16(S[8 * j + 2 * e], S[8 * j + 2 * e + 1]);
-                    const float2 r = unpack_bf16(hi[e]);
-                    lo[e] = pack_bf16(S[8 * j + 2 * e] - r.x, S[8 * j + 2 * e + 1] - r.y);
-                }
-                sts128(sbase + OFF_S + sw_off(row, PC * qt + j), make_uint4(hi[0], hi[1], hi[2], hi[3]));
-                sts128(sbase + OFF_SLO + sw_off(row, PC * qt + j), make_uint4(lo[0], lo[1], lo[2], lo[3]));
-            }
-        };
-        store_S();
-
-        // TMA loads of chunk c into buffer `buf`: B and C as two 64-column boxes each, x one.
-        auto issue_loads = [&](int64_t c, int buf) {
-            const int t0 = int(c * Q);
-            mbar_arrive_expect_tx(&bar_load[buf], kLoadBytes);
-            unsigned char *bb = smem + OFF_B + buf * kTile128, *cc = smem + OFF_C + buf * kTile128;
-            tma_load_3d(bb, &tm_b, &bar_load[buf], 0, t0, b);
-            tma_load_3d(bb + kTile64, &tm_b, &bar_load[buf], 64, t0, b);
-            tma_load_3d(cc, &tm_c, &bar_load[buf], 0, t0, b);
-            tma_load_3d(cc + kTile64, &tm_c, &bar_load[buf], 64, t0, b);
-            tma_load_3d(smem + OFF_X + buf * kTile64, &tm_x, &bar_load[buf], h * P, t0, b);
-        };
-        // G = C B^T and Y_off = C S of chunk c (buffer buf), once its tiles have landed and S is
-        // in shared memory: issued as soon as possible, ahead of the chunk's own work
-        auto issue_G_Yoff = [&](int buf) {
-            if (!wait_phase(&bar_load[buf], ph_load[buf])) ok = false;
-            ph_load[buf] ^= 1u;
-            if (tid == 0) {
+        if (warp == NCW) {
+            // ---------------- load / MMA warp: lane 0 issues, every lane waits
+            const bool lead = lane == 0;
+            const float bias = p.dt_bias ? __ldg(p.dt_bias + h) : 0.f;
+            auto issue_loads = [&](int64_t c, int buf) {  // B and C as two 64-column boxes each, x one
+                if (!lead || *abort_flag) return;
+                const int t0 = int(c * Q);
+                mbar_arrive_expect_tx(&bar_full[buf], kLoadBytes);
+                unsigned char *bb = smem + OFF_B + buf * kTile128, *cc = smem + OFF_C + buf * kTile128;
+                tma_load_3d(bb, &tm_b, &bar_full[buf], 0, t0, b);
+                tma_load_3d(bb + kTile64, &tm_b, &bar_full[buf], 64, t0, b);
+                tma_load_3d(cc, &tm_c, &bar_full[buf], 0, t0, b);
+                tma_load_3d(cc + kTile64, &tm_c, &bar_full[buf], 64, t0, b);
+                tma_load_3d(smem + OFF_X + buf * kTile64, &tm_x, &bar_full[buf], h * P, t0, b);
+            };
+            auto issue_z = [&](int64_t c) {
+                if (!gate || !lead || *abort_flag) return;
+                mbar_arrive_expect_tx(bar_z, kTile64);
+                tma_load_3d(smem + OFF_Z, &tm_z, bar_z, h * P, int(c * Q), b);
+            };
+            // G = C B^T of the chunk in buffer buf, once its tiles have landed
+            auto issue_G = [&](int buf) {
+                uint32_t &ph = buf ? ph_full1 : ph_full0;
+                wait_phase(&bar_full[buf], ph, abort_flag);
+                ph ^= 1u;
                 tc_fence_after();
+                if (!lead || *abort_flag) return;
                 const uint32_t sB = sbase + OFF_B + buf * kTile128, sC = sbase + OFF_C + buf * kTile128;
                 constexpr uint32_t iG = idesc_bf16(128, 128, 0, 0);
 #pragma unroll
@@ -343,108 +371,188 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                     const uint32_t koff = (kk >> 2) * kTile64 + (kk & 3) * 32;  // K block, 32 bytes per 16 columns
                     umma(tmem + TM_G, sw128_desc(sC + koff, 16, 1024), sw128_desc(sB + koff, 16, 1024), iG, kk > 0);
                 }
-                umma_commit(bar_mma);
-            } else if (tid == 128) {  // another warp issues C S at the same time (a thread's MMA issue waits)
-                tc_fence_after();
+                umma_commit(bar_g);
+            };
+            // C [S_hi | S_lo]: one N = 128 product (S_lo's block follows S_hi's, 16 KB on)
+            auto issue_Yoff = [&](int buf) {
+                if (!lead || *abort_flag) return;
                 const uint32_t sC = sbase + OFF_C + buf * kTile128;
-                const uint32_t sS = sbase + OFF_S;
-                constexpr uint32_t iO = idesc_bf16(128, 64, 0, 1);
+                constexpr uint32_t iO = idesc_bf16(128, 128, 0, 1);
 #pragma unroll
-                for (int kk = 0; kk < 2 * (NS / 16); ++kk) {  // C S_hi, then C S_lo into the same accumulator
-                    const int k8 = kk & 7;
-                    const uint32_t koff = (k8 >> 2) * kTile64 + (k8 & 3) * 32;
-                    const uint32_t sPart = kk < 8 ? sS : sbase + OFF_SLO;
-                    umma(tmem + TM_YOFF, sw128_desc(sC + koff, 16, 1024), sw128_desc(sPart + k8 * 2048, kTile64, 1024),
+                for (int kk = 0; kk < NS / 16; ++kk) {
+                    const uint32_t koff = (kk >> 2) * kTile64 + (kk & 3) * 32;
+                    umma(tmem + TM_YOFF, sw128_desc(sC + koff, 16, 1024), sw128_desc(sbase + OFF_S + kk * 2048, kTile64, 1024),
                          iO, kk > 0);
                 }
-                umma_commit(bar_yoff);
-            }
-        };
-        if (tid == 0) issue_loads(c0, 0);
-        // make S (written by threads) visible to the tensor cores before the first C S
-        fence_proxy_async_smem();
-        tc_fence_before();
-        __syncthreads();
-        tc_fence_after();
-        issue_G_Yoff(0);
-
-        // dt of this thread's row for the first chunk (prefetched one chunk ahead; first quarter)
-        const __nv_bfloat16 *dtp = p.dt + (int64_t(b) * p.L) * p.H + h;
-        auto load_dt = [&](int64_t c) -> float {
-            const int64_t t = c * Q + row;
-            return (qt == 0 && t < p.L) ? __uint_as_float(uint32_t(ldg_u16_early(dtp + t * p.H)) << 16) : 0.f;
-        };
-        float dt_next = load_dt(c0);
-
-        for (int64_t c = c0; c < c1; ++c) {
-            const int buf = int((c - c0) & 1);
-            const int64_t t0 = c * Q;
-            const int64_t trow = t0 + row;
-            const bool rvalid = trow < p.L;
-            // the next chunk's loads go into the other buffer, whose last readers (the
-            // previous chunk's MMAs) have completed
-            if (tid == 0 && c + 1 < c1) issue_loads(c + 1, buf ^ 1);
-            const float dtv = dt_next;
-            if (c + 1 < c1) dt_next = load_dt(c + 1);
-            // z of this row's column quarter (the gate), read early so its latency overlaps the MMAs
-            uint4 zr[PC];
-            if (p.z && rvalid) {
-                const uint4 *zp = reinterpret_cast<const uint4 *>(p.z + (int64_t(b) * p.L + trow) * (p.H * P) + h * P);
+                umma_commit(bar_yo);
+            };
+            // M X (M from tensor memory) and (w B)^T x: both read the chunk's unscaled x
+            auto issue_YdS = [&](int buf) {
+                if (!lead || *abort_flag) return;
+                const uint32_t sB = sbase + OFF_B + buf * kTile128, sX = sbase + OFF_X + buf * kTile64;
+                constexpr uint32_t iY = idesc_bf16(128, 64, 0, 1);
 #pragma unroll
-                for (int j = 0; j < PC; ++j) zr[j] = ldg_v4_early(zp + PC * qt + j);
-            }
-
-            // Delta and the running sum of A Delta (log2 units) over the chunk's rows (first quarter)
-            float d = 0.f, a = 0.f;
-            if (qt == 0) {
-                if (rvalid) {
-                    const float v = dtv + bias;
-                    d = p.softplus ? softplus_f(v) : v;
+                for (int kk = 0; kk < Q / 16; ++kk)
+                    umma_ts(tmem + TM_YDIAG, tmem + TM_M + kk * 8, sw128_desc(sX + kk * 2048, kTile64, 1024), iY, kk > 0);
+                constexpr uint32_t iS = idesc_bf16(128, 64, 1, 1);  // A is B read N-major (rows n across its two blocks)
+#pragma unroll
+                for (int kk = 0; kk < Q / 16; ++kk)
+                    umma(tmem + TM_S, sw128_desc(sB + kk * 2048, kTile64, 1024), sw128_desc(sX + kk * 2048, kTile64, 1024),
+                         iS, kk > 0);
+                umma_commit(bar_ys);
+            };
+            // dt of chunk c's rows 4 lane .. 4 lane + 3 (zero past L), read a loader iteration
+            // before its use: the registers carry it over the loop's back edge
+            auto load_dt4 = [&](int64_t c, float (&v)[4]) {
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    const int64_t t = c * Q + 4 * lane + j;
+                    v[j] = t < p.L ? __uint_as_float(uint32_t(ldg_u16_early(p.dt + (int64_t(b) * p.L + t) * p.H + h)) << 16) : 0.f;
                 }
-                a = d * A2;
+            };
+            // Delta_t and a_t = A (Delta_1 + ... + Delta_t) log2 e of chunk c (slot = its parity in the
+            // item) from its dt: lane l takes rows 4l .. 4l+3, a running sum over them, then a scan of
+            // the lanes' totals; every lane arrives once its rows are stored
+            auto prefix = [&](int64_t c, int slot, const float (&dtv)[4]) {
+                float d4[4], a4[4];
+                float run = 0.f;
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    const int64_t t = c * Q + 4 * lane + j;
+                    float d = 0.f;
+                    if (t < p.L) {
+                        const float v = dtv[j] + bias;
+                        d = p.softplus ? softplus_f(v) : v;
+                    }
+                    d4[j] = d;
+                    run = fmaf(d, A2, run);
+                    a4[j] = run;
+                }
+                float excl = run;
 #pragma unroll
                 for (int o = 1; o < 32; o <<= 1) {
-                    const float n = __shfl_up_sync(0xffffffffu, a, o);
-                    if (lane >= o) a += n;
+                    const float n = __shfl_up_sync(0xffffffffu, excl, o);
+                    if (lane >= o) excl += n;
                 }
-                if (lane == 31) wsum[quarter] = a;
+                excl -= run;  // sum of the preceding lanes' rows
+                *reinterpret_cast<float4 *>(alpha + slot * Q + 4 * lane) =
+                    make_float4(a4[0] + excl, a4[1] + excl, a4[2] + excl, a4[3] + excl);
+                *reinterpret_cast<float4 *>(dlt + slot * Q + 4 * lane) = make_float4(d4[0], d4[1], d4[2], d4[3]);
+                mbar_arrive1(&bar_pf[slot]);
+            };
+
+            float dta[4], dtb[4];
+            load_dt4(c0, dta);
+            load_dt4(c0 + 1, dtb);
+            issue_loads(c0, 0);
+            if (nch > 1) issue_loads(c0 + 1, 1);
+            issue_z(c0);
+            prefix(c0, 0, dta);
+            issue_G(0);
+            wait_bar(bar_sr, ph_sr);  // the segment's start state is in shared memory
+            issue_Yoff(0);
+            if (nch > 1) prefix(c0 + 1, 1, dtb);
+            load_dt4(c0 + 2, dta);
+            wait_bar(bar_mr, ph_mr);  // chunk c0's M
+            issue_YdS(0);
+            if (nch > 1) issue_G(1);
+            for (int i = 0; i < nch; ++i) {
+                wait_bar(bar_sr, ph_sr);  // chunk c0+i finished: its buffer and z's are free, the new state stored
+                if (i + 2 < nch) issue_loads(c0 + i + 2, i & 1);
+                if (i + 1 < nch) {
+                    issue_z(c0 + i + 1);
+                    issue_Yoff((i + 1) & 1);
+                    wait_bar(bar_mr, ph_mr);  // chunk c0+i+1's M
+                    issue_YdS((i + 1) & 1);
+                    if (i + 2 < nch) {
+                        issue_G(i & 1);
+                        prefix(c0 + i + 2, i & 1, dta);
+                        load_dt4(c0 + i + 3, dta);
+                    }
+                }
             }
-            __syncthreads();
-            if (qt == 0) {
+            __syncwarp();
+        } else {
+            // ---------------- compute warps
+            const float dskip = p.Dskip ? __ldg(p.Dskip + h) : 0.f;
+
+            // The state at the segment's start: this thread holds S[row][PH qt .. +PH) in float32.
+            float S[PH];
+            if (k == 0) {
 #pragma unroll
-                for (int w = 0; w < 3; ++w)
-                    if (w < quarter) a += wsum[w];
-                alpha[row] = a;
-                dlt[row] = d;
+                for (int q = 0; q < PH; ++q)
+                    S[q] = p.h0 ? __ldg(p.h0 + ((int64_t(b) * p.H + h) * P + PH * qt + q) * NS + row) : 0.f;
+            } else {
+                if (tid == 0 && ld_acquire_gpu(p.flags + bh) < uint32_t(k)) {
+                    const uint64_t start = globaltimer_ns();
+                    for (uint32_t n = 1;; ++n) {
+                        if (ld_acquire_gpu(p.flags + bh) >= uint32_t(k)) break;
+                        __nanosleep(256);
+                        if ((n & 63u) == 0 && globaltimer_ns() - start > kWaitLimitNs) {
+                            atomicExch(p.status, uint32_t(SSM_ERR_TIMEOUT));
+                            break;
+                        }
+                    }
+                }
+                comp_sync();
+                __threadfence();
+                const float4 *src = reinterpret_cast<const float4 *>(p.carry + (bh * NS + row) * P + PH * qt);
+#pragma unroll
+                for (int q = 0; q < PH / 4; ++q) {
+                    const float4 v = __ldcg(src + q);
+                    S[4 * q] = v.x;
+                    S[4 * q + 1] = v.y;
+                    S[4 * q + 2] = v.z;
+                    S[4 * q + 3] = v.w;
+                }
             }
+            // S as the operand of C S: row n, 64 p contiguous (N-major, 128-byte swizzle), in two
+            // bfloat16 parts, S = hi + lo to about 2^-17, so that C S keeps the float32 state's
+            // precision; then the hand-off to the MMA warp (every thread fences its stores for
+            // the tensor cores and orders its tensor-memory reads before arriving)
+            auto store_S = [&]() {
+#pragma unroll
+                for (int j = 0; j < PC; ++j) {
+                    uint32_t hi[4], lo[4];
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        hi[e] = pack_bf16(S[8 * j + 2 * e], S[8 * j + 2 * e + 1]);
+                        const float2 r = unpack_bf16(hi[e]);
+                        lo[e] = pack_bf16(S[8 * j + 2 * e] - r.x, S[8 * j + 2 * e + 1] - r.y);
+                    }
+                    sts128(sbase + OFF_S + sw_off(row, PC * qt + j), make_uint4(hi[0], hi[1], hi[2], hi[3]));
+                    sts128(sbase + OFF_SLO + sw_off(row, PC * qt + j), make_uint4(lo[0], lo[1], lo[2], lo[3]));
+                }
+                fence_proxy_async_smem();
+                tc_fence_before();
+                mbar_arrive1(bar_sr);
+            };
+            store_S();
 
-            __syncthreads();  // alpha, delta visible
-
-            const uint32_t sB = sbase + OFF_B + buf * kTile128;
-            const uint32_t sX = sbase + OFF_X + buf * kTile64, sM = sbase + OFF_M;
-            mma_wait();  // G and Y_off of this chunk, issued when its tiles and the state were ready
-            if (!wait_phase(bar_yoff, ph_yoff)) ok = false;
-            ph_yoff ^= 1u;
-            tc_fence_after();
-
-            // ---- M = G o exp(a_t - a_s) Delta_s [s <= t], bfloat16: row t, columns of this quarter
-            {
-                const float at = alpha[row];
+            // M = G o exp(a_t - a_s) Delta_s [s <= t] (bfloat16 pairs, row t, this quarter's 32
+            // columns) into tensor memory, and B's row s scaled in place by w_s = exp(a_Q - a_s)
+            // Delta_s (this quarter's 32 columns; G has read B); then the hand-off
+            auto build_M = [&](int slot) {
+                wait_bar(&bar_pf[slot], slot ? ph_pf1 : ph_pf0);
+                wait_bar(bar_g, ph_g);
+                const float *al = alpha + slot * Q, *dl = dlt + slot * Q;
+                const float at = al[row];
                 const int t = row;
 #pragma unroll
-                for (int qq = 0; qq < Q / NQ / 32; ++qq) {  // 32 columns at a time
-                    const int q = (Q / NQ / 32) * qt + qq;
-                    float g[32];
-                    tmem_ld32(tmem + tlane + TM_G + q * 32, g);
-                    const bool any = q * 32 <= quarter * 32 + 31;  // some row of this warp reaches these columns
+                for (int qq = 0; qq < Q / NQ / 16; ++qq) {  // 16 columns at a time
+                    const int q = (Q / NQ / 16) * qt + qq;
+                    float g[16];
+                    tmem_ld16(tmem + tlane + TM_G + q * 16, g);
+                    const bool any = q * 16 <= quarter * 32 + 31;  // some row of this warp reaches these columns
+                    uint32_t mp[8];
 #pragma unroll
-                    for (int j4 = 0; j4 < 4; ++j4) {  // 8 columns per 16-byte chunk
-                        const int sb = q * 32 + j4 * 8;
+                    for (int j4 = 0; j4 < 2; ++j4) {  // 8 columns at a time
+                        const int sb = q * 16 + j4 * 8;
                         float as[8], ds[8];
-                        *reinterpret_cast<float4 *>(as) = *reinterpret_cast<const float4 *>(alpha + sb);  // uniform
-                        *reinterpret_cast<float4 *>(as + 4) = *reinterpret_cast<const float4 *>(alpha + sb + 4);
-                        *reinterpret_cast<float4 *>(ds) = *reinterpret_cast<const float4 *>(dlt + sb);
-                        *reinterpret_cast<float4 *>(ds + 4) = *reinterpret_cast<const float4 *>(dlt + sb + 4);
+                        *reinterpret_cast<float4 *>(as) = *reinterpret_cast<const float4 *>(al + sb);  // uniform
+                        *reinterpret_cast<float4 *>(as + 4) = *reinterpret_cast<const float4 *>(al + sb + 4);
+                        *reinterpret_cast<float4 *>(ds) = *reinterpret_cast<const float4 *>(dl + sb);
+                        *reinterpret_cast<float4 *>(ds + 4) = *reinterpret_cast<const float4 *>(dl + sb + 4);
                         float m[8];
 #pragma unroll
                         for (int e = 0; e < 8; ++e) {
@@ -453,127 +561,102 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                             if (any && s <= t) v = g[j4 * 8 + e] * ex2_approx(at - as[e]) * ds[e];
                             m[e] = v;
                         }
-                        sts128(sM + (sb >> 6) * kTile64 + sw_off(t, (sb & 63) >> 3),
-                               make_uint4(pack_bf16(m[0], m[1]), pack_bf16(m[2], m[3]), pack_bf16(m[4], m[5]),
-                                          pack_bf16(m[6], m[7])));
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) mp[j4 * 4 + e] = pack_bf16(m[2 * e], m[2 * e + 1]);
                     }
+                    tmem_st8(tmem + tlane + TM_M + q * 8, mp);
                 }
-            }
-            fence_proxy_async_smem();
-            tc_fence_before();
-            __syncthreads();
-
-            // ---- Y_diag = M X
-            if (tid == 0) {
-                tc_fence_after();
-                constexpr uint32_t iY = idesc_bf16(128, 64, 0, 1);
+                const float w = ex2_approx(al[Q - 1] - at) * dl[row];
+                const uint32_t sBq = sbase + OFF_B + slot * kTile128 + (qt >> 1) * kTile64;
 #pragma unroll
-                for (int kk = 0; kk < Q / 16; ++kk) {
-                    const uint32_t koff = (kk >> 2) * kTile64 + (kk & 3) * 32;
-                    umma(tmem + TM_YDIAG, sw128_desc(sM + koff, 16, 1024), sw128_desc(sX + kk * 2048, kTile64, 1024),
-                         iY, kk > 0);
-                }
-                umma_commit(bar_mma);
-            }
-            mma_wait();
-
-            // ---- x rows scaled in place by w_s = exp(a_Q - a_s) Delta_s: the operand of the state
-            // update; the raw row stays in registers for the skip D x of the epilogue (float32: a
-            // skip term rounded to bfloat16 inside M would cost up to 2^-9 |D x| where C h and D x
-            // nearly cancel)
-            const float alast = alpha[Q - 1];
-            uint4 xr[PC];
-            {
-                const int s = row;
-                const float w = ex2_approx(alast - alpha[s]) * dlt[s];
-#pragma unroll
-                for (int j = 0; j < PC; ++j) {
-                    const uint32_t ad = sX + sw_off(s, PC * qt + j);
+                for (int j = 0; j < 4; ++j) {
+                    const uint32_t ad = sBq + sw_off(row, (qt & 1) * 4 + j);
                     const uint4 v = lds128(ad);
-                    xr[j] = v;
                     const float2 e0 = unpack_bf16(v.x), e1 = unpack_bf16(v.y), e2 = unpack_bf16(v.z), e3 = unpack_bf16(v.w);
                     sts128(ad, make_uint4(pack_bf16(e0.x * w, e0.y * w), pack_bf16(e1.x * w, e1.y * w),
                                           pack_bf16(e2.x * w, e2.y * w), pack_bf16(e3.x * w, e3.y * w)));
                 }
-            }
-            fence_proxy_async_smem();
-            tc_fence_before();
-            __syncthreads();
+                tmem_wait_st();
+                fence_proxy_async_smem();
+                tc_fence_before();
+                mbar_arrive1(bar_mr);
+            };
+            build_M(0);
 
-            // ---- S_acc = B^T (w x): A is B read N-major (rows n across the two 64-column blocks)
-            if (tid == 0) {
-                tc_fence_after();
-                constexpr uint32_t iS = idesc_bf16(128, 64, 1, 1);
-#pragma unroll
-                for (int kk = 0; kk < Q / 16; ++kk)
-                    umma(tmem + TM_S, sw128_desc(sB + kk * 2048, kTile64, 1024), sw128_desc(sX + kk * 2048, kTile64, 1024),
-                         iS, kk > 0);
-                umma_commit(bar_mma);
-            }
+            for (int i = 0; i < nch; ++i) {
+                const int64_t c = c0 + i;
+                const int slot = i & 1;
+                const int64_t trow = c * Q + row;
+                const bool rvalid = trow < p.L;
 
-            // ---- epilogue (overlaps the state MMA): y = Y_diag + exp(a_t) Y_off + D x, gate, store
-            {
-                const float et = ex2_approx(alpha[row]);
-                float yd[PH], yo[PH];
-                tmem_ld16(tmem + tlane + TM_YDIAG + qt * PH, yd);
-                tmem_ld16(tmem + tlane + TM_YOFF + qt * PH, yo);
-                uint32_t out[PH / 2];
-#pragma unroll
-                for (int e = 0; e < PH; e += 2) {
-                    const float2 xx = unpack_bf16((&xr[0].x)[e >> 1]);
-                    float v0 = fmaf(dskip, xx.x, fmaf(et, yo[e], yd[e]));
-                    float v1 = fmaf(dskip, xx.y, fmaf(et, yo[e + 1], yd[e + 1]));
-                    if (p.z) {
-                        const float2 zz = unpack_bf16(rvalid ? (&zr[0].x)[e >> 1] : 0u);
-                        v0 *= silu_1sfu(zz.x);
-                        v1 *= silu_1sfu(zz.y);
-                    }
-                    out[e >> 1] = pack_bf16(v0, v1);
-                }
-                if (rvalid) {
+                // ---- y = M X + exp(a_t) C S + D x, gate, store (this row, this quarter)
+                wait_bar(bar_yo, ph_yo);
+                wait_bar(bar_ys, ph_ys);
+                if (gate) wait_bar(bar_z, ph_z);
+                {
+                    const float et = ex2_approx(alpha[slot * Q + row]);
                     uint4 *dst = reinterpret_cast<uint4 *>(p.y + (int64_t(b) * p.L + trow) * (p.H * P) + h * P + qt * PH);
 #pragma unroll
-                    for (int j = 0; j < PC; ++j) dst[j] = make_uint4(out[4 * j], out[4 * j + 1], out[4 * j + 2], out[4 * j + 3]);
+                    for (int j = 0; j < PC; ++j) {  // 8 columns at a time
+                        uint32_t rd[8], rh[8], rl[8];
+                        tmem_ld8_nw(tmem + tlane + TM_YDIAG + qt * PH + 8 * j, rd);
+                        tmem_ld8_nw(tmem + tlane + TM_YOFF + qt * PH + 8 * j, rh);
+                        tmem_ld8_nw(tmem + tlane + TM_YOFF + P + qt * PH + 8 * j, rl);
+                        const uint4 xv = lds128(sbase + OFF_X + slot * kTile64 + sw_off(row, PC * qt + j));
+                        const uint4 zv = gate ? lds128(sbase + OFF_Z + sw_off(row, PC * qt + j)) : make_uint4(0, 0, 0, 0);
+                        tmem_wait8(rd);
+                        tmem_wait8(rh);
+                        tmem_wait8(rl);
+                        uint32_t out[4];
+#pragma unroll
+                        for (int e = 0; e < 8; e += 2) {
+                            const float2 xx = unpack_bf16((&xv.x)[e >> 1]);
+                            const float yo0 = __uint_as_float(rh[e]) + __uint_as_float(rl[e]);
+                            const float yo1 = __uint_as_float(rh[e + 1]) + __uint_as_float(rl[e + 1]);
+                            float v0 = fmaf(dskip, xx.x, fmaf(et, yo0, __uint_as_float(rd[e])));
+                            float v1 = fmaf(dskip, xx.y, fmaf(et, yo1, __uint_as_float(rd[e + 1])));
+                            if (gate) {
+                                const float2 zz = unpack_bf16((&zv.x)[e >> 1]);
+                                v0 *= silu_1sfu(zz.x);
+                                v1 *= silu_1sfu(zz.y);
+                            }
+                            out[e >> 1] = pack_bf16(v0, v1);
+                        }
+                        if (rvalid) dst[j] = make_uint4(out[0], out[1], out[2], out[3]);
+                    }
                 }
-            }
-            mma_wait();
 
-            // ---- S <- exp(a_Q) S + S_acc (row n, this quarter's columns), and its bfloat16 parts
-            {
-                const float eq = ex2_approx(alast);
-                float sa[PH];
-                tmem_ld16(tmem + tlane + TM_S + qt * PH, sa);
+                // ---- S <- exp(a_Q) S + B^T (w x) (row n, this quarter's columns), stored for C S
+                {
+                    const float eq = ex2_approx(alpha[slot * Q + Q - 1]);
+                    uint32_t rs[PH];
+                    tmem_ld16_nw(tmem + tlane + TM_S + qt * PH, rs);
+                    tmem_wait16(rs);
 #pragma unroll
-                for (int e = 0; e < PH; ++e) S[e] = fmaf(eq, S[e], sa[e]);
+                    for (int e = 0; e < PH; ++e) S[e] = fmaf(eq, S[e], __uint_as_float(rs[e]));
+                }
+                store_S();
+                if (i + 1 < nch) build_M(slot ^ 1);
             }
-            store_S();
-            fence_proxy_async_smem();
-            tc_fence_before();
-            // a wait that gave up ends the block's work (every later wait would give up too)
-            const int all_ok = __syncthreads_and(ok);
-            tc_fence_after();
-            if (!all_ok) break;
-            if (c + 1 < c1) issue_G_Yoff(buf ^ 1);
-        }
-        if (!__syncthreads_and(ok)) break;
 
-        // ---- the segment's end state: published for the next segment, or h_last
-        if (k == p.K - 1) {
-            if (p.h_last) {
+            // ---- the segment's end state: published for the next segment, or h_last
+            if (k == p.K - 1) {
+                if (p.h_last) {
 #pragma unroll
-                for (int q = 0; q < PH; ++q) p.h_last[((int64_t(b) * p.H + h) * P + PH * qt + q) * NS + row] = S[q];
+                    for (int q = 0; q < PH; ++q) p.h_last[((int64_t(b) * p.H + h) * P + PH * qt + q) * NS + row] = S[q];
+                }
+            } else {
+                float4 *dst = reinterpret_cast<float4 *>(p.carry + (bh * NS + row) * P + PH * qt);
+#pragma unroll
+                for (int q = 0; q < PH / 4; ++q) dst[q] = make_float4(S[4 * q], S[4 * q + 1], S[4 * q + 2], S[4 * q + 3]);
+                __threadfence();
+                comp_sync();
+                if (tid == 0) st_release_gpu(p.flags + bh, uint32_t(k + 1));
             }
-        } else {
-            float4 *dst = reinterpret_cast<float4 *>(p.carry + (bh * NS + row) * P + PH * qt);
-#pragma unroll
-            for (int q = 0; q < PH / 4; ++q) dst[q] = make_float4(S[4 * q], S[4 * q + 1], S[4 * q + 2], S[4 * q + 3]);
-            __threadfence();
-            __syncthreads();
-            if (tid == 0) st_release_gpu(p.flags + bh, uint32_t(k + 1));
         }
         __syncthreads();
     }
-    if (!ok) atomicExch(p.status, uint32_t(SSM_ERR_TIMEOUT));
+    if (tid == 0 && *abort_flag) atomicExch(p.status, uint32_t(SSM_ERR_TIMEOUT));
     tc_fence_before();
     __syncthreads();
     if (warp == 0) tmem_dealloc(tmem, kTmemCols);
@@ -678,10 +761,10 @@ ssm_status ssm_ssd_fwd(const ssm_ssd_args *a, void *stream_) {
             attr_set[dev] = true;
         }
     }
-    CUtensorMap tb, tc, tx;
+    CUtensorMap tb, tc, tx, tz;
     const int64_t D = a->nheads * P;
     if (!map_sw128(&tb, a->Bm, a->batch, a->seqlen, NS) || !map_sw128(&tc, a->Cm, a->batch, a->seqlen, NS) ||
-        !map_sw128(&tx, a->x, a->batch, a->seqlen, D))
+        !map_sw128(&tx, a->x, a->batch, a->seqlen, D) || !map_sw128(&tz, a->z ? a->z : a->x, a->batch, a->seqlen, D))
         return SSM_ERR_CUDA;
     unsigned char *ws = static_cast<unsigned char *>(a->workspace);
     const int64_t BH = a->batch * a->nheads;
@@ -707,7 +790,7 @@ ssm_status ssm_ssd_fwd(const ssm_ssd_args *a, void *stream_) {
     p.carry = reinterpret_cast<float *>(ws + up256(kSsdHeader + size_t(BH) * 4));
     p.softplus = (a->flags & SSM_DELTA_SOFTPLUS) != 0;
     const int grid = int(std::min<int64_t>(p.items, sms));
-    void *args[] = {&tb, &tc, &tx, &p};
+    void *args[] = {&tb, &tc, &tx, &tz, &p};
     const cudaError_t e = cudaLaunchKernel(reinterpret_cast<void *>(ssd_kernel), dim3(grid), dim3(NTHREADS), args,
                                            SMEM_BYTES, stream);
     return e == cudaSuccess ? SSM_OK : SSM_ERR_CUDA;
