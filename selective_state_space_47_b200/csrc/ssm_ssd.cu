@@ -401,19 +401,20 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                          iS, kk > 0);
                 umma_commit(bar_ys);
             };
-            // dt of chunk c's rows 4 lane .. 4 lane + 3 (zero past L), read a loader iteration
-            // before its use: the registers carry it over the loop's back edge
-            auto load_dt4 = [&](int64_t c, float (&v)[4]) {
+            // dt of the chunk's rows 4 lane .. 4 lane + 3 (rows past L read row L - 1; the prefix
+            // zeroes them), loaded a loader iteration before its use: the raw bits ride in registers
+            // over the loop's back edge and are widened only there
+            auto load_dt4 = [&](int64_t c, uint16_t (&v)[4]) {  // raw bits: widened where used, so no wait here
 #pragma unroll
                 for (int j = 0; j < 4; ++j) {
                     const int64_t t = c * Q + 4 * lane + j;
-                    v[j] = t < p.L ? __uint_as_float(uint32_t(ldg_u16_early(p.dt + (int64_t(b) * p.L + t) * p.H + h)) << 16) : 0.f;
+                    v[j] = ldg_u16_early(p.dt + (int64_t(b) * p.L + (t < p.L ? t : p.L - 1)) * p.H + h);
                 }
             };
             // Delta_t and a_t = A (Delta_1 + ... + Delta_t) log2 e of chunk c (slot = its parity in the
             // item) from its dt: lane l takes rows 4l .. 4l+3, a running sum over them, then a scan of
             // the lanes' totals; every lane arrives once its rows are stored
-            auto prefix = [&](int64_t c, int slot, const float (&dtv)[4]) {
+            auto prefix = [&](int64_t c, int slot, const uint16_t (&dtv)[4]) {
                 float d4[4], a4[4];
                 float run = 0.f;
 #pragma unroll
@@ -421,7 +422,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                     const int64_t t = c * Q + 4 * lane + j;
                     float d = 0.f;
                     if (t < p.L) {
-                        const float v = dtv[j] + bias;
+                        const float v = __uint_as_float(uint32_t(dtv[j]) << 16) + bias;
                         d = p.softplus ? softplus_f(v) : v;
                     }
                     d4[j] = d;
@@ -441,7 +442,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                 mbar_arrive1(&bar_pf[slot]);
             };
 
-            float dta[4], dtb[4];
+            uint16_t dta[4], dtb[4];
             load_dt4(c0, dta);
             load_dt4(c0 + 1, dtb);
             issue_loads(c0, 0);
