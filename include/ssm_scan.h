@@ -345,10 +345,11 @@ ssm_status ssm_scan_bwd(const ssm_scan_bwd_args *args, void *stream);
  *   state[p, n] <- exp(Delta_t A[h]) state[p, n] + Delta_t B_t[n] x_t[d]
  *   y_t[d] = (sum_n C_t[n] state[p, n] + D[h] x_t[d]) * silu(z_t[d])   (no gate if z NULL)
  * Evaluated per chunk of 128 steps as four tcgen05 matrix products with float32
- * accumulation: C B^T, the decay-masked matrix times x (the skip D x on its diagonal), C
- * times the chunk's starting state, and B^T times the decay-weighted x for the next state.
- * The operands of the products are rounded to bfloat16 (the decay matrix and the state
- * among them); the state is carried between chunks in float32.
+ * accumulation: C B^T, the decay-masked matrix times x, C times the chunk's starting
+ * state, and the decay-weighted B^T times x for the next state; the skip D x is added in
+ * float32. The operands of the products are bfloat16 (the decay matrix rounded to it; the
+ * state entering C S as two bfloat16 parts, high and low, to keep its float32
+ * precision); the state is carried between chunks in float32.
  * Shapes: x, z, y [B, L, H, P]; dt [B, L, H]; Bm, Cm [B, L, N]; A, Dskip, dt_bias [H];
  * h0, h_last [B, H, P, N] float32 (state[p, n] of head h), NULL for 0 / not wanted.
  * Supported: dtype SSM_BF16, headdim P = 64, dstate N = 128 (the Mamba-2 head shape);
