@@ -70,7 +70,8 @@ constexpr uint32_t OFF_SLO = OFF_S + kTile64;        // S - high part, rounded t
 constexpr uint32_t OFF_MISC = OFF_SLO + kTile64;
 constexpr uint32_t OFF_ALPHA = OFF_MISC;             // a_t log2 e per row [2][Q] f32, by the chunk's parity
 constexpr uint32_t OFF_DELTA = OFF_ALPHA + 2 * Q * 4;  // Delta_t per row [2][Q] f32, by the chunk's parity
-constexpr uint32_t OFF_BAR = OFF_DELTA + 2 * Q * 4;  // mbarriers (10)
+constexpr uint32_t OFF_CF = OFF_DELTA + 2 * Q * 4;   // column factors exp(a_r - a_s) Delta_s [2][4][Q] f32, r = 32 rb
+constexpr uint32_t OFF_BAR = OFF_CF + 2 * 4 * Q * 4; // mbarriers (10)
 constexpr uint32_t OFF_TMEM = OFF_BAR + 128;         // tensor-memory base address
 constexpr uint32_t OFF_ITEM = OFF_TMEM + 16;         // claimed item, abort flag
 constexpr uint32_t SMEM_BYTES = OFF_ITEM + 16 + 1024;  // + slack to align the base to 1024
@@ -239,19 +240,6 @@ __device__ __forceinline__ uint4 ldg_v4_early(const void *p) {
     return v;
 }
 
-// silu(z) = z / (1 + e^-z) with one special-function-unit operation: the exponential there,
-// the reciprocal of d = 1 + e^-z by Newton's method from a seed taken from d's bits
-// (0x7EF311C2 minus them: at most 5% relative error, the constant chosen to minimise that
-// over a binade) and three steps r <- r + r (1 - d r) (6e-8). -z log2 e is clamped at 125,
-// which keeps d inside the seed's range; silu(z) is then z 2^-125, zero to float precision.
-__device__ __forceinline__ float silu_1sfu(float z) {
-    const float d = 1.0f + ex2_approx(fminf(-z * kLog2e, 125.f));
-    float r = __int_as_float(0x7EF311C2 - __float_as_int(d));
-#pragma unroll
-    for (int i = 0; i < 3; ++i) r = fmaf(r, fmaf(-d, r, 1.f), r);
-    return z * r;
-}
-
 __device__ __forceinline__ void sts128(uint32_t saddr, uint4 v) {
     asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(saddr), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w)
                  : "memory");
@@ -272,6 +260,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     const uint32_t sbase = smem_u32(smem);
     float *alpha = reinterpret_cast<float *>(smem + OFF_ALPHA);
     float *dlt = reinterpret_cast<float *>(smem + OFF_DELTA);
+    float *cfac = reinterpret_cast<float *>(smem + OFF_CF);
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + OFF_BAR);
     uint64_t *bar_full = bars;    // [2] a chunk's B, C and x tiles have landed (TMA)
     uint64_t *bar_g = bars + 2;   // G done
@@ -439,6 +428,17 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                 *reinterpret_cast<float4 *>(alpha + slot * Q + 4 * lane) =
                     make_float4(a4[0] + excl, a4[1] + excl, a4[2] + excl, a4[3] + excl);
                 *reinterpret_cast<float4 *>(dlt + slot * Q + 4 * lane) = make_float4(d4[0], d4[1], d4[2], d4[3]);
+                // the factors exp(a_r - a_s) Delta_s of the columns s < r = 32 rb wholly left of row
+                // block rb (a_r - a_s <= 0: at most 1); the other columns' entries are not read
+#pragma unroll
+                for (int rb = 1; rb < 4; ++rb) {
+                    const float ar = __shfl_sync(0xffffffffu, a4[0] + excl, 8 * rb);  // row 32 rb is lane 8 rb's first
+                    float cfv[4];
+#pragma unroll
+                    for (int j = 0; j < 4; ++j)
+                        cfv[j] = 4 * lane + j < 32 * rb ? ex2_approx(ar - (a4[j] + excl)) * d4[j] : 0.f;
+                    *reinterpret_cast<float4 *>(cfac + (slot * 4 + rb) * Q + 4 * lane) = make_float4(cfv[0], cfv[1], cfv[2], cfv[3]);
+                }
                 mbar_arrive1(&bar_pf[slot]);
             };
 
@@ -539,16 +539,30 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                 const float *al = alpha + slot * Q, *dl = dlt + slot * Q;
                 const float at = al[row];
                 const int t = row;
+                // columns wholly left of this warp's row block r = 32 quarter: exp(a_t - a_s) =
+                // exp(a_t - a_r) exp(a_r - a_s), the second factor (times Delta_s) per column
+                const float rt = quarter ? ex2_approx(at - al[32 * quarter]) : 1.f;
+                const float *cf = cfac + (slot * 4 + quarter) * Q;
 #pragma unroll
                 for (int qq = 0; qq < Q / NQ / 16; ++qq) {  // 16 columns at a time
                     const int q = (Q / NQ / 16) * qt + qq;
                     float g[16];
                     tmem_ld16(tmem + tlane + TM_G + q * 16, g);
                     const bool any = q * 16 <= quarter * 32 + 31;  // some row of this warp reaches these columns
+                    const bool left = q * 16 + 15 < quarter * 32;  // every row of this warp is past these columns
                     uint32_t mp[8];
 #pragma unroll
                     for (int j4 = 0; j4 < 2; ++j4) {  // 8 columns at a time
                         const int sb = q * 16 + j4 * 8;
+                        if (left) {
+                            float cs[8];
+                            *reinterpret_cast<float4 *>(cs) = *reinterpret_cast<const float4 *>(cf + sb);  // uniform
+                            *reinterpret_cast<float4 *>(cs + 4) = *reinterpret_cast<const float4 *>(cf + sb + 4);
+#pragma unroll
+                            for (int e = 0; e < 4; ++e)
+                                mp[j4 * 4 + e] = pack_bf16(g[j4 * 8 + 2 * e] * rt * cs[2 * e], g[j4 * 8 + 2 * e + 1] * rt * cs[2 * e + 1]);
+                            continue;
+                        }
                         float as[8], ds[8];
                         *reinterpret_cast<float4 *>(as) = *reinterpret_cast<const float4 *>(al + sb);  // uniform
                         *reinterpret_cast<float4 *>(as + 4) = *reinterpret_cast<const float4 *>(al + sb + 4);
@@ -618,8 +632,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                             float v1 = fmaf(dskip, xx.y, fmaf(et, yo1, __uint_as_float(rd[e + 1])));
                             if (gate) {
                                 const float2 zz = unpack_bf16((&zv.x)[e >> 1]);
-                                v0 *= silu_1sfu(zz.x);
-                                v1 *= silu_1sfu(zz.y);
+                                v0 *= silu_f(zz.x);
+                                v1 *= silu_f(zz.y);
                             }
                             out[e >> 1] = pack_bf16(v0, v1);
                         }
