@@ -356,7 +356,9 @@ ssm_status ssm_scan_bwd(const ssm_scan_bwd_args *args, void *stream);
  * anything else returns SSM_ERR_UNSUPPORTED (ssm_scan_fwd computes the same model for
  * other shapes and float32, one exponential per state). Alignment: x, z, y, Bm, Cm, h0,
  * h_last and the workspace on 16 bytes, A, Dskip, dt_bias on 4. flags: SSM_DELTA_SOFTPLUS
- * only. The workspace (ssm_ssd_workspace_size bytes, caller-owned device memory, one
+ * and the test hook SSM_TEST_DROP_HANDOFF (the first time segment of sequence 0, head 0
+ * does not publish its state: its successor's bounded wait runs out, the status word then
+ * reads SSM_ERR_TIMEOUT and that call's outputs are not valid). The workspace (ssm_ssd_workspace_size bytes, caller-owned device memory, one
  * per concurrently running call) holds a counter, a status word (ssm_workspace_status
  * reads it: SSM_ERR_TIMEOUT if a bounded device wait gave up), a flag per (sequence,
  * head) and the float32 state handed between the time segments of each (B x H x 32 KB).

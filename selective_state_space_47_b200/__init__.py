@@ -368,13 +368,13 @@ def step(x, dt, A, B, C, h, D=None, z=None, dt_bias=None, *, delta_softplus=True
 
 
 def ssd_fwd(x, dt, A, B, C, D=None, z=None, dt_bias=None, h0=None, *, delta_softplus=True,
-            return_last_state=False, out=None, h_last=None, workspace=None, stream=None):
+            return_last_state=False, out=None, h_last=None, workspace=None, stream=None, _test_flags=0):
     """The chunked (Mamba-2) form on the tensor cores (see include/ssm_scan.h, ssm_ssd_fwd).
 
     x, z: [B, L, H, P] bfloat16 (P = 64); dt: [B, L, H] bfloat16 (one step size per head);
     B, C: [B, L, N] bfloat16 (N = 128); A, D, dt_bias: [H] float32 (one scalar A per head);
     h0: [B, H, P, N] float32. Returns y [B, L, H, P] and, with return_last_state, the final
-    state [B, H, P, N] float32.
+    state [B, H, P, N] float32. _test_flags: test hooks of the C ABI (SSM_TEST_DROP_HANDOFF).
     """
     dev = x.device
     if x.dim() != 4:
@@ -405,7 +405,7 @@ def ssd_fwd(x, dt, A, B, C, D=None, z=None, dt_bias=None, h0=None, *, delta_soft
     a = _native.SsdArgs()
     a.batch, a.seqlen, a.nheads, a.headdim, a.dstate = Bsz, L, H, Pd, N
     a.dtype = _TOKEN_DTYPES[tok]
-    a.flags = SSM_DELTA_SOFTPLUS if delta_softplus else 0
+    a.flags = (SSM_DELTA_SOFTPLUS if delta_softplus else 0) | int(_test_flags)
     a.x, a.dt, a.z, a.Bm, a.Cm = (_ptr(t) for t in (x, dt, z, B, C))
     a.A, a.Dskip, a.dt_bias, a.h0 = (_ptr(t) for t in (A, D, dt_bias, h0))
     a.y, a.h_last = _ptr(y), _ptr(h_last)

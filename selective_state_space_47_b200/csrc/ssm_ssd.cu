@@ -92,7 +92,7 @@ struct Params {
     float *h_last;
     uint32_t *counter, *status, *flags;
     float *carry;  // [B*H][NS][P]
-    int softplus;
+    int softplus, drop_handoff;
 };
 
 // ---------------------------------------------------------------- tcgen05
@@ -666,7 +666,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                 for (int q = 0; q < PH / 4; ++q) dst[q] = make_float4(S[4 * q], S[4 * q + 1], S[4 * q + 2], S[4 * q + 3]);
                 __threadfence();
                 comp_sync();
-                if (tid == 0) st_release_gpu(p.flags + bh, uint32_t(k + 1));
+                // (test hook: the first segment of sequence 0, head 0 keeps its state to itself)
+                if (tid == 0 && !(p.drop_handoff && bh == 0 && k == 0)) st_release_gpu(p.flags + bh, uint32_t(k + 1));
             }
         }
         __syncthreads();
@@ -723,7 +724,7 @@ size_t ssd_ws_bytes(int64_t Bsz, int64_t H) {
 ssm_status ssd_validate(const ssm_ssd_args *a) {
     if (!a) return SSM_ERR_INVALID;
     if (a->batch < 0 || a->seqlen < 0 || a->nheads < 0) return SSM_ERR_INVALID;
-    if (a->flags & ~uint32_t(SSM_DELTA_SOFTPLUS)) return SSM_ERR_INVALID;
+    if (a->flags & ~uint32_t(SSM_DELTA_SOFTPLUS | SSM_TEST_DROP_HANDOFF)) return SSM_ERR_INVALID;
     if (a->dtype != SSM_BF16 || a->headdim != ssm::ssd::P || a->dstate != ssm::ssd::NS) return SSM_ERR_UNSUPPORTED;
     if (a->batch > INT32_MAX || a->seqlen > INT32_MAX || a->nheads > (int64_t(1) << 20)) return SSM_ERR_UNSUPPORTED;
     const bool work = a->batch > 0 && a->nheads > 0 && a->seqlen > 0;
@@ -804,6 +805,7 @@ ssm_status ssm_ssd_fwd(const ssm_ssd_args *a, void *stream_) {
     p.flags = reinterpret_cast<uint32_t *>(ws + kSsdHeader);
     p.carry = reinterpret_cast<float *>(ws + up256(kSsdHeader + size_t(BH) * 4));
     p.softplus = (a->flags & SSM_DELTA_SOFTPLUS) != 0;
+    p.drop_handoff = (a->flags & SSM_TEST_DROP_HANDOFF) != 0;
     const int grid = int(std::min<int64_t>(p.items, sms));
     void *args[] = {&tb, &tc, &tx, &tz, &p};
     const cudaError_t e = cudaLaunchKernel(reinterpret_cast<void *>(ssd_kernel), dim3(grid), dim3(NTHREADS), args,

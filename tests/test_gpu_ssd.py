@@ -97,3 +97,21 @@ def test_ssd_rejects_unsupported(ssm):
     dev = {k: (v.cuda() if isinstance(v, torch.Tensor) else v) for k, v in inp.items()}
     with pytest.raises(RuntimeError):
         ssm.ssd_fwd(dev["x"], dev["dt"], dev["A"], dev["B"], dev["C"], dev["D"], dev["z"], dev["dt_bias"])
+
+
+def test_ssd_handoff_timeout_is_reported(ssm):
+    """A dropped state hand-off between time segments (host-requested test hook) makes the
+    successor's bounded wait run out: the call reports SSM_ERR_TIMEOUT, and the next call
+    on the same workspace is correct again (the GPU stays usable)."""
+    from selective_state_space_47_b200 import _native
+    inp = synth.ssd_inputs(1, 4097, 2, seed=4097 + 90, gate=True, h0=False)  # three segments per head
+    dev = {k: (v.cuda() if isinstance(v, torch.Tensor) else v) for k, v in inp.items()}
+    args = [dev[k] for k in ("x", "dt", "A", "B", "C", "D", "z", "dt_bias")]
+    ws = ssm.ScanWorkspace()
+    ssm.ssd_fwd(*args, workspace=ws, _test_flags=_native.SSM_TEST_DROP_HANDOFF)
+    assert ssm.workspace_status(ws) == _native.SSM_ERR_TIMEOUT
+    y = ssm.ssd_fwd(*args, workspace=ws)
+    assert ssm.workspace_status(ws) == _native.SSM_OK
+    y_ref, _ = oracle_ssd(inp)
+    err = rowwise_rel(y.float().cpu().numpy().reshape(1, 4097, 2 * 64), y_ref.reshape(1, 4097, 2 * 64), axis=1)
+    assert err <= 1e-2, err
