@@ -16,9 +16,9 @@
 //   S'    = exp(a_Q) S + B^T diag(exp(a_Q - a_s) Delta_s) X   [N x P] (tensor cores)
 //
 // where S[n, p] is the state at the chunk's start. Every product is a 128-row tcgen05.mma
-// (kind::f16, bfloat16 operands from shared memory, float32 accumulators in tensor memory):
-// G 128x128x128, C S 128x64x128 (twice: S in two bfloat16 parts), M X 128x64x128, B^T (w X)
-// 128x64x128.
+// (kind::f16, bfloat16 operands from shared memory, M from tensor memory, float32
+// accumulators in tensor memory): G 128x128x128, C [S_hi S_lo] 128x128x128 (S in two
+// bfloat16 parts side by side), M X 128x64x128, (w B)^T X 128x64x128.
 //
 // Work decomposition: one persistent block per SM claims (sequence, head, segment) items in
 // order; a segment of SEG chunks starts from the state its predecessor segment published
