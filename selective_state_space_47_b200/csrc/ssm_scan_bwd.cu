@@ -36,6 +36,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <type_traits>
+
 #include "../../include/ssm_scan.h"
 #include "ssm_device.cuh"
 
@@ -83,8 +85,10 @@ struct Smem {
     static constexpr size_t off_del = off_dq + size_t(TH) * CH * 4;
     static constexpr size_t off_sig = off_del + size_t(TH) * CH * 4;
     static constexpr size_t total = off_sig + size_t(TH) * CH * 4;
-    // the local pass needs only the chunk buffers and a chunk's Delta and dq
-    static constexpr size_t local_total = off_h + size_t(2) * KC * CH * 4;
+    // the local pass needs only the chunk buffers, a chunk's Delta and dq, and (bfloat16
+    // tokens) the chunk's B and C rows widened to float [2][KC][16]
+    static constexpr size_t off_lbc = off_h + size_t(2) * KC * CH * 4;
+    static constexpr size_t local_total = off_lbc + (sizeof(T) == 2 ? size_t(2) * KC * kMaxN * 4 : 0);
     static_assert(buf % 16 == 0 && off_h % 16 == 0, "16-byte copies and float4 rows");
 };
 
@@ -333,6 +337,8 @@ __global__ void __launch_bounds__(NT) scan_bwd_local_kernel(const Params p) {
     const int64_t slot = (it.g * p.K + it.k) * (CW * CH) + warp * CH + lane;
     float *dc = reinterpret_cast<float *>(smem + S::off_h);            // [KC][CH] Delta of the chunk
     float *dqc = reinterpret_cast<float *>(smem + S::off_h) + KC * CH;  // [KC][CH] dq of the chunk
+    float *lbc = reinterpret_cast<float *>(smem + S::off_lbc);          // [2][KC][16] B | C rows as float
+    constexpr bool kWiden = !std::is_same<T, float>::value;
 
     float4 *ck = p.ckpt + (it.g * p.nchunks) * (CW * CH) + warp * CH + lane;
     float4 h = make_float4(0.f, 0.f, 0.f, 0.f);
@@ -362,13 +368,23 @@ __global__ void __launch_bounds__(NT) scan_bwd_local_kernel(const Params p) {
                 if (gate) dq *= silu_f(Tok<T>::to_f(sz[t * CH]));
                 dqc[t * CH + lane] = dq;
             }
+            if (kWiden) {  // thread: matrix tid / 64, rows (tid / 4) % 16 and that + 16, states 4 (tid % 4) ..
+                const int m = threadIdx.x >> 6, r = (threadIdx.x >> 2) & 15, n0 = 4 * (threadIdx.x & 3);
+                const size_t src = m ? S::o_c : S::o_b;
+#pragma unroll
+                for (int rr = 0; rr < 2; ++rr)
+                    *reinterpret_cast<float4 *>(lbc + (m * KC + r + 16 * rr) * kMaxN + n0) = row4<T>(buf + src, r + 16 * rr, n0);
+            }
         }
         __syncthreads();
         const int tn = p.L - j * KC < KC ? int(p.L - j * KC) : KC;  // valid steps of the chunk
         for (int t = 0; t < tn; ++t) {
             const float delta = dc[t * CH + lane], dq = dqc[t * CH + lane];
             const float4 a = abar4(delta * kLog2e, Aq);
-            const float4 bv = row4<T>(buf + S::o_b, t, 4 * warp), cv = row4<T>(buf + S::o_c, t, 4 * warp);
+            const float4 bv = kWiden ? *reinterpret_cast<const float4 *>(lbc + t * kMaxN + 4 * warp)
+                                     : row4<T>(buf + S::o_b, t, 4 * warp);
+            const float4 cv = kWiden ? *reinterpret_cast<const float4 *>(lbc + (KC + t) * kMaxN + 4 * warp)
+                                     : row4<T>(buf + S::o_c, t, 4 * warp);
             const float xv = Tok<T>::to_f(sx[t * CH]);
             h = fma4(a, h, ZOH ? mul4(mul4s(zoh_w4(delta, Aq, iAq, a), xv), bv) : mul4s(bv, delta * xv));
             P = mul4(P, a);
