@@ -282,3 +282,60 @@ def test_bwd_rejects_on_host(lib, bad, code):
     assert lib.ssm_scan_bwd(ctypes.byref(a), None) == code
     assert lib.ssm_scan_bwd(None, None) == _native.SSM_ERR_INVALID
     assert lib.ssm_scan_bwd(ctypes.byref(_bwd_args(batch=0)), None) == _native.SSM_OK
+
+
+def _ssd_args(**kw):
+    a = _native.SsdArgs()
+    a.batch, a.seqlen, a.nheads, a.headdim, a.dstate = 2, 300, 3, 64, 128
+    a.dtype = _native.SSM_BF16
+    a.flags = _native.SSM_DELTA_SOFTPLUS
+    fake = 1 << 20  # host-side stand-ins: never dereferenced, the calls must fail first
+    for name in ("x", "dt", "z", "Bm", "Cm", "A", "Dskip", "dt_bias", "h0", "y", "h_last"):
+        setattr(a, name, fake)
+        fake += 1 << 16
+    a.workspace = fake
+    a.workspace_bytes = 1 << 40
+    for k, v in kw.items():
+        setattr(a, k, v)
+    return a
+
+
+def test_ssd_workspace_size(lib):
+    """The chunked form's workspace: a 256-byte header (item counter, status word) and a
+    32-bit flag per (sequence, head), rounded up to 256 bytes, then the float32 state handed
+    between time segments, N x P floats per (sequence, head)."""
+    a = _ssd_args()
+    bh = 2 * 3
+    head = (256 + bh * 4 + 255) // 256 * 256
+    assert lib.ssm_ssd_workspace_size(ctypes.byref(a)) == head + bh * 128 * 64 * 4
+    assert lib.ssm_ssd_workspace_size(ctypes.byref(_ssd_args(batch=-1))) == 0
+    assert lib.ssm_ssd_workspace_size(None) == 0
+
+
+@pytest.mark.parametrize("bad,code", [
+    (dict(flags=_native.SSM_DELTA_SOFTPLUS | _native.SSM_EXACT_ZOH), _native.SSM_ERR_INVALID),      # the scan's flags only
+    (dict(flags=_native.SSM_DELTA_SOFTPLUS | _native.SSM_SEQ_PARALLEL), _native.SSM_ERR_INVALID),
+    (dict(headdim=32), _native.SSM_ERR_UNSUPPORTED),       # the Mamba-2 head shape only
+    (dict(dstate=64), _native.SSM_ERR_UNSUPPORTED),
+    (dict(dtype=_native.SSM_F32), _native.SSM_ERR_UNSUPPORTED),
+    (dict(seqlen=-1), _native.SSM_ERR_INVALID),
+    (dict(x=None), _native.SSM_ERR_INVALID),
+    (dict(A=None), _native.SSM_ERR_INVALID),
+    (dict(y=None), _native.SSM_ERR_INVALID),
+    (dict(y=(1 << 20) + 8), _native.SSM_ERR_UNSUPPORTED),  # tiles move 16 bytes at a time
+    (dict(A=(1 << 20) + 2), _native.SSM_ERR_UNSUPPORTED),
+    (dict(dt=(1 << 20) + 1), _native.SSM_ERR_UNSUPPORTED),
+    (dict(workspace=None), _native.SSM_ERR_INVALID),
+    (dict(workspace_bytes=64), _native.SSM_ERR_INVALID),
+])
+def test_ssd_rejects_on_host(lib, bad, code):
+    assert lib.ssm_ssd_fwd(ctypes.byref(_ssd_args(**bad)), None) == code
+
+
+def test_ssd_accepts_its_test_hook_and_empty_shapes(lib):
+    """The dropped-hand-off hook passes validation; an empty batch or no heads is a no-op
+    that returns before any CUDA call."""
+    hook = _native.SSM_DELTA_SOFTPLUS | _native.SSM_TEST_DROP_HANDOFF
+    assert lib.ssm_ssd_fwd(ctypes.byref(_ssd_args(batch=0, flags=hook)), None) == _native.SSM_OK
+    assert lib.ssm_ssd_fwd(ctypes.byref(_ssd_args(nheads=0)), None) == _native.SSM_OK
+    assert lib.ssm_ssd_fwd(None, None) == _native.SSM_ERR_INVALID
