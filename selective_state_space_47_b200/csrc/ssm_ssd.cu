@@ -71,7 +71,7 @@ constexpr uint32_t OFF_MISC = OFF_SLO + kTile64;
 constexpr uint32_t OFF_ALPHA = OFF_MISC;             // a_t log2 e per row [2][Q] f32, by the chunk's parity
 constexpr uint32_t OFF_DELTA = OFF_ALPHA + 2 * Q * 4;  // Delta_t per row [2][Q] f32, by the chunk's parity
 constexpr uint32_t OFF_CF = OFF_DELTA + 2 * Q * 4;   // column factors exp(a_r - a_s) Delta_s [2][4][Q] f32, r = 32 rb
-constexpr uint32_t OFF_BAR = OFF_CF + 2 * 4 * Q * 4; // mbarriers (10)
+constexpr uint32_t OFF_BAR = OFF_CF + 2 * 4 * Q * 4; // mbarriers (12)
 constexpr uint32_t OFF_TMEM = OFF_BAR + 128;         // tensor-memory base address
 constexpr uint32_t OFF_ITEM = OFF_TMEM + 16;         // claimed item, abort flag
 constexpr uint32_t SMEM_BYTES = OFF_ITEM + 16 + 1024;  // + slack to align the base to 1024
@@ -264,10 +264,12 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + OFF_BAR);
     uint64_t *bar_full = bars;    // [2] a chunk's B, C and x tiles have landed (TMA)
     uint64_t *bar_g = bars + 2;   // G done
-    uint64_t *bar_ys = bars + 3;  // M X and B^T (w x) done
+    uint64_t *bar_yd = bars + 3;  // M X done
+    uint64_t *bar_sa = bars + 10; // B^T (w x) done
+    uint64_t *bar_br = bars + 11; // the compute threads: B scaled
     uint64_t *bar_yo = bars + 4;  // C S done
     uint64_t *bar_sr = bars + 5;  // the compute threads: state stored, the chunk's accumulators, x and z read
-    uint64_t *bar_mr = bars + 6;  // the compute threads: M written, B scaled, G read
+    uint64_t *bar_mr = bars + 6;  // the compute threads: M written, G read
     uint64_t *bar_pf = bars + 7;  // [2] the load warp: a chunk's Delta and prefix stored (by the chunk's parity)
     uint64_t *bar_z = bars + 9;   // z of the next chunk to finish has landed (TMA)
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + OFF_TMEM);
@@ -283,7 +285,9 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         mbar_init(&bar_full[0], 1);
         mbar_init(&bar_full[1], 1);
         mbar_init(bar_g, 1);
-        mbar_init(bar_ys, 1);
+        mbar_init(bar_yd, 1);
+        mbar_init(bar_sa, 1);
+        mbar_init(bar_br, NCOMP);
         mbar_init(bar_yo, 1);
         mbar_init(bar_sr, NCOMP);
         mbar_init(bar_mr, NCOMP);
@@ -307,8 +311,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     const uint32_t tmem = *tmem_slot;
     const uint32_t tlane = uint32_t(quarter * 32) << 16;  // this warp's lane block in tensor-memory addresses
     // mbarrier phases, carried across items (each role uses its own)
-    uint32_t ph_full0 = 0, ph_full1 = 0, ph_g = 0, ph_ys = 0, ph_yo = 0, ph_sr = 0, ph_mr = 0, ph_pf0 = 0, ph_pf1 = 0,
-             ph_z = 0;
+    uint32_t ph_full0 = 0, ph_full1 = 0, ph_g = 0, ph_yd = 0, ph_sa = 0, ph_br = 0, ph_yo = 0, ph_sr = 0;
+    uint32_t ph_mr = 0, ph_pf0 = 0, ph_pf1 = 0, ph_z = 0;
     auto wait_bar = [&](uint64_t *bar, uint32_t &ph) {
         wait_phase(bar, ph, abort_flag);
         ph ^= 1u;
@@ -375,20 +379,26 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                 }
                 umma_commit(bar_yo);
             };
-            // M X (M from tensor memory) and (w B)^T x: both read the chunk's unscaled x
-            auto issue_YdS = [&](int buf) {
+            // M X (M from tensor memory), as soon as M is written; then (w B)^T x, once B's rows
+            // are scaled: both read the chunk's unscaled x, each has its own completion
+            auto issue_Yd = [&](int buf) {
                 if (!lead || *abort_flag) return;
-                const uint32_t sB = sbase + OFF_B + buf * kTile128, sX = sbase + OFF_X + buf * kTile64;
+                const uint32_t sX = sbase + OFF_X + buf * kTile64;
                 constexpr uint32_t iY = idesc_bf16(128, 64, 0, 1);
 #pragma unroll
                 for (int kk = 0; kk < Q / 16; ++kk)
                     umma_ts(tmem + TM_YDIAG, tmem + TM_M + kk * 8, sw128_desc(sX + kk * 2048, kTile64, 1024), iY, kk > 0);
+                umma_commit(bar_yd);
+            };
+            auto issue_Sa = [&](int buf) {
+                if (!lead || *abort_flag) return;
+                const uint32_t sB = sbase + OFF_B + buf * kTile128, sX = sbase + OFF_X + buf * kTile64;
                 constexpr uint32_t iS = idesc_bf16(128, 64, 1, 1);  // A is B read N-major (rows n across its two blocks)
 #pragma unroll
                 for (int kk = 0; kk < Q / 16; ++kk)
                     umma(tmem + TM_S, sw128_desc(sB + kk * 2048, kTile64, 1024), sw128_desc(sX + kk * 2048, kTile64, 1024),
                          iS, kk > 0);
-                umma_commit(bar_ys);
+                umma_commit(bar_sa);
             };
             // dt of the chunk's rows 4 lane .. 4 lane + 3 (rows past L read row L - 1; the prefix
             // zeroes them), loaded a loader iteration before its use: the raw bits ride in registers
@@ -455,7 +465,9 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             if (nch > 1) prefix(c0 + 1, 1, dtb);
             load_dt4(c0 + 2, dta);
             wait_bar(bar_mr, ph_mr);  // chunk c0's M
-            issue_YdS(0);
+            issue_Yd(0);
+            wait_bar(bar_br, ph_br);  // chunk c0's B scaled
+            issue_Sa(0);
             if (nch > 1) issue_G(1);
             for (int i = 0; i < nch; ++i) {
                 wait_bar(bar_sr, ph_sr);  // chunk c0+i finished: its buffer and z's are free, the new state stored
@@ -464,7 +476,9 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                     issue_z(c0 + i + 1);
                     issue_Yoff((i + 1) & 1);
                     wait_bar(bar_mr, ph_mr);  // chunk c0+i+1's M
-                    issue_YdS((i + 1) & 1);
+                    issue_Yd((i + 1) & 1);
+                    wait_bar(bar_br, ph_br);  // chunk c0+i+1's B scaled
+                    issue_Sa((i + 1) & 1);
                     if (i + 2 < nch) {
                         issue_G(i & 1);
                         prefix(c0 + i + 2, i & 1, dta);
@@ -581,6 +595,9 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                     }
                     tmem_st8(tmem + tlane + TM_M + q * 8, mp);
                 }
+                tmem_wait_st();
+                tc_fence_before();
+                mbar_arrive1(bar_mr);  // M X can start
                 const float w = ex2_approx(al[Q - 1] - at) * dl[row];
                 const uint32_t sBq = sbase + OFF_B + slot * kTile128 + (qt >> 1) * kTile64;
 #pragma unroll
@@ -591,10 +608,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                     sts128(ad, make_uint4(pack_bf16(e0.x * w, e0.y * w), pack_bf16(e1.x * w, e1.y * w),
                                           pack_bf16(e2.x * w, e2.y * w), pack_bf16(e3.x * w, e3.y * w)));
                 }
-                tmem_wait_st();
                 fence_proxy_async_smem();
-                tc_fence_before();
-                mbar_arrive1(bar_mr);
+                mbar_arrive1(bar_br);
             };
             build_M(0);
 
@@ -606,7 +621,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
 
                 // ---- y = M X + exp(a_t) C S + D x, gate, store (this row, this quarter)
                 wait_bar(bar_yo, ph_yo);
-                wait_bar(bar_ys, ph_ys);
+                wait_bar(bar_yd, ph_yd);
                 if (gate) wait_bar(bar_z, ph_z);
                 {
                     const float et = ex2_approx(alpha[slot * Q + row]);
@@ -644,6 +659,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                 // ---- S <- exp(a_Q) S + B^T (w x) (row n, this quarter's columns), stored for C S
                 {
                     const float eq = ex2_approx(alpha[slot * Q + Q - 1]);
+                    wait_bar(bar_sa, ph_sa);
                     uint32_t rs[PH];
                     tmem_ld16_nw(tmem + tlane + TM_S + qt * PH, rs);
                     tmem_wait16(rs);
