@@ -620,38 +620,49 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                 const bool rvalid = trow < p.L;
 
                 // ---- y = M X + exp(a_t) C S + D x, gate, store (this row, this quarter)
+                // first the parts that do not need M X: pre = D x + exp(a_t) C S and the gate
+                // silu(z) of the thread's 16 columns, while M X may still be running
                 wait_bar(bar_yo, ph_yo);
-                wait_bar(bar_yd, ph_yd);
                 if (gate) wait_bar(bar_z, ph_z);
+                float pre[PH], gz[PH];
                 {
                     const float et = ex2_approx(alpha[slot * Q + row]);
-                    uint4 *dst = reinterpret_cast<uint4 *>(p.y + (int64_t(b) * p.L + trow) * (p.H * P) + h * P + qt * PH);
 #pragma unroll
                     for (int j = 0; j < PC; ++j) {  // 8 columns at a time
-                        uint32_t rd[8], rh[8], rl[8];
-                        tmem_ld8_nw(tmem + tlane + TM_YDIAG + qt * PH + 8 * j, rd);
+                        uint32_t rh[8], rl[8];
                         tmem_ld8_nw(tmem + tlane + TM_YOFF + qt * PH + 8 * j, rh);
                         tmem_ld8_nw(tmem + tlane + TM_YOFF + P + qt * PH + 8 * j, rl);
                         const uint4 xv = lds128(sbase + OFF_X + slot * kTile64 + sw_off(row, PC * qt + j));
                         const uint4 zv = gate ? lds128(sbase + OFF_Z + sw_off(row, PC * qt + j)) : make_uint4(0, 0, 0, 0);
-                        tmem_wait8(rd);
                         tmem_wait8(rh);
                         tmem_wait8(rl);
-                        uint32_t out[4];
 #pragma unroll
                         for (int e = 0; e < 8; e += 2) {
                             const float2 xx = unpack_bf16((&xv.x)[e >> 1]);
                             const float yo0 = __uint_as_float(rh[e]) + __uint_as_float(rl[e]);
                             const float yo1 = __uint_as_float(rh[e + 1]) + __uint_as_float(rl[e + 1]);
-                            float v0 = fmaf(dskip, xx.x, fmaf(et, yo0, __uint_as_float(rd[e])));
-                            float v1 = fmaf(dskip, xx.y, fmaf(et, yo1, __uint_as_float(rd[e + 1])));
-                            if (gate) {
-                                const float2 zz = unpack_bf16((&zv.x)[e >> 1]);
-                                v0 *= silu_f(zz.x);
-                                v1 *= silu_f(zz.y);
-                            }
-                            out[e >> 1] = pack_bf16(v0, v1);
+                            pre[8 * j + e] = fmaf(dskip, xx.x, et * yo0);
+                            pre[8 * j + e + 1] = fmaf(dskip, xx.y, et * yo1);
+                            const float2 zz = unpack_bf16((&zv.x)[e >> 1]);
+                            gz[8 * j + e] = gate ? silu_f(zz.x) : 1.f;
+                            gz[8 * j + e + 1] = gate ? silu_f(zz.y) : 1.f;
                         }
+                    }
+                }
+                // then y = (M X + pre) silu(z), stored
+                wait_bar(bar_yd, ph_yd);
+                {
+                    uint4 *dst = reinterpret_cast<uint4 *>(p.y + (int64_t(b) * p.L + trow) * (p.H * P) + h * P + qt * PH);
+#pragma unroll
+                    for (int j = 0; j < PC; ++j) {
+                        uint32_t rd[8];
+                        tmem_ld8_nw(tmem + tlane + TM_YDIAG + qt * PH + 8 * j, rd);
+                        tmem_wait8(rd);
+                        uint32_t out[4];
+#pragma unroll
+                        for (int e = 0; e < 8; e += 2)
+                            out[e >> 1] = pack_bf16((__uint_as_float(rd[e]) + pre[8 * j + e]) * gz[8 * j + e],
+                                                    (__uint_as_float(rd[e + 1]) + pre[8 * j + e + 1]) * gz[8 * j + e + 1]);
                         if (rvalid) dst[j] = make_uint4(out[0], out[1], out[2], out[3]);
                     }
                 }
