@@ -599,10 +599,11 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                 tc_fence_before();
                 mbar_arrive1(bar_mr);  // M X can start
                 const float w = ex2_approx(al[Q - 1] - at) * dl[row];
-                const uint32_t sBq = sbase + OFF_B + slot * kTile128 + (qt >> 1) * kTile64;
+                constexpr int BC = NS / NQ;  // B columns of this thread's part of row s
+                const uint32_t sBq = sbase + OFF_B + slot * kTile128 + (qt * BC / 64) * kTile64;
 #pragma unroll
-                for (int j = 0; j < 4; ++j) {
-                    const uint32_t ad = sBq + sw_off(row, (qt & 1) * 4 + j);
+                for (int j = 0; j < BC / 8; ++j) {
+                    const uint32_t ad = sBq + sw_off(row, (qt * BC % 64) / 8 + j);
                     const uint4 v = lds128(ad);
                     const float2 e0 = unpack_bf16(v.x), e1 = unpack_bf16(v.y), e2 = unpack_bf16(v.z), e3 = unpack_bf16(v.w);
                     sts128(ad, make_uint4(pack_bf16(e0.x * w, e0.y * w), pack_bf16(e1.x * w, e1.y * w),
@@ -671,11 +672,14 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                 {
                     const float eq = ex2_approx(alpha[slot * Q + Q - 1]);
                     wait_bar(bar_sa, ph_sa);
-                    uint32_t rs[PH];
-                    tmem_ld16_nw(tmem + tlane + TM_S + qt * PH, rs);
-                    tmem_wait16(rs);
 #pragma unroll
-                    for (int e = 0; e < PH; ++e) S[e] = fmaf(eq, S[e], __uint_as_float(rs[e]));
+                    for (int k16 = 0; k16 < PH / 16; ++k16) {
+                        uint32_t rs[16];
+                        tmem_ld16_nw(tmem + tlane + TM_S + qt * PH + 16 * k16, rs);
+                        tmem_wait16(rs);
+#pragma unroll
+                        for (int e = 0; e < 16; ++e) S[16 * k16 + e] = fmaf(eq, S[16 * k16 + e], __uint_as_float(rs[e]));
+                    }
                 }
                 store_S();
                 if (i + 1 < nch) build_M(slot ^ 1);
