@@ -184,6 +184,23 @@ def test_python_binding_refuses_cpu_tensors():
         ssm.scan_fwd(x, x, torch.zeros(8, 16), torch.zeros(1, 4, 16), torch.zeros(1, 4, 16))
 
 
+def test_python_binding_checks_chunked_form_arguments():
+    """ssd_fwd refuses host tensors and wrong shapes before any CUDA call."""
+    import torch
+    import selective_state_space_47_b200 as ssm
+    Bsz, L, H = 1, 4, 2
+    x = torch.zeros(Bsz, L, H, 64, dtype=torch.bfloat16)
+    dt = torch.zeros(Bsz, L, H, dtype=torch.bfloat16)
+    Bm = torch.zeros(Bsz, L, 128, dtype=torch.bfloat16)
+    A = torch.zeros(H)
+    with pytest.raises(ValueError):  # host tensors
+        ssm.ssd_fwd(x, dt, A, Bm, Bm)
+    with pytest.raises(ValueError):  # x must be [B, L, H, P]
+        ssm.ssd_fwd(x[0], dt, A, Bm, Bm)
+    with pytest.raises(ValueError):  # dt per head, not per channel
+        ssm.ssd_fwd(x, torch.zeros(Bsz, L, H * 64, dtype=torch.bfloat16), A, Bm, Bm)
+
+
 def test_host_scan_staging_size_and_argument_checks(lib):
     """ssm_scan_fwd_host: staging size arithmetic and the checks made before any CUDA call."""
     a = _args()
