@@ -46,3 +46,23 @@ def test_single_rank_helpers_are_identity():
     import bench
     assert bench.max_over_ranks(3.5, 1) == 3.5
     assert bench.sum_over_ranks(2.0, 1) == 2.0
+
+
+def test_reference_arm_prints_the_contract_line():
+    """`bench.py --impl reference` (the float64 oracle on the host cores) prints one JSON line
+    with the contract's keys, its cpu_baseline and an e2e object without host copies."""
+    import json
+    import subprocess
+    import sys
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    out = subprocess.run([sys.executable, os.path.join(root, "bench.py"), "--impl", "reference", "--workload",
+                          "tiny_f32", "--steps", "1", "--warmup", "0"], capture_output=True, text=True, timeout=600,
+                         cwd=root)
+    assert out.returncode == 0, out.stderr[-2000:]
+    line = json.loads(out.stdout.strip().splitlines()[-1])
+    for key in ("impl", "metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step", "higher_is_better",
+                "scaling", "dtype", "data", "config", "cpu_baseline", "e2e"):
+        assert key in line, key
+    assert line["impl"] == "reference" and line["value"] > 0 and line["config"]["workload"] == "tiny_f32"
+    assert line["cpu_baseline"]["kind"] == "oracle" and line["cpu_baseline"]["cores"] >= 1
+    assert line["e2e"]["h2d_bytes_per_step"] == 0 and line["e2e"]["d2h_bytes_per_step"] == 0
